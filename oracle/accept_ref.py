@@ -1,0 +1,235 @@
+"""CPU float64 oracle of the DSpark block verify/accept step.
+
+TEST INFRASTRUCTURE. Only ``tests/``, ``__graft_entry__.smoke()`` and ``bench.py``'s
+CPU-baseline / reference arm may import or run this module. The product path never
+does: it shares no code with this file and imports nothing from ``oracle/``.
+
+What it computes, and where that comes from:
+
+* The logit block. Row 0 of P is p_1, the base distribution for the first drafted
+  token, produced by the anchor step; rows 1..K are p_2..p_{K+1} from one verify
+  forward over the K drafts; row K is the bonus position. Page "dspark-mlx
+  0.1.0__py3-none-any.whl", ``dspark_mlx/adapter.py`` module docstring ("Logit
+  conventions") and the ``StepOut`` / ``BlockOut`` dataclasses.
+* The two accept policies, ``greedy_accept`` and ``speculative_sample_accept``, and the
+  ``AcceptResult`` they return, are named by the same wheel's ``dspark_mlx/__init__.py``
+  (imports from ``.verify``); their bodies are not on the pages. The wheel calls the
+  policy lossless (adapter.py docstring), the mlx-dspark README ("How it works") calls
+  greedy verification identical to plain greedy decoding up to near-tie breaking, and
+  the DeepSeek-V4-Flash DSpark drafter model card calls decoding lossless because the
+  target's verify forward is the only token source.
+* The rule itself is the published speculative-sampling rule (Leviathan, Kalman &
+  Matias 2023; Chen et al. 2023): accept draft x_i with probability min(1, p_i(x_i) /
+  q_i(x_i)); at the first rejection draw from normalize(max(p_i - q_i, 0)); when every
+  draft is accepted draw the bonus token from p_{K+1}. Greedy: accept while the draft
+  equals the base argmax, then emit the argmax of the first mismatching (or bonus) row.
+
+Readings where the pages are silent (each restated in the design notes):
+  temperature divides both P and Q logits; T == 0 means greedy; u[b, i] tests draft i
+  and u[b, K] is the single draw for the resample or bonus token; accept iff
+  u * q(x) < p(x) (strict; q == 0 < p accepts); the inverse CDF runs in ascending token
+  id and returns the smallest v with C(v) > u * Z; argmax ties go to the lowest index
+  and -0.0 equals +0.0; a zero residual mass after a rejection (possible only through
+  rounding) falls back to p_j; a draft id outside [0, V) or a row holding NaN or +inf,
+  or no finite value at all, makes the whole sequence an error (n = 0, tokens -1).
+
+Parity pins: every function here is pinned in ``tests/test_oracle_pins.py`` against
+things other than itself (exact enumeration of losslessness, sequential greedy
+decoding, library inverse-CDF draws, closed-form acceptance rates, chi-square).
+"""
+
+from __future__ import annotations
+
+from dataclasses import dataclass
+from typing import Optional
+
+import numpy as np
+
+STATUS_BAD_DRAFT = 1      # a draft id outside [0, V)
+STATUS_NONFINITE = 2      # a row with NaN / +inf, or with no finite value
+STATUS_ZERO_RESIDUAL = 4  # residual mass was 0 after a rejection; drew from p_j instead
+
+
+@dataclass
+class OracleResult:
+    """Per-sequence outcome of one verify call (the pages' ``AcceptResult``)."""
+
+    n_accepted: np.ndarray          # [B] int32, j in [0, K]; the host's n_keep
+    tokens: np.ndarray              # [B, K+1] int32: x_0..x_{j-1}, then the drawn token, then -1
+    next_token: np.ndarray          # [B] int32: correction (j < K) or bonus (j == K); -1 on error
+    status: np.ndarray              # [B] int32 bit flags (STATUS_*)
+    p_draft: Optional[np.ndarray] = None   # [B, K] float64 p_i(x_i)
+    q_draft: Optional[np.ndarray] = None   # [B, K] float64 q_i(x_i)
+    resid_mass: Optional[np.ndarray] = None  # [B] float64: Z_j if j < K, else 1
+    accept_margin: Optional[np.ndarray] = None  # [B, K] |u_i - p_i/q_i| (inf where q == 0)
+    cdf_margin: Optional[np.ndarray] = None     # [B] distance of u_K to the nearest CDF boundary
+    argmax: Optional[np.ndarray] = None         # [B, K+1] greedy row argmax
+
+    def near_boundary(self, eps: float = 1e-6) -> np.ndarray:
+        """[B] bool: some decision of this sequence had its uniform within eps of a boundary.
+
+        Only the accept tests that were actually taken (i <= j) and the final inverse-CDF
+        draw count.
+        """
+        B = self.n_accepted.shape[0]
+        out = np.zeros(B, dtype=bool)
+        if self.accept_margin is None:
+            return out
+        for b in range(B):
+            j = int(self.n_accepted[b])
+            K = self.accept_margin.shape[1]
+            taken = self.accept_margin[b, : min(j + 1, K)]
+            out[b] = bool(np.any(taken < eps)) or bool(self.cdf_margin[b] < eps)
+        return out
+
+
+def _row_is_bad(z: np.ndarray) -> bool:
+    """NaN or +inf anywhere, or no finite value at all."""
+    return bool(np.isnan(z).any() or np.isposinf(z).any() or not np.isfinite(z).any())
+
+
+def row_argmax(z: np.ndarray) -> int:
+    """a = min{v : z[v] = max_w z[w]}. Float equality treats -0.0 and +0.0 as equal."""
+    m = z.max()
+    return int(np.flatnonzero(z == m)[0])
+
+
+def softmax(z: np.ndarray, T: float) -> np.ndarray:
+    """softmax(z / T) in float64, max subtracted; -inf entries get probability 0."""
+    y = z / T
+    y = y - y.max()
+    e = np.exp(y)
+    return e / e.sum()
+
+
+def inverse_cdf(w: np.ndarray, u: float):
+    """Smallest v with sum_{t<=v} w[t] > u * sum(w), ascending token id.
+
+    Returns (v, margin): margin is the distance, in normalised units, from u to the
+    nearer of the two CDF boundaries that bracket v.
+    """
+    C = np.cumsum(w)
+    Z = C[-1]
+    target = u * Z
+    hits = np.flatnonzero(C > target)
+    v = int(hits[0]) if hits.size else int(np.flatnonzero(w > 0)[-1])
+    lo = C[v - 1] / Z if v > 0 else 0.0
+    hi = C[v] / Z
+    return v, float(min(u - lo, hi - u))
+
+
+def _error_row(K: int):
+    return 0, np.full(K + 1, -1, dtype=np.int32), -1
+
+
+def greedy_accept(P: np.ndarray, drafts: np.ndarray) -> OracleResult:
+    """Greedy block verify.
+
+    P: [B, K+1, V] float64 base logits (row 0 = p_1, row K = bonus); drafts: [B, K] ints.
+    a_r = lowest-index argmax of row r; j = first i < K with x_i != a_i, else K; emit
+    x_0..x_{j-1} and a_j.
+    """
+    P = np.asarray(P, dtype=np.float64)
+    drafts = np.asarray(drafts)
+    B, K1, V = P.shape
+    K = K1 - 1
+    n = np.zeros(B, dtype=np.int32)
+    tokens = np.full((B, K + 1), -1, dtype=np.int32)
+    nxt = np.full(B, -1, dtype=np.int32)
+    status = np.zeros(B, dtype=np.int32)
+    amax = np.full((B, K + 1), -1, dtype=np.int32)
+    for b in range(B):
+        st = 0
+        if K and (np.any(drafts[b] < 0) or np.any(drafts[b] >= V)):
+            st |= STATUS_BAD_DRAFT
+        if any(_row_is_bad(P[b, r]) for r in range(K + 1)):
+            st |= STATUS_NONFINITE
+        status[b] = st
+        if st:
+            continue
+        a = [row_argmax(P[b, r]) for r in range(K + 1)]
+        amax[b] = a
+        j = K
+        for i in range(K):
+            if int(drafts[b, i]) != a[i]:
+                j = i
+                break
+        n[b] = j
+        tokens[b, :j] = drafts[b, :j]
+        tokens[b, j] = a[j]
+        nxt[b] = a[j]
+    return OracleResult(n, tokens, nxt, status, argmax=amax)
+
+
+def speculative_sample_accept(P: np.ndarray, Q: np.ndarray, drafts: np.ndarray, T: float,
+                              u: np.ndarray) -> OracleResult:
+    """Lossless rejection-sampling block verify.
+
+    P: [B, K+1, V], Q: [B, K, V] float64 logits; drafts [B, K]; T >= 0; u: [B, K+1] uniforms
+    in [0, 1). T == 0 gives exactly ``greedy_accept``.
+
+    For each sequence: p_r = softmax(P_r / T), q_i = softmax(Q_i / T). Walk i = 0..K-1 and
+    accept draft x_i iff u_i * q_i(x_i) < p_i(x_i); stop at the first rejection j. If j < K
+    draw the correction from r = max(p_j - q_j, 0) with u_K by inverse CDF; else draw the
+    bonus token from p_K with u_K.
+    """
+    if T == 0:
+        return greedy_accept(P, drafts)
+    if not (T > 0 and np.isfinite(T)):
+        raise ValueError("temperature must be finite and >= 0")
+    P = np.asarray(P, dtype=np.float64)
+    Q = np.asarray(Q, dtype=np.float64)
+    u = np.asarray(u, dtype=np.float64)
+    drafts = np.asarray(drafts)
+    B, K1, V = P.shape
+    K = K1 - 1
+    n = np.zeros(B, dtype=np.int32)
+    tokens = np.full((B, K + 1), -1, dtype=np.int32)
+    nxt = np.full(B, -1, dtype=np.int32)
+    status = np.zeros(B, dtype=np.int32)
+    pd = np.full((B, K), np.nan)
+    qd = np.full((B, K), np.nan)
+    zm = np.full(B, np.nan)
+    am = np.full((B, K), np.inf)
+    cm = np.full(B, np.inf)
+    for b in range(B):
+        st = 0
+        if K and (np.any(drafts[b] < 0) or np.any(drafts[b] >= V)):
+            st |= STATUS_BAD_DRAFT
+        if any(_row_is_bad(P[b, r]) for r in range(K + 1)) or \
+                any(_row_is_bad(Q[b, i]) for i in range(K)):
+            st |= STATUS_NONFINITE
+        if st:
+            status[b] = st
+            continue
+        p = [softmax(P[b, r], T) for r in range(K + 1)]
+        q = [softmax(Q[b, i], T) for i in range(K)]
+        j = K
+        for i in range(K):
+            x = int(drafts[b, i])
+            pd[b, i], qd[b, i] = p[i][x], q[i][x]
+        for i in range(K):
+            px, qx = pd[b, i], qd[b, i]
+            if qx > 0:
+                am[b, i] = abs(u[b, i] - px / qx)
+            if not (u[b, i] * qx < px):
+                j = i
+                break
+        if j < K:
+            r = np.maximum(p[j] - q[j], 0.0)
+            Z = r.sum()
+            if not Z > 0:
+                st |= STATUS_ZERO_RESIDUAL
+                r, Z = p[j], 1.0
+            zm[b] = Z
+        else:
+            r = p[K]
+            zm[b] = 1.0
+        v, cm[b] = inverse_cdf(r, float(u[b, K]))
+        status[b] = st
+        n[b] = j
+        tokens[b, :j] = drafts[b, :j]
+        tokens[b, j] = v
+        nxt[b] = v
+    return OracleResult(n, tokens, nxt, status, p_draft=pd, q_draft=qd, resid_mass=zm,
+                        accept_margin=am, cdf_margin=cm)
