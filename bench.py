@@ -1,0 +1,458 @@
+"""Benchmark of the DSpark block verify step (greedy_accept + speculative_sample_accept).
+
+One step = one verify call per temperature of the workload over one batch of B sequences:
+for the DeepSeek-V4-Flash-shaped serving workload (B=64, K=7, V=129280, bf16) that is
+greedy_accept (T=0), then speculative_sample_accept at T=0.7 and at T=1.0. Each call reads
+a distinct copy of the inputs (4 rotating sets of ~248 MB, each larger than L2), so every
+call streams its logits from HBM.
+
+    python bench.py [--gpus N --steps K --warmup W]      # the CUDA path
+    python bench.py --impl reference ...                  # the CPU float64 oracle
+
+Under torchrun every rank verifies its own batch (B-sharded replicas, no collective); the
+reported value is all ranks' verified blocks over the max-over-ranks device time.
+"""
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "verified blocks/s and HBM GB/s vs B200 peak at B=64,K=7,V=129280 bf16"
+FALLBACK_HBM_GBS = 6650.0
+N_SETS = 4
+PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "sample_rowstats_dsv4_flash_serving.md")
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=3000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="dsv4_flash_serving")
+    ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--cpu-steps", type=int, default=2,
+                    help="full steps of the oracle timed for the CPU baseline")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    return ap.parse_args()
+
+
+def source_hash():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "lossless_draft_verification_speculative_b200", "csrc")
+    for f in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic():
+    """Per-launch DRAM bytes of the sampling pass from the committed ncu summary, if the
+    kernel sources are unchanged since it was taken; else None."""
+    try:
+        kv = {}
+        for line in open(PROFILE_SUMMARY):
+            if ":" in line and line.strip().startswith("- "):
+                k, v = line.strip()[2:].split(":", 1)
+                kv[k.strip()] = v.strip().strip("`")
+        if kv.get("source_hash") != source_hash():
+            return None
+        return float(kv["traffic_bytes_per_launch"])
+    except (OSError, KeyError, ValueError):
+        return None
+
+
+def measured_peaks():
+    try:
+        return json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json")))
+    except (OSError, ValueError):
+        return None
+
+
+class ClockSampler:
+    """nvidia-smi clock and throttle-reason samples while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except OSError:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.thread.join(timeout=2)
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx.append(float(parts[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx),
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def build_calls(w):
+    return [("greedy" if T == 0 else "sample", float(T)) for T in w.temperatures]
+
+
+# ------------------------------------------------------------------------- reference arm
+
+def run_reference(args, w):
+    """The oracle as it stands, on the host cores, on bounded samples of the workload."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    from lossless_draft_verification_speculative_b200 import workloads as wl
+    from oracle import accept_ref as ora
+
+    calls = build_calls(w)
+    nseq = 4  # sequences per call per step: a bounded sample of the batch
+    seqs = list(range(nseq))
+    P, Q = wl.logits(w, seqs)
+    Pf, Qf = wl.as_float64(P, w.dtype), wl.as_float64(Q, w.dtype)
+    inputs = [(T, wl.drafts(w, Q, T, seqs), wl.uniforms(w, seqs, T=T).astype(np.float64))
+              for _, T in calls]
+
+    def step():
+        for T, d, u in inputs:
+            if T == 0:
+                ora.greedy_accept(Pf, d)
+            else:
+                ora.speculative_sample_accept(Pf, Qf, d, T, u)
+
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    dt = time.perf_counter() - t0
+    blocks = args.steps * len(calls) * nseq
+    value = blocks / dt
+    sample = (f"{nseq} of {w.B} sequences per call, {len(calls)} calls (T={list(w.temperatures)}) "
+              f"per step, float64 NumPy, one process")
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "blocks/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": dt * 1000 / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "K": w.K, "V": w.V,
+                   "temperatures": list(w.temperatures), "sampled_sequences": nseq},
+        "cpu_baseline": {"value": value, "unit": "blocks/s", "cores": 1, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "blocks/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }), flush=True)
+
+
+def cpu_baseline(w, steps):
+    """The oracle timed on the host on `steps` full steps of sequence samples (1 core)."""
+    from lossless_draft_verification_speculative_b200 import workloads as wl
+    from oracle import accept_ref as ora
+
+    calls = build_calls(w)
+    nseq = 8
+    seqs = list(range(nseq))
+    P, Q = wl.logits(w, seqs)
+    Pf, Qf = wl.as_float64(P, w.dtype), wl.as_float64(Q, w.dtype)
+    inputs = [(T, wl.drafts(w, Q, T, seqs), wl.uniforms(w, seqs, T=T).astype(np.float64))
+              for _, T in calls]
+    t0 = time.perf_counter()
+    for _ in range(steps):
+        for T, d, u in inputs:
+            if T == 0:
+                ora.greedy_accept(Pf, d)
+            else:
+                ora.speculative_sample_accept(Pf, Qf, d, T, u)
+    dt = time.perf_counter() - t0
+    blocks = steps * len(calls) * nseq
+    return {"value": blocks / dt, "unit": "blocks/s", "cores": 1, "kind": "oracle",
+            "sample": f"{steps} x {len(calls)} calls x {nseq} of {w.B} sequences "
+                      f"({dt:.1f} s of float64 NumPy on one host core)"}
+
+
+# ----------------------------------------------------------------------------- our arm
+
+def run_ours(args, w):
+    import torch
+    import torch.distributed as dist
+
+    import lossless_draft_verification_speculative_b200 as pkg
+    from lossless_draft_verification_speculative_b200 import binding as bd
+    from lossless_draft_verification_speculative_b200 import workloads as wl
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    pkg.load_library()
+    calls = build_calls(w)
+    # inputs: this rank's own batch (distinct sequences per rank)
+    P, Q, D = wl.generate(w, w.temperatures, seed=wl.SEED_LOGITS + 1000 * rank,
+                          processes=min(16, os.cpu_count() or 1))
+    U = {T: wl.uniforms(w, T=T) for T in w.temperatures}
+    tdt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+
+    def host_tensor(a):
+        if w.dtype == "bf16":
+            return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16)
+        return torch.from_numpy(a)
+
+    Ph, Qh = host_tensor(P), host_tensor(Q)
+    sets = []
+    for s in range(N_SETS):
+        if s == 0:
+            sets.append((Ph.to(dev), Qh.to(dev)))
+        else:
+            sets.append((sets[0][0].clone(), sets[0][1].clone()))
+    Dd = {T: torch.from_numpy(D[T]).to(dev) for T in w.temperatures}
+    Ud = {T: torch.from_numpy(U[T]).to(dev) for T in w.temperatures}
+    wsb = bd.workspace_bytes(w.B, w.K, w.V, tdt)
+    workspace = torch.empty(wsb, dtype=torch.uint8, device=dev)
+    outs = [bd._alloc_result(w.B, w.K, dev, diagnostics=(kind == "sample")) for kind, _ in calls]
+
+    # one prepared call per (call, input set)
+    prepared = []
+    for c, (kind, T) in enumerate(calls):
+        row = []
+        for s in range(N_SETS):
+            Pd, Qd = sets[s]
+            row.append(bd.PreparedCall(kind, Pd, Qd, Dd[T], T, Ud[T], outs[c], workspace))
+        prepared.append(row)
+    ncalls = len(calls)
+
+    def step(s, evs=None):
+        for c in range(ncalls):
+            k = (s * ncalls + c) % N_SETS
+            if evs is not None:
+                evs[c][0].record()
+            prepared[c][k]()
+            if evs is not None:
+                evs[c][1].record()
+
+    for s in range(args.warmup):
+        step(s)
+    torch.cuda.synchronize()
+
+    # per-call events over the whole timed region
+    per_call = [[] for _ in range(ncalls)]
+    ev_pool = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                for _ in range(args.steps)] for _ in range(ncalls)]
+    clocks = ClockSampler(local) if rank == 0 else None
+    barrier()
+    torch.cuda.synchronize()
+    if clocks:
+        clocks.start()
+        time.sleep(0.3)
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    t_start.record()
+    for s in range(args.steps):
+        step(s, [ev_pool[c][s] for c in range(ncalls)])
+    t_end.record()
+    torch.cuda.synchronize()
+    clk = clocks.stop() if clocks else None
+    barrier()
+    ms = t_start.elapsed_time(t_end)
+    for c in range(ncalls):
+        per_call[c] = [a.elapsed_time(b) for a, b in ev_pool[c]]
+    ms_t = torch.tensor([ms], device=dev, dtype=torch.float64)
+    if world > 1:
+        dist.all_reduce(ms_t, op=dist.ReduceOp.MAX)
+    ms_max = float(ms_t.item())
+    blocks = args.steps * ncalls * w.B * world
+    value = blocks / (ms_max / 1000.0)
+
+    # results of the last step: committed tokens per verified block
+    committed = []
+    for c in range(ncalls):
+        committed.append(float((outs[c].n_accepted.double() + 1).mean().item()))
+
+    # e2e: the public API with pinned host inputs, copies and the result read inside
+    e2e = None
+    if not args.no_e2e:
+        e2e = run_e2e(args, w, calls, P, Q, D, U, dev, tdt, outs, workspace, world)
+
+    if world > 1:
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+
+    peaks = measured_peaks()
+    peak = peaks["hbm_gbs"] if peaks else FALLBACK_HBM_GBS
+    call_stats = {}
+    samp_ms = []
+    for c, (kind, T) in enumerate(calls):
+        mean_ms = statistics.mean(per_call[c])
+        nbytes = w.greedy_bytes() if kind == "greedy" else w.sampling_bytes()
+        call_stats[f"{kind}_T{T}"] = {
+            "us_per_call": mean_ms * 1000, "median_us": statistics.median(per_call[c]) * 1000,
+            "algorithmic_bytes": nbytes, "GB_per_s": nbytes / (mean_ms / 1000) / 1e9,
+            "frac_of_peak": nbytes / (mean_ms / 1000) / 1e9 / peak,
+            "committed_tokens_per_block": committed[c]}
+        if kind == "sample":
+            samp_ms.extend(per_call[c])
+    samp_mean = statistics.mean(samp_ms)
+    achieved = w.sampling_bytes() / (samp_mean / 1000) / 1e9
+    traffic = recorded_traffic()
+    line = {
+        "metric": METRIC, "value": value, "unit": "blocks/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_max / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16"
+        if w.dtype == "bf16" else "f32",
+        "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "K": w.K, "V": w.V,
+                   "temperatures": list(w.temperatures), "calls_per_step": ncalls,
+                   "global_batch": w.B * world,
+                   "l2": f"inputs larger than L2: {N_SETS} rotating input sets of "
+                         f"{w.sampling_bytes() / 1e6:.1f} MB, a different set every call",
+                   "parallelism": f"B-sharded replicas x{world}, no collective"},
+        "gpu_launches": 2 * ncalls * args.steps,
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "traffic": traffic,
+                     "kernel": "speculative_sample_accept (pass-1 row stream + finish), "
+                               "mean over the timed T>0 calls",
+                     "peak_source": "MEASURED_PEAKS.json hbm_gbs (measured)" if peaks
+                     else "fallback 6.65 TB/s"},
+        "committed_token_equivalents_per_s": value * statistics.mean(committed),
+        "calls": call_stats,
+    }
+    if clk:
+        line["clocks"] = clk
+    if e2e:
+        line["e2e"] = e2e
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(w, args.cpu_steps)
+    print(json.dumps(line), flush=True)
+
+
+def run_e2e(args, w, calls, P, Q, D, U, dev, tdt, outs, workspace, world):
+    import torch
+    import torch.distributed as dist
+    import lossless_draft_verification_speculative_b200 as pkg
+
+    def pinned(a, dt=None):
+        t = torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16) \
+            if dt == "bf16" else torch.from_numpy(np.ascontiguousarray(a))
+        return t.pin_memory()
+
+    Ph, Qh = pinned(P, w.dtype), pinned(Q, w.dtype)
+    Dh = {T: pinned(D[T]) for T in w.temperatures}
+    Uh = {T: pinned(U[T]) for T in w.temperatures}
+    Pd = torch.empty(Ph.shape, dtype=tdt, device=dev)
+    Qd = torch.empty(Qh.shape, dtype=tdt, device=dev)
+    Dd = {T: torch.empty_like(Dh[T], device=dev) for T in w.temperatures}
+    Ud = {T: torch.empty_like(Uh[T], device=dev) for T in w.temperatures}
+    res_h = [(torch.empty(w.B, dtype=torch.int32).pin_memory(),
+              torch.empty(w.B, w.K + 1, dtype=torch.int32).pin_memory()) for _ in calls]
+    h2d = 0
+    d2h = 0
+    for kind, T in calls:
+        h2d += Ph.numel() * Ph.element_size() + Dh[T].numel() * 4
+        if kind == "sample":
+            h2d += Qh.numel() * Qh.element_size() + Uh[T].numel() * 4
+        d2h += w.B * 4 + w.B * (w.K + 1) * 4
+
+    def step():
+        for c, (kind, T) in enumerate(calls):
+            Pd.copy_(Ph, non_blocking=True)
+            Dd[T].copy_(Dh[T], non_blocking=True)
+            if kind == "greedy":
+                r = pkg.greedy_accept(Pd, Dd[T], out=outs[c], workspace=workspace)
+            else:
+                Qd.copy_(Qh, non_blocking=True)
+                Ud[T].copy_(Uh[T], non_blocking=True)
+                r = pkg.speculative_sample_accept(Pd, Qd, Dd[T], T, Ud[T], out=outs[c],
+                                                  workspace=workspace)
+            res_h[c][0].copy_(r.n_accepted, non_blocking=True)
+            res_h[c][1].copy_(r.tokens, non_blocking=True)
+        torch.cuda.current_stream().synchronize()
+
+    step()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record()
+    for _ in range(args.e2e_steps):
+        step()
+    t1.record()
+    torch.cuda.synchronize()
+    ms = torch.tensor([t0.elapsed_time(t1)], device=dev, dtype=torch.float64)
+    if world > 1:
+        dist.all_reduce(ms, op=dist.ReduceOp.MAX)
+    blocks = args.e2e_steps * len(calls) * w.B * world
+    return {"value": blocks / (float(ms.item()) / 1000), "unit": "blocks/s",
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+            "ms_per_step": float(ms.item()) / args.e2e_steps}
+
+
+def main():
+    args = parse_args()
+    from lossless_draft_verification_speculative_b200 import workloads as wl
+    w = wl.WORKLOADS[args.workload]
+    if args.impl == "reference":
+        run_reference(args, w)
+    else:
+        run_ours(args, w)
+
+
+if __name__ == "__main__":
+    main()

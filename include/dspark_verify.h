@@ -1,0 +1,149 @@
+/*
+ * dspark_verify.h - C ABI of the DSpark block-draft verify/accept step on B200 (sm_100a).
+ *
+ * What the calls compute
+ * ----------------------
+ * One decode cycle of block speculative decoding ends with a verify step. The base model
+ * has produced, for every sequence b of the batch, a logit block of K+1 rows:
+ *   row 0      p_1          from the step that produced the anchor token (free, never recomputed)
+ *   rows 1..K  p_2..p_{K+1} from ONE verify forward over the K drafted tokens; row K is the
+ *                           bonus position.
+ * (Page "dspark-mlx 0.1.0__py3-none-any.whl", dspark_mlx/adapter.py, module docstring
+ * "Logit conventions", and the StepOut / BlockOut dataclasses: StepOut.logits [b, V] is p_1,
+ * BlockOut.per_pos_logits [b, K, V] is p_2..p_{K+1}.) The drafter supplied K draft tokens
+ * x_0..x_{K-1} and, for the sampling policy, the K draft logit rows q_1..q_K they were drawn
+ * from. The same wheel's dspark_mlx/__init__.py exports the two accept policies
+ * greedy_accept and speculative_sample_accept and their AcceptResult; this header is their
+ * device form.
+ *
+ *  - greedy_accept: accepted prefix = the leading drafts equal to the lowest-index argmax of
+ *    their base row; the emitted token is the argmax of the first mismatching row (or of the
+ *    bonus row when all K match). Output equals plain greedy decoding (mlx-dspark 0.0.1
+ *    README, "How it works").
+ *  - speculative_sample_accept: the lossless rejection rule (Leviathan et al. 2023, Chen et
+ *    al. 2023): with p_i = softmax(P_i / T), q_i = softmax(Q_i / T), draft x_i is accepted iff
+ *    u[b,i] * q_i(x_i) < p_i(x_i); at the first rejection j the correction is drawn from
+ *    normalize(max(p_j - q_j, 0)); when all K are accepted the bonus is drawn from p_{K+1}.
+ *    Both draws use u[b,K] by inverse CDF in ascending token order: the smallest v with
+ *    sum_{t<=v} r[t] > u[b,K] * sum(r). The emitted tokens are distributed exactly as the
+ *    target's (the adapter.py docstring's "lossless accept policy"; the DeepSeek-V4-Flash
+ *    DSpark drafter card's "lossless by construction").
+ *
+ * Conventions common to every entry point
+ * ---------------------------------------
+ *  - Every buffer pointer is a DEVICE pointer owned by the caller. The library allocates no
+ *    device memory, never synchronizes the stream, and returns as soon as its kernels are
+ *    enqueued on `stream` (a cudaStream_t passed as void*; NULL = the legacy default stream).
+ *  - Logits are row-major, contiguous along V, of type `dtype` (bf16 or fp32), consumed as
+ *    given (soft-capping, masking etc. are the producer's job). -inf entries are allowed
+ *    (masked tokens).
+ *  - Returned synchronously: DSPARK_ERR_INVALID_ARG for a bad argument (nothing enqueued),
+ *    DSPARK_ERR_UNSUPPORTED for a shape beyond the kernels' limits or a pointer not aligned to
+ *    its element size, DSPARK_ERR_WORKSPACE for a missing or short workspace, DSPARK_ERR_CUDA
+ *    if a launch failed. B == 0 is a no-op returning DSPARK_OK.
+ *  - Data errors are reported per sequence on the device, never by a trap: a draft id outside
+ *    [0, V), or a row holding NaN or +inf or no finite value, makes that sequence's result
+ *    n_accepted = 0, tokens all -1, next_token = -1, with the cause in status[b].
+ *  - Limits: 0 <= K <= 32; 1 <= V <= 262144; B * (K+1) < 2^31.
+ *  - Calls that share a workspace must not overlap on the GPU (same stream, or ordered).
+ */
+#ifndef DSPARK_VERIFY_H
+#define DSPARK_VERIFY_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  DSPARK_OK = 0,
+  DSPARK_ERR_INVALID_ARG = 1,
+  DSPARK_ERR_UNSUPPORTED = 2,
+  DSPARK_ERR_CUDA = 3,
+  DSPARK_ERR_WORKSPACE = 4
+} dspark_status_t;
+
+typedef enum { DSPARK_BF16 = 0, DSPARK_F32 = 1 } dspark_dtype_t;
+
+/* Per-sequence bits written to out.status[b]. */
+#define DSPARK_SEQ_BAD_DRAFT 1     /* a draft id outside [0, V)                           */
+#define DSPARK_SEQ_NONFINITE 2     /* a row with NaN / +inf, or with no finite value       */
+#define DSPARK_SEQ_ZERO_RESIDUAL 4 /* not an error: residual mass rounded to 0 after a
+                                      rejection; the correction was drawn from p_j          */
+#define DSPARK_SEQ_TIMEOUT 8       /* an internal bounded wait gave up (never expected)     */
+
+/* AcceptResult: device buffers, caller-allocated. Required: n_accepted, tokens, next_token.
+ * The optional ones (NULL = not written) are diagnostics of the sampling policy. */
+typedef struct {
+  int32_t* n_accepted; /* [B]      j in [0, K]: accepted drafts = n_keep for the host's KV rollback */
+  int32_t* tokens;     /* [B, K+1] x_0..x_{j-1}, then the correction / bonus token, then -1      */
+  int32_t* next_token; /* [B]      the correction (j < K) or the bonus token (j == K)            */
+  int32_t* status;     /* [B] or NULL: DSPARK_SEQ_* bits, 0 = ok                                 */
+  float* p_draft;      /* [B, K] or NULL: p_i(x_i)  (sampling only)                              */
+  float* q_draft;      /* [B, K] or NULL: q_i(x_i)  (sampling only)                              */
+  float* resid_mass;   /* [B] or NULL: Z_j = sum max(p_j - q_j, 0) if j < K, else 1 (sampling)  */
+} dspark_accept_out_t;
+
+/* Human-readable name of a dspark_status_t value. Never NULL. */
+const char* dspark_status_string(int status);
+
+/* Library ABI version (bumped on any incompatible change). */
+int dspark_version(void);
+
+/* Bytes of device workspace the verify calls need for this shape (valid for both policies).
+ * Returns 0 when the shape is invalid or unsupported. The workspace needs no initialisation
+ * and its contents after a call are unspecified. */
+size_t dspark_workspace_bytes(int B, int K, int V, dspark_dtype_t dtype);
+
+/* Launch geometry the sampling call would use for this shape (for tests and reports).
+ * Returns DSPARK_OK and fills the fields, or an error for an invalid / unsupported shape.
+ * `aligned16` says whether every row start will be 16-byte aligned (vector path). */
+typedef struct {
+  int elems_per_load;   /* 8 (bf16) / 4 (fp32) on the 16-byte vector path, 1 on the scalar path */
+  int elems_per_lane;   /* register-resident logits per lane per row                             */
+  int chunk_elems;      /* contiguous V elements per warp chunk (32 * elems_per_lane)            */
+  int n_chunks;         /* chunks per row                                                        */
+  int warps_per_cta;
+  int cluster_ctas;     /* CTAs per thread-block cluster sharing one row pair                    */
+  int stages;           /* shared-memory pipeline depth (0 = direct register loads)             */
+  int greedy_slices;    /* CTAs per row in the greedy pass                                      */
+} dspark_plan_t;
+dspark_status_t dspark_plan(int B, int K, int V, dspark_dtype_t dtype, int aligned16,
+                            dspark_plan_t* plan);
+
+/* greedy_accept.
+ *  p1      [B, V] base logits p_1; row b starts at p1 + b * ld_p1 (elements, ld_p1 >= V).
+ *  pv      [B, K, V] base logits p_2..p_{K+1}; sequence b starts at pv + b * ld_pv
+ *          (elements, ld_pv >= K * V), its K rows are V apart. May be NULL when K == 0.
+ *          A contiguous [B, K+1, V] block is p1 = blk, pv = blk + V, ld_p1 = ld_pv = (K+1) * V.
+ *  drafts  [B, K] int32 draft token ids (NULL allowed when K == 0).
+ *  Writes n_accepted, tokens, next_token and status; ignores the sampling diagnostics. */
+dspark_status_t dspark_greedy_accept(const void* p1, int64_t ld_p1, const void* pv, int64_t ld_pv,
+                                     dspark_dtype_t dtype, const int32_t* drafts, int B, int K,
+                                     int V, dspark_accept_out_t out, void* workspace,
+                                     size_t workspace_bytes, void* stream);
+
+/* speculative_sample_accept.
+ *  p1, ld_p1, pv, ld_pv, drafts as for greedy_accept.
+ *  q         [B, K, V] draft logits q_1..q_K, contiguous (row (b, i) at q + (b*K + i) * V); the
+ *            distribution the drafts were drawn from, before temperature.
+ *  temperature  T > 0 divides both P and Q logits; T == 0 runs greedy_accept (q and uniforms
+ *            are then not read); T < 0 or non-finite is INVALID_ARG.
+ *  uniforms  [B, K+1] float32 in [0, 1): u[b, i] is the accept test of draft i, u[b, K] the one
+ *            draw used for the correction or the bonus token. The caller supplies the randomness,
+ *            so a call is a pure function of its inputs. */
+dspark_status_t dspark_speculative_sample_accept(const void* p1, int64_t ld_p1, const void* pv,
+                                                 int64_t ld_pv, const void* q,
+                                                 dspark_dtype_t dtype, const int32_t* drafts,
+                                                 int B, int K, int V, float temperature,
+                                                 const float* uniforms, dspark_accept_out_t out,
+                                                 void* workspace, size_t workspace_bytes,
+                                                 void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DSPARK_VERIFY_H */

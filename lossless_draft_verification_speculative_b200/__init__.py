@@ -1,0 +1,35 @@
+"""DSpark block-draft verify/accept on B200 (sm_100a).
+
+``greedy_accept`` and ``speculative_sample_accept`` verify a block of K drafted tokens per
+sequence against the base model's [B, K+1, V] logit block and return an ``AcceptResult``.
+The work runs in hand-written CUDA kernels behind a C ABI (``include/dspark_verify.h``);
+this package is the thin Python binding over it plus the seeded synthetic workloads.
+"""
+
+from .binding import (  # noqa: F401
+    SEQ_BAD_DRAFT,
+    SEQ_NONFINITE,
+    SEQ_TIMEOUT,
+    SEQ_ZERO_RESIDUAL,
+    AcceptResult,
+    DsparkError,
+    greedy_accept,
+    load_library,
+    plan,
+    speculative_sample_accept,
+    workspace_bytes,
+)
+
+__all__ = [
+    "AcceptResult",
+    "DsparkError",
+    "greedy_accept",
+    "speculative_sample_accept",
+    "load_library",
+    "plan",
+    "workspace_bytes",
+    "SEQ_BAD_DRAFT",
+    "SEQ_NONFINITE",
+    "SEQ_ZERO_RESIDUAL",
+    "SEQ_TIMEOUT",
+]

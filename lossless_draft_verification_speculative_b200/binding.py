@@ -1,0 +1,293 @@
+"""Python binding of the C ABI in ``include/dspark_verify.h`` (argument marshalling only).
+
+The names follow the dspark-mlx wheel's verify module (page "dspark-mlx
+0.1.0__py3-none-any.whl", ``dspark_mlx/__init__.py``: ``AcceptResult``, ``greedy_accept``,
+``speculative_sample_accept``). Every step of the verify runs in the CUDA library; this
+module only checks tensor layouts, allocates the result tensors and a workspace with
+PyTorch, and passes raw device pointers and the current CUDA stream. There is no CPU
+fallback: without the built library or a CUDA device every call raises.
+
+Logit inputs follow the wheel's block convention (``dspark_mlx/adapter.py``): either the
+full ``[B, K+1, V]`` block, or the pair ``(p1, pv)`` with ``p1 = StepOut.logits`` ``[B, V]``
+and ``pv = BlockOut.per_pos_logits`` ``[B, K, V]``, passed without concatenation.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+from dataclasses import dataclass
+from typing import Optional, Tuple, Union
+
+import torch
+
+from . import build_lib
+
+DSPARK_OK = 0
+STATUS_NAMES = {0: "DSPARK_OK", 1: "DSPARK_ERR_INVALID_ARG", 2: "DSPARK_ERR_UNSUPPORTED",
+                3: "DSPARK_ERR_CUDA", 4: "DSPARK_ERR_WORKSPACE"}
+DTYPE_CODES = {torch.bfloat16: 0, torch.float32: 1}
+
+SEQ_BAD_DRAFT = 1
+SEQ_NONFINITE = 2
+SEQ_ZERO_RESIDUAL = 4
+SEQ_TIMEOUT = 8
+
+
+class DsparkError(RuntimeError):
+    def __init__(self, code: int, what: str):
+        super().__init__(f"{what}: {STATUS_NAMES.get(code, code)}")
+        self.code = code
+
+
+class AcceptOut(ctypes.Structure):
+    _fields_ = [
+        ("n_accepted", ctypes.c_void_p),
+        ("tokens", ctypes.c_void_p),
+        ("next_token", ctypes.c_void_p),
+        ("status", ctypes.c_void_p),
+        ("p_draft", ctypes.c_void_p),
+        ("q_draft", ctypes.c_void_p),
+        ("resid_mass", ctypes.c_void_p),
+    ]
+
+
+class Plan(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int) for n in (
+        "elems_per_load", "elems_per_lane", "chunk_elems", "n_chunks", "warps_per_cta",
+        "cluster_ctas", "stages", "greedy_slices")]
+
+
+_LIB = None
+
+
+def header_functions() -> list:
+    """Names of every function declared in include/dspark_verify.h."""
+    path = os.path.join(build_lib.INCLUDE, "dspark_verify.h")
+    text = open(path).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(dspark_[a-z0-9_]+)\s*\(", text)))
+
+
+def library_path() -> str:
+    return build_lib.LIB_PATH
+
+
+def load_library(build_if_missing: bool = True) -> ctypes.CDLL:
+    """Load (building first if needed) the CUDA library and declare its signatures."""
+    global _LIB
+    if _LIB is not None:
+        return _LIB
+    path = build_lib.LIB_PATH
+    if not os.path.exists(path):
+        if not build_if_missing:
+            raise RuntimeError(f"CUDA library not built: {path}")
+        build_lib.build()
+    lib = ctypes.CDLL(path)
+    vp, i32, i64, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_size_t
+    lib.dspark_status_string.restype = ctypes.c_char_p
+    lib.dspark_status_string.argtypes = [i32]
+    lib.dspark_version.restype = i32
+    lib.dspark_version.argtypes = []
+    lib.dspark_workspace_bytes.restype = sz
+    lib.dspark_workspace_bytes.argtypes = [i32, i32, i32, i32]
+    lib.dspark_plan.restype = i32
+    lib.dspark_plan.argtypes = [i32, i32, i32, i32, i32, ctypes.POINTER(Plan)]
+    lib.dspark_greedy_accept.restype = i32
+    lib.dspark_greedy_accept.argtypes = [vp, i64, vp, i64, i32, vp, i32, i32, i32, AcceptOut,
+                                         vp, sz, vp]
+    lib.dspark_speculative_sample_accept.restype = i32
+    lib.dspark_speculative_sample_accept.argtypes = [vp, i64, vp, i64, vp, i32, vp, i32, i32,
+                                                     i32, ctypes.c_float, vp, AcceptOut, vp, sz,
+                                                     vp]
+    _LIB = lib
+    return lib
+
+
+@dataclass
+class AcceptResult:
+    """Per-sequence result of one verify call (device tensors)."""
+
+    n_accepted: torch.Tensor           # [B] int32: accepted drafts j (the host's n_keep)
+    tokens: torch.Tensor               # [B, K+1] int32: x_0..x_{j-1}, token, then -1
+    next_token: torch.Tensor           # [B] int32: correction (j < K) or bonus (j == K)
+    status: torch.Tensor               # [B] int32 SEQ_* bits
+    p_draft: Optional[torch.Tensor] = None     # [B, K] float32 p_i(x_i) (sampling)
+    q_draft: Optional[torch.Tensor] = None     # [B, K] float32 q_i(x_i) (sampling)
+    resid_mass: Optional[torch.Tensor] = None  # [B] float32 residual mass Z_j or 1 (sampling)
+
+    @property
+    def n_committed(self) -> torch.Tensor:
+        """Tokens committed by the cycle: accepted drafts plus the correction / bonus."""
+        return torch.where(self.next_token >= 0, self.n_accepted + 1, 0)
+
+
+def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
+    return None if t is None else t.data_ptr()
+
+
+def _split_block(P) -> Tuple[torch.Tensor, Optional[torch.Tensor], int, int]:
+    """(p1, pv, ld_p1, ld_pv) in elements from a [B, K+1, V] block or a (p1, pv) pair."""
+    if isinstance(P, (tuple, list)):
+        p1, pv = P
+        if p1.dim() != 2 or p1.stride(1) != 1:
+            raise ValueError("p1 must be [B, V] with unit stride along V")
+        if pv is not None and pv.shape[1] > 0:
+            if pv.dim() != 3 or pv.stride(2) != 1 or pv.stride(1) != pv.shape[2]:
+                raise ValueError("pv must be [B, K, V] with rows V apart")
+            if pv.dtype != p1.dtype or pv.device != p1.device or pv.shape[0] != p1.shape[0] \
+                    or pv.shape[2] != p1.shape[1]:
+                raise ValueError("p1 and pv disagree in dtype, device or shape")
+            return p1, pv, p1.stride(0), pv.stride(0)
+        return p1, None, p1.stride(0), 0
+    if P.dim() != 3 or P.stride(2) != 1 or P.stride(1) != P.shape[2]:
+        raise ValueError("P must be [B, K+1, V] with rows V apart")
+    K = P.shape[1] - 1
+    return P[:, 0], (P[:, 1:] if K > 0 else None), P.stride(0), P.stride(0)
+
+
+class _Workspace:
+    """A per-device byte buffer reused across calls, grown on demand."""
+
+    def __init__(self):
+        self.bufs = {}
+
+    def get(self, device: torch.device, nbytes: int) -> torch.Tensor:
+        key = device.index if device.index is not None else torch.cuda.current_device()
+        buf = self.bufs.get(key)
+        if buf is None or buf.numel() < nbytes:
+            buf = torch.empty(max(nbytes, 256), dtype=torch.uint8, device=device)
+            self.bufs[key] = buf
+        return buf
+
+
+_WS = _Workspace()
+
+
+def workspace_bytes(B: int, K: int, V: int, dtype: torch.dtype) -> int:
+    return int(load_library().dspark_workspace_bytes(B, K, V, DTYPE_CODES[dtype]))
+
+
+def plan(B: int, K: int, V: int, dtype: torch.dtype, aligned16: bool = True) -> dict:
+    p = Plan()
+    rc = load_library().dspark_plan(B, K, V, DTYPE_CODES[dtype], int(aligned16), ctypes.byref(p))
+    if rc != DSPARK_OK:
+        raise DsparkError(rc, "dspark_plan")
+    return {n: getattr(p, n) for n, _ in Plan._fields_}
+
+
+def _alloc_result(B: int, K: int, device, diagnostics: bool) -> AcceptResult:
+    i32 = dict(dtype=torch.int32, device=device)
+    res = AcceptResult(torch.empty(B, **i32), torch.empty(B, K + 1, **i32),
+                       torch.empty(B, **i32), torch.empty(B, **i32))
+    if diagnostics:
+        res.p_draft = torch.empty(B, K, dtype=torch.float32, device=device)
+        res.q_draft = torch.empty(B, K, dtype=torch.float32, device=device)
+        res.resid_mass = torch.empty(B, dtype=torch.float32, device=device)
+    return res
+
+
+def _out_struct(r: AcceptResult) -> AcceptOut:
+    return AcceptOut(_ptr(r.n_accepted), _ptr(r.tokens), _ptr(r.next_token), _ptr(r.status),
+                     _ptr(r.p_draft), _ptr(r.q_draft), _ptr(r.resid_mass))
+
+
+def _stream_handle(device) -> int:
+    return torch.cuda.current_stream(device).cuda_stream
+
+
+def greedy_accept(P: Union[torch.Tensor, Tuple[torch.Tensor, torch.Tensor]],
+                  drafts: torch.Tensor, *, out: Optional[AcceptResult] = None,
+                  workspace: Optional[torch.Tensor] = None) -> AcceptResult:
+    """Greedy block verify on the GPU: accept drafts while they equal the base argmax."""
+    lib = load_library()
+    p1, pv, ld_p1, ld_pv = _split_block(P)
+    if not p1.is_cuda:
+        raise RuntimeError("greedy_accept runs on CUDA tensors only")
+    B, V = p1.shape
+    K = 0 if pv is None else pv.shape[1]
+    drafts = _check_drafts(drafts, B, K, p1.device)
+    res = out if out is not None else _alloc_result(B, K, p1.device, diagnostics=False)
+    nbytes = lib.dspark_workspace_bytes(B, K, V, DTYPE_CODES[p1.dtype])
+    ws = workspace if workspace is not None else _WS.get(p1.device, nbytes)
+    rc = lib.dspark_greedy_accept(_ptr(p1), ld_p1, _ptr(pv), ld_pv, DTYPE_CODES[p1.dtype],
+                                  _ptr(drafts), B, K, V, _out_struct(res), _ptr(ws),
+                                  ws.numel() * ws.element_size(), _stream_handle(p1.device))
+    if rc != DSPARK_OK:
+        raise DsparkError(rc, "dspark_greedy_accept")
+    return res
+
+
+def speculative_sample_accept(P: Union[torch.Tensor, Tuple[torch.Tensor, torch.Tensor]],
+                              Q: Optional[torch.Tensor], drafts: torch.Tensor,
+                              temperature: float, uniforms: torch.Tensor, *,
+                              out: Optional[AcceptResult] = None,
+                              workspace: Optional[torch.Tensor] = None) -> AcceptResult:
+    """Lossless rejection-sampling block verify on the GPU (T == 0 is greedy_accept)."""
+    lib = load_library()
+    p1, pv, ld_p1, ld_pv = _split_block(P)
+    if not p1.is_cuda:
+        raise RuntimeError("speculative_sample_accept runs on CUDA tensors only")
+    B, V = p1.shape
+    K = 0 if pv is None else pv.shape[1]
+    drafts = _check_drafts(drafts, B, K, p1.device)
+    if Q is not None and K > 0:
+        if Q.shape != (B, K, V) or not Q.is_contiguous() or Q.dtype != p1.dtype:
+            raise ValueError("Q must be a contiguous [B, K, V] tensor of P's dtype")
+    if uniforms.dtype != torch.float32 or uniforms.shape != (B, K + 1) or \
+            not uniforms.is_contiguous() or uniforms.device != p1.device:
+        raise ValueError("uniforms must be a contiguous float32 [B, K+1] tensor on P's device")
+    res = out if out is not None else _alloc_result(B, K, p1.device, diagnostics=True)
+    nbytes = lib.dspark_workspace_bytes(B, K, V, DTYPE_CODES[p1.dtype])
+    ws = workspace if workspace is not None else _WS.get(p1.device, nbytes)
+    rc = lib.dspark_speculative_sample_accept(
+        _ptr(p1), ld_p1, _ptr(pv), ld_pv, _ptr(Q), DTYPE_CODES[p1.dtype], _ptr(drafts), B, K,
+        V, float(temperature), _ptr(uniforms), _out_struct(res), _ptr(ws),
+        ws.numel() * ws.element_size(), _stream_handle(p1.device))
+    if rc != DSPARK_OK:
+        raise DsparkError(rc, "dspark_speculative_sample_accept")
+    return res
+
+
+def _check_drafts(drafts: Optional[torch.Tensor], B: int, K: int, device) -> Optional[torch.Tensor]:
+    if K == 0:
+        return drafts
+    if drafts.dtype != torch.int32 or drafts.shape != (B, K) or not drafts.is_contiguous() \
+            or drafts.device != device:
+        raise ValueError("drafts must be a contiguous int32 [B, K] tensor on P's device")
+    return drafts
+
+
+class PreparedCall:
+    """A verify call with its arguments marshalled once, for tight timing loops.
+
+    Holds references to every tensor it points at. Calling it enqueues the same kernels as
+    the corresponding function above on the stream captured at construction.
+    """
+
+    def __init__(self, policy: str, P, Q, drafts, temperature, uniforms, out: AcceptResult,
+                 workspace: torch.Tensor):
+        self.lib = load_library()
+        p1, pv, ld_p1, ld_pv = _split_block(P)
+        B, V = p1.shape
+        K = 0 if pv is None else pv.shape[1]
+        self.keep = (P, Q, drafts, uniforms, out, workspace, p1, pv)
+        dt = DTYPE_CODES[p1.dtype]
+        stream = _stream_handle(p1.device)
+        nbytes = workspace.numel() * workspace.element_size()
+        if policy == "greedy":
+            self.fn = self.lib.dspark_greedy_accept
+            self.args = (_ptr(p1), ld_p1, _ptr(pv), ld_pv, dt, _ptr(drafts), B, K, V,
+                         _out_struct(out), _ptr(workspace), nbytes, stream)
+        else:
+            self.fn = self.lib.dspark_speculative_sample_accept
+            self.args = (_ptr(p1), ld_p1, _ptr(pv), ld_pv, _ptr(Q), dt, _ptr(drafts), B, K, V,
+                         float(temperature), _ptr(uniforms), _out_struct(out), _ptr(workspace),
+                         nbytes, stream)
+        self.name = policy
+
+    def __call__(self):
+        rc = self.fn(*self.args)
+        if rc != DSPARK_OK:
+            raise DsparkError(rc, self.name)

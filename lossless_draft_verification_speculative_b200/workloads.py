@@ -24,6 +24,7 @@ that the verifier will see.
 
 from __future__ import annotations
 
+import os
 from dataclasses import dataclass, field
 from typing import Iterable, Optional, Sequence
 
@@ -220,3 +221,65 @@ def tiny_cycles(w: Workload, cycles: int, T: float = 1.0):
     d = np.concatenate([drafts(w, Q1, T, [0], cycle=c) for c in range(cycles)], axis=0)
     u = np.concatenate([uniforms(w, [0], T, cycle=c) for c in range(cycles)], axis=0)
     return P, Q, d, u
+
+
+# ------------------------------------------------------------- parallel generation
+
+def _fill_worker(args):
+    from multiprocessing import shared_memory
+    name, w, seqs, seed, p_name, q_name, T_list, d_names = args
+    shp = shared_memory.SharedMemory(name=p_name)
+    shq = shared_memory.SharedMemory(name=q_name)
+    store = np.float32 if w.dtype == "f32" else np.uint16
+    P = np.ndarray((w.B, w.K + 1, w.V), dtype=store, buffer=shp.buf)
+    Q = np.ndarray((w.B, w.K, w.V), dtype=store, buffer=shq.buf)
+    dsh = [shared_memory.SharedMemory(name=n) for n in d_names]
+    D = [np.ndarray((w.B, w.K), dtype=np.int32, buffer=s.buf) for s in dsh]
+    for b in seqs:
+        p, q = logits(w, [b], seed)
+        P[b], Q[b] = p[0], q[0]
+        for T, d in zip(T_list, D):
+            d[b] = drafts(w, q, T, [b])[0]
+    del P, Q, D
+    shp.close()
+    shq.close()
+    for s in dsh:
+        s.close()
+    return len(seqs)
+
+
+def generate(w: Workload, temperatures=(), processes: Optional[int] = None,
+             seed: int = SEED_LOGITS):
+    """Whole-batch P, Q and per-temperature drafts, built by a spawn-started process pool.
+
+    Returns (P, Q, {T: drafts}). Identical to calling ``logits`` and ``drafts`` sequence by
+    sequence; only faster for the large workloads.
+    """
+    import multiprocessing as mp
+    from multiprocessing import shared_memory
+
+    procs = processes or min(w.B, max(1, (os.cpu_count() or 1)))
+    if procs <= 1 or w.B <= 2:
+        P, Q = logits(w, seed=seed)
+        return P, Q, {T: drafts(w, Q, T) for T in temperatures}
+    store = np.float32 if w.dtype == "f32" else np.uint16
+    isz = np.dtype(store).itemsize
+    shp = shared_memory.SharedMemory(create=True, size=w.B * (w.K + 1) * w.V * isz)
+    shq = shared_memory.SharedMemory(create=True, size=max(1, w.B * w.K * w.V * isz))
+    dsh = [shared_memory.SharedMemory(create=True, size=max(4, w.B * w.K * 4))
+           for _ in temperatures]
+    try:
+        groups = [list(range(k, w.B, procs)) for k in range(procs)]
+        args = [(w.name, w, g, seed, shp.name, shq.name, tuple(temperatures),
+                 [s.name for s in dsh]) for g in groups if g]
+        with mp.get_context("spawn").Pool(len(args)) as pool:
+            pool.map(_fill_worker, args)
+        P = np.ndarray((w.B, w.K + 1, w.V), dtype=store, buffer=shp.buf).copy()
+        Q = np.ndarray((w.B, w.K, w.V), dtype=store, buffer=shq.buf).copy()
+        D = {T: np.ndarray((w.B, w.K), dtype=np.int32, buffer=s.buf).copy()
+             for T, s in zip(temperatures, dsh)}
+    finally:
+        for s in [shp, shq] + dsh:
+            s.close()
+            s.unlink()
+    return P, Q, D

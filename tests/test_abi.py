@@ -1,0 +1,118 @@
+"""The C ABI without a GPU: the library builds, loads, exports what the header declares,
+and rejects bad arguments synchronously, before any CUDA call."""
+
+import ctypes
+
+import pytest
+
+from lossless_draft_verification_speculative_b200 import binding, build_lib
+
+BF16, F32 = 0, 1
+FAKE = 0x10000  # a 64 KiB-aligned fake device address: never dereferenced by these calls
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build_lib.build()
+    return binding.load_library()
+
+
+def _out(n=FAKE, t=FAKE, nx=FAKE):
+    return binding.AcceptOut(n, t, nx, None, None, None, None)
+
+
+def test_exports_every_declared_symbol(lib):
+    names = binding.header_functions()
+    assert {"dspark_greedy_accept", "dspark_speculative_sample_accept",
+            "dspark_workspace_bytes", "dspark_status_string"} <= set(names)
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_status_strings_and_version(lib):
+    for code, name in binding.STATUS_NAMES.items():
+        assert lib.dspark_status_string(code).decode() == name
+    assert lib.dspark_status_string(99).decode() == "DSPARK_ERR_UNKNOWN"
+    assert lib.dspark_version() >= 1
+
+
+def test_workspace_bytes(lib):
+    assert lib.dspark_workspace_bytes(64, 7, 129280, BF16) > 0
+    assert lib.dspark_workspace_bytes(64, 7, 129280, BF16) < 8 << 20
+    assert lib.dspark_workspace_bytes(1, 33, 100, BF16) == 0      # K > 32
+    assert lib.dspark_workspace_bytes(1, 3, 0, BF16) == 0         # V < 1
+    assert lib.dspark_workspace_bytes(1, 3, 262145, BF16) == 0    # V beyond the limit
+    assert lib.dspark_workspace_bytes(1, 3, 64, 7) == 0           # unknown dtype
+    a = lib.dspark_workspace_bytes(8, 7, 262144, BF16)
+    b = lib.dspark_workspace_bytes(16, 7, 262144, BF16)
+    assert b > a
+
+
+def test_plans_cover_every_workload_shape(lib):
+    for V, want_cluster, want_warps in [(64, 1, 1), (129280, 16, 8), (151936, 16, 10),
+                                        (262144, 16, 16), (5000, 1, 5), (20000, 4, 5)]:
+        p = binding.Plan()
+        assert lib.dspark_plan(4, 7, V, BF16, 1, ctypes.byref(p)) == 0
+        assert p.cluster_ctas == want_cluster and p.warps_per_cta == want_warps, V
+        assert p.cluster_ctas * p.warps_per_cta * p.chunk_elems >= V
+        assert p.n_chunks == -(-V // p.chunk_elems)
+        assert p.elems_per_load == 8 and p.stages >= 2
+        assert lib.dspark_plan(4, 7, V, BF16, 0, ctypes.byref(p)) == 0
+        assert p.elems_per_load == 1 and p.stages == 0
+    assert lib.dspark_plan(4, 7, 262145, BF16, 1, ctypes.byref(binding.Plan())) == 2
+
+
+def _greedy(lib, **kw):
+    a = dict(p1=FAKE, ld=1024, pv=FAKE, ldv=7 * 1024, dt=BF16, d=FAKE, B=4, K=7, V=1024,
+             out=_out(), ws=FAKE, wsb=1 << 30, s=None)
+    a.update(kw)
+    return lib.dspark_greedy_accept(a["p1"], a["ld"], a["pv"], a["ldv"], a["dt"], a["d"], a["B"],
+                                    a["K"], a["V"], a["out"], a["ws"], a["wsb"], a["s"])
+
+
+def _sample(lib, **kw):
+    a = dict(p1=FAKE, ld=1024, pv=FAKE, ldv=7 * 1024, q=FAKE, dt=BF16, d=FAKE, B=4, K=7, V=1024,
+             T=1.0, u=FAKE, out=_out(), ws=FAKE, wsb=1 << 30, s=None)
+    a.update(kw)
+    return lib.dspark_speculative_sample_accept(a["p1"], a["ld"], a["pv"], a["ldv"], a["q"], a["dt"],
+                                                a["d"], a["B"], a["K"], a["V"], a["T"], a["u"],
+                                                a["out"], a["ws"], a["wsb"], a["s"])
+
+
+@pytest.mark.parametrize("call", [_greedy, _sample])
+def test_invalid_arguments(lib, call):
+    INV, UNS, WS = 1, 2, 4
+    assert call(lib, B=-1) == INV
+    assert call(lib, K=-1) == INV
+    assert call(lib, K=33, ldv=33 * 1024) == INV
+    assert call(lib, V=0) == INV
+    assert call(lib, dt=5) == INV
+    assert call(lib, p1=None) == INV
+    assert call(lib, pv=None) == INV
+    assert call(lib, d=None) == INV
+    assert call(lib, ld=1000) == INV              # rows of p1 would overlap
+    assert call(lib, ldv=6 * 1024) == INV         # sequences of pv would overlap
+    assert call(lib, out=_out(n=None)) == INV
+    assert call(lib, out=_out(t=None)) == INV
+    assert call(lib, out=_out(nx=None)) == INV
+    assert call(lib, p1=FAKE + 1) == UNS          # not aligned to the element size
+    assert call(lib, V=262145, ld=262145, ldv=7 * 262145) == UNS
+    assert call(lib, ws=None) == WS
+    assert call(lib, wsb=16) == WS
+    assert call(lib, ws=FAKE + 16) == WS          # workspace must be 256-byte aligned
+    assert call(lib, B=0) == 0                    # empty batch: a no-op
+
+
+def test_sampling_specific_arguments(lib):
+    INV, UNS = 1, 2
+    assert _sample(lib, T=-0.5) == INV
+    assert _sample(lib, T=float("nan")) == INV
+    assert _sample(lib, T=float("inf")) == INV
+    assert _sample(lib, T=1e-45) == INV           # log2(e)/T overflows float
+    assert _sample(lib, q=None) == INV
+    assert _sample(lib, u=None) == INV
+    assert _sample(lib, q=FAKE + 1) == UNS
+    # T == 0 is greedy_accept: q and uniforms are not needed, the greedy checks apply
+    assert _sample(lib, T=0.0, q=None, u=None, ws=None) == 4
+    # K == 0: no draft rows, pv / q / drafts may be NULL; workspace still checked
+    assert _sample(lib, K=0, pv=None, q=None, d=None, ldv=0, ws=None) == 4
