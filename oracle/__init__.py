@@ -9,6 +9,8 @@ from .accept_ref import (  # noqa: F401
     STATUS_NONFINITE,
     STATUS_ZERO_RESIDUAL,
     OracleResult,
+    cdf_interval,
+    draw_law,
     greedy_accept,
     inverse_cdf,
     row_argmax,

@@ -118,8 +118,35 @@ def inverse_cdf(w: np.ndarray, u: float):
     return v, float(min(u - lo, hi - u))
 
 
-def _error_row(K: int):
-    return 0, np.full(K + 1, -1, dtype=np.int32), -1
+def _draw_law(p, q, j):
+    """Unnormalised law of the correction / bonus token after j accepted drafts.
+
+    j < K: the residual max(p_j - q_j, 0); if its mass is not positive (only rounding can
+    cause that) p_j instead. j == K: the bonus row p_K. Returns (weights, fell_back).
+    """
+    K = len(q)
+    if j < K:
+        r = np.maximum(p[j] - q[j], 0.0)
+        if r.sum() > 0:
+            return r, False
+        return p[j], True
+    return p[K], False
+
+
+def draw_law(P_b: np.ndarray, Q_b: np.ndarray, j: int, T: float) -> np.ndarray:
+    """The law ``speculative_sample_accept`` draws from for one sequence (P_b: [K+1, V],
+    Q_b: [K, V] float64 logits) after j accepted drafts, unnormalised."""
+    K = P_b.shape[0] - 1
+    p = [softmax(P_b[r], T) for r in range(K + 1)]
+    q = [softmax(Q_b[i], T) for i in range(K)]
+    return _draw_law(p, q, j)[0]
+
+
+def cdf_interval(w: np.ndarray, v: int):
+    """[C(v-1), C(v)) / Z: the range of u for which the inverse CDF of w returns v."""
+    C = np.cumsum(w)
+    Z = C[-1]
+    return (C[v - 1] / Z if v > 0 else 0.0), C[v] / Z
 
 
 def greedy_accept(P: np.ndarray, drafts: np.ndarray) -> OracleResult:
@@ -215,16 +242,10 @@ def speculative_sample_accept(P: np.ndarray, Q: np.ndarray, drafts: np.ndarray, 
             if not (u[b, i] * qx < px):
                 j = i
                 break
-        if j < K:
-            r = np.maximum(p[j] - q[j], 0.0)
-            Z = r.sum()
-            if not Z > 0:
-                st |= STATUS_ZERO_RESIDUAL
-                r, Z = p[j], 1.0
-            zm[b] = Z
-        else:
-            r = p[K]
-            zm[b] = 1.0
+        r, fell_back = _draw_law(p, q, j)
+        if fell_back:
+            st |= STATUS_ZERO_RESIDUAL
+        zm[b] = r.sum() if (j < K and not fell_back) else (0.0 if fell_back else 1.0)
         v, cm[b] = inverse_cdf(r, float(u[b, K]))
         status[b] = st
         n[b] = j

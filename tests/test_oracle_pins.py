@@ -438,3 +438,25 @@ def test_near_boundary_flag():
     near = ora.speculative_sample_accept(zP, zQ, d, 1.0, np.asarray([[0.5 - 1e-9, 0.3]]))
     far = ora.speculative_sample_accept(zP, zQ, d, 1.0, np.asarray([[0.499, 0.3]]))
     assert near.near_boundary()[0] and not far.near_boundary()[0]
+
+
+def test_draw_law_and_cdf_interval():
+    """draw_law after a rejection under a point-mass q is p without x (library softmax), and
+    cdf_interval brackets exactly the uniforms whose library inverse-CDF draw is v."""
+    rng = np.random.default_rng(11)
+    V, K = 17, 2
+    zP = rng.normal(0, 1.5, (K + 1, V))
+    zQ = np.full((K, V), -np.inf)
+    zQ[0, 5] = 0.0
+    zQ[1] = rng.normal(0, 1.5, V)
+    w = ora.draw_law(zP, zQ, 0, 1.0)
+    p0 = special.softmax(zP[0])
+    want = p0.copy()
+    want[5] = 0.0
+    np.testing.assert_allclose(w, want, rtol=1e-13, atol=1e-16)
+    np.testing.assert_allclose(ora.draw_law(zP, zQ, K, 1.0), special.softmax(zP[K]), rtol=1e-13)
+    c = np.cumsum(want)
+    for uu in rng.random(200):
+        v = int(np.searchsorted(c, uu * c[-1], side="right"))
+        lo, hi = ora.cdf_interval(want, v)
+        assert lo <= uu < hi
