@@ -16,6 +16,7 @@ constexpr int kMaxWarps = 16;        // warps per CTA in the sampling pass
 constexpr int kMaxCluster = 16;      // CTAs per cluster (non-portable size, opt-in)
 constexpr int kMaxChunks = kMaxWarps * kMaxCluster;
 constexpr int kLaneElems = 32;       // register-resident logits per lane per row
+constexpr int kChunkElems = 32 * kLaneElems;  // contiguous tokens per warp chunk
 constexpr int kFinishThreads = 256;  // finish kernel block (>= kMaxChunks)
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;  // bounded waits give up after 2 s
 
@@ -124,10 +125,81 @@ __device__ __forceinline__ float warp_sum(float v) {
 
 __device__ __forceinline__ bool is_finite(float x) { return fabsf(x) <= 3.402823466e38f; }
 
+// ---------------------------------------------------------------- packed / warp arithmetic
+
+// Two floats in one 64-bit register pair, for the sm_100 f32x2 FMA-pipe instructions. Each
+// lane of a packed op rounds exactly like the scalar op (round to nearest, no flush).
+__device__ __forceinline__ uint64_t pk2(float a, float b) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+  return r;
+}
+__device__ __forceinline__ void upk2(uint64_t v, float& a, float& b) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(v));
+}
+__device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t add2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ uint64_t mul2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+
+// max of three with NaN propagation (a NaN anywhere gives NaN).
+__device__ __forceinline__ float max3_nan(float a, float b, float c) {
+  float d;
+  asm("max.NaN.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+__device__ __forceinline__ float max_nan(float a, float b) {
+  float d;
+  asm("max.NaN.f32 %0, %1, %2;" : "=f"(d) : "f"(a), "f"(b));
+  return d;
+}
+// Elementwise max of two bf16 pairs, NaN-propagating.
+__device__ __forceinline__ uint32_t max_nan_bf16x2(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("max.NaN.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+// Warp-wide max (every lane gets it), NaN-propagating.
+__device__ __forceinline__ float warp_max_nan(float v) {
+  float d;
+  asm volatile("redux.sync.max.NaN.f32 %0, %1, 0xffffffff;" : "=f"(d) : "f"(v));
+  return d;
+}
+
+// Merge 32 lane-held softmax parts (m = reference, s = sum against it; empty = (-inf, 0))
+// into one, identical on every lane: M = max m, S = sum s * 2^(m - M).
+__device__ __forceinline__ SoftPart warp_soft_merge_lanes(float m, float s) {
+  const float M = warp_max_nan(m);
+  float w = s == 0.f ? 0.f : __fmul_rn(s, ex2(__fsub_rn(m, M)));
+  w = warp_sum(w);
+  return {M, w};
+}
+
 // ---------------------------------------------------------------- mbarrier / bulk copy
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+// Shared-memory fetch-add with acquire-release ordering at CTA scope; returns the old value.
+__device__ __forceinline__ unsigned smem_atomic_add_acq_rel(unsigned* p, unsigned v) {
+  unsigned old;
+  asm volatile("atom.acq_rel.cta.shared::cta.add.u32 %0, [%1], %2;"
+               : "=r"(old)
+               : "r"(smem_u32(p)), "r"(v)
+               : "memory");
+  return old;
 }
 
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
@@ -169,6 +241,41 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity
     if (mbar_try_wait(bar, parity)) return true;
     if ((it & 255u) == 255u && globaltimer_ns() - t0 > kWaitLimitNs) return false;
   }
+}
+
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t* bar, uint32_t parity) {
+  uint32_t done;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(done)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return done != 0;
+}
+
+// Bounded wait for a phase completed by other CTAs of the cluster (st.async data).
+__device__ __forceinline__ bool mbar_wait_cluster_bounded(uint64_t* bar, uint32_t parity) {
+  if (mbar_try_wait_cluster(bar, parity)) return true;
+  const unsigned long long t0 = globaltimer_ns();
+  for (uint32_t it = 0;; ++it) {
+    if (mbar_try_wait_cluster(bar, parity)) return true;
+    if ((it & 255u) == 255u && globaltimer_ns() - t0 > kWaitLimitNs) return false;
+  }
+}
+
+// Store 16 bytes into CTA `rank`'s shared memory at the address that `local` has in this CTA,
+// completing 16 transaction bytes on that CTA's mbarrier at the address `local_bar` has here.
+__device__ __forceinline__ void st_async_peer(const void* local, const uint64_t* local_bar,
+                                              uint32_t rank, float4 v) {
+  uint32_t dst, bar;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(dst) : "r"(smem_u32(local)), "r"(rank));
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(bar) : "r"(smem_u32(local_bar)), "r"(rank));
+  asm volatile(
+      "st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.f32 [%0], {%1, %2, %3, %4}, [%5];" ::"r"(dst),
+      "f"(v.x), "f"(v.y), "f"(v.z), "f"(v.w), "r"(bar)
+      : "memory");
 }
 
 // 1-D bulk copy global -> this CTA's shared memory, completing on `bar` (no multicast).

@@ -71,7 +71,7 @@ bool make_plan(int V, dspark_dtype_t dt, bool aligned16, Plan* pl) {
   pl->stages = 0;
   if (aligned16 && !tuning().no_tma) {
     // Aim for two CTAs per SM up to 8 warps, one above; at least 2 and at most 4 stages.
-    const size_t stage_bytes = pass1_ring_bytes(1, pl->slice_elems, es);
+    const size_t stage_bytes = pass1_ring_bytes(warps, 1, es);
     const int ctas_per_sm = warps <= 8 ? 2 : 1;
     int st = static_cast<int>(kSmemBudgetPerSm / ctas_per_sm / stage_bytes);
     st = st < 2 ? 2 : (st > kMaxStages ? kMaxStages : st);
@@ -98,7 +98,7 @@ WsLayout ws_layout(long long B, long long K, const Plan& pl) {
   w.chunk_r = off;
   off = align256(off + sizeof(ChunkRec) * static_cast<size_t>(B * K * pl.n_chunks));
   w.unit_flags = off;
-  off = align256(off + static_cast<size_t>(B * (K + 1) * pl.cluster));
+  off = align256(off + static_cast<size_t>(B * (K + 1) * pl.cluster * pl.warps));
   w.greedy_part = off;
   off = align256(off + sizeof(int4) * static_cast<size_t>(B * (K + 1) * pl.greedy_slices));
   w.total = off;
@@ -218,8 +218,8 @@ template <typename T, int VEC, bool kTma>
 dspark_status_t run_sample(SampleParams prm, const FinishParams& fin, const Plan& pl, int fn_id,
                            cudaStream_t stream) {
   const int threads = pl.warps * 32;
-  const size_t smem = (kTma ? pass1_ring_bytes(pl.stages, pl.slice_elems, Elem<T>::kBytes) : 0) +
-                      sizeof(Pass1Smem);
+  const size_t smem =
+      (kTma ? pass1_ring_bytes(pl.warps, pl.stages, Elem<T>::kBytes) : 0) + sizeof(Pass1Smem);
   void* fn = Pass1Kernel<T, VEC, kTma>::fn();
   cudaError_t e = cudaSuccess;
   const int mc = max_clusters(fn, fn_id, threads, smem, pl.cluster, &e);
@@ -374,7 +374,6 @@ dspark_status_t dspark_speculative_sample_accept(const void* p1, int64_t ld_p1, 
   prm.cluster = pl.cluster;
   prm.n_units = B * (K + 1);
   prm.stages = pl.stages;
-  prm.slice_elems = pl.slice_elems;
   prm.rowstat = reinterpret_cast<float2*>(ws + w.rowstat);
   prm.chunk_p = reinterpret_cast<ChunkRec*>(ws + w.chunk_p);
   prm.chunk_r = reinterpret_cast<ChunkRec*>(ws + w.chunk_r);
@@ -394,6 +393,7 @@ dspark_status_t dspark_speculative_sample_accept(const void* p1, int64_t ld_p1, 
   fin.uniforms = uniforms;
   fin.n_chunks = pl.n_chunks;
   fin.cluster = pl.cluster;
+  fin.warps = pl.warps;
   fin.rowstat = prm.rowstat;
   fin.chunk_p = prm.chunk_p;
   fin.chunk_r = prm.chunk_r;

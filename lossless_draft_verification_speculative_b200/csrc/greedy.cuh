@@ -1,10 +1,11 @@
 // greedy_accept on sm_100a.
 //
-// Pass 1 streams the K+1 base rows of every sequence once (P only; Q is never read) and
-// computes, per 8192-token slice of a row, the lowest-index maximum and whether a NaN was
-// seen. Each thread walks its 32 elements in ascending token order with a strict ">" so it
-// keeps the first of equal maxima; the warp/CTA merges break ties toward the lower index.
-// Float comparison makes -0.0 and +0.0 equal, as the definition asks.
+// Pass 1 streams the K+1 base rows of every sequence once (P only; Q is never read). Per
+// 8192-token slice of a row it takes the maximum with a NaN-propagating max (two bf16 tokens
+// per packed instruction, so a NaN anywhere shows up as a NaN maximum at no extra cost), then
+// the lowest index holding it: only the threads whose own maximum equals the slice maximum
+// (usually one) walk their tokens. Float equality makes -0.0 and +0.0 equal, as the
+// definition asks.
 // The finish kernel (one CTA per sequence) merges the slices of each row into a_r, accepts
 // drafts while x_i == a_i, and emits a_j (the greedy semantics of plain sequential decoding).
 #pragma once
@@ -50,6 +51,32 @@ __device__ __forceinline__ ArgBest warp_arg_best(ArgBest a) {
   return a;
 }
 
+// Max of this thread's logits. bf16 vectors use the packed NaN-propagating max (two tokens
+// per instruction); a NaN anywhere makes the result NaN, so NaN rows are caught for free.
+template <typename T, int VEC>
+__device__ __forceinline__ float thread_max(const uint4* raw, const float* z);
+
+template <>
+__device__ __forceinline__ float thread_max<bf16_t, 8>(const uint4* raw, const float*) {
+  uint32_t m = 0xff80ff80u;  // (-inf, -inf)
+#pragma unroll
+  for (int g = 0; g < kGreedyThreadElems / 8; ++g) {
+    m = max_nan_bf16x2(m, raw[g].x);
+    m = max_nan_bf16x2(m, raw[g].y);
+    m = max_nan_bf16x2(m, raw[g].z);
+    m = max_nan_bf16x2(m, raw[g].w);
+  }
+  return max_nan(__uint_as_float(m << 16), __uint_as_float(m & 0xffff0000u));
+}
+
+template <typename T, int VEC>
+__device__ __forceinline__ float thread_max(const uint4*, const float* z) {
+  float m = -__int_as_float(0x7f800000);
+#pragma unroll
+  for (int k = 0; k < kGreedyThreadElems; k += 2) m = max3_nan(m, z[k], z[k + 1]);
+  return m;
+}
+
 template <typename T, int VEC>
 __global__ void __launch_bounds__(kGreedyThreads) greedy_argmax_kernel(const GreedyParams prm) {
   constexpr int G = kGreedyThreadElems / VEC;  // loads per thread
@@ -64,73 +91,84 @@ __global__ void __launch_bounds__(kGreedyThreads) greedy_argmax_kernel(const Gre
   const T* base = rows.prow(b, i);
   const int V = prm.V;
   const int sbase = sl * kGreedySliceElems;
+  // token of this thread's k-th value (ascending in k)
+  auto token = [&](int k) {
+    return VEC == 1 ? sbase + k * kGreedyThreads + tid
+                    : sbase + ((k / VEC) * kGreedyThreads + tid) * VEC + (k % VEC);
+  };
 
+  uint4 raw[VEC == 1 ? 1 : G];
   float z[kGreedyThreadElems];
   if constexpr (VEC == 1) {
 #pragma unroll
-    for (int g = 0; g < G; ++g) {
-      const int e = sbase + g * kGreedyThreads + tid;
-      z[g] = e < V ? Elem<T>::load1(base + e) : ninf;
+    for (int k = 0; k < G; ++k) {
+      const int e = token(k);
+      z[k] = e < V ? Elem<T>::load1(base + e) : ninf;
     }
   } else {
-    uint4 raw[G];
 #pragma unroll
     for (int g = 0; g < G; ++g) {
       const int e = sbase + (g * kGreedyThreads + tid) * VEC;
-      if (e < V) raw[g] = ld_stream16(base + e);
+      raw[g] = e < V ? ld_stream16(base + e)
+                     : (Elem<T>::kBytes == 2 ? make_uint4(0xff80ff80u, 0xff80ff80u, 0xff80ff80u,
+                                                          0xff80ff80u)
+                                             : make_uint4(0xff800000u, 0xff800000u, 0xff800000u,
+                                                          0xff800000u));
     }
+    if constexpr (Elem<T>::kBytes == 4) {
 #pragma unroll
-    for (int g = 0; g < G; ++g) {
-      const int e = sbase + (g * kGreedyThreads + tid) * VEC;
-      if (e < V) {
-        Elem<T>::unpack(raw[g], z + g * VEC);
-      } else {
-#pragma unroll
-        for (int k = 0; k < VEC; ++k) z[g * VEC + k] = ninf;
-      }
+      for (int g = 0; g < G; ++g) Elem<T>::unpack(raw[g], z + g * VEC);
     }
   }
 
-  ArgBest best{ninf, INT_MAX};
-  bool nan = false;
-#pragma unroll
-  for (int g = 0; g < G; ++g) {
-#pragma unroll
-    for (int k = 0; k < VEC; ++k) {
-      const float v = z[g * VEC + k];
-      const int e = VEC == 1 ? sbase + g * kGreedyThreads + tid
-                             : sbase + (g * kGreedyThreads + tid) * VEC + k;
-      if (v > best.v) best = ArgBest{v, e};
-      nan |= v != v;
-    }
-  }
-  best = warp_arg_best(best);
-  const bool any_nan = __any_sync(0xffffffffu, nan);
-
-  __shared__ ArgBest s_best[kGreedyThreads / 32];
-  __shared__ int s_nan[kGreedyThreads / 32];
-  if (lane == 0) {
-    s_best[warp] = best;
-    s_nan[warp] = any_nan;
-  }
+  const float tm = thread_max<T, VEC>(raw, z);
+  const float wm = warp_max_nan(tm);
+  __shared__ float s_wmax[kGreedyThreads / 32];
+  __shared__ float s_max;
+  __shared__ int s_idx;
+  if (lane == 0) s_wmax[warp] = wm;
+  if (tid == 0) s_idx = INT_MAX;
   __syncthreads();
   if (warp == 0) {
-    ArgBest a = lane < kGreedyThreads / 32 ? s_best[lane] : ArgBest{ninf, INT_MAX};
-    int n = lane < kGreedyThreads / 32 ? s_nan[lane] : 0;
-    a = warp_arg_best(a);
-    n = __reduce_or_sync(0xffffffffu, n);
-    if (lane == 0)
-      prm.part[static_cast<size_t>(row) * prm.slices + sl] = make_int4(__float_as_int(a.v), a.i, n, 0);
+    const float v = lane < kGreedyThreads / 32 ? s_wmax[lane] : ninf;
+    const float m = warp_max_nan(v);
+    if (lane == 0) s_max = m;
+  }
+  __syncthreads();
+  const float M = s_max;
+  // Only threads holding the slice maximum look for its first position (usually one thread).
+  if (tm == M && M > ninf) {
+    float zz[kGreedyThreadElems];
+    if constexpr (VEC == 1 || Elem<T>::kBytes == 4) {
+#pragma unroll
+      for (int k = 0; k < kGreedyThreadElems; ++k) zz[k] = z[k];
+    } else {
+#pragma unroll
+      for (int g = 0; g < G; ++g) Elem<T>::unpack(raw[g], zz + g * VEC);
+    }
+    int first = INT_MAX;
+#pragma unroll
+    for (int k = kGreedyThreadElems - 1; k >= 0; --k)
+      if (zz[k] == M) first = token(k);
+    atomicMin(&s_idx, first);
+  }
+  __syncthreads();
+  if (tid == 0) {
+    const bool nan = M != M;
+    prm.part[static_cast<size_t>(row) * prm.slices + sl] =
+        make_int4(__float_as_int(nan ? ninf : M), nan || !(M > ninf) ? INT_MAX : s_idx, nan, 0);
   }
   grid_dependents_launch();
 }
 
 template <int WARPS>
 __global__ void __launch_bounds__(WARPS * 32) greedy_finish_kernel(const GreedyParams prm) {
-  grid_dependency_wait();
   const float ninf = -__int_as_float(0x7f800000);
   const int b = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int K = prm.K, K1 = K + 1;
+  // The drafts are an input, not a result of pass 1: read them before waiting for it.
+  const int x = (warp == 0 && lane < K) ? prm.drafts[static_cast<size_t>(b) * K + lane] : 0;
+  grid_dependency_wait();
   __shared__ int s_arg[kMaxK + 1];
   __shared__ int s_bad[kMaxK + 1];
   __shared__ int s_j, s_err;
@@ -149,7 +187,7 @@ __global__ void __launch_bounds__(WARPS * 32) greedy_finish_kernel(const GreedyP
     if (lane == 0) {
       s_arg[r] = a.i;
       // NaN anywhere, a +inf maximum, or no value above -inf: not a usable row.
-      s_bad[r] = n || a.i == INT_MAX || !(a.v < __int_as_float(0x7f800000));
+      s_bad[r] = n || a.i == INT_MAX || !(a.v < __int_as_float(0x7f800000)) || !(a.v > ninf);
     }
   }
   __syncthreads();
@@ -157,7 +195,6 @@ __global__ void __launch_bounds__(WARPS * 32) greedy_finish_kernel(const GreedyP
     int err = 0;
     bool match = false;
     if (lane < K) {
-      const int x = prm.drafts[static_cast<size_t>(b) * K + lane];
       if (x < 0 || x >= prm.V) err |= DSPARK_SEQ_BAD_DRAFT;
       match = x == s_arg[lane];
     }
