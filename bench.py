@@ -264,7 +264,7 @@ def run_ours(args, w):
     Dd = {T: torch.from_numpy(D[T]).to(dev) for T in w.temperatures}
     Ud = {T: torch.from_numpy(U[T]).to(dev) for T in w.temperatures}
     wsb = bd.workspace_bytes(w.B, w.K, w.V, tdt)
-    workspace = torch.empty(wsb, dtype=torch.uint8, device=dev)
+    workspace = bd.new_workspace(wsb, dev)
     outs = [bd._alloc_result(w.B, w.K, dev, diagnostics=(kind == "sample")) for kind, _ in calls]
 
     # one prepared call per (call, input set)

@@ -44,7 +44,7 @@
  *  - Data errors are reported per sequence on the device, never by a trap: a draft id outside
  *    [0, V), or a row holding NaN or +inf or no finite value, makes that sequence's result
  *    n_accepted = 0, tokens all -1, next_token = -1, with the cause in status[b].
- *  - Limits: 0 <= K <= 32; 1 <= V <= 262144; B * (K+1) < 2^31.
+ *  - Limits: 0 <= K <= 32; 1 <= V <= 262144; B * (2K+1) < 2^31.
  *  - Calls that share a workspace must not overlap on the GPU (same stream, or ordered).
  */
 #ifndef DSPARK_VERIFY_H
@@ -93,22 +93,26 @@ const char* dspark_status_string(int status);
 int dspark_version(void);
 
 /* Bytes of device workspace the verify calls need for this shape (valid for both policies).
- * Returns 0 when the shape is invalid or unsupported. The workspace needs no initialisation
- * and its contents after a call are unspecified. */
+ * Returns 0 when the shape is invalid or unsupported.
+ * Contract: the first dspark_workspace_zero_bytes(B, K) bytes of a workspace must be zero
+ * before its first call (e.g. cudaMemsetAsync once after allocating it); every call that
+ * returns DSPARK_OK leaves them zero again, so no per-call clearing is needed. After a call
+ * reported DSPARK_SEQ_TIMEOUT for some sequence, clear them again. The rest of the workspace
+ * needs no initialisation. One workspace serves one call at a time. */
 size_t dspark_workspace_bytes(int B, int K, int V, dspark_dtype_t dtype);
+size_t dspark_workspace_zero_bytes(int B, int K);
 
-/* Launch geometry the sampling call would use for this shape (for tests and reports).
+/* Launch geometry the calls would use for this shape (for tests and reports).
  * Returns DSPARK_OK and fills the fields, or an error for an invalid / unsupported shape.
  * `aligned16` says whether every row start will be 16-byte aligned (vector path). */
 typedef struct {
-  int elems_per_load;   /* 8 (bf16) / 4 (fp32) on the 16-byte vector path, 1 on the scalar path */
-  int elems_per_lane;   /* register-resident logits per lane per row                             */
-  int chunk_elems;      /* contiguous V elements per warp chunk (32 * elems_per_lane)            */
-  int n_chunks;         /* chunks per row                                                        */
-  int warps_per_cta;
-  int cluster_ctas;     /* CTAs per thread-block cluster sharing one row pair                    */
-  int stages;           /* shared-memory pipeline depth (0 = direct register loads)             */
-  int greedy_slices;    /* CTAs per row in the greedy pass                                      */
+  int elems_per_load;              /* 8 (bf16) / 4 (fp32) on the 16-byte path, 1 on the scalar path */
+  int chunk_elems;                 /* tokens per streaming task (one warp)                    */
+  int n_chunks;                    /* chunks per row                                          */
+  int threads_per_cta;
+  int stages;                      /* shared-memory ring depth per warp (0 = direct loads)    */
+  int sampling_tasks_per_sequence; /* warp tasks of one sequence, sampling policy            */
+  int greedy_tasks_per_sequence;   /* warp tasks of one sequence, greedy policy              */
 } dspark_plan_t;
 dspark_status_t dspark_plan(int B, int K, int V, dspark_dtype_t dtype, int aligned16,
                             dspark_plan_t* plan);

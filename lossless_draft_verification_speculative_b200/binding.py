@@ -55,8 +55,8 @@ class AcceptOut(ctypes.Structure):
 
 class Plan(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int) for n in (
-        "elems_per_load", "elems_per_lane", "chunk_elems", "n_chunks", "warps_per_cta",
-        "cluster_ctas", "stages", "greedy_slices")]
+        "elems_per_load", "chunk_elems", "n_chunks", "threads_per_cta", "stages",
+        "sampling_tasks_per_sequence", "greedy_tasks_per_sequence")]
 
 
 _LIB = None
@@ -92,6 +92,8 @@ def load_library(build_if_missing: bool = True) -> ctypes.CDLL:
     lib.dspark_version.argtypes = []
     lib.dspark_workspace_bytes.restype = sz
     lib.dspark_workspace_bytes.argtypes = [i32, i32, i32, i32]
+    lib.dspark_workspace_zero_bytes.restype = sz
+    lib.dspark_workspace_zero_bytes.argtypes = [i32, i32]
     lib.dspark_plan.restype = i32
     lib.dspark_plan.argtypes = [i32, i32, i32, i32, i32, ctypes.POINTER(Plan)]
     lib.dspark_greedy_accept.restype = i32
@@ -148,18 +150,33 @@ def _split_block(P) -> Tuple[torch.Tensor, Optional[torch.Tensor], int, int]:
 
 
 class _Workspace:
-    """A per-device byte buffer reused across calls, grown on demand."""
+    """A per-device byte buffer reused across calls, grown on demand.
+
+    The library needs the workspace's counter region (a prefix whose length depends on B and
+    K) to be zero before a call, and leaves it zero after every call. A fresh buffer is
+    allocated zero-filled; when the (B, K) of consecutive calls differ the prefix moves, so
+    it is cleared again (a memset on the current stream; nothing is allocated).
+    """
 
     def __init__(self):
         self.bufs = {}
+        self.shape = {}
 
-    def get(self, device: torch.device, nbytes: int) -> torch.Tensor:
+    def get(self, device: torch.device, nbytes: int, B: int, K: int) -> torch.Tensor:
         key = device.index if device.index is not None else torch.cuda.current_device()
         buf = self.bufs.get(key)
         if buf is None or buf.numel() < nbytes:
-            buf = torch.empty(max(nbytes, 256), dtype=torch.uint8, device=device)
+            buf = new_workspace(max(nbytes, 256), device)
             self.bufs[key] = buf
+        elif self.shape.get(key) != (B, K):
+            buf[: load_library().dspark_workspace_zero_bytes(B, K)].zero_()
+        self.shape[key] = (B, K)
         return buf
+
+
+def new_workspace(nbytes: int, device) -> torch.Tensor:
+    """A workspace buffer in the state the library requires before its first call."""
+    return torch.zeros(nbytes, dtype=torch.uint8, device=device)
 
 
 _WS = _Workspace()
@@ -200,7 +217,12 @@ def _stream_handle(device) -> int:
 def greedy_accept(P: Union[torch.Tensor, Tuple[torch.Tensor, torch.Tensor]],
                   drafts: torch.Tensor, *, out: Optional[AcceptResult] = None,
                   workspace: Optional[torch.Tensor] = None) -> AcceptResult:
-    """Greedy block verify on the GPU: accept drafts while they equal the base argmax."""
+    """Greedy block verify on the GPU: accept drafts while they equal the base argmax.
+
+    ``workspace``, if given, must follow the library's contract: its first
+    ``dspark_workspace_zero_bytes(B, K)`` bytes zero before the first call with this (B, K)
+    (``new_workspace`` returns such a buffer); calls leave them zero.
+    """
     lib = load_library()
     p1, pv, ld_p1, ld_pv = _split_block(P)
     if not p1.is_cuda:
@@ -210,7 +232,7 @@ def greedy_accept(P: Union[torch.Tensor, Tuple[torch.Tensor, torch.Tensor]],
     drafts = _check_drafts(drafts, B, K, p1.device)
     res = out if out is not None else _alloc_result(B, K, p1.device, diagnostics=False)
     nbytes = lib.dspark_workspace_bytes(B, K, V, DTYPE_CODES[p1.dtype])
-    ws = workspace if workspace is not None else _WS.get(p1.device, nbytes)
+    ws = workspace if workspace is not None else _WS.get(p1.device, nbytes, B, K)
     rc = lib.dspark_greedy_accept(_ptr(p1), ld_p1, _ptr(pv), ld_pv, DTYPE_CODES[p1.dtype],
                                   _ptr(drafts), B, K, V, _out_struct(res), _ptr(ws),
                                   ws.numel() * ws.element_size(), _stream_handle(p1.device))
@@ -240,7 +262,7 @@ def speculative_sample_accept(P: Union[torch.Tensor, Tuple[torch.Tensor, torch.T
         raise ValueError("uniforms must be a contiguous float32 [B, K+1] tensor on P's device")
     res = out if out is not None else _alloc_result(B, K, p1.device, diagnostics=True)
     nbytes = lib.dspark_workspace_bytes(B, K, V, DTYPE_CODES[p1.dtype])
-    ws = workspace if workspace is not None else _WS.get(p1.device, nbytes)
+    ws = workspace if workspace is not None else _WS.get(p1.device, nbytes, B, K)
     rc = lib.dspark_speculative_sample_accept(
         _ptr(p1), ld_p1, _ptr(pv), ld_pv, _ptr(Q), DTYPE_CODES[p1.dtype], _ptr(drafts), B, K,
         V, float(temperature), _ptr(uniforms), _out_struct(res), _ptr(ws),

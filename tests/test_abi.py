@@ -49,17 +49,26 @@ def test_workspace_bytes(lib):
 
 
 def test_plans_cover_every_workload_shape(lib):
-    for V, want_cluster, want_warps in [(64, 1, 1), (129280, 16, 8), (151936, 16, 10),
-                                        (262144, 16, 16), (5000, 1, 5), (20000, 4, 5)]:
+    for V in (1, 64, 2048, 2049, 129280, 151936, 262144):
         p = binding.Plan()
         assert lib.dspark_plan(4, 7, V, BF16, 1, ctypes.byref(p)) == 0
-        assert p.cluster_ctas == want_cluster and p.warps_per_cta == want_warps, V
-        assert p.cluster_ctas * p.warps_per_cta * p.chunk_elems >= V
-        assert p.n_chunks == -(-V // p.chunk_elems)
-        assert p.elems_per_load == 8 and p.stages >= 2
+        assert p.n_chunks == -(-V // p.chunk_elems) and p.n_chunks * p.chunk_elems >= V
+        assert p.elems_per_load == 8 and p.stages >= 2 and p.threads_per_cta % 32 == 0
+        nc = p.n_chunks
+        assert p.sampling_tasks_per_sequence == 15 * nc + (nc + 1) // 2 + 2  # STREAM, RESID, rest
+        assert p.greedy_tasks_per_sequence == 8 * nc + 1          # STREAM, DECIDE
         assert lib.dspark_plan(4, 7, V, BF16, 0, ctypes.byref(p)) == 0
         assert p.elems_per_load == 1 and p.stages == 0
+        assert lib.dspark_plan(4, 7, V, F32, 1, ctypes.byref(p)) == 0
+        assert p.elems_per_load == 4
     assert lib.dspark_plan(4, 7, 262145, BF16, 1, ctypes.byref(binding.Plan())) == 2
+
+
+def test_workspace_zero_region_is_a_prefix(lib):
+    for B, K in ((1, 0), (64, 7), (256, 15), (3, 32)):
+        z = lib.dspark_workspace_zero_bytes(B, K)
+        assert 0 < z <= lib.dspark_workspace_bytes(B, K, 129280, BF16)
+        assert z >= 16 * B
 
 
 def _greedy(lib, **kw):
