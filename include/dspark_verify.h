@@ -146,6 +146,30 @@ dspark_status_t dspark_speculative_sample_accept(const void* p1, int64_t ld_p1, 
                                                  void* workspace, size_t workspace_bytes,
                                                  void* stream);
 
+/* speculative_sample_accept without a workspace argument. The pages have no counterpart of
+ * this entry point: it exists for callers that cannot allocate device memory where they
+ * verify (a serving loop whose KV-cache pool took all free HBM at start-up and left no
+ * allocator to draw a workspace from; a host runtime with no device allocator of its own).
+ *  Arguments, results and T == 0 behaviour are those of dspark_speculative_sample_accept.
+ *  Scratch: one fixed array of DSPARK_STATIC_SCRATCH_BYTES per device, in the library's own
+ *    module image; the call allocates nothing. A shape whose dspark_workspace_bytes exceeds
+ *    that size is rejected with DSPARK_ERR_WORKSPACE before anything is enqueued (the limit
+ *    holds e.g. B = 64, K = 7, V = 129280 bf16, about 0.5 MB; not B = 256, K = 15, V = 262144).
+ *  Set-up: the first call on a device, with that device current, looks up the array's device
+ *    address (cudaGetSymbolAddress) and keeps it; make that first call before any stream
+ *    capture on that device. A failed look-up returns DSPARK_ERR_CUDA.
+ *  Each call clears the array's counter region (dspark_workspace_zero_bytes(B, K) bytes) on
+ *    `stream` before its kernel, so an earlier DSPARK_SEQ_TIMEOUT needs no clean-up.
+ *  All calls on one device share the array: calls that overlap on the GPU race and give
+ *    wrong results. Order them (one stream, or events). */
+#define DSPARK_STATIC_SCRATCH_BYTES ((size_t)4 << 20)
+dspark_status_t dspark_speculative_sample_accept_static(const void* p1, int64_t ld_p1,
+                                                        const void* pv, int64_t ld_pv,
+                                                        const void* q, dspark_dtype_t dtype,
+                                                        const int32_t* drafts, int B, int K, int V,
+                                                        float temperature, const float* uniforms,
+                                                        dspark_accept_out_t out, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -17,6 +17,7 @@ from .binding import (  # noqa: F401
     load_library,
     plan,
     speculative_sample_accept,
+    speculative_sample_accept_static,
     workspace_bytes,
 )
 
@@ -25,6 +26,7 @@ __all__ = [
     "DsparkError",
     "greedy_accept",
     "speculative_sample_accept",
+    "speculative_sample_accept_static",
     "load_library",
     "plan",
     "workspace_bytes",

@@ -25,6 +25,7 @@ import torch
 from . import build_lib
 
 DSPARK_OK = 0
+STATIC_SCRATCH_BYTES = 4 << 20  # DSPARK_STATIC_SCRATCH_BYTES of the C header
 STATUS_NAMES = {0: "DSPARK_OK", 1: "DSPARK_ERR_INVALID_ARG", 2: "DSPARK_ERR_UNSUPPORTED",
                 3: "DSPARK_ERR_CUDA", 4: "DSPARK_ERR_WORKSPACE"}
 DTYPE_CODES = {torch.bfloat16: 0, torch.float32: 1}
@@ -103,6 +104,10 @@ def load_library(build_if_missing: bool = True) -> ctypes.CDLL:
     lib.dspark_speculative_sample_accept.argtypes = [vp, i64, vp, i64, vp, i32, vp, i32, i32,
                                                      i32, ctypes.c_float, vp, AcceptOut, vp, sz,
                                                      vp]
+    lib.dspark_speculative_sample_accept_static.restype = i32
+    lib.dspark_speculative_sample_accept_static.argtypes = [vp, i64, vp, i64, vp, i32, vp, i32,
+                                                            i32, i32, ctypes.c_float, vp,
+                                                            AcceptOut, vp]
     _LIB = lib
     return lib
 
@@ -270,6 +275,31 @@ def speculative_sample_accept(P: Union[torch.Tensor, Tuple[torch.Tensor, torch.T
     if rc != DSPARK_OK:
         raise DsparkError(rc, "dspark_speculative_sample_accept")
     return res
+
+
+def speculative_sample_accept_static(P: Union[torch.Tensor, Tuple[torch.Tensor, torch.Tensor]],
+                                     Q: Optional[torch.Tensor], drafts: torch.Tensor,
+                                     temperature: float, uniforms: torch.Tensor, *,
+                                     out: AcceptResult) -> AcceptResult:
+    """speculative_sample_accept on the library's fixed per-device scratch: no workspace.
+
+    ``out`` is required, so that the call itself allocates nothing. Shapes whose workspace
+    exceeds STATIC_SCRATCH_BYTES raise DsparkError(DSPARK_ERR_WORKSPACE). Calls on one
+    device that overlap on the GPU share the scratch and race.
+    """
+    lib = load_library()
+    p1, pv, ld_p1, ld_pv = _split_block(P)
+    if not p1.is_cuda:
+        raise RuntimeError("speculative_sample_accept_static runs on CUDA tensors only")
+    B, V = p1.shape
+    K = 0 if pv is None else pv.shape[1]
+    drafts = _check_drafts(drafts, B, K, p1.device)
+    rc = lib.dspark_speculative_sample_accept_static(
+        _ptr(p1), ld_p1, _ptr(pv), ld_pv, _ptr(Q), DTYPE_CODES[p1.dtype], _ptr(drafts), B, K,
+        V, float(temperature), _ptr(uniforms), _out_struct(out), _stream_handle(p1.device))
+    if rc != DSPARK_OK:
+        raise DsparkError(rc, "dspark_speculative_sample_accept_static")
+    return out
 
 
 def _check_drafts(drafts: Optional[torch.Tensor], B: int, K: int, device) -> Optional[torch.Tensor]:

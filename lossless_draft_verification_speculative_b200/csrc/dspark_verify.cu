@@ -221,6 +221,34 @@ TaskParams base_params(const void* p1, int64_t ld_p1, const void* pv, int64_t ld
   return prm;
 }
 
+// ----------------------------------------------------- fixed scratch, no allocation
+// Scratch of dspark_speculative_sample_accept_static. Some callers cannot allocate device
+// memory where they verify: a serving loop that gave every free byte of HBM to its KV-cache
+// pool at start-up has no allocator left to draw a workspace from, and a host runtime in
+// another language may hold no device allocator at all. For them the library keeps one
+// fixed array per device, part of its own module image, so a call allocates nothing.
+// Every call on a device uses the same array: calls that overlap on the GPU race on it.
+static __device__ __align__(256) unsigned char g_static_scratch[DSPARK_STATIC_SCRATCH_BYTES];
+
+std::mutex g_scratch_mu;
+void* g_scratch_addr[kMaxDevices] = {};
+
+// Device address of the fixed scratch on the current device, looked up once per device
+// (cudaGetSymbolAddress, with that device current) and cached.
+dspark_status_t static_scratch_address(void** addr) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return DSPARK_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return DSPARK_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lk(g_scratch_mu);
+  if (!g_scratch_addr[dev]) {
+    void* a = nullptr;
+    if (cudaGetSymbolAddress(&a, g_static_scratch) != cudaSuccess || !a) return DSPARK_ERR_CUDA;
+    g_scratch_addr[dev] = a;
+  }
+  *addr = g_scratch_addr[dev];
+  return DSPARK_OK;
+}
+
 }  // namespace
 }  // namespace dspark
 
@@ -334,6 +362,35 @@ dspark_status_t dspark_speculative_sample_accept(const void* p1, int64_t ld_p1, 
   if (!a16) return run_tasks<float, 1, true, false>(prm, pl, 9, s);
   if (pl.stages) return run_tasks<float, 4, true, true>(prm, pl, 10, s);
   return run_tasks<float, 4, true, false>(prm, pl, 11, s);
+}
+
+dspark_status_t dspark_speculative_sample_accept_static(const void* p1, int64_t ld_p1,
+                                                        const void* pv, int64_t ld_pv,
+                                                        const void* q, dspark_dtype_t dtype,
+                                                        const int32_t* drafts, int B, int K, int V,
+                                                        float temperature, const float* uniforms,
+                                                        dspark_accept_out_t out, void* stream) {
+  // every synchronous check first, so that a rejected call enqueues nothing
+  if (!(temperature >= 0.f) || !std::isfinite(temperature)) return DSPARK_ERR_INVALID_ARG;
+  dspark_status_t st = check_common(p1, ld_p1, pv, ld_pv, dtype, drafts, B, K, V, out);
+  if (st != DSPARK_OK || B == 0) return st;
+  if (temperature > 0.f) {
+    if (!uniforms || (K > 0 && !q)) return DSPARK_ERR_INVALID_ARG;
+    if (K > 0 && !aligned(q, static_cast<size_t>(elem_bytes(dtype)))) return DSPARK_ERR_UNSUPPORTED;
+  }
+  const size_t need = dspark_workspace_bytes(B, K, V, dtype);
+  if (need == 0) return DSPARK_ERR_UNSUPPORTED;
+  if (need > DSPARK_STATIC_SCRATCH_BYTES) return DSPARK_ERR_WORKSPACE;
+  void* scratch = nullptr;
+  st = static_scratch_address(&scratch);
+  if (st != DSPARK_OK) return st;
+  // the counters at the front of the scratch must start at zero
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cudaMemsetAsync(scratch, 0, dspark_workspace_zero_bytes(B, K), s) != cudaSuccess)
+    return DSPARK_ERR_CUDA;
+  return dspark_speculative_sample_accept(p1, ld_p1, pv, ld_pv, q, dtype, drafts, B, K, V,
+                                          temperature, uniforms, out, scratch,
+                                          DSPARK_STATIC_SCRATCH_BYTES, stream);
 }
 
 }  // extern "C"
