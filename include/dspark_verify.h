@@ -72,7 +72,7 @@ typedef enum { DSPARK_BF16 = 0, DSPARK_F32 = 1 } dspark_dtype_t;
 #define DSPARK_SEQ_NONFINITE 2     /* a row with NaN / +inf, or with no finite value       */
 #define DSPARK_SEQ_ZERO_RESIDUAL 4 /* not an error: residual mass rounded to 0 after a
                                       rejection; the correction was drawn from p_j          */
-#define DSPARK_SEQ_TIMEOUT 8       /* an internal bounded wait gave up (never expected)     */
+#define DSPARK_SEQ_TIMEOUT 8       /* reserved: the kernels have no waits that can give up  */
 
 /* AcceptResult: device buffers, caller-allocated. Required: n_accepted, tokens, next_token.
  * The optional ones (NULL = not written) are diagnostics of the sampling policy. */
@@ -94,25 +94,31 @@ int dspark_version(void);
 
 /* Bytes of device workspace the verify calls need for this shape (valid for both policies).
  * Returns 0 when the shape is invalid or unsupported.
- * Contract: the first dspark_workspace_zero_bytes(B, K) bytes of a workspace must be zero
- * before its first call (e.g. cudaMemsetAsync once after allocating it); every call that
- * returns DSPARK_OK leaves them zero again, so no per-call clearing is needed. After a call
- * reported DSPARK_SEQ_TIMEOUT for some sequence, clear them again. The rest of the workspace
- * needs no initialisation. One workspace serves one call at a time. */
+ * Contract: the first dspark_workspace_zero_bytes(B, K) bytes of a workspace (one arrival
+ * counter per sequence) must be zero before its first call (e.g. cudaMemsetAsync once after
+ * allocating it); every call that returns DSPARK_OK leaves them zero again once it has run,
+ * so no per-call clearing is needed. The rest of the workspace needs no initialisation. One
+ * workspace serves one call at a time. */
 size_t dspark_workspace_bytes(int B, int K, int V, dspark_dtype_t dtype);
 size_t dspark_workspace_zero_bytes(int B, int K);
 
-/* Launch geometry the calls would use for this shape (for tests and reports).
+/* Launch geometry of the calls for this shape (for tests and reports).
  * Returns DSPARK_OK and fills the fields, or an error for an invalid / unsupported shape.
- * `aligned16` says whether every row start will be 16-byte aligned (vector path). */
+ * `aligned16` says whether every row start will be 16-byte aligned (vector path).
+ * A call runs two kernels on `stream`. Pass 1 reads every logit row once: its units are the
+ * (row, chunk) pairs, and each warp of one full wave streams an equal contiguous run of them
+ * and writes one statistics record per unit. Pass 2, a programmatic dependent launch, takes
+ * the per-sequence decisions and, when sampling, computes the draw's law chunk by chunk and
+ * draws the token. */
 typedef struct {
   int elems_per_load;              /* 8 (bf16) / 4 (fp32) on the 16-byte path, 1 on the scalar path */
-  int chunk_elems;                 /* tokens per streaming task (one warp)                    */
-  int n_chunks;                    /* chunks per row                                          */
-  int threads_per_cta;
-  int stages;                      /* shared-memory ring depth per warp (0 = direct loads)    */
-  int sampling_tasks_per_sequence; /* warp tasks of one sequence, sampling policy            */
-  int greedy_tasks_per_sequence;   /* warp tasks of one sequence, greedy policy              */
+  int loads_in_flight;             /* loads each lane of pass 1 keeps in flight                    */
+  int threads_per_cta;             /* both passes                                                 */
+  int chunk_elems;                 /* tokens per chunk (pass-1 unit, pass-2 chunk)                */
+  int n_chunks;                    /* chunks per row                                              */
+  int greedy_units_per_sequence;   /* pass-1 units of one sequence, greedy: (K+1) * n_chunks      */
+  int sampling_units_per_sequence; /* pass-1 units of one sequence, sampling: (2K+1) * n_chunks   */
+  int finish_ctas_per_sequence;    /* pass-2 CTAs per sequence, sampling policy                   */
 } dspark_plan_t;
 dspark_status_t dspark_plan(int B, int K, int V, dspark_dtype_t dtype, int aligned16,
                             dspark_plan_t* plan);
@@ -159,7 +165,7 @@ dspark_status_t dspark_speculative_sample_accept(const void* p1, int64_t ld_p1, 
  *    address (cudaGetSymbolAddress) and keeps it; make that first call before any stream
  *    capture on that device. A failed look-up returns DSPARK_ERR_CUDA.
  *  Each call clears the array's counter region (dspark_workspace_zero_bytes(B, K) bytes) on
- *    `stream` before its kernel, so an earlier DSPARK_SEQ_TIMEOUT needs no clean-up.
+ *    `stream` before its kernels.
  *  All calls on one device share the array: calls that overlap on the GPU race and give
  *    wrong results. Order them (one stream, or events). */
 #define DSPARK_STATIC_SCRATCH_BYTES ((size_t)4 << 20)

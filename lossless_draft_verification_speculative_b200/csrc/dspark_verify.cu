@@ -1,38 +1,27 @@
 // C ABI of the DSpark block verify/accept step: argument checks, launch planning and the
-// kernel launch. The device work is the task kernel of tasks.cuh.
+// two kernel launches of a call (pass 1 in stream.cuh, pass 2 in finish.cuh).
 #include <cmath>
 #include <cstdlib>
 #include <mutex>
 
 #include "common.cuh"
-#include "tasks.cuh"
+#include "finish.cuh"
+#include "stream.cuh"
 
 namespace dspark {
 namespace {
 
-constexpr int kAbiVersion = 2;
+constexpr int kAbiVersion = 3;
 constexpr int kMaxDevices = 64;
-constexpr size_t kRingBudgetPerCta = 100 * 1024;  // shared memory for one CTA's rings
 
-// ------------------------------------------------------------------------- tuning knobs
-
-struct Tuning {
-  int stages = 0;        // 0 = automatic
-  bool no_tma = false;   // direct loads instead of the bulk-copy rings
-  int max_ctas = 0;      // 0 = as many as fit
-};
-
-const Tuning& tuning() {
-  static const Tuning t = [] {
-    Tuning v;
-    if (const char* s = std::getenv("DSPARK_STAGES")) v.stages = std::atoi(s);
-    if (const char* s = std::getenv("DSPARK_NO_TMA")) v.no_tma = std::atoi(s) != 0;
-    if (const char* s = std::getenv("DSPARK_MAX_CTAS")) v.max_ctas = std::atoi(s);
-    if (v.stages < 0 || v.stages > kMaxTaskStages) v.stages = 0;
-    if (v.max_ctas < 0) v.max_ctas = 0;
-    return v;
+// Pass-1 CTAs may be capped for experiments (DSPARK_MAX_CTAS); 0 = one full wave.
+int max_ctas_override() {
+  static const int v = [] {
+    const char* s = std::getenv("DSPARK_MAX_CTAS");
+    const int n = s ? std::atoi(s) : 0;
+    return n > 0 ? n : 0;
   }();
-  return t;
+  return v;
 }
 
 // ------------------------------------------------------------------------------ plans
@@ -48,9 +37,9 @@ bool shape_ok(int B, int K, int V) {
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
 struct Plan {
-  int vec;     // elements per load: 16-byte vectors (8 bf16 / 4 fp32) or 1
-  int nch;     // 2048-token chunks per row
-  int stages;  // ring depth per warp, 0 = direct loads
+  int vec;  // elements per load: 16-byte vectors (8 bf16 / 4 fp32) or 1
+  int nch;  // 2048-token chunks per row
+  int G;    // pass-2 CTAs per sequence, sampling
 };
 
 bool make_plan(int V, dspark_dtype_t dt, bool aligned16, Plan* pl) {
@@ -59,40 +48,28 @@ bool make_plan(int V, dspark_dtype_t dt, bool aligned16, Plan* pl) {
   if (nch < 1 || nch > kMaxChunkCount) return false;
   pl->vec = aligned16 ? 16 / es : 1;
   pl->nch = static_cast<int>(nch);
-  pl->stages = 0;
-  if (aligned16 && !tuning().no_tma) {
-    int st = static_cast<int>(kRingBudgetPerCta / (static_cast<size_t>(kStreamWarps) * kCE * es));
-    st = st < 2 ? 2 : (st > kMaxTaskStages ? kMaxTaskStages : st);
-    if (tuning().stages) st = tuning().stages;
-    pl->stages = st;
-  }
+  pl->G = (pl->nch + kWarps - 1) / kWarps;
   return true;
 }
 
 size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
-// Workspace regions. The counters come first: they must be zero before a call, and every
-// call leaves them zero again. The rest needs no initialisation.
+// Workspace regions. The per-sequence arrival counters come first: they must be zero before
+// a call, and every call leaves them zero again. The rest needs no initialisation.
 struct WsLayout {
-  size_t dq, seq_cnt, chunk_stat, row_stat, dec, resid, total;
+  size_t arrive, rec, mass, total;
 };
 
 WsLayout ws_layout(long long B, long long K, int nch) {
   const long long rows = 2 * K + 1;
   WsLayout w{};
   size_t off = 0;
-  w.dq = off;
-  off = align256(off + sizeof(DepQueue));
-  w.seq_cnt = off;
-  off = align256(off + sizeof(SeqCounters) * static_cast<size_t>(B));
-  w.chunk_stat = off;
+  w.arrive = off;
+  off = align256(off + sizeof(unsigned) * static_cast<size_t>(B));
+  w.rec = off;
   off = align256(off + sizeof(float2) * static_cast<size_t>(B * rows * nch));
-  w.row_stat = off;
-  off = align256(off + sizeof(float2) * static_cast<size_t>(B * rows));
-  w.dec = off;
-  off = align256(off + sizeof(SeqDecision) * static_cast<size_t>(B));
-  w.resid = off;
-  off = align256(off + sizeof(float) * static_cast<size_t>(B * nch));
+  w.mass = off;
+  off = align256(off + sizeof(float2) * static_cast<size_t>(B * nch));
   w.total = off;
   return w;
 }
@@ -101,76 +78,94 @@ WsLayout ws_layout(long long B, long long K, int nch) {
 
 std::mutex g_mu;
 struct OccEntry {
-  void* fn;
+  const void* fn;
   int dev;
-  size_t smem;
-  int ctas;  // co-resident CTAs on the device
+  int ctas;  // co-resident CTAs of the kernel on the device
 };
 OccEntry g_occ[64];
 int g_occ_n = 0;
-bool g_attr_done[kMaxDevices][16] = {};
 
-// CTAs of the task kernel that fit on the device at once (the schedule needs them all
-// resident); 0 if it cannot launch.
-int resident_ctas(void* fn, int fn_id, size_t smem, cudaError_t* err) {
+int resident_ctas(const void* fn, cudaError_t* err) {
   int dev = 0;
   *err = cudaGetDevice(&dev);
   if (*err != cudaSuccess) return 0;
   std::lock_guard<std::mutex> lk(g_mu);
   for (int n = 0; n < g_occ_n; ++n)
-    if (g_occ[n].fn == fn && g_occ[n].dev == dev && g_occ[n].smem == smem) return g_occ[n].ctas;
-  if (dev < kMaxDevices && !g_attr_done[dev][fn_id]) {
-    // allow the largest dynamic shared memory the device takes next to the static part
-    int optin = 0;
-    *err = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
-    if (*err != cudaSuccess) return 0;
-    cudaFuncAttributes fa;
-    *err = cudaFuncGetAttributes(&fa, fn);
-    if (*err != cudaSuccess) return 0;
-    if (smem + fa.sharedSizeBytes > static_cast<size_t>(optin)) return 0;
-    *err = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                optin - static_cast<int>(fa.sharedSizeBytes));
-    if (*err != cudaSuccess) return 0;
-    g_attr_done[dev][fn_id] = true;
-  }
+    if (g_occ[n].fn == fn && g_occ[n].dev == dev) return g_occ[n].ctas;
   int per_sm = 0, sms = 0;
-  *err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, kTaskThreads, smem);
+  *err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, kThreads, 0);
   if (*err != cudaSuccess) return 0;
   *err = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   if (*err != cudaSuccess) return 0;
   const int n = per_sm * sms;
-  if (g_occ_n < 64) g_occ[g_occ_n++] = OccEntry{fn, dev, smem, n};
+  if (g_occ_n < 64) g_occ[g_occ_n++] = OccEntry{fn, dev, n};
   return n;
 }
 
-template <typename T, int VEC, bool kSample, bool kTma>
-dspark_status_t run_tasks(TaskParams prm, const Plan& pl, int fn_id, cudaStream_t stream) {
-  const size_t smem =
-      kTma ? static_cast<size_t>(kStreamWarps) * pl.stages * kCE * Elem<T>::kBytes +
-                 static_cast<size_t>(kStreamWarps) * kMaxTaskStages * sizeof(uint64_t)
-           : 0;
-  void* fn = reinterpret_cast<void*>(&verify_tasks_kernel<T, VEC, kSample, kTma>);
+struct Call {
+  RowSet rs;
+  int B;
+  const int32_t* drafts;
+  const float* uniforms;
+  float scale;
+  dspark_accept_out_t out;
+  char* ws;
+};
+
+// Pass 1 over every (row, chunk) unit (one wave of warps, equal contiguous runs of units),
+// then pass 2 launched as a programmatic dependent of it.
+template <typename T, int VEC, bool kSample>
+dspark_status_t run_call(const Call& c, const Plan& pl, cudaStream_t stream) {
+  const void* k1 = reinterpret_cast<const void*>(&stream_stats_kernel<T, VEC, kSample>);
   cudaError_t e = cudaSuccess;
-  int ctas = resident_ctas(fn, fn_id, smem, &e);
+  int ctas = resident_ctas(k1, &e);
   if (e != cudaSuccess) return DSPARK_ERR_CUDA;
   if (ctas < 1) return DSPARK_ERR_UNSUPPORTED;
-  if (tuning().max_ctas) ctas = ctas < tuning().max_ctas ? ctas : tuning().max_ctas;
-  prm.n_stream = static_cast<long long>(prm.B) * prm.rows * prm.nch;
-  prm.n_resid = (prm.nch + kResidGroup - 1) / kResidGroup;
-  prm.n_dep_per_seq = kSample ? prm.n_resid + 2 : 1;
-  // no more CTAs than there is streaming work for
-  const long long want = (prm.n_stream + kStreamWarps - 1) / kStreamWarps;
-  if (want < ctas) ctas = static_cast<int>(want < 1 ? 1 : want);
-  prm.stages = pl.stages;
-  prm.stream_warps = ctas * kStreamWarps;
-  prm.dep_warps = ctas;
+  if (max_ctas_override() && max_ctas_override() < ctas) ctas = max_ctas_override();
+  const WsLayout w = ws_layout(c.B, c.rs.K, pl.nch);
+  const long long n_units = static_cast<long long>(c.B) * c.rs.rows * pl.nch;
+  const long long warps = static_cast<long long>(ctas) * kWarps;
+  const long long upw = (n_units + warps - 1) / warps;
+  const long long need = (n_units + upw - 1) / upw;
+  const int grid1 = static_cast<int>((need + kWarps - 1) / kWarps);
+
+  StreamParams sp{};
+  sp.rs = c.rs;
+  sp.n_units = n_units;
+  sp.upw = upw;
+  sp.nch = pl.nch;
+  sp.scale = c.scale;
+  sp.rec = reinterpret_cast<float2*>(c.ws + w.rec);
+  stream_stats_kernel<T, VEC, kSample><<<grid1, kThreads, 0, stream>>>(sp);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return DSPARK_ERR_CUDA;
+
+  FinishParams fp{};
+  fp.rs = c.rs;
+  fp.drafts = c.drafts;
+  fp.uniforms = c.uniforms;
+  fp.B = c.B;
+  fp.G = pl.G;
+  fp.nch = pl.nch;
+  fp.scale = c.scale;
+  fp.rec = sp.rec;
+  fp.mass = reinterpret_cast<float2*>(c.ws + w.mass);
+  fp.arrive = reinterpret_cast<unsigned*>(c.ws + w.arrive);
+  fp.out = c.out;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(static_cast<unsigned>(ctas), 1, 1);
-  cfg.blockDim = dim3(kTaskThreads, 1, 1);
-  cfg.dynamicSmemBytes = smem;
+  cfg.gridDim = dim3(static_cast<unsigned>(kSample ? static_cast<long long>(c.B) * pl.G : c.B), 1, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = 0;
   cfg.stream = stream;
-  cfg.numAttrs = 0;
-  e = cudaLaunchKernelEx(&cfg, verify_tasks_kernel<T, VEC, kSample, kTma>, prm);
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if constexpr (kSample)
+    e = cudaLaunchKernelEx(&cfg, finish_sample_kernel<T, VEC>, fp);
+  else
+    e = cudaLaunchKernelEx(&cfg, finish_greedy_kernel<T>, fp);
   return e == cudaSuccess ? DSPARK_OK : DSPARK_ERR_CUDA;
 }
 
@@ -191,34 +186,25 @@ dspark_status_t check_common(const void* p1, int64_t ld_p1, const void* pv, int6
   return DSPARK_OK;
 }
 
-TaskParams base_params(const void* p1, int64_t ld_p1, const void* pv, int64_t ld_pv, const void* q,
-                       const int32_t* drafts, const float* uniforms, int B, int K, int V,
-                       float scale, int rows, const Plan& pl, void* workspace,
-                       const dspark_accept_out_t& out) {
-  const WsLayout w = ws_layout(B, K, pl.nch);
-  char* ws = static_cast<char*>(workspace);
-  TaskParams prm{};
-  prm.p1 = p1;
-  prm.pv = pv;
-  prm.q = q;
-  prm.ld_p1 = ld_p1;
-  prm.ld_pv = ld_pv;
-  prm.B = B;
-  prm.K = K;
-  prm.V = V;
-  prm.scale = scale;
-  prm.drafts = drafts;
-  prm.uniforms = uniforms;
-  prm.nch = pl.nch;
-  prm.rows = rows;
-  prm.chunk_stat = reinterpret_cast<float2*>(ws + w.chunk_stat);
-  prm.row_stat = reinterpret_cast<float2*>(ws + w.row_stat);
-  prm.seq_cnt = reinterpret_cast<SeqCounters*>(ws + w.seq_cnt);
-  prm.dq = reinterpret_cast<DepQueue*>(ws + w.dq);
-  prm.dec = reinterpret_cast<SeqDecision*>(ws + w.dec);
-  prm.resid_mass = reinterpret_cast<float*>(ws + w.resid);
-  prm.out = out;
-  return prm;
+Call make_call(const void* p1, int64_t ld_p1, const void* pv, int64_t ld_pv, const void* q,
+               const int32_t* drafts, const float* uniforms, int B, int K, int V, float scale,
+               int rows, void* workspace, const dspark_accept_out_t& out) {
+  Call c{};
+  c.rs.p1 = p1;
+  c.rs.pv = pv;
+  c.rs.q = q;
+  c.rs.ld_p1 = ld_p1;
+  c.rs.ld_pv = ld_pv;
+  c.rs.K = K;
+  c.rs.V = V;
+  c.rs.rows = rows;
+  c.B = B;
+  c.drafts = drafts;
+  c.uniforms = uniforms;
+  c.scale = scale;
+  c.out = out;
+  c.ws = static_cast<char*>(workspace);
+  return c;
 }
 
 // ----------------------------------------------------- fixed scratch, no allocation
@@ -279,8 +265,7 @@ size_t dspark_workspace_bytes(int B, int K, int V, dspark_dtype_t dtype) {
 
 size_t dspark_workspace_zero_bytes(int B, int K) {
   if (!shape_ok(B, K, 1)) return 0;
-  Plan pl{1, 1, 0};
-  return ws_layout(B, K, pl.nch).chunk_stat;
+  return ws_layout(B, K, 1).rec;
 }
 
 dspark_status_t dspark_plan(int B, int K, int V, dspark_dtype_t dtype, int aligned16,
@@ -290,13 +275,13 @@ dspark_status_t dspark_plan(int B, int K, int V, dspark_dtype_t dtype, int align
   Plan pl;
   if (!make_plan(V, dtype, aligned16 != 0, &pl)) return DSPARK_ERR_UNSUPPORTED;
   plan->elems_per_load = pl.vec;
+  plan->loads_in_flight = kBatchVecs;
+  plan->threads_per_cta = kThreads;
   plan->chunk_elems = kCE;
   plan->n_chunks = pl.nch;
-  plan->threads_per_cta = kTaskThreads;
-  plan->stages = pl.stages;
-  plan->sampling_tasks_per_sequence =
-      (2 * K + 1) * pl.nch + (pl.nch + kResidGroup - 1) / kResidGroup + 2;
-  plan->greedy_tasks_per_sequence = (K + 1) * pl.nch + 1;
+  plan->greedy_units_per_sequence = (K + 1) * pl.nch;
+  plan->sampling_units_per_sequence = (2 * K + 1) * pl.nch;
+  plan->finish_ctas_per_sequence = pl.G;
   return DSPARK_OK;
 }
 
@@ -313,17 +298,12 @@ dspark_status_t dspark_greedy_accept(const void* p1, int64_t ld_p1, const void* 
   if (!make_plan(V, dtype, a16, &pl)) return DSPARK_ERR_UNSUPPORTED;
   if (!workspace || workspace_bytes < ws_layout(B, K, pl.nch).total || !aligned(workspace, 256))
     return DSPARK_ERR_WORKSPACE;
-  TaskParams prm = base_params(p1, ld_p1, pv, ld_pv, nullptr, drafts, nullptr, B, K, V, 0.f,
-                               K + 1, pl, workspace, out);
+  const Call c = make_call(p1, ld_p1, pv, ld_pv, nullptr, drafts, nullptr, B, K, V, 0.f, K + 1,
+                           workspace, out);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (dtype == DSPARK_BF16) {
-    if (!a16) return run_tasks<bf16_t, 1, false, false>(prm, pl, 0, s);
-    if (pl.stages) return run_tasks<bf16_t, 8, false, true>(prm, pl, 1, s);
-    return run_tasks<bf16_t, 8, false, false>(prm, pl, 2, s);
-  }
-  if (!a16) return run_tasks<float, 1, false, false>(prm, pl, 3, s);
-  if (pl.stages) return run_tasks<float, 4, false, true>(prm, pl, 4, s);
-  return run_tasks<float, 4, false, false>(prm, pl, 5, s);
+  if (dtype == DSPARK_BF16)
+    return a16 ? run_call<bf16_t, 8, false>(c, pl, s) : run_call<bf16_t, 1, false>(c, pl, s);
+  return a16 ? run_call<float, 4, false>(c, pl, s) : run_call<float, 1, false>(c, pl, s);
 }
 
 dspark_status_t dspark_speculative_sample_accept(const void* p1, int64_t ld_p1, const void* pv,
@@ -351,17 +331,12 @@ dspark_status_t dspark_speculative_sample_accept(const void* p1, int64_t ld_p1, 
     return DSPARK_ERR_WORKSPACE;
   const float scale = static_cast<float>(1.4426950408889634 / static_cast<double>(temperature));
   if (!std::isfinite(scale)) return DSPARK_ERR_INVALID_ARG;
-  TaskParams prm = base_params(p1, ld_p1, pv, ld_pv, q, drafts, uniforms, B, K, V, scale,
-                               2 * K + 1, pl, workspace, out);
+  const Call c = make_call(p1, ld_p1, pv, ld_pv, q, drafts, uniforms, B, K, V, scale, 2 * K + 1,
+                           workspace, out);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (dtype == DSPARK_BF16) {
-    if (!a16) return run_tasks<bf16_t, 1, true, false>(prm, pl, 6, s);
-    if (pl.stages) return run_tasks<bf16_t, 8, true, true>(prm, pl, 7, s);
-    return run_tasks<bf16_t, 8, true, false>(prm, pl, 8, s);
-  }
-  if (!a16) return run_tasks<float, 1, true, false>(prm, pl, 9, s);
-  if (pl.stages) return run_tasks<float, 4, true, true>(prm, pl, 10, s);
-  return run_tasks<float, 4, true, false>(prm, pl, 11, s);
+  if (dtype == DSPARK_BF16)
+    return a16 ? run_call<bf16_t, 8, true>(c, pl, s) : run_call<bf16_t, 1, true>(c, pl, s);
+  return a16 ? run_call<float, 4, true>(c, pl, s) : run_call<float, 1, true>(c, pl, s);
 }
 
 dspark_status_t dspark_speculative_sample_accept_static(const void* p1, int64_t ld_p1,
