@@ -72,7 +72,8 @@ typedef enum { DSPARK_BF16 = 0, DSPARK_F32 = 1 } dspark_dtype_t;
 #define DSPARK_SEQ_NONFINITE 2     /* a row with NaN / +inf, or with no finite value       */
 #define DSPARK_SEQ_ZERO_RESIDUAL 4 /* not an error: residual mass rounded to 0 after a
                                       rejection; the correction was drawn from p_j          */
-#define DSPARK_SEQ_TIMEOUT 8       /* reserved: the kernels have no waits that can give up  */
+#define DSPARK_SEQ_TIMEOUT 8       /* a bounded wait for staged logits gave up (2 s); the
+                                      sequence's result is the error result            */
 
 /* AcceptResult: device buffers, caller-allocated. Required: n_accepted, tokens, next_token.
  * The optional ones (NULL = not written) are diagnostics of the sampling policy. */
@@ -94,11 +95,10 @@ int dspark_version(void);
 
 /* Bytes of device workspace the verify calls need for this shape (valid for both policies).
  * Returns 0 when the shape is invalid or unsupported.
- * Contract: the first dspark_workspace_zero_bytes(B, K) bytes of a workspace (one arrival
- * counter per sequence) must be zero before its first call (e.g. cudaMemsetAsync once after
- * allocating it); every call that returns DSPARK_OK leaves them zero again once it has run,
- * so no per-call clearing is needed. The rest of the workspace needs no initialisation. One
- * workspace serves one call at a time. */
+ * A workspace needs no initialisation: a call writes every word of it that it reads.
+ * dspark_workspace_zero_bytes returns the size of the prefix that must be zero before a call,
+ * which is 0 for this library (kept so that callers can clear generically). One workspace
+ * serves one call at a time. */
 size_t dspark_workspace_bytes(int B, int K, int V, dspark_dtype_t dtype);
 size_t dspark_workspace_zero_bytes(int B, int K);
 
@@ -164,8 +164,7 @@ dspark_status_t dspark_speculative_sample_accept(const void* p1, int64_t ld_p1, 
  *  Set-up: the first call on a device, with that device current, looks up the array's device
  *    address (cudaGetSymbolAddress) and keeps it; make that first call before any stream
  *    capture on that device. A failed look-up returns DSPARK_ERR_CUDA.
- *  Each call clears the array's counter region (dspark_workspace_zero_bytes(B, K) bytes) on
- *    `stream` before its kernels.
+ *  The array needs no clearing: each call writes every word of it that it reads.
  *  All calls on one device share the array: calls that overlap on the GPU race and give
  *    wrong results. Order them (one stream, or events). */
 #define DSPARK_STATIC_SCRATCH_BYTES ((size_t)4 << 20)

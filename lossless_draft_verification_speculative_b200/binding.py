@@ -155,33 +155,24 @@ def _split_block(P) -> Tuple[torch.Tensor, Optional[torch.Tensor], int, int]:
 
 
 class _Workspace:
-    """A per-device byte buffer reused across calls, grown on demand.
-
-    The library needs the workspace's counter region (a prefix whose length depends on B and
-    K) to be zero before a call, and leaves it zero after every call. A fresh buffer is
-    allocated zero-filled; when the (B, K) of consecutive calls differ the prefix moves, so
-    it is cleared again (a memset on the current stream; nothing is allocated).
-    """
+    """A per-device byte buffer reused across calls, grown on demand. The library needs no
+    initialisation of it (a call writes every word it reads)."""
 
     def __init__(self):
         self.bufs = {}
-        self.shape = {}
 
-    def get(self, device: torch.device, nbytes: int, B: int, K: int) -> torch.Tensor:
+    def get(self, device: torch.device, nbytes: int) -> torch.Tensor:
         key = device.index if device.index is not None else torch.cuda.current_device()
         buf = self.bufs.get(key)
         if buf is None or buf.numel() < nbytes:
             buf = new_workspace(max(nbytes, 256), device)
             self.bufs[key] = buf
-        elif self.shape.get(key) != (B, K):
-            buf[: load_library().dspark_workspace_zero_bytes(B, K)].zero_()
-        self.shape[key] = (B, K)
         return buf
 
 
 def new_workspace(nbytes: int, device) -> torch.Tensor:
-    """A workspace buffer in the state the library requires before its first call."""
-    return torch.zeros(nbytes, dtype=torch.uint8, device=device)
+    """A workspace buffer of `nbytes` bytes (256-byte aligned, as every CUDA allocation)."""
+    return torch.empty(max(nbytes, 256), dtype=torch.uint8, device=device)
 
 
 _WS = _Workspace()
@@ -224,9 +215,8 @@ def greedy_accept(P: Union[torch.Tensor, Tuple[torch.Tensor, torch.Tensor]],
                   workspace: Optional[torch.Tensor] = None) -> AcceptResult:
     """Greedy block verify on the GPU: accept drafts while they equal the base argmax.
 
-    ``workspace``, if given, must follow the library's contract: its first
-    ``dspark_workspace_zero_bytes(B, K)`` bytes zero before the first call with this (B, K)
-    (``new_workspace`` returns such a buffer); calls leave them zero.
+    ``workspace``, if given, is a device byte buffer of at least ``workspace_bytes(...)``
+    bytes that no other call uses at the same time.
     """
     lib = load_library()
     p1, pv, ld_p1, ld_pv = _split_block(P)
@@ -237,7 +227,7 @@ def greedy_accept(P: Union[torch.Tensor, Tuple[torch.Tensor, torch.Tensor]],
     drafts = _check_drafts(drafts, B, K, p1.device)
     res = out if out is not None else _alloc_result(B, K, p1.device, diagnostics=False)
     nbytes = lib.dspark_workspace_bytes(B, K, V, DTYPE_CODES[p1.dtype])
-    ws = workspace if workspace is not None else _WS.get(p1.device, nbytes, B, K)
+    ws = workspace if workspace is not None else _WS.get(p1.device, nbytes)
     rc = lib.dspark_greedy_accept(_ptr(p1), ld_p1, _ptr(pv), ld_pv, DTYPE_CODES[p1.dtype],
                                   _ptr(drafts), B, K, V, _out_struct(res), _ptr(ws),
                                   ws.numel() * ws.element_size(), _stream_handle(p1.device))
@@ -267,7 +257,7 @@ def speculative_sample_accept(P: Union[torch.Tensor, Tuple[torch.Tensor, torch.T
         raise ValueError("uniforms must be a contiguous float32 [B, K+1] tensor on P's device")
     res = out if out is not None else _alloc_result(B, K, p1.device, diagnostics=True)
     nbytes = lib.dspark_workspace_bytes(B, K, V, DTYPE_CODES[p1.dtype])
-    ws = workspace if workspace is not None else _WS.get(p1.device, nbytes, B, K)
+    ws = workspace if workspace is not None else _WS.get(p1.device, nbytes)
     rc = lib.dspark_speculative_sample_accept(
         _ptr(p1), ld_p1, _ptr(pv), ld_pv, _ptr(Q), DTYPE_CODES[p1.dtype], _ptr(drafts), B, K,
         V, float(temperature), _ptr(uniforms), _out_struct(res), _ptr(ws),

@@ -67,6 +67,25 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
+// 2^x on the FMA pipe, for loops whose SFU is the bottleneck. x = n + f with n = rint(x)
+// (the 1.5 * 2^23 shift) and |f| <= 1/2; 2^f = p(f), the degree-5 polynomial with p(0) = 1
+// fitted to the relative error on [-1/2, 1/2] by gen_exp2_poly.py (max relative error of the
+// whole float32 evaluation 1.7e-7, as the SFU's); 2^n is added to the exponent bits. Results
+// below 2^-125 (and x = -inf) are 0, as on the flush-to-zero SFU path. Not for NaN or +inf.
+__device__ __forceinline__ float exp2_poly(float x) {
+  const float xc = fmaxf(x, -125.f);
+  const float t = __fadd_rn(xc, 12582912.f);
+  const float f = __fsub_rn(xc, __fsub_rn(t, 12582912.f));
+  float p = __int_as_float(0x3aade4f2);
+  p = __fmaf_rn(p, f, __int_as_float(0x3c1e7545));
+  p = __fmaf_rn(p, f, __int_as_float(0x3d635b93));
+  p = __fmaf_rn(p, f, __int_as_float(0x3e75fcde));
+  p = __fmaf_rn(p, f, __int_as_float(0x3f317215));
+  p = __fmaf_rn(p, f, 1.f);
+  const float r = __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
+  return x < -125.f ? 0.f : r;
+}
+
 __device__ __forceinline__ unsigned long long globaltimer_ns() {
   unsigned long long t;
   asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));

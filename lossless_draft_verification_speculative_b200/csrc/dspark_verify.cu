@@ -2,6 +2,7 @@
 // two kernel launches of a call (pass 1 in stream.cuh, pass 2 in finish.cuh).
 #include <cmath>
 #include <cstdlib>
+#include <cstring>
 #include <mutex>
 
 #include "common.cuh"
@@ -14,12 +15,30 @@ namespace {
 constexpr int kAbiVersion = 3;
 constexpr int kMaxDevices = 64;
 
-// Pass-1 CTAs may be capped for experiments (DSPARK_MAX_CTAS); 0 = one full wave.
+constexpr size_t kRingBudget = 100 * 1024;  // shared memory of one ring CTA's stages
+
+// Tuning switches read once: DSPARK_MAX_CTAS caps the pass-1 CTAs (0 = one full wave);
+// DSPARK_STREAM=ring stages pass 1 through per-warp bulk-copy rings instead of plain loads.
 int max_ctas_override() {
   static const int v = [] {
     const char* s = std::getenv("DSPARK_MAX_CTAS");
     const int n = s ? std::atoi(s) : 0;
     return n > 0 ? n : 0;
+  }();
+  return v;
+}
+// DSPARK_ORDER=run gives each pass-1 warp a contiguous run of units instead of a grid stride.
+bool run_order() {
+  static const bool v = [] {
+    const char* s = std::getenv("DSPARK_ORDER");
+    return s && std::strcmp(s, "run") == 0;
+  }();
+  return v;
+}
+bool ring_stream() {
+  static const bool v = [] {
+    const char* s = std::getenv("DSPARK_STREAM");
+    return s && std::strcmp(s, "ring") == 0;
   }();
   return v;
 }
@@ -39,7 +58,8 @@ bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) %
 struct Plan {
   int vec;  // elements per load: 16-byte vectors (8 bf16 / 4 fp32) or 1
   int nch;  // 2048-token chunks per row
-  int G;    // pass-2 CTAs per sequence, sampling
+  int G;    // pass-2 CTAs per sequence (one cluster), sampling
+  int cpc;  // chunks per pass-2 CTA
 };
 
 bool make_plan(int V, dspark_dtype_t dt, bool aligned16, Plan* pl) {
@@ -48,29 +68,26 @@ bool make_plan(int V, dspark_dtype_t dt, bool aligned16, Plan* pl) {
   if (nch < 1 || nch > kMaxChunkCount) return false;
   pl->vec = aligned16 ? 16 / es : 1;
   pl->nch = static_cast<int>(nch);
-  pl->G = (pl->nch + kWarps - 1) / kWarps;
+  pl->G = pl->nch < kMaxFinishCluster ? pl->nch : kMaxFinishCluster;
+  pl->cpc = (pl->nch + pl->G - 1) / pl->G;
   return true;
 }
 
 size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
-// Workspace regions. The per-sequence arrival counters come first: they must be zero before
-// a call, and every call leaves them zero again. The rest needs no initialisation.
+// Workspace: the pass-1 records, one float2 per (row, chunk) unit, then the draft tokens'
+// logits (sampling). Pass 1 writes every record, and the gather of every draft id in [0, V),
+// before pass 2 reads them, so the workspace needs no initialisation.
 struct WsLayout {
-  size_t arrive, rec, mass, total;
+  size_t rec, gather, total;
 };
 
 WsLayout ws_layout(long long B, long long K, int nch) {
   const long long rows = 2 * K + 1;
   WsLayout w{};
-  size_t off = 0;
-  w.arrive = off;
-  off = align256(off + sizeof(unsigned) * static_cast<size_t>(B));
-  w.rec = off;
-  off = align256(off + sizeof(float2) * static_cast<size_t>(B * rows * nch));
-  w.mass = off;
-  off = align256(off + sizeof(float2) * static_cast<size_t>(B * nch));
-  w.total = off;
+  w.rec = 0;
+  w.gather = align256(sizeof(float2) * static_cast<size_t>(B * rows * nch));
+  w.total = w.gather + align256(sizeof(float2) * static_cast<size_t>(B * K));
   return w;
 }
 
@@ -80,26 +97,48 @@ std::mutex g_mu;
 struct OccEntry {
   const void* fn;
   int dev;
+  size_t smem;
   int ctas;  // co-resident CTAs of the kernel on the device
 };
 OccEntry g_occ[64];
 int g_occ_n = 0;
 
-int resident_ctas(const void* fn, cudaError_t* err) {
+// CTAs of `fn` (kThreads threads, `smem` dynamic shared memory) resident on the current
+// device at once; sets the kernel's dynamic shared-memory limit first when it needs one.
+int resident_ctas(const void* fn, size_t smem, cudaError_t* err) {
   int dev = 0;
   *err = cudaGetDevice(&dev);
   if (*err != cudaSuccess) return 0;
   std::lock_guard<std::mutex> lk(g_mu);
   for (int n = 0; n < g_occ_n; ++n)
-    if (g_occ[n].fn == fn && g_occ[n].dev == dev) return g_occ[n].ctas;
+    if (g_occ[n].fn == fn && g_occ[n].dev == dev && g_occ[n].smem == smem) return g_occ[n].ctas;
+  if (smem > 0) {
+    *err = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                static_cast<int>(smem));
+    if (*err != cudaSuccess) return 0;
+  }
   int per_sm = 0, sms = 0;
-  *err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, kThreads, 0);
+  *err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, kThreads, smem);
   if (*err != cudaSuccess) return 0;
   *err = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   if (*err != cudaSuccess) return 0;
   const int n = per_sm * sms;
-  if (g_occ_n < 64) g_occ[g_occ_n++] = OccEntry{fn, dev, n};
+  if (g_occ_n < 64) g_occ[g_occ_n++] = OccEntry{fn, dev, smem, n};
   return n;
+}
+
+// Shared-memory stages per warp of the ring kernel for this element type.
+template <typename T>
+int ring_stages() {
+  const size_t ub = static_cast<size_t>(kCE) * Elem<T>::kBytes;
+  int st = static_cast<int>(kRingBudget / (static_cast<size_t>(kWarps) * ub));
+  return st < 2 ? 2 : (st > kMaxStages ? kMaxStages : st);
+}
+
+template <typename T>
+size_t ring_smem(int stages) {
+  return static_cast<size_t>(kWarps) * stages * kCE * Elem<T>::kBytes +
+         static_cast<size_t>(kWarps) * kMaxStages * sizeof(uint64_t);
 }
 
 struct Call {
@@ -116,9 +155,13 @@ struct Call {
 // then pass 2 launched as a programmatic dependent of it.
 template <typename T, int VEC, bool kSample>
 dspark_status_t run_call(const Call& c, const Plan& pl, cudaStream_t stream) {
-  const void* k1 = reinterpret_cast<const void*>(&stream_stats_kernel<T, VEC, kSample>);
+  const bool ring = VEC > 1 && ring_stream();
+  const int stages = ring ? ring_stages<T>() : 0;
+  const size_t smem = ring ? ring_smem<T>(stages) : 0;
+  const void* k1 = ring ? reinterpret_cast<const void*>(&stream_stats_ring_kernel<T, kSample>)
+                        : reinterpret_cast<const void*>(&stream_stats_kernel<T, VEC, kSample>);
   cudaError_t e = cudaSuccess;
-  int ctas = resident_ctas(k1, &e);
+  int ctas = resident_ctas(k1, smem, &e);
   if (e != cudaSuccess) return DSPARK_ERR_CUDA;
   if (ctas < 1) return DSPARK_ERR_UNSUPPORTED;
   if (max_ctas_override() && max_ctas_override() < ctas) ctas = max_ctas_override();
@@ -133,10 +176,18 @@ dspark_status_t run_call(const Call& c, const Plan& pl, cudaStream_t stream) {
   sp.rs = c.rs;
   sp.n_units = n_units;
   sp.upw = upw;
+  sp.warps = static_cast<long long>(grid1) * kWarps;
+  sp.strided = ring ? 0 : (run_order() ? 0 : 1);
   sp.nch = pl.nch;
+  sp.stages = stages;
   sp.scale = c.scale;
   sp.rec = reinterpret_cast<float2*>(c.ws + w.rec);
-  stream_stats_kernel<T, VEC, kSample><<<grid1, kThreads, 0, stream>>>(sp);
+  sp.drafts = c.drafts;
+  sp.gather = reinterpret_cast<float*>(c.ws + w.gather);
+  if (ring)
+    stream_stats_ring_kernel<T, kSample><<<grid1, kThreads, smem, stream>>>(sp);
+  else
+    stream_stats_kernel<T, VEC, kSample><<<grid1, kThreads, 0, stream>>>(sp);
   e = cudaGetLastError();
   if (e != cudaSuccess) return DSPARK_ERR_CUDA;
 
@@ -146,22 +197,26 @@ dspark_status_t run_call(const Call& c, const Plan& pl, cudaStream_t stream) {
   fp.uniforms = c.uniforms;
   fp.B = c.B;
   fp.G = pl.G;
+  fp.cpc = pl.cpc;
   fp.nch = pl.nch;
   fp.scale = c.scale;
   fp.rec = sp.rec;
-  fp.mass = reinterpret_cast<float2*>(c.ws + w.mass);
-  fp.arrive = reinterpret_cast<unsigned*>(c.ws + w.arrive);
+  fp.gather = sp.gather;
   fp.out = c.out;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
+  attr[1].id = cudaLaunchAttributeClusterDimension;
+  attr[1].val.clusterDim.x = static_cast<unsigned>(pl.G);
+  attr[1].val.clusterDim.y = 1;
+  attr[1].val.clusterDim.z = 1;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(kSample ? static_cast<long long>(c.B) * pl.G : c.B), 1, 1);
   cfg.blockDim = dim3(kThreads, 1, 1);
-  cfg.dynamicSmemBytes = 0;
+  cfg.dynamicSmemBytes = kSample ? static_cast<size_t>(pl.cpc) * 2 * kGroups * sizeof(float) : 0;
   cfg.stream = stream;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = kSample ? 2 : 1;
   if constexpr (kSample)
     e = cudaLaunchKernelEx(&cfg, finish_sample_kernel<T, VEC>, fp);
   else
@@ -264,8 +319,9 @@ size_t dspark_workspace_bytes(int B, int K, int V, dspark_dtype_t dtype) {
 }
 
 size_t dspark_workspace_zero_bytes(int B, int K) {
-  if (!shape_ok(B, K, 1)) return 0;
-  return ws_layout(B, K, 1).rec;
+  (void)B;
+  (void)K;
+  return 0;  // no part of the workspace needs initialisation
 }
 
 dspark_status_t dspark_plan(int B, int K, int V, dspark_dtype_t dtype, int aligned16,
@@ -359,10 +415,7 @@ dspark_status_t dspark_speculative_sample_accept_static(const void* p1, int64_t 
   void* scratch = nullptr;
   st = static_scratch_address(&scratch);
   if (st != DSPARK_OK) return st;
-  // the counters at the front of the scratch must start at zero
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (cudaMemsetAsync(scratch, 0, dspark_workspace_zero_bytes(B, K), s) != cudaSuccess)
-    return DSPARK_ERR_CUDA;
+  // nothing in the scratch needs clearing: each call writes every word of it that it reads
   return dspark_speculative_sample_accept(p1, ld_p1, pv, ld_pv, q, dtype, drafts, B, K, V,
                                           temperature, uniforms, out, scratch,
                                           DSPARK_STATIC_SCRATCH_BYTES, stream);

@@ -3,13 +3,14 @@
 // Greedy: one CTA per sequence merges the pass-1 argmax records of its K+1 rows (a warp per
 // row), compares the drafts with the row argmaxes and writes the AcceptResult.
 //
-// Sampling: G CTAs per sequence, G = ceil(n_chunks / 8). Every CTA of a sequence merges the
-// 2K+1 rows' softmax records and takes the accept decisions (the same inputs and arithmetic
-// in each, so the same j). It then computes, one 2048-token chunk per warp, the mass of the
-// draw's law: r = max(p_j - q_j, 0) after a rejection (j < K), p_K for the bonus (j = K).
-// The last CTA of the sequence to finish (a counter in the workspace) draws the token by
-// inverse CDF: float64 prefix over the chunk masses, then a re-read and scan of the one
-// chunk that holds the target. No CTA waits for another.
+// Sampling: one thread-block cluster of G = min(8, n_chunks) CTAs per sequence. Every CTA
+// merges the 2K+1 rows' softmax records and takes the accept decisions (the same inputs and
+// arithmetic in each, so the same j). It then computes, one 2048-token chunk per warp, the
+// mass of the draw's law: r = max(p_j - q_j, 0) after a rejection (j < K), p_K for the bonus
+// (j = K), keeping the sums of every 8-token group in shared memory and sending each chunk's
+// mass to every CTA of the cluster (distributed shared memory). After one cluster barrier all
+// CTAs locate the chunk that holds the draw (float64 prefix over the chunk masses); its owner
+// finds the group from its group sums, re-reads that group's 8 tokens and scans them.
 //
 // Both kernels start with the loads that do not depend on pass 1 (drafts, uniforms, the
 // draft-token logits) and then wait for pass 1 to complete (programmatic dependent launch).
@@ -21,18 +22,19 @@ namespace dspark {
 
 constexpr int kErrBits = DSPARK_SEQ_BAD_DRAFT | DSPARK_SEQ_NONFINITE | DSPARK_SEQ_TIMEOUT;
 constexpr int kMaxRows = 2 * kMaxK + 1;
+constexpr int kMaxFinishCluster = 8;  // CTAs per sampling cluster (portable size)
 
 struct FinishParams {
   RowSet rs;
   const int32_t* drafts;    // [B, K]
   const float* uniforms;    // [B, K+1] (sampling)
   int B;
-  int G;                    // CTAs per sequence (sampling)
+  int G;                    // CTAs per sequence = cluster size (sampling)
+  int cpc;                  // chunks per CTA (sampling)
   int nch;                  // chunks per row
   float scale;              // log2(e) / T
   const float2* rec;        // pass-1 records [B * rows, nch]
-  float2* mass;             // [B, nch]: (mass of the draw's law, mass of p_j) per chunk
-  unsigned* arrive;         // [B], zero between calls
+  const float* gather;      // [B, K, 2]: P_i[x_i], Q_i[x_i] written by pass 1 (sampling)
   dspark_accept_out_t out;
 };
 
@@ -80,17 +82,27 @@ __device__ __forceinline__ float2 reduce_row(const RowRecs& rr) {
   }
 }
 
+// Whether any record of the row marks a unit whose data never arrived.
+__device__ __forceinline__ bool row_timed_out(const RowRecs& rr) {
+  bool t = false;
+#pragma unroll
+  for (int k = 0; k < kRecPerLane; ++k) t |= __float_as_uint(rr.v[k].y) == kTimeoutRecBits;
+  return __any_sync(0xffffffffu, t);
+}
+
 // Rows 0..rows-1 of sequence b into s_stat: warp w merges rows w, w + 8, ..., two at a time
-// so that their loads overlap.
+// so that their loads overlap. A timed-out unit sets DSPARK_SEQ_TIMEOUT in *s_flags.
 template <bool kSample>
 __device__ __forceinline__ void merge_rows(const FinishParams& p, int b, int rows, int wi,
-                                           int lane, float2* s_stat) {
+                                           int lane, float2* s_stat, int* s_flags) {
   const long long r0 = static_cast<long long>(b) * rows;
   for (int r = wi; r < rows; r += 2 * kWarps) {
     RowRecs a, c;
     load_row<kSample>(p, r0 + r, lane, a);
     const bool two = r + kWarps < rows;
     if (two) load_row<kSample>(p, r0 + r + kWarps, lane, c);
+    if ((row_timed_out(a) || (two && row_timed_out(c))) && lane == 0)
+      atomicOr(s_flags, DSPARK_SEQ_TIMEOUT);
     const float2 sa = reduce_row<kSample>(a);
     if (lane == 0) s_stat[r] = sa;
     if (two) {
@@ -117,13 +129,12 @@ __device__ __forceinline__ void write_error(const FinishParams& p, int b, int st
   }
 }
 
-// x_0..x_{j-1}, then `token` at j, then -1.
-__device__ __forceinline__ void write_tokens(const FinishParams& p, int b, int j, int token, int t,
-                                             int nt) {
-  const int K = p.rs.K, K1 = K + 1;
+// x_0..x_{j-1} (from the shared-memory copy xs of the drafts), then `token` at j, then -1.
+__device__ __forceinline__ void write_tokens(const FinishParams& p, int b, int j, int token,
+                                             const int* xs, int t, int nt) {
+  const int K1 = p.rs.K + 1;
   for (int k = t; k < K1; k += nt)
-    p.out.tokens[static_cast<size_t>(b) * K1 + k] =
-        k < j ? p.drafts[static_cast<size_t>(b) * K + k] : (k == j ? token : -1);
+    p.out.tokens[static_cast<size_t>(b) * K1 + k] = k < j ? xs[k] : (k == j ? token : -1);
   if (t == 0) {
     p.out.n_accepted[b] = j;
     p.out.next_token[b] = token;
@@ -135,13 +146,20 @@ __device__ __forceinline__ void write_tokens(const FinishParams& p, int b, int j
 template <typename T>
 __global__ void __launch_bounds__(kThreads) finish_greedy_kernel(const FinishParams p) {
   __shared__ float2 s_arg[kMaxK + 1];
+  __shared__ int s_x[kMaxK];
+  __shared__ int s_flags;
   const int lane = threadIdx.x & 31, wi = threadIdx.x >> 5;
   const int b = blockIdx.x;
   const int K = p.rs.K, K1 = K + 1;
   int x = 0;
-  if (wi == 0 && lane < K) x = p.drafts[static_cast<size_t>(b) * K + lane];
+  if (wi == 0 && lane < K) {
+    x = p.drafts[static_cast<size_t>(b) * K + lane];
+    s_x[lane] = x;
+  }
+  if (threadIdx.x == 0) s_flags = 0;
   grid_dependency_wait();
-  merge_rows<false>(p, b, K1, wi, lane, s_arg);
+  __syncthreads();
+  merge_rows<false>(p, b, K1, wi, lane, s_arg, &s_flags);
   __syncthreads();
   if (wi != 0) return;
   const float ninf = -__int_as_float(0x7f800000);
@@ -151,7 +169,8 @@ __global__ void __launch_bounds__(kThreads) finish_greedy_kernel(const FinishPar
     // NaN anywhere, a +inf maximum, or nothing above -inf: not a usable row
     bad |= !(a.x > ninf) || !(a.x < -ninf) || __float_as_int(a.y) == INT_MAX;
   }
-  int status = __any_sync(0xffffffffu, bad) ? DSPARK_SEQ_NONFINITE : 0;
+  int status = s_flags;
+  if (!(status & DSPARK_SEQ_TIMEOUT) && __any_sync(0xffffffffu, bad)) status |= DSPARK_SEQ_NONFINITE;
   if (__any_sync(0xffffffffu, lane < K && (x < 0 || x >= p.rs.V))) status |= DSPARK_SEQ_BAD_DRAFT;
   const int arg = lane < K ? __float_as_int(s_arg[lane].y) : -1;
   const unsigned mis = __ballot_sync(0xffffffffu, lane < K && x != arg);
@@ -160,7 +179,7 @@ __global__ void __launch_bounds__(kThreads) finish_greedy_kernel(const FinishPar
     write_error(p, b, status, lane, 32);
     return;
   }
-  write_tokens(p, b, j, __float_as_int(s_arg[j].y), lane, 32);
+  write_tokens(p, b, j, __float_as_int(s_arg[j].y), s_x, lane, 32);
   if (lane == 0 && p.out.status) p.out.status[b] = 0;
 }
 
@@ -174,139 +193,160 @@ struct Decision {
   float mq, iq;  // q_j: reference and 1 / sum (iq = 0 for the bonus)
 };
 
-// Per-token mass of the draw's law. The chunk masses and the draw's scan use exactly this
-// arithmetic, so the scan reproduces the masses it located.
-__device__ __forceinline__ float p_value(float zp, float s, const Decision& d) {
-  return __fmul_rn(ex2(__fmaf_rn(zp, s, -d.mp)), d.ip);
-}
-__device__ __forceinline__ float resid_value(float zp, float zq, float s, const Decision& d) {
+// Per-token values of the draw's law. The group sums, the chunk masses and the draw's scan all
+// come from exactly this arithmetic, so the scan reproduces the sums it located.
+//   p value:        p_j(v) = 2^(z_p[v]*s - m_p) / S_p
+//   residual value: max(p_j(v) - q_j(v), 0)
+struct TokenVals {
+  float r;  // residual (equals p on the bonus row)
+  float p;
+};
+__device__ __forceinline__ TokenVals token_vals(float zp, float zq, bool has_q, float s,
+                                                const Decision& d) {
   const float ep = ex2(__fmaf_rn(zp, s, -d.mp));
+  const float pv = __fmul_rn(ep, d.ip);
+  if (!has_q) return {pv, pv};
   const float eq = ex2(__fmaf_rn(zq, s, -d.mq));
-  return fmaxf(__fmaf_rn(ep, d.ip, -__fmul_rn(eq, d.iq)), 0.f);
+  return {fmaxf(__fmaf_rn(ep, d.ip, -__fmul_rn(eq, d.iq)), 0.f), pv};
 }
 
-// The 8 consecutive tokens t0 .. t0+7 of a row (t0 a multiple of 8); -inf past V.
+// A group: 8 consecutive tokens 8q .. 8q+7 of a chunk (q = 0..255). Lane l of a warp handles
+// groups q = l + 32k, k = 0..7, so a round of loads is coalesced across the warp.
+constexpr int kGroups = kCE / 8;
+
+// The 8 logits of a group of one row (t0 = first token, a multiple of 8); -inf past V.
 template <typename T, int VEC>
-__device__ __forceinline__ void load8(const T* row, int t0, int V, float* z) {
-  const float ninf = -__int_as_float(0x7f800000);
-  if constexpr (VEC == 1) {
+struct GroupRaw {
+  static constexpr int NW = VEC == 1 ? 1 : 8 / VEC;
+  uint4 w[NW];   // vector path: raw words
+  float z[VEC == 1 ? 8 : 1];  // scalar path: values
+  __device__ __forceinline__ void load(const T* row, int t0, int V) {
+    const float ninf = -__int_as_float(0x7f800000);
+    if constexpr (VEC == 1) {
 #pragma unroll
-    for (int e = 0; e < 8; ++e) z[e] = t0 + e < V ? Elem<T>::load1(row + t0 + e) : ninf;
-  } else {
+      for (int e = 0; e < 8; ++e) z[e] = t0 + e < V ? Elem<T>::load1(row + t0 + e) : ninf;
+    } else {
+      const uint32_t nb = Elem<T>::kBytes == 2 ? 0xff80ff80u : 0xff800000u;
 #pragma unroll
-    for (int h = 0; h < 8; h += VEC) {
-      if (t0 + h < V) {
-        Elem<T>::unpack(ld_stream16(row + t0 + h), z + h);
-      } else {
-#pragma unroll
-        for (int e = 0; e < VEC; ++e) z[h + e] = ninf;
-      }
+      for (int h = 0; h < NW; ++h)
+        w[h] = t0 + h * VEC < V ? ld_stream16(row + t0 + h * VEC) : make_uint4(nb, nb, nb, nb);
     }
   }
-}
-
-// Sum of the draw's law and of p_j over 8 raw tokens groups (accumulated in place).
-template <typename T>
-__device__ __forceinline__ void mass_terms(const uint4& wp, const uint4& wq, bool has_q,
-                                           const FinishParams& p, const Decision& d, float& acc_r,
-                                           float& acc_p) {
-  constexpr int VEC = Elem<T>::kPerVec16;
-  float zp[VEC];
-  Elem<T>::unpack(wp, zp);
-  if (has_q) {
-    float zq[VEC];
-    Elem<T>::unpack(wq, zq);
+  __device__ __forceinline__ void values(float* out) const {
+    if constexpr (VEC == 1) {
 #pragma unroll
-    for (int e = 0; e < VEC; ++e) {
-      acc_r = __fadd_rn(acc_r, resid_value(zp[e], zq[e], p.scale, d));
-      acc_p = __fadd_rn(acc_p, p_value(zp[e], p.scale, d));
+      for (int e = 0; e < 8; ++e) out[e] = z[e];
+    } else {
+#pragma unroll
+      for (int h = 0; h < NW; ++h) Elem<T>::unpack(w[h], out + h * VEC);
     }
-  } else {
-#pragma unroll
-    for (int e = 0; e < VEC; ++e) acc_p = __fadd_rn(acc_p, p_value(zp[e], p.scale, d));
   }
+};
+
+// Sums over a group's 8 tokens in token order.
+template <typename T, int VEC>
+__device__ __forceinline__ TokenVals group_sums(const GroupRaw<T, VEC>& gp,
+                                                const GroupRaw<T, VEC>& gq, bool has_q, float s,
+                                                const Decision& d) {
+  float zp[8], zq[8];
+  gp.values(zp);
+  if (has_q) gq.values(zq);
+  TokenVals acc{0.f, 0.f};
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+    const TokenVals v = token_vals(zp[e], has_q ? zq[e] : 0.f, has_q, s, d);
+    acc.r = __fadd_rn(acc.r, v.r);
+    acc.p = __fadd_rn(acc.p, v.p);
+  }
+  return acc;
 }
 
-// (mass of the draw's law, mass of p_j) over chunk c, one warp. The order of the sum is free:
-// the draw's scan recomputes the per-token values and only locates the chunk with these.
+// Chunk c of the draw's law, one warp: the 256 group sums into part_r / part_p (token order)
+// and the chunk's (residual mass, p mass) on every lane.
 template <typename T, int VEC>
-__device__ __forceinline__ float2 chunk_mass(const FinishParams& p, int b, int c, const Decision& d,
-                                             int lane) {
+__device__ __forceinline__ float2 chunk_work(const FinishParams& p, int b, int c, const Decision& d,
+                                             int lane, float* part_r, float* part_p) {
   const int K = p.rs.K, V = p.rs.V;
-  const T* pr = row_ptr<T>(p.rs, b, d.j) + static_cast<size_t>(c) * kCE;
-  const T* qr = d.j < K ? row_ptr<T>(p.rs, b, K + 1 + d.j) + static_cast<size_t>(c) * kCE : nullptr;
-  const int valid = min(kCE, V - c * kCE);
-  float acc_r = 0.f, acc_p = 0.f;
-  if constexpr (VEC == 1) {
-    for (int t = lane; t < valid; t += 32) {
-      const float zp = Elem<T>::load1(pr + t);
-      if (qr) acc_r = __fadd_rn(acc_r, resid_value(zp, Elem<T>::load1(qr + t), p.scale, d));
-      acc_p = __fadd_rn(acc_p, p_value(zp, p.scale, d));
-    }
-  } else {
-    // 8 vectors of each row in flight per lane (bf16: the whole chunk)
-    constexpr int NV = kCE / VEC / 32;
-    constexpr int NB = NV < 8 ? NV : 8;
-    const int nvv = valid / VEC;
+  const bool has_q = d.j < K;
+  const T* pr = row_ptr<T>(p.rs, b, d.j);
+  const T* qr = has_q ? row_ptr<T>(p.rs, b, K + 1 + d.j) : pr;
+  constexpr int kPerLane = kGroups / 32;                      // groups per lane
+  constexpr int kRound = VEC == 8 ? 4 : (VEC == 4 ? 2 : 1);  // groups in flight per row
+  float lr = 0.f, lp = 0.f;
+  GroupRaw<T, VEC> gp[kRound], gq[kRound];
+  auto load = [&](int k, int slot) {
+    const int t0 = c * kCE + (k * 32 + lane) * 8;
+    gp[slot].load(pr, t0, V);
+    if (has_q) gq[slot].load(qr, t0, V);
+  };
 #pragma unroll
-    for (int k0 = 0; k0 < NV; k0 += NB) {
-      uint4 wp[NB], wq[NB] = {};
+  for (int k = 0; k < kRound; ++k) load(k, k);
+  // group k is summed from slot k % kRound, whose registers then take group k + kRound, so
+  // the next loads are in flight while this round's groups are computed
 #pragma unroll
-      for (int k = 0; k < NB; ++k) {
-        const int vi = (k0 + k) * 32 + lane;
-        const bool ok = vi < nvv;
-        const uint32_t ninf = Elem<T>::kBytes == 2 ? 0xff80ff80u : 0xff800000u;
-        wp[k] = ok ? ld_stream16(pr + vi * VEC) : make_uint4(ninf, ninf, ninf, ninf);
-        if (qr) wq[k] = ok ? ld_stream16(qr + vi * VEC) : make_uint4(ninf, ninf, ninf, ninf);
-      }
-#pragma unroll
-      for (int k = 0; k < NB; ++k) mass_terms<T>(wp[k], wq[k], qr != nullptr, p, d, acc_r, acc_p);
-    }
+  for (int k = 0; k < kPerLane; ++k) {
+    const int slot = k % kRound;
+    const TokenVals gsum = group_sums<T, VEC>(gp[slot], gq[slot], has_q, p.scale, d);
+    if (k + kRound < kPerLane) load(k + kRound, slot);
+    const int q = k * 32 + lane;
+    part_r[q] = gsum.r;
+    part_p[q] = gsum.p;
+    lr = __fadd_rn(lr, gsum.r);
+    lp = __fadd_rn(lp, gsum.p);
   }
-  acc_p = warp_sum(acc_p);
-  acc_r = qr ? warp_sum(acc_r) : acc_p;
-  return make_float2(acc_r, acc_p);
+  return make_float2(warp_sum(lr), warp_sum(lp));
 }
 
+// L2 prefetch of `bytes` bytes (a multiple of 16, 16-byte aligned) from global memory.
+__device__ __forceinline__ void prefetch_l2(const void* src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
+
+// Sampling finish. Launched as clusters of G CTAs, one cluster per sequence; CTA g of the
+// cluster owns chunks g*cpc .. g*cpc + cpc - 1 of the draw's law (warp w: local chunks w, w+8).
 template <typename T, int VEC>
-__global__ void __launch_bounds__(kThreads) finish_sample_kernel(const FinishParams p) {
+__global__ void __launch_bounds__(kThreads, 4) finish_sample_kernel(const FinishParams p) {
+  extern __shared__ float s_part[];  // [cpc][2][kGroups]: group sums (residual, p)
   __shared__ float2 s_stat[kMaxRows];
+  __shared__ float2 s_mass[kMaxChunkCount];  // every chunk's (residual, p) mass
   __shared__ float s_zp[kMaxK], s_zq[kMaxK], s_u[kMaxK + 1];
   __shared__ int s_x[kMaxK];
   __shared__ Decision s_dec;
-  __shared__ int s_last;
-  __shared__ float s_wtot[kWarps];
   __shared__ double s_tin;
-  __shared__ int s_chunk, s_use_p, s_token, s_lastpos;
+  __shared__ int s_chunk, s_use_p, s_flags;
+  cg::cluster_group cluster = cg::this_cluster();
   const int tid = threadIdx.x, lane = tid & 31, wi = tid >> 5;
-  const int b = blockIdx.x / p.G, g = blockIdx.x - b * p.G;
+  const int G = p.G;
+  const int b = blockIdx.x / G;
+  const int g = static_cast<int>(cluster.block_rank());
   const int K = p.rs.K, K1 = K + 1, V = p.rs.V, rows = p.rs.rows;
 
-  // inputs that pass 1 does not write: drafts, uniforms, the draft tokens' logits
-  if (tid < K) {
-    const int x = p.drafts[static_cast<size_t>(b) * K + tid];
-    s_x[tid] = x;
-    float zp = 0.f, zq = 0.f;
-    if (x >= 0 && x < V) {
-      zp = Elem<T>::load1(row_ptr<T>(p.rs, b, tid) + x);
-      zq = Elem<T>::load1(row_ptr<T>(p.rs, b, K1 + tid) + x);
-    }
-    s_zp[tid] = zp;
-    s_zq[tid] = zq;
-  }
+  // inputs that pass 1 does not write: drafts, uniforms
+  int x = -1;
+  if (tid < K) x = p.drafts[static_cast<size_t>(b) * K + tid];
   if (tid <= K) s_u[tid] = p.uniforms[static_cast<size_t>(b) * K1 + tid];
+  if (tid == 0) s_flags = 0;
   grid_dependency_wait();
+  // the draft tokens' logits, gathered by pass 1
+  if (tid < K) {
+    s_x[tid] = x;
+    float2 zg = make_float2(0.f, 0.f);
+    if (x >= 0 && x < V) zg = __ldcg(reinterpret_cast<const float2*>(p.gather) + static_cast<size_t>(b) * K + tid);
+    s_zp[tid] = zg.x;
+    s_zq[tid] = zg.y;
+  }
+  __syncthreads();
 
   // every row's (reference, sum)
-  merge_rows<true>(p, b, rows, wi, lane, s_stat);
+  merge_rows<true>(p, b, rows, wi, lane, s_stat, &s_flags);
   __syncthreads();
 
   // decisions (warp 0; draft i on lane i)
   if (wi == 0) {
-    int status = 0;
+    int status = s_flags;
     bool bad = false;
     for (int r = lane; r < rows; r += 32) bad |= !stat_ok(s_stat[r]);
-    if (__any_sync(0xffffffffu, bad)) status |= DSPARK_SEQ_NONFINITE;
+    if (!(status & DSPARK_SEQ_TIMEOUT) && __any_sync(0xffffffffu, bad)) status |= DSPARK_SEQ_NONFINITE;
     const int x = lane < K ? s_x[lane] : 0;
     const bool bad_draft = lane < K && (x < 0 || x >= V);
     if (__any_sync(0xffffffffu, bad_draft)) status |= DSPARK_SEQ_BAD_DRAFT;
@@ -315,8 +355,9 @@ __global__ void __launch_bounds__(kThreads) finish_sample_kernel(const FinishPar
     bool accept = false;
     if (lane < K && !bad_draft) {
       const float2 sp = s_stat[lane], sq = s_stat[K1 + lane];
-      px = __fdiv_rn(ex2(__fmaf_rn(s_zp[lane], p.scale, -sp.x)), sp.y);
-      qx = __fdiv_rn(ex2(__fmaf_rn(s_zq[lane], p.scale, -sq.x)), sq.y);
+      // p_i(x_i) = 2^(z*s - M) / S (division within 2 ulp: no IEEE slow path)
+      px = __fdividef(ex2(__fmaf_rn(s_zp[lane], p.scale, -sp.x)), sp.y);
+      qx = __fdividef(ex2(__fmaf_rn(s_zq[lane], p.scale, -sq.x)), sq.y);
       accept = __fmul_rn(s_u[lane], qx) < px;
     }
     const unsigned rej = __ballot_sync(0xffffffffu, lane < K && !accept);
@@ -331,11 +372,11 @@ __global__ void __launch_bounds__(kThreads) finish_sample_kernel(const FinishPar
       d.j = j;
       d.status = status;
       d.mp = sp.x;
-      d.ip = __fdiv_rn(1.f, sp.y);
+      d.ip = __fdividef(1.f, sp.y);
       if (j < K) {
         const float2 sq = s_stat[K1 + j];
         d.mq = sq.x;
-        d.iq = __fdiv_rn(1.f, sq.y);
+        d.iq = __fdividef(1.f, sq.y);
       } else {
         d.mq = 0.f;
         d.iq = 0.f;
@@ -345,56 +386,52 @@ __global__ void __launch_bounds__(kThreads) finish_sample_kernel(const FinishPar
   }
   __syncthreads();
   const Decision d = s_dec;
-
-  // this CTA's chunks of the draw's law
-  if (!(d.status & kErrBits)) {
-    const int c = g * kWarps + wi;
-    if (c < p.nch) {
-      const float2 m = chunk_mass<T, VEC>(p, b, c, d, lane);
-      if (lane == 0) {
-        p.mass[static_cast<size_t>(b) * p.nch + c] = m;
-        __threadfence();  // the mass is visible before this CTA's arrival is counted
-      }
+  // this CTA's chunk range of the draw's rows into L2, ahead of the warps' second loads
+  if (VEC > 1 && lane == 0 && wi >= kWarps - 2 && !(d.status & kErrBits)) {
+    const int t0 = g * p.cpc * kCE;
+    const int t1 = min(V, t0 + p.cpc * kCE);
+    const bool q_row = wi == kWarps - 1;
+    if (t0 < t1 && (!q_row || d.j < K)) {
+      const uint32_t bytes = static_cast<uint32_t>(t1 - t0) * Elem<T>::kBytes;
+      prefetch_l2(row_ptr<T>(p.rs, b, q_row ? K1 + d.j : d.j) + t0, bytes);
     }
   }
-  __syncthreads();
-  if (tid == 0) {
-    __threadfence();
-    const unsigned old = atomicAdd(p.arrive + b, 1u);
-    s_last = old == static_cast<unsigned>(p.G - 1);
-    if (s_last) p.arrive[b] = 0;  // every CTA of b has arrived: reset for the next call
+
+  // this CTA's chunks: group sums into shared memory, chunk masses to every CTA of the cluster
+  if (!(d.status & kErrBits)) {
+    for (int lc = wi; lc < p.cpc; lc += kWarps) {
+      const int c = g * p.cpc + lc;
+      if (c >= p.nch) break;
+      float* pr = s_part + static_cast<size_t>(lc) * 2 * kGroups;
+      const float2 m = chunk_work<T, VEC>(p, b, c, d, lane, pr, pr + kGroups);
+      if (lane < G) cluster.map_shared_rank(s_mass, lane)[c] = m;
+    }
   }
-  __syncthreads();
-  if (!s_last) return;
-  __threadfence();
+  cluster.sync();  // every chunk mass has landed in every CTA; group sums are visible CTA-wide
 
   if (d.status & kErrBits) {
-    write_error(p, b, d.status, tid, kThreads);
+    if (g == 0) write_error(p, b, d.status, tid, kThreads);
     return;
   }
 
-  // ---- the draw (the last CTA of the sequence)
+  // ---- which chunk holds the draw (every CTA, the same float64 arithmetic on the same masses)
   const int j = d.j;
-  int status = d.status;
-  const float uK = s_u[K];
-  // chunk masses in float64: warp 0, lane l holds chunks 4l .. 4l+3 (token order)
   constexpr int NPL = kMaxChunkCount / 32;
-  bool use_p = j == K;
   if (wi == 0) {
+    int status = d.status;
+    bool use_p = j == K;
     double mr[NPL], mp[NPL];
     double zr = 0.0, zpm = 0.0;
 #pragma unroll
     for (int k = 0; k < NPL; ++k) {
       const int c = lane * NPL + k;
-      float2 m = make_float2(0.f, 0.f);
-      if (c < p.nch) m = __ldcg(p.mass + static_cast<size_t>(b) * p.nch + c);
+      const float2 m = c < p.nch ? s_mass[c] : make_float2(0.f, 0.f);
       mr[k] = m.x;
       mp[k] = m.y;
       zr += mr[k];
       zpm += mp[k];
     }
-    // totals over lanes (every lane the same sums in the same order)
-    double Zr = zr, Zp = zpm;
+    double Zr = zr, Zp = zpm;  // inclusive prefixes over lanes
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
       const double a = __shfl_up_sync(0xffffffffu, Zr, o), c2 = __shfl_up_sync(0xffffffffu, Zp, o);
@@ -403,7 +440,6 @@ __global__ void __launch_bounds__(kThreads) finish_sample_kernel(const FinishPar
         Zp += c2;
       }
     }
-    // Zr / Zp now hold inclusive prefixes over lanes; the totals sit on lane 31
     const double Zres = __shfl_sync(0xffffffffu, Zr, 31);
     if (!use_p && !(Zres > 0.0)) {  // residual mass rounded to zero: draw from p_j instead
       use_p = true;
@@ -415,7 +451,7 @@ __global__ void __launch_bounds__(kThreads) finish_sample_kernel(const FinishPar
     const double incl = use_p ? Zp : Zr;
     const double ls = use_p ? zpm : zr;
     const double Z = __shfl_sync(0xffffffffu, incl, 31);
-    const double target = static_cast<double>(uK) * Z;
+    const double target = static_cast<double>(s_u[K]) * Z;
     double run = incl - ls;
     int cfound = -1, clast = -1;
     double before = 0.0;
@@ -438,50 +474,44 @@ __global__ void __launch_bounds__(kThreads) finish_sample_kernel(const FinishPar
       const int hl = __ffs(hit) - 1;
       c = __shfl_sync(0xffffffffu, cfound, hl);
       tin = target - __shfl_sync(0xffffffffu, before, hl);
-    } else {  // rounding left the target past the last mass: the chunk's last token
+    } else {  // rounding left the target past the last mass: the last token with mass
       int cl = clast;
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) cl = max(cl, __shfl_xor_sync(0xffffffffu, cl, o));
       c = cl;
       tin = __int_as_float(0x7f800000);
     }
+    const int owner = c >= 0 ? c / p.cpc : 0;
     if (lane == 0) {
-      s_tin = tin;
-      s_chunk = c;
+      s_chunk = owner == g ? c : -2;  // -2: another CTA draws
       s_use_p = use_p;
-      s_token = INT_MAX;
-      s_lastpos = -1;
-      if (p.out.resid_mass) p.out.resid_mass[b] = j < K ? (use_p ? 0.f : static_cast<float>(Zres)) : 1.f;
-      if (p.out.status) p.out.status[b] = status;
+      s_tin = tin;
+      if (owner == g) {
+        if (p.out.resid_mass)
+          p.out.resid_mass[b] = j < K ? (use_p ? 0.f : static_cast<float>(Zres)) : 1.f;
+        if (p.out.status) p.out.status[b] = status;
+      }
     }
   }
   __syncthreads();
   const int c = s_chunk;
-  const float tin = static_cast<float>(s_tin);
-  use_p = s_use_p != 0;
+  if (c == -2) return;
+  if (wi != 0) return;
+  int token = -1;
   if (c >= 0) {
-    // per-token masses of chunk c exactly as chunk_mass computed them; warp w scans tokens
-    // c*2048 + 256w .. +255, lane l holds 8 consecutive ones
-    const T* pr = row_ptr<T>(p.rs, b, j);
-    const T* qr = !use_p ? row_ptr<T>(p.rs, b, K1 + j) : nullptr;
-    const int t0 = c * kCE + wi * 256 + lane * 8;
-    float zp[8], val[8];
-    load8<T, VEC>(pr, t0, V, zp);
-    if (qr) {
-      float zq[8];
-      load8<T, VEC>(qr, t0, V, zq);
-#pragma unroll
-      for (int e = 0; e < 8; ++e) val[e] = resid_value(zp[e], zq[e], p.scale, d);
-    } else {
-#pragma unroll
-      for (int e = 0; e < 8; ++e) val[e] = p_value(zp[e], p.scale, d);
-    }
+    // the group holding the target: lane l scans the chunk's groups 8l .. 8l+7 (token order)
+    const bool use_p = s_use_p != 0;
+    const float tin = static_cast<float>(s_tin);
+    const float* part = s_part + static_cast<size_t>(c - g * p.cpc) * 2 * kGroups +
+                        (use_p ? kGroups : 0);
+    float gv[8];
     float lsum = 0.f;
-    int lastv = -1;
+    int lastg = -1;
 #pragma unroll
     for (int e = 0; e < 8; ++e) {
-      lsum = __fadd_rn(lsum, val[e]);
-      if (val[e] > 0.f) lastv = t0 + e;
+      gv[e] = part[lane * 8 + e];
+      lsum = __fadd_rn(lsum, gv[e]);
+      if (gv[e] > 0.f) lastg = lane * 8 + e;
     }
     float inc = lsum;
 #pragma unroll
@@ -489,34 +519,65 @@ __global__ void __launch_bounds__(kThreads) finish_sample_kernel(const FinishPar
       const float y = __shfl_up_sync(0xffffffffu, inc, o);
       if (lane >= o) inc = __fadd_rn(inc, y);
     }
-    if (lane == 31) s_wtot[wi] = inc;
-    if (lastv >= 0) atomicMax(&s_lastpos, lastv);
-    __syncthreads();
-    float wbase = 0.f;
-    for (int w = 0; w < wi; ++w) wbase = __fadd_rn(wbase, s_wtot[w]);
     float ex = __shfl_up_sync(0xffffffffu, inc, 1);
     if (lane == 0) ex = 0.f;
-    float r = __fadd_rn(wbase, ex);
-    if (r <= tin && tin < __fadd_rn(wbase, inc)) {
-      int cand = -1;
+    int qsel = -1;
+    float gin = 0.f;
+    if (ex <= tin && tin < inc) {
+      float r = ex;
 #pragma unroll
       for (int e = 0; e < 8; ++e) {
-        const float nx = __fadd_rn(r, val[e]);
-        if (cand < 0 && val[e] > 0.f && r <= tin && tin < nx) cand = t0 + e;
+        const float nx = __fadd_rn(r, gv[e]);
+        if (qsel < 0 && gv[e] > 0.f && r <= tin && tin < nx) {
+          qsel = lane * 8 + e;
+          gin = __fsub_rn(tin, r);
+        }
         r = nx;
       }
-      if (cand < 0) cand = lastv;
-      if (cand >= 0) atomicMin(&s_token, cand);
     }
-    __syncthreads();
+    const unsigned h = __ballot_sync(0xffffffffu, qsel >= 0);
+    bool last_mode = false;
+    if (h) {
+      const int hl = __ffs(h) - 1;
+      qsel = __shfl_sync(0xffffffffu, qsel, hl);
+      gin = __shfl_sync(0xffffffffu, gin, hl);
+    } else {  // rounding: the chunk's last group with mass, its last token with mass
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) lastg = max(lastg, __shfl_xor_sync(0xffffffffu, lastg, o));
+      qsel = lastg;
+      last_mode = true;
+    }
+    if (qsel >= 0) {
+      // the group's 8 tokens, recomputed exactly as their sum was; lane 0 scans them
+      if (lane == 0) {
+        const int K_ = p.rs.K;
+        const bool has_q = j < K_;
+        const T* pr = row_ptr<T>(p.rs, b, j);
+        const T* qr = has_q ? row_ptr<T>(p.rs, b, K_ + 1 + j) : pr;
+        const int t0 = c * kCE + qsel * 8;
+        GroupRaw<T, VEC> gp, gq;
+        gp.load(pr, t0, V);
+        if (has_q) gq.load(qr, t0, V);
+        float zp[8], zq[8];
+        gp.values(zp);
+        if (has_q) gq.values(zq);
+        float r = 0.f;
+        int cand = -1, lastv = -1;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const TokenVals v = token_vals(zp[e], has_q ? zq[e] : 0.f, has_q, p.scale, d);
+          const float val = use_p ? v.p : v.r;
+          const float nx = __fadd_rn(r, val);
+          if (val > 0.f) lastv = t0 + e;
+          if (!last_mode && cand < 0 && val > 0.f && r <= gin && gin < nx) cand = t0 + e;
+          r = nx;
+        }
+        token = cand >= 0 ? cand : lastv;
+      }
+    }
   }
-  if (tid == 0) {
-    int token = s_token;
-    if (token == INT_MAX) token = s_lastpos;  // rounding: the last token with mass
-    s_token = token;
-  }
-  __syncthreads();
-  write_tokens(p, b, j, s_token, tid, kThreads);
+  token = __shfl_sync(0xffffffffu, token, 0);
+  write_tokens(p, b, j, token, s_x, lane, 32);
 }
 
 }  // namespace dspark
