@@ -32,7 +32,7 @@ if ROOT not in sys.path:
 METRIC = "verified blocks/s and HBM GB/s vs B200 peak at B=64,K=7,V=129280 bf16"
 FALLBACK_HBM_GBS = 6650.0
 N_SETS = 4
-PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "sample_rowstats_dsv4_flash_serving.md")
+PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "stream_stats_kernel_dsv4_flash_serving.md")
 
 
 def parse_args():
@@ -54,14 +54,15 @@ def source_hash():
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "lossless_draft_verification_speculative_b200", "csrc")
     for f in sorted(os.listdir(csrc)):
-        with open(os.path.join(csrc, f), "rb") as fh:
-            h.update(fh.read())
+        if f.endswith((".cu", ".cuh")):
+            with open(os.path.join(csrc, f), "rb") as fh:
+                h.update(fh.read())
     return h.hexdigest()[:16]
 
 
 def recorded_traffic():
-    """Per-launch DRAM bytes of the sampling pass from the committed ncu summary, if the
-    kernel sources are unchanged since it was taken; else None."""
+    """Per-launch DRAM bytes (read + write) of the sampling call's stream kernel from the
+    committed ncu summary, if the kernel sources are unchanged since it was taken; else None."""
     try:
         kv = {}
         for line in open(PROFILE_SUMMARY):
@@ -366,8 +367,9 @@ def run_ours(args, w):
         "gpu_launches": 2 * ncalls * args.steps,
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "traffic": traffic,
-                     "kernel": "speculative_sample_accept (pass-1 row stream + finish), "
-                               "mean over the timed T>0 calls",
+                     "kernel": "stream_stats_kernel + finish_sample_kernel: the whole "
+                               "speculative_sample_accept call (both launches), mean over the "
+                               "timed T>0 calls",
                      "peak_source": "MEASURED_PEAKS.json hbm_gbs (measured)" if peaks
                      else "fallback 6.65 TB/s"},
         "committed_token_equivalents_per_s": value * statistics.mean(committed),

@@ -72,8 +72,7 @@ typedef enum { DSPARK_BF16 = 0, DSPARK_F32 = 1 } dspark_dtype_t;
 #define DSPARK_SEQ_NONFINITE 2     /* a row with NaN / +inf, or with no finite value       */
 #define DSPARK_SEQ_ZERO_RESIDUAL 4 /* not an error: residual mass rounded to 0 after a
                                       rejection; the correction was drawn from p_j          */
-#define DSPARK_SEQ_TIMEOUT 8       /* a bounded wait for staged logits gave up (2 s); the
-                                      sequence's result is the error result            */
+#define DSPARK_SEQ_TIMEOUT 8       /* reserved: the kernels have no waits that can give up  */
 
 /* AcceptResult: device buffers, caller-allocated. Required: n_accepted, tokens, next_token.
  * The optional ones (NULL = not written) are diagnostics of the sampling policy. */
@@ -106,14 +105,15 @@ size_t dspark_workspace_zero_bytes(int B, int K);
  * Returns DSPARK_OK and fills the fields, or an error for an invalid / unsupported shape.
  * `aligned16` says whether every row start will be 16-byte aligned (vector path).
  * A call runs two kernels on `stream`. Pass 1 reads every logit row once: its units are the
- * (row, chunk) pairs, and each warp of one full wave streams an equal contiguous run of them
- * and writes one statistics record per unit. Pass 2, a programmatic dependent launch, takes
+ * (row, chunk) pairs; each SM's CTA owns an equal contiguous range of them, hands them to its
+ * warps in order, and each unit gets one statistics record. Pass 2, a programmatic dependent launch, takes
  * the per-sequence decisions and, when sampling, computes the draw's law chunk by chunk and
  * draws the token. */
 typedef struct {
   int elems_per_load;              /* 8 (bf16) / 4 (fp32) on the 16-byte path, 1 on the scalar path */
   int loads_in_flight;             /* loads each lane of pass 1 keeps in flight                    */
-  int threads_per_cta;             /* both passes                                                 */
+  int stream_threads_per_cta;      /* pass 1: one CTA of this many threads per SM                  */
+  int threads_per_cta;             /* pass 2                                                      */
   int chunk_elems;                 /* tokens per chunk (pass-1 unit, pass-2 chunk)                */
   int n_chunks;                    /* chunks per row                                              */
   int greedy_units_per_sequence;   /* pass-1 units of one sequence, greedy: (K+1) * n_chunks      */

@@ -56,7 +56,8 @@ class AcceptOut(ctypes.Structure):
 
 class Plan(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int) for n in (
-        "elems_per_load", "loads_in_flight", "threads_per_cta", "chunk_elems", "n_chunks",
+        "elems_per_load", "loads_in_flight", "stream_threads_per_cta", "threads_per_cta",
+        "chunk_elems", "n_chunks",
         "greedy_units_per_sequence", "sampling_units_per_sequence", "finish_ctas_per_sequence")]
 
 

@@ -15,30 +15,12 @@ namespace {
 constexpr int kAbiVersion = 3;
 constexpr int kMaxDevices = 64;
 
-constexpr size_t kRingBudget = 100 * 1024;  // shared memory of one ring CTA's stages
-
-// Tuning switches read once: DSPARK_MAX_CTAS caps the pass-1 CTAs (0 = one full wave);
-// DSPARK_STREAM=ring stages pass 1 through per-warp bulk-copy rings instead of plain loads.
+// Tuning switch read once: DSPARK_MAX_CTAS caps the pass-1 CTAs (0 = one full wave).
 int max_ctas_override() {
   static const int v = [] {
     const char* s = std::getenv("DSPARK_MAX_CTAS");
     const int n = s ? std::atoi(s) : 0;
     return n > 0 ? n : 0;
-  }();
-  return v;
-}
-// DSPARK_ORDER=run gives each pass-1 warp a contiguous run of units instead of a grid stride.
-bool run_order() {
-  static const bool v = [] {
-    const char* s = std::getenv("DSPARK_ORDER");
-    return s && std::strcmp(s, "run") == 0;
-  }();
-  return v;
-}
-bool ring_stream() {
-  static const bool v = [] {
-    const char* s = std::getenv("DSPARK_STREAM");
-    return s && std::strcmp(s, "ring") == 0;
   }();
   return v;
 }
@@ -91,6 +73,19 @@ WsLayout ws_layout(long long B, long long K, int nch) {
   return w;
 }
 
+// Constants of FastDiv for divisor d >= 1 (see stream.cuh).
+FastDiv fast_div(uint32_t d) {
+  FastDiv f{};
+  uint32_t s = 0;
+  while ((1ull << s) < d) ++s;
+  const unsigned __int128 num = static_cast<unsigned __int128>(1) << (32 + s);
+  const unsigned __int128 m = (num + d - 1) / d;
+  f.m_lo = static_cast<uint32_t>(m & 0xffffffffu);
+  f.m_hi = static_cast<uint32_t>(m >> 32);
+  f.s = s;
+  return f;
+}
+
 // --------------------------------------------------------------- per-device launch state
 
 std::mutex g_mu;
@@ -105,7 +100,7 @@ int g_occ_n = 0;
 
 // CTAs of `fn` (kThreads threads, `smem` dynamic shared memory) resident on the current
 // device at once; sets the kernel's dynamic shared-memory limit first when it needs one.
-int resident_ctas(const void* fn, size_t smem, cudaError_t* err) {
+int resident_ctas(const void* fn, int threads, size_t smem, cudaError_t* err) {
   int dev = 0;
   *err = cudaGetDevice(&dev);
   if (*err != cudaSuccess) return 0;
@@ -118,27 +113,13 @@ int resident_ctas(const void* fn, size_t smem, cudaError_t* err) {
     if (*err != cudaSuccess) return 0;
   }
   int per_sm = 0, sms = 0;
-  *err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, kThreads, smem);
+  *err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, threads, smem);
   if (*err != cudaSuccess) return 0;
   *err = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   if (*err != cudaSuccess) return 0;
   const int n = per_sm * sms;
   if (g_occ_n < 64) g_occ[g_occ_n++] = OccEntry{fn, dev, smem, n};
   return n;
-}
-
-// Shared-memory stages per warp of the ring kernel for this element type.
-template <typename T>
-int ring_stages() {
-  const size_t ub = static_cast<size_t>(kCE) * Elem<T>::kBytes;
-  int st = static_cast<int>(kRingBudget / (static_cast<size_t>(kWarps) * ub));
-  return st < 2 ? 2 : (st > kMaxStages ? kMaxStages : st);
-}
-
-template <typename T>
-size_t ring_smem(int stages) {
-  return static_cast<size_t>(kWarps) * stages * kCE * Elem<T>::kBytes +
-         static_cast<size_t>(kWarps) * kMaxStages * sizeof(uint64_t);
 }
 
 struct Call {
@@ -155,39 +136,29 @@ struct Call {
 // then pass 2 launched as a programmatic dependent of it.
 template <typename T, int VEC, bool kSample>
 dspark_status_t run_call(const Call& c, const Plan& pl, cudaStream_t stream) {
-  const bool ring = VEC > 1 && ring_stream();
-  const int stages = ring ? ring_stages<T>() : 0;
-  const size_t smem = ring ? ring_smem<T>(stages) : 0;
-  const void* k1 = ring ? reinterpret_cast<const void*>(&stream_stats_ring_kernel<T, kSample>)
-                        : reinterpret_cast<const void*>(&stream_stats_kernel<T, VEC, kSample>);
+  const void* k1 = reinterpret_cast<const void*>(&stream_stats_kernel<T, VEC, kSample>);
   cudaError_t e = cudaSuccess;
-  int ctas = resident_ctas(k1, smem, &e);
+  int ctas = resident_ctas(k1, kStreamThreads, 0, &e);
   if (e != cudaSuccess) return DSPARK_ERR_CUDA;
   if (ctas < 1) return DSPARK_ERR_UNSUPPORTED;
   if (max_ctas_override() && max_ctas_override() < ctas) ctas = max_ctas_override();
   const WsLayout w = ws_layout(c.B, c.rs.K, pl.nch);
   const long long n_units = static_cast<long long>(c.B) * c.rs.rows * pl.nch;
-  const long long warps = static_cast<long long>(ctas) * kWarps;
-  const long long upw = (n_units + warps - 1) / warps;
-  const long long need = (n_units + upw - 1) / upw;
-  const int grid1 = static_cast<int>((need + kWarps - 1) / kWarps);
+  if (n_units >= (1LL << 31)) return DSPARK_ERR_UNSUPPORTED;  // unit indices stay in 32 bits
+  const long long want = (n_units + kStreamWarps - 1) / kStreamWarps;
+  const int grid1 = static_cast<int>(want < ctas ? want : ctas);
 
   StreamParams sp{};
   sp.rs = c.rs;
-  sp.n_units = n_units;
-  sp.upw = upw;
-  sp.warps = static_cast<long long>(grid1) * kWarps;
-  sp.strided = ring ? 0 : (run_order() ? 0 : 1);
+  sp.n_units = static_cast<uint32_t>(n_units);
   sp.nch = pl.nch;
-  sp.stages = stages;
+  sp.by_nch = fast_div(static_cast<uint32_t>(pl.nch));
+  sp.by_rows = fast_div(static_cast<uint32_t>(c.rs.rows));
   sp.scale = c.scale;
   sp.rec = reinterpret_cast<float2*>(c.ws + w.rec);
   sp.drafts = c.drafts;
   sp.gather = reinterpret_cast<float*>(c.ws + w.gather);
-  if (ring)
-    stream_stats_ring_kernel<T, kSample><<<grid1, kThreads, smem, stream>>>(sp);
-  else
-    stream_stats_kernel<T, VEC, kSample><<<grid1, kThreads, 0, stream>>>(sp);
+  stream_stats_kernel<T, VEC, kSample><<<grid1, kStreamThreads, 0, stream>>>(sp);
   e = cudaGetLastError();
   if (e != cudaSuccess) return DSPARK_ERR_CUDA;
 
@@ -332,6 +303,7 @@ dspark_status_t dspark_plan(int B, int K, int V, dspark_dtype_t dtype, int align
   if (!make_plan(V, dtype, aligned16 != 0, &pl)) return DSPARK_ERR_UNSUPPORTED;
   plan->elems_per_load = pl.vec;
   plan->loads_in_flight = kBatchVecs;
+  plan->stream_threads_per_cta = kStreamThreads;
   plan->threads_per_cta = kThreads;
   plan->chunk_elems = kCE;
   plan->n_chunks = pl.nch;

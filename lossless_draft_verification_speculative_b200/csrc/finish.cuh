@@ -82,27 +82,17 @@ __device__ __forceinline__ float2 reduce_row(const RowRecs& rr) {
   }
 }
 
-// Whether any record of the row marks a unit whose data never arrived.
-__device__ __forceinline__ bool row_timed_out(const RowRecs& rr) {
-  bool t = false;
-#pragma unroll
-  for (int k = 0; k < kRecPerLane; ++k) t |= __float_as_uint(rr.v[k].y) == kTimeoutRecBits;
-  return __any_sync(0xffffffffu, t);
-}
-
 // Rows 0..rows-1 of sequence b into s_stat: warp w merges rows w, w + 8, ..., two at a time
-// so that their loads overlap. A timed-out unit sets DSPARK_SEQ_TIMEOUT in *s_flags.
+// so that their loads overlap.
 template <bool kSample>
 __device__ __forceinline__ void merge_rows(const FinishParams& p, int b, int rows, int wi,
-                                           int lane, float2* s_stat, int* s_flags) {
+                                           int lane, float2* s_stat) {
   const long long r0 = static_cast<long long>(b) * rows;
   for (int r = wi; r < rows; r += 2 * kWarps) {
     RowRecs a, c;
     load_row<kSample>(p, r0 + r, lane, a);
     const bool two = r + kWarps < rows;
     if (two) load_row<kSample>(p, r0 + r + kWarps, lane, c);
-    if ((row_timed_out(a) || (two && row_timed_out(c))) && lane == 0)
-      atomicOr(s_flags, DSPARK_SEQ_TIMEOUT);
     const float2 sa = reduce_row<kSample>(a);
     if (lane == 0) s_stat[r] = sa;
     if (two) {
@@ -147,7 +137,6 @@ template <typename T>
 __global__ void __launch_bounds__(kThreads) finish_greedy_kernel(const FinishParams p) {
   __shared__ float2 s_arg[kMaxK + 1];
   __shared__ int s_x[kMaxK];
-  __shared__ int s_flags;
   const int lane = threadIdx.x & 31, wi = threadIdx.x >> 5;
   const int b = blockIdx.x;
   const int K = p.rs.K, K1 = K + 1;
@@ -156,10 +145,8 @@ __global__ void __launch_bounds__(kThreads) finish_greedy_kernel(const FinishPar
     x = p.drafts[static_cast<size_t>(b) * K + lane];
     s_x[lane] = x;
   }
-  if (threadIdx.x == 0) s_flags = 0;
   grid_dependency_wait();
-  __syncthreads();
-  merge_rows<false>(p, b, K1, wi, lane, s_arg, &s_flags);
+  merge_rows<false>(p, b, K1, wi, lane, s_arg);
   __syncthreads();
   if (wi != 0) return;
   const float ninf = -__int_as_float(0x7f800000);
@@ -169,8 +156,7 @@ __global__ void __launch_bounds__(kThreads) finish_greedy_kernel(const FinishPar
     // NaN anywhere, a +inf maximum, or nothing above -inf: not a usable row
     bad |= !(a.x > ninf) || !(a.x < -ninf) || __float_as_int(a.y) == INT_MAX;
   }
-  int status = s_flags;
-  if (!(status & DSPARK_SEQ_TIMEOUT) && __any_sync(0xffffffffu, bad)) status |= DSPARK_SEQ_NONFINITE;
+  int status = __any_sync(0xffffffffu, bad) ? DSPARK_SEQ_NONFINITE : 0;
   if (__any_sync(0xffffffffu, lane < K && (x < 0 || x >= p.rs.V))) status |= DSPARK_SEQ_BAD_DRAFT;
   const int arg = lane < K ? __float_as_int(s_arg[lane].y) : -1;
   const unsigned mis = __ballot_sync(0xffffffffu, lane < K && x != arg);
@@ -273,26 +259,24 @@ __device__ __forceinline__ float2 chunk_work(const FinishParams& p, int b, int c
   constexpr int kPerLane = kGroups / 32;                      // groups per lane
   constexpr int kRound = VEC == 8 ? 4 : (VEC == 4 ? 2 : 1);  // groups in flight per row
   float lr = 0.f, lp = 0.f;
-  GroupRaw<T, VEC> gp[kRound], gq[kRound];
-  auto load = [&](int k, int slot) {
-    const int t0 = c * kCE + (k * 32 + lane) * 8;
-    gp[slot].load(pr, t0, V);
-    if (has_q) gq[slot].load(qr, t0, V);
-  };
 #pragma unroll
-  for (int k = 0; k < kRound; ++k) load(k, k);
-  // group k is summed from slot k % kRound, whose registers then take group k + kRound, so
-  // the next loads are in flight while this round's groups are computed
+  for (int k0 = 0; k0 < kPerLane; k0 += kRound) {
+    GroupRaw<T, VEC> gp[kRound], gq[kRound];
 #pragma unroll
-  for (int k = 0; k < kPerLane; ++k) {
-    const int slot = k % kRound;
-    const TokenVals gsum = group_sums<T, VEC>(gp[slot], gq[slot], has_q, p.scale, d);
-    if (k + kRound < kPerLane) load(k + kRound, slot);
-    const int q = k * 32 + lane;
-    part_r[q] = gsum.r;
-    part_p[q] = gsum.p;
-    lr = __fadd_rn(lr, gsum.r);
-    lp = __fadd_rn(lp, gsum.p);
+    for (int k = 0; k < kRound; ++k) {
+      const int t0 = c * kCE + ((k0 + k) * 32 + lane) * 8;
+      gp[k].load(pr, t0, V);
+      if (has_q) gq[k].load(qr, t0, V);
+    }
+#pragma unroll
+    for (int k = 0; k < kRound; ++k) {
+      const TokenVals gsum = group_sums<T, VEC>(gp[k], gq[k], has_q, p.scale, d);
+      const int q = (k0 + k) * 32 + lane;
+      part_r[q] = gsum.r;
+      part_p[q] = gsum.p;
+      lr = __fadd_rn(lr, gsum.r);
+      lp = __fadd_rn(lp, gsum.p);
+    }
   }
   return make_float2(warp_sum(lr), warp_sum(lp));
 }
@@ -313,7 +297,7 @@ __global__ void __launch_bounds__(kThreads, 4) finish_sample_kernel(const Finish
   __shared__ int s_x[kMaxK];
   __shared__ Decision s_dec;
   __shared__ double s_tin;
-  __shared__ int s_chunk, s_use_p, s_flags;
+  __shared__ int s_chunk, s_use_p;
   cg::cluster_group cluster = cg::this_cluster();
   const int tid = threadIdx.x, lane = tid & 31, wi = tid >> 5;
   const int G = p.G;
@@ -325,7 +309,6 @@ __global__ void __launch_bounds__(kThreads, 4) finish_sample_kernel(const Finish
   int x = -1;
   if (tid < K) x = p.drafts[static_cast<size_t>(b) * K + tid];
   if (tid <= K) s_u[tid] = p.uniforms[static_cast<size_t>(b) * K1 + tid];
-  if (tid == 0) s_flags = 0;
   grid_dependency_wait();
   // the draft tokens' logits, gathered by pass 1
   if (tid < K) {
@@ -338,15 +321,15 @@ __global__ void __launch_bounds__(kThreads, 4) finish_sample_kernel(const Finish
   __syncthreads();
 
   // every row's (reference, sum)
-  merge_rows<true>(p, b, rows, wi, lane, s_stat, &s_flags);
+  merge_rows<true>(p, b, rows, wi, lane, s_stat);
   __syncthreads();
 
   // decisions (warp 0; draft i on lane i)
   if (wi == 0) {
-    int status = s_flags;
+    int status = 0;
     bool bad = false;
     for (int r = lane; r < rows; r += 32) bad |= !stat_ok(s_stat[r]);
-    if (!(status & DSPARK_SEQ_TIMEOUT) && __any_sync(0xffffffffu, bad)) status |= DSPARK_SEQ_NONFINITE;
+    if (__any_sync(0xffffffffu, bad)) status |= DSPARK_SEQ_NONFINITE;
     const int x = lane < K ? s_x[lane] : 0;
     const bool bad_draft = lane < K && (x < 0 || x >= V);
     if (__any_sync(0xffffffffu, bad_draft)) status |= DSPARK_SEQ_BAD_DRAFT;

@@ -2,12 +2,13 @@
 //
 // The work is split into units (row, chunk): chunk c of a row is its tokens
 // [2048c, min(V, 2048(c+1))). Units are numbered sequence-major (sequence b: P rows 0..K,
-// then for the sampling policy Q rows 0..K-1; within a row, chunks in order), and each warp
-// of one full wave takes an equal contiguous run of them. A warp streams a unit with 16-byte
+// then for the sampling policy Q rows 0..K-1; within a row, chunks in order); each SM's CTA
+// owns an equal contiguous range of them and hands them to its warps in order. A warp streams a
+// unit with 16-byte
 // loads, several in flight per lane, keeps per-lane running statistics, merges its lanes and
 // writes one record for the unit. A record is a function of the unit's logits alone (not of
 // the launch geometry), so identical rows give identical statistics. No warp waits for
-// another: all warps of the wave finish together and the kernel is a plain stream.
+// another.
 //
 // Records. Sampling: (ref, sum) with ref = max_v z[v] * scale and sum = sum_v 2^(z[v]*scale
 // - ref), the online-softmax pair (Milakov & Gimelshein 2018) in base 2; (-inf, 0) for a
@@ -21,9 +22,10 @@
 
 namespace dspark {
 
-constexpr int kThreads = 256;            // both kernels
+constexpr int kThreads = 256;            // pass-2 CTAs
 constexpr int kWarps = kThreads / 32;
-constexpr int kStreamCtasPerSm = 4;      // 4 x 256 threads x 64 registers fill the SM
+constexpr int kStreamThreads = 1024;     // pass 1: one CTA of 32 warps per SM (64 registers)
+constexpr int kStreamWarps = kStreamThreads / 32;
 constexpr int kBatchVecs = 8;            // loads each lane keeps in flight
 constexpr int kCE = 2048;                // tokens per chunk (pass-1 unit, pass-2 chunk)
 constexpr int kMaxChunkCount = 128;      // chunks per row (V <= 262144)
@@ -51,75 +53,33 @@ __device__ __forceinline__ const T* row_ptr(const RowSet& rs, int b, int i) {
          (static_cast<int64_t>(b) * rs.K + (i - rs.K - 1)) * rs.V;
 }
 
+// Unsigned division by a divisor fixed per call, by multiplication: q = floor(n * m / 2^(32+s))
+// with m = ceil(2^(32+s) / d), s = ceil(log2 d), exact for every n < 2^32 (m < 2^33 is kept as
+// m_hi * 2^32 + m_lo). Integer multiplies only: no SFU or conversion instructions.
+struct FastDiv {
+  uint32_t m_lo, m_hi, s;
+  __device__ __forceinline__ uint32_t div(uint32_t n) const {
+    const uint64_t t = static_cast<uint64_t>(__umulhi(n, m_lo)) + (m_hi ? n : 0u);
+    return static_cast<uint32_t>(t >> s);
+  }
+};
+
 struct StreamParams {
   RowSet rs;
-  long long n_units;  // B * rows * nch
-  long long upw;      // units per warp (contiguous runs)
-  long long warps;    // warps of the grid (strided order)
-  int strided;        // 1: warp w takes units w, w + warps, ...; 0: a contiguous run
+  uint32_t n_units;   // B * rows * nch (< 2^32)
   int nch;            // chunks per row
-  int stages;         // ring kernel: shared-memory stages per warp
+  FastDiv by_nch;     // division by nch
+  FastDiv by_rows;    // division by rows
+
   float scale;        // log2(e) / T (sampling)
   float2* rec;        // [n_units]: record of unit u at u
   const int32_t* drafts;  // [B, K] (sampling)
   float* gather;      // [B, K, 2] (sampling): P_i[x_i], Q_i[x_i] as float
 };
 
-
-
-// Record of a unit whose data never arrived (a bounded wait gave up): its second word has
-// these bits, which no statistics record has (arithmetic NaNs are 0x7fffffff, indices >= 0).
-constexpr uint32_t kTimeoutRecBits = 0xffffffffu;
-
-// (sequence b, row i, chunk c) of a unit, stepped through a warp's run in order.
+// (sequence b, row i, chunk c) of a unit.
 struct UnitPos {
   int b, i, c;
-  __device__ __forceinline__ void init(long long u, int nch, int rows) {
-    const long long r = u / nch;
-    c = static_cast<int>(u - r * nch);
-    b = static_cast<int>(r / rows);
-    i = static_cast<int>(r - static_cast<long long>(b) * rows);
-  }
-  __device__ __forceinline__ void next(int nch, int rows) {
-    if (++c == nch) {
-      c = 0;
-      if (++i == rows) {
-        i = 0;
-        ++b;
-      }
-    }
-  }
-};
-
-// Steps a unit position by a fixed stride n = q * nch + rc (rc < nch) without dividing:
-// c += rc with a carry into the row, the row advances by q or q + 1, and the row index
-// (b * rows + i) is split the same way with precomputed quotients of both row steps.
-struct UnitStride {
-  int rc;                   // stride mod nch
-  int qi0, qb0, qi1, qb1;   // row steps q and q + 1 as (mod rows, div rows)
-  __device__ __forceinline__ void init(long long n, int nch, int rows) {
-    const long long q = n / nch;
-    rc = static_cast<int>(n - q * nch);
-    qb0 = static_cast<int>(q / rows);
-    qi0 = static_cast<int>(q - static_cast<long long>(qb0) * rows);
-    qb1 = static_cast<int>((q + 1) / rows);
-    qi1 = static_cast<int>(q + 1 - static_cast<long long>(qb1) * rows);
-  }
-  __device__ __forceinline__ void step(UnitPos& at, int nch, int rows) const {
-    at.c += rc;
-    int di = qi0, db = qb0;
-    if (at.c >= nch) {
-      at.c -= nch;
-      di = qi1;
-      db = qb1;
-    }
-    at.i += di;
-    at.b += db;
-    if (at.i >= rows) {
-      at.i -= rows;
-      ++at.b;
-    }
-  }
 };
 
 // Sampling: the unit that holds a draft token x_i of a draft row (P row i < K, or Q row i)
@@ -232,19 +192,13 @@ __device__ __forceinline__ float2 soft_record(const LaneSoft& st, float scale) {
   return make_float2(w.m, w.m == ninf ? 0.f : w.s);
 }
 
-// Where a unit's 16-byte vectors come from: global memory (vector vi of the row) or this
-// warp's shared-memory stage (vector vi - nv0 of the stage).
+// Where a unit's 16-byte vectors come from: vector vi of the row in global memory.
 template <typename T>
 struct GlobalVecs {
   const T* row;
   __device__ __forceinline__ uint4 operator()(long long vi) const {
     return ld_stream16(row + vi * Elem<T>::kPerVec16);
   }
-};
-struct StageVecs {
-  const uint4* stage;
-  long long nv0;
-  __device__ __forceinline__ uint4 operator()(long long vi) const { return stage[vi - nv0]; }
 };
 
 template <typename T, class Src>
@@ -380,24 +334,34 @@ __device__ __forceinline__ float2 piece_argmax(const T* row, long long o0, long 
 
 // --------------------------------------------------------------------------- kernel
 
+// One CTA per SM. CTA k owns units [k n / grid, (k+1) n / grid) and hands them to its warps
+// in order from a shared-memory counter, one at a time: lane 0 asks for the next unit while
+// the warp works on the current one, so the atomic's latency is hidden, and the warps that the
+// SM's scheduler favours simply take more units. Every SM holds the same share of the work
+// and its warps finish together; no global atomic, fence or barrier is involved.
 template <typename T, int VEC, bool kSample>
-__global__ void __launch_bounds__(kThreads, kStreamCtasPerSm) stream_stats_kernel(
-    const StreamParams p) {
+__global__ void __launch_bounds__(kStreamThreads, 1) stream_stats_kernel(const StreamParams p) {
+  __shared__ unsigned s_next;
   // the finish kernel may be scheduled as soon as these CTAs retire
   grid_dependents_launch();
   const int lane = threadIdx.x & 31;
-  const long long w = static_cast<long long>(blockIdx.x) * kWarps + (threadIdx.x >> 5);
-  // units of this warp: u0, u0 + du, ... below u1 (a contiguous run, or a grid stride)
-  const long long u0 = p.strided ? w : w * p.upw;
-  const long long u1 = p.strided ? p.n_units : min(u0 + p.upw, p.n_units);
-  const long long du = p.strided ? p.warps : 1;
-  if (u0 >= u1) return;
-  UnitPos at;
-  at.init(u0, p.nch, p.rs.rows);
-  UnitStride stride;
-  stride.init(du, p.nch, p.rs.rows);
+  const int wi = threadIdx.x >> 5;
   const int V = p.rs.V;
-  for (long long u = u0; u < u1; u += du) {
+  const unsigned u_begin =
+      static_cast<unsigned>(static_cast<uint64_t>(blockIdx.x) * p.n_units / gridDim.x);
+  const unsigned u_end =
+      static_cast<unsigned>(static_cast<uint64_t>(blockIdx.x + 1) * p.n_units / gridDim.x);
+  if (threadIdx.x == 0) s_next = u_begin + kStreamWarps;  // first units are fixed: u_begin + w
+  __syncthreads();
+  unsigned nxt = 0;
+  unsigned u = u_begin + wi;
+  while (u < u_end) {
+    if (lane == 0) nxt = atomicAdd(&s_next, 1u);
+    UnitPos at;
+    const uint32_t r = p.by_nch.div(u);
+    at.c = static_cast<int>(u - r * static_cast<uint32_t>(p.nch));
+    at.b = static_cast<int>(p.by_rows.div(r));
+    at.i = static_cast<int>(r - static_cast<uint32_t>(at.b) * static_cast<uint32_t>(p.rs.rows));
     const T* row = row_ptr<T>(p.rs, at.b, at.i);
     const int o0 = at.c * kCE;
     const int o1 = min(V, o0 + kCE);
@@ -410,98 +374,7 @@ __global__ void __launch_bounds__(kThreads, kStreamCtasPerSm) stream_stats_kerne
       rec = piece_argmax<T, VEC>(row, o0, o1, lane);
     }
     if (lane == 0) p.rec[u] = rec;
-    stride.step(at, p.nch, p.rs.rows);
-  }
-}
-
-// ---------------------------------------------------------------- ring kernel (16-byte path)
-
-// The same pass with each warp's next units staged in shared memory by 1-D bulk copies
-// (cp.async.bulk, one per unit, issued by lane 0 `stages` units ahead), so a warp's loads stay
-// in flight while it computes. Stage and mbarrier per (warp, slot); no data is shared between
-// warps. A unit's bytes: min(V - 2048c, 2048) tokens, a multiple of 16 bytes on this path.
-constexpr int kRingCtasPerSm = 2;
-constexpr int kMaxStages = 4;
-
-template <typename T>
-__device__ __forceinline__ void issue_unit(const StreamParams& p, const UnitPos& at,
-                                           unsigned char* stage, uint64_t* bar) {
-  const int o0 = at.c * kCE;
-  const int n = min(p.rs.V - o0, kCE);
-  const uint32_t bytes = static_cast<uint32_t>(n) * Elem<T>::kBytes;
-  mbar_arrive_expect_tx(bar, bytes);
-  bulk_g2s(stage, row_ptr<T>(p.rs, at.b, at.i) + o0, bytes, bar);
-}
-
-template <typename T, bool kSample>
-__global__ void __launch_bounds__(kThreads, kRingCtasPerSm) stream_stats_ring_kernel(
-    const StreamParams p) {
-  extern __shared__ __align__(128) unsigned char smem[];
-  grid_dependents_launch();
-  constexpr int VEC = Elem<T>::kPerVec16;
-  constexpr int UB = kCE * Elem<T>::kBytes;  // bytes per stage
-  const int lane = threadIdx.x & 31, wi = threadIdx.x >> 5;
-  const int S = p.stages;
-  unsigned char* ring = smem + static_cast<size_t>(wi) * S * UB;
-  uint64_t* bar = reinterpret_cast<uint64_t*>(smem + static_cast<size_t>(kWarps) * S * UB) +
-                  wi * kMaxStages;
-  const long long w = static_cast<long long>(blockIdx.x) * kWarps + wi;
-  const long long u0 = w * p.upw;
-  const long long u1 = min(u0 + p.upw, p.n_units);
-  if (u0 >= u1) return;
-  const int n = static_cast<int>(u1 - u0);
-  UnitPos at, ahead;
-  at.init(u0, p.nch, p.rs.rows);
-  ahead = at;
-  if (lane == 0) {
-    for (int s = 0; s < S; ++s) mbar_init(&bar[s], 1);
-    fence_mbar_init();
-    for (int k = 0; k < S && k < n; ++k) {
-      issue_unit<T>(p, ahead, ring + k * UB, &bar[k]);
-      ahead.next(p.nch, p.rs.rows);
-    }
-  }
-  __syncwarp();
-  const int V = p.rs.V;
-  int issued = S < n ? S : n;  // units whose copies were issued (lane 0's count, kept warp-wide)
-  int first_failed = -1;       // first unit whose wait gave up
-  bool failed = false;
-  for (int k = 0; k < n; ++k) {
-    const int st = k % S;
-    float2 rec;
-    if (!failed) {
-      failed = !__all_sync(0xffffffffu, mbar_wait_bounded(&bar[st], (k / S) & 1));
-      if (failed) first_failed = k;
-    }
-    if (!failed) {
-      const int o0 = at.c * kCE;
-      const int o1 = min(V, o0 + kCE);
-      const StageVecs src{reinterpret_cast<const uint4*>(ring + st * UB), o0 / VEC};
-      if constexpr (kSample) {
-        const int xd = unit_draft<T>(p, at, lane);
-        rec = unit_softmax_vec<T>(src, o0 / VEC, o1 / VEC, lane, p.scale);
-        unit_gather<T>(p, at, row_ptr<T>(p.rs, at.b, at.i), xd, o0, o1);
-      } else {
-        rec = unit_argmax_vec<T>(src, o0 / VEC, o1 / VEC, lane);
-      }
-    } else {
-      rec = make_float2(0.f, __uint_as_float(kTimeoutRecBits));
-    }
-    __syncwarp();  // every lane is done with the stage
-    if (lane == 0) {
-      p.rec[u0 + k] = rec;
-      if (!failed && k + S < n) {
-        fence_proxy_async_smem();  // the stage's reads come before the copy that refills it
-        issue_unit<T>(p, ahead, ring + st * UB, &bar[st]);
-        ahead.next(p.nch, p.rs.rows);
-      }
-    }
-    if (!failed && k + S < n) ++issued;
-    at.next(p.nch, p.rs.rows);
-  }
-  if (failed) {
-    // copies still in flight land in this warp's stages: wait for them (bounded) before exit
-    for (int k = first_failed; k < issued; ++k) mbar_wait_bounded(&bar[k % S], (k / S) & 1);
+    u = __shfl_sync(0xffffffffu, nxt, 0);
   }
 }
 

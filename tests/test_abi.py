@@ -54,6 +54,7 @@ def test_plans_cover_every_workload_shape(lib):
         assert lib.dspark_plan(4, 7, V, BF16, 1, ctypes.byref(p)) == 0
         assert p.n_chunks == -(-V // p.chunk_elems) and p.n_chunks * p.chunk_elems >= V
         assert p.elems_per_load == 8 and p.threads_per_cta % 32 == 0 and p.loads_in_flight >= 1
+        assert p.stream_threads_per_cta % 32 == 0 and p.stream_threads_per_cta <= 1024
         # pass-1 units: one per (row, chunk); K+1 rows (greedy), 2K+1 rows (sampling)
         assert p.greedy_units_per_sequence == 8 * p.n_chunks
         assert p.sampling_units_per_sequence == 15 * p.n_chunks
@@ -69,9 +70,9 @@ def test_plans_cover_every_workload_shape(lib):
 def test_workspace_needs_no_initialisation(lib):
     for B, K in ((1, 0), (64, 7), (256, 15), (3, 32)):
         assert lib.dspark_workspace_zero_bytes(B, K) == 0
-        # the workspace holds one float2 record per (row, chunk) unit, 2K+1 rows per sequence
+        # one float2 record per (row, chunk) unit, 2K+1 rows per sequence, then the gathers
         nch = -(-129280 // 2048)
-        assert lib.dspark_workspace_bytes(B, K, 129280, BF16) >= 8 * B * (2 * K + 1) * nch
+        assert lib.dspark_workspace_bytes(B, K, 129280, BF16) >= 8 * B * (2 * K + 1) * nch + 8 * B * K
 
 
 def _greedy(lib, **kw):
