@@ -156,24 +156,36 @@ def _split_block(P) -> Tuple[torch.Tensor, Optional[torch.Tensor], int, int]:
 
 
 class _Workspace:
-    """A per-device byte buffer reused across calls, grown on demand. The library needs no
-    initialisation of it (a call writes every word it reads)."""
+    """A per-device byte buffer reused across calls, grown on demand.
+
+    The library needs the first ``dspark_workspace_zero_bytes(B, K)`` bytes (one counter per
+    sequence) zero before a call, and a call leaves exactly its own such prefix zero; the bytes
+    after it hold that call's other data. So the prefix is cleared again (a memset on the
+    current stream; nothing is allocated) whenever a call needs more of it than the previous
+    call left zero.
+    """
 
     def __init__(self):
         self.bufs = {}
+        self.zeroed = {}
 
-    def get(self, device: torch.device, nbytes: int) -> torch.Tensor:
+    def get(self, device: torch.device, nbytes: int, B: int, K: int) -> torch.Tensor:
         key = device.index if device.index is not None else torch.cuda.current_device()
+        need = int(load_library().dspark_workspace_zero_bytes(B, K))
         buf = self.bufs.get(key)
         if buf is None or buf.numel() < nbytes:
             buf = new_workspace(max(nbytes, 256), device)
             self.bufs[key] = buf
+        elif need > self.zeroed.get(key, 0):
+            buf[:need].zero_()
+        self.zeroed[key] = need
         return buf
 
 
 def new_workspace(nbytes: int, device) -> torch.Tensor:
-    """A workspace buffer of `nbytes` bytes (256-byte aligned, as every CUDA allocation)."""
-    return torch.empty(max(nbytes, 256), dtype=torch.uint8, device=device)
+    """A zeroed workspace buffer of `nbytes` bytes (256-byte aligned, as every CUDA
+    allocation): the state the library requires before its first call."""
+    return torch.zeros(max(nbytes, 256), dtype=torch.uint8, device=device)
 
 
 _WS = _Workspace()
@@ -217,7 +229,10 @@ def greedy_accept(P: Union[torch.Tensor, Tuple[torch.Tensor, torch.Tensor]],
     """Greedy block verify on the GPU: accept drafts while they equal the base argmax.
 
     ``workspace``, if given, is a device byte buffer of at least ``workspace_bytes(...)``
-    bytes that no other call uses at the same time.
+    bytes that no other call uses at the same time, whose first
+    ``dspark_workspace_zero_bytes(B, K)`` bytes are zero (``new_workspace`` returns such a
+    buffer; a call leaves its own prefix zero, so only a call with a larger B needs a clear).
+    The current kernels need no zero prefix (the size is 0); the contract is kept general.
     """
     lib = load_library()
     p1, pv, ld_p1, ld_pv = _split_block(P)
@@ -228,7 +243,7 @@ def greedy_accept(P: Union[torch.Tensor, Tuple[torch.Tensor, torch.Tensor]],
     drafts = _check_drafts(drafts, B, K, p1.device)
     res = out if out is not None else _alloc_result(B, K, p1.device, diagnostics=False)
     nbytes = lib.dspark_workspace_bytes(B, K, V, DTYPE_CODES[p1.dtype])
-    ws = workspace if workspace is not None else _WS.get(p1.device, nbytes)
+    ws = workspace if workspace is not None else _WS.get(p1.device, nbytes, B, K)
     rc = lib.dspark_greedy_accept(_ptr(p1), ld_p1, _ptr(pv), ld_pv, DTYPE_CODES[p1.dtype],
                                   _ptr(drafts), B, K, V, _out_struct(res), _ptr(ws),
                                   ws.numel() * ws.element_size(), _stream_handle(p1.device))
@@ -258,7 +273,7 @@ def speculative_sample_accept(P: Union[torch.Tensor, Tuple[torch.Tensor, torch.T
         raise ValueError("uniforms must be a contiguous float32 [B, K+1] tensor on P's device")
     res = out if out is not None else _alloc_result(B, K, p1.device, diagnostics=True)
     nbytes = lib.dspark_workspace_bytes(B, K, V, DTYPE_CODES[p1.dtype])
-    ws = workspace if workspace is not None else _WS.get(p1.device, nbytes)
+    ws = workspace if workspace is not None else _WS.get(p1.device, nbytes, B, K)
     rc = lib.dspark_speculative_sample_accept(
         _ptr(p1), ld_p1, _ptr(pv), ld_pv, _ptr(Q), DTYPE_CODES[p1.dtype], _ptr(drafts), B, K,
         V, float(temperature), _ptr(uniforms), _out_struct(res), _ptr(ws),

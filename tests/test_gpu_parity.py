@@ -271,3 +271,13 @@ def test_chi_square_first_token_one_million_cycles():
     expect = sum(np.prod(alpha[:k]) for k in range(1, w.K + 1))
     n = r.n_accepted.double()
     assert abs(n.mean().item() - expect) < 4 * n.std().item() / np.sqrt(N)
+
+
+def test_shared_workspace_across_growing_batches():
+    """The binding's shared workspace: a small batch, then a larger one whose per-sequence
+    counters lie where the small call kept its records; results must not depend on it."""
+    small = wl.Workload("s", B=5, K=3, V=4096, dtype="bf16", kind="shared_noise",
+                        params={"sd": 2.0, "noise": 1.0})
+    big = wl.Workload("g", B=700, K=3, V=64, dtype="f32", kind="iid", params={"sd": 2.0})
+    for w in (small, big, small, big):
+        _check(w, 1.0, label=f"{w.name} B={w.B}")
