@@ -3,8 +3,8 @@
 // The work is split into units (row, chunk): chunk c of a row is its tokens
 // [2048c, min(V, 2048(c+1))). Units are numbered sequence-major (sequence b: P rows 0..K,
 // then for the sampling policy Q rows 0..K-1; within a row, chunks in order); each SM's CTA
-// owns an equal contiguous range of them and hands them to its warps in order. A warp streams a
-// unit with 16-byte
+// owns every grid-th unit and hands them to its warps in order. A warp streams a unit with
+// 16-byte
 // loads, several in flight per lane, keeps per-lane running statistics, merges its lanes and
 // writes one record for the unit. A record is a function of the unit's logits alone (not of
 // the launch geometry), so identical rows give identical statistics. No warp waits for
@@ -334,11 +334,13 @@ __device__ __forceinline__ float2 piece_argmax(const T* row, long long o0, long 
 
 // --------------------------------------------------------------------------- kernel
 
-// One CTA per SM. CTA k owns units [k n / grid, (k+1) n / grid) and hands them to its warps
-// in order from a shared-memory counter, one at a time: lane 0 asks for the next unit while
-// the warp works on the current one, so the atomic's latency is hidden, and the warps that the
-// SM's scheduler favours simply take more units. Every SM holds the same share of the work
-// and its warps finish together; no global atomic, fence or barrier is involved.
+// One CTA per SM. CTA k owns units k, k + grid, k + 2 grid, ... and hands them to its warps in
+// order from a shared-memory counter, one at a time: lane 0 asks for the next unit while the
+// warp works on the current one, so the atomic's latency is hidden, and the warps that the SM's
+// scheduler favours simply take more units. Every SM holds the same share of the work and its
+// warps finish together; no global atomic, fence or barrier is involved. The whole grid sweeps
+// the units front to back, so the rows read last, still in L2 when pass 2 re-reads a row pair,
+// are those of the last sequences.
 template <typename T, int VEC, bool kSample>
 __global__ void __launch_bounds__(kStreamThreads, 1) stream_stats_kernel(const StreamParams p) {
   __shared__ unsigned s_next;
@@ -347,16 +349,15 @@ __global__ void __launch_bounds__(kStreamThreads, 1) stream_stats_kernel(const S
   const int lane = threadIdx.x & 31;
   const int wi = threadIdx.x >> 5;
   const int V = p.rs.V;
-  const unsigned u_begin =
-      static_cast<unsigned>(static_cast<uint64_t>(blockIdx.x) * p.n_units / gridDim.x);
-  const unsigned u_end =
-      static_cast<unsigned>(static_cast<uint64_t>(blockIdx.x + 1) * p.n_units / gridDim.x);
-  if (threadIdx.x == 0) s_next = u_begin + kStreamWarps;  // first units are fixed: u_begin + w
+  const unsigned k = blockIdx.x, G = gridDim.x;
+  const unsigned n_mine = k < p.n_units ? (p.n_units - 1 - k) / G + 1 : 0;  // this CTA's units
+  if (threadIdx.x == 0) s_next = kStreamWarps;  // the first kStreamWarps go to warps 0..31
   __syncthreads();
   unsigned nxt = 0;
-  unsigned u = u_begin + wi;
-  while (u < u_end) {
+  unsigned m = wi;
+  while (m < n_mine) {
     if (lane == 0) nxt = atomicAdd(&s_next, 1u);
+    const unsigned u = k + m * G;
     UnitPos at;
     const uint32_t r = p.by_nch.div(u);
     at.c = static_cast<int>(u - r * static_cast<uint32_t>(p.nch));
@@ -374,7 +375,7 @@ __global__ void __launch_bounds__(kStreamThreads, 1) stream_stats_kernel(const S
       rec = piece_argmax<T, VEC>(row, o0, o1, lane);
     }
     if (lane == 0) p.rec[u] = rec;
-    u = __shfl_sync(0xffffffffu, nxt, 0);
+    m = __shfl_sync(0xffffffffu, nxt, 0);
   }
 }
 
