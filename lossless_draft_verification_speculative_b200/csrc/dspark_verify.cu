@@ -15,14 +15,11 @@ namespace {
 constexpr int kAbiVersion = 3;
 constexpr int kMaxDevices = 64;
 
-// Tuning switch read once: DSPARK_MAX_CTAS caps the pass-1 CTAs (0 = one full wave).
+// Tuning switch, read at every call: DSPARK_MAX_CTAS caps the pass-1 CTAs (0 = one per SM).
 int max_ctas_override() {
-  static const int v = [] {
-    const char* s = std::getenv("DSPARK_MAX_CTAS");
-    const int n = s ? std::atoi(s) : 0;
-    return n > 0 ? n : 0;
-  }();
-  return v;
+  const char* s = std::getenv("DSPARK_MAX_CTAS");
+  const int n = s ? std::atoi(s) : 0;
+  return n > 0 ? n : 0;
 }
 
 // ------------------------------------------------------------------------------ plans
@@ -97,21 +94,38 @@ struct OccEntry {
 };
 OccEntry g_occ[64];
 int g_occ_n = 0;
+struct SmemLimit {
+  const void* fn;
+  int dev;
+  size_t bytes;  // the kernel's dynamic shared-memory limit, as last raised
+};
+SmemLimit g_lim[64];
+int g_lim_n = 0;
 
-// CTAs of `fn` (kThreads threads, `smem` dynamic shared memory) resident on the current
-// device at once; sets the kernel's dynamic shared-memory limit first when it needs one.
+// CTAs of `fn` (`threads` threads, `smem` dynamic shared memory) resident on the current
+// device at once. Raises the kernel's dynamic shared-memory limit first when `smem` is above
+// it; the limit is never lowered, so a call that needs less shared memory cannot break a
+// later call that needs more.
 int resident_ctas(const void* fn, int threads, size_t smem, cudaError_t* err) {
   int dev = 0;
   *err = cudaGetDevice(&dev);
   if (*err != cudaSuccess) return 0;
   std::lock_guard<std::mutex> lk(g_mu);
-  for (int n = 0; n < g_occ_n; ++n)
-    if (g_occ[n].fn == fn && g_occ[n].dev == dev && g_occ[n].smem == smem) return g_occ[n].ctas;
-  if (smem > 0) {
+  SmemLimit* lim = nullptr;
+  for (int n = 0; n < g_lim_n; ++n)
+    if (g_lim[n].fn == fn && g_lim[n].dev == dev) lim = &g_lim[n];
+  if (smem > 0 && (!lim || smem > lim->bytes)) {
     *err = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 static_cast<int>(smem));
     if (*err != cudaSuccess) return 0;
+    if (!lim && g_lim_n < 64) {
+      g_lim[g_lim_n] = SmemLimit{fn, dev, 0};
+      lim = &g_lim[g_lim_n++];
+    }
+    if (lim) lim->bytes = smem;
   }
+  for (int n = 0; n < g_occ_n; ++n)
+    if (g_occ[n].fn == fn && g_occ[n].dev == dev && g_occ[n].smem == smem) return g_occ[n].ctas;
   int per_sm = 0, sms = 0;
   *err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, threads, smem);
   if (*err != cudaSuccess) return 0;
@@ -152,8 +166,9 @@ dspark_status_t run_call(const Call& c, const Plan& pl, cudaStream_t stream) {
   sp.rs = c.rs;
   sp.n_units = static_cast<uint32_t>(n_units);
   sp.nch = pl.nch;
+  sp.B = c.B;
   sp.by_nch = fast_div(static_cast<uint32_t>(pl.nch));
-  sp.by_rows = fast_div(static_cast<uint32_t>(c.rs.rows));
+  sp.by_seqs = fast_div(static_cast<uint32_t>(c.B));
   sp.scale = c.scale;
   sp.rec = reinterpret_cast<float2*>(c.ws + w.rec);
   sp.drafts = c.drafts;

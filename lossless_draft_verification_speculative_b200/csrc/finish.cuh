@@ -247,15 +247,16 @@ __device__ __forceinline__ TokenVals group_sums(const GroupRaw<T, VEC>& gp,
   return acc;
 }
 
-// Chunk c of the draw's law, one warp: the 256 group sums into part_r / part_p (token order)
-// and the chunk's (residual mass, p mass) on every lane.
+// Chunk c of the draw's law, one warp: the 256 group sums into part_r / part_p (token order;
+// either may be null) and the chunk's (residual mass, p mass) on every lane.
 template <typename T, int VEC>
-__device__ __forceinline__ float2 chunk_work(const FinishParams& p, int b, int c, const Decision& d,
-                                             int lane, float* part_r, float* part_p) {
-  const int K = p.rs.K, V = p.rs.V;
+__device__ __forceinline__ float2 chunk_work(const RowSet& rs, float scale, int b, int c,
+                                             const Decision& d, int lane, float* part_r,
+                                             float* part_p) {
+  const int K = rs.K, V = rs.V;
   const bool has_q = d.j < K;
-  const T* pr = row_ptr<T>(p.rs, b, d.j);
-  const T* qr = has_q ? row_ptr<T>(p.rs, b, K + 1 + d.j) : pr;
+  const T* pr = row_ptr<T>(rs, b, d.j);
+  const T* qr = has_q ? row_ptr<T>(rs, b, K + 1 + d.j) : pr;
   constexpr int kPerLane = kGroups / 32;                      // groups per lane
   constexpr int kRound = VEC == 8 ? 4 : (VEC == 4 ? 2 : 1);  // groups in flight per row
   float lr = 0.f, lp = 0.f;
@@ -270,15 +271,178 @@ __device__ __forceinline__ float2 chunk_work(const FinishParams& p, int b, int c
     }
 #pragma unroll
     for (int k = 0; k < kRound; ++k) {
-      const TokenVals gsum = group_sums<T, VEC>(gp[k], gq[k], has_q, p.scale, d);
+      const TokenVals gsum = group_sums<T, VEC>(gp[k], gq[k], has_q, scale, d);
       const int q = (k0 + k) * 32 + lane;
-      part_r[q] = gsum.r;
-      part_p[q] = gsum.p;
+      if (part_r) part_r[q] = gsum.r;
+      if (part_p) part_p[q] = gsum.p;
       lr = __fadd_rn(lr, gsum.r);
       lp = __fadd_rn(lp, gsum.p);
     }
   }
   return make_float2(warp_sum(lr), warp_sum(lp));
+}
+
+// Where the draw falls among the chunks of its row: float64 prefix over the chunk masses
+// (lane l holds chunks l*kMassPerLane .. l*kMassPerLane + kMassPerLane - 1, zero past the
+// row), target u*Z, first chunk whose inclusive prefix passes it. Every lane gets the result.
+constexpr int kMassPerLane = kMaxChunkCount / 32;
+struct ChunkPick {
+  int c;        // chunk that holds the draw; -1 when no chunk has mass
+  int status;   // the decision's status, plus DSPARK_SEQ_ZERO_RESIDUAL when that applies
+  bool use_p;   // draw from p_j itself: the bonus row, or a residual that rounded to zero
+  double tin;   // the target measured from the chunk's start (+inf: past the last mass)
+  double zres;  // the residual mass (rejection rows)
+};
+
+__device__ __forceinline__ ChunkPick pick_chunk(const float2 (&ms)[kMassPerLane], bool bonus,
+                                                float u, int status, int lane) {
+  constexpr int NPL = kMassPerLane;
+  bool use_p = bonus;
+  double mr[NPL], mp[NPL];
+  double zr = 0.0, zpm = 0.0;
+#pragma unroll
+  for (int k = 0; k < NPL; ++k) {
+    mr[k] = ms[k].x;
+    mp[k] = ms[k].y;
+    zr += mr[k];
+    zpm += mp[k];
+  }
+  double Zr = zr, Zp = zpm;  // inclusive prefixes over lanes
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const double a = __shfl_up_sync(0xffffffffu, Zr, o), c2 = __shfl_up_sync(0xffffffffu, Zp, o);
+    if (lane >= o) {
+      Zr += a;
+      Zp += c2;
+    }
+  }
+  const double Zres = __shfl_sync(0xffffffffu, Zr, 31);
+  if (!use_p && !(Zres > 0.0)) {  // residual mass rounded to zero: draw from p_j instead
+    use_p = true;
+    status |= DSPARK_SEQ_ZERO_RESIDUAL;
+  }
+  double m[NPL];
+#pragma unroll
+  for (int k = 0; k < NPL; ++k) m[k] = use_p ? mp[k] : mr[k];
+  const double incl = use_p ? Zp : Zr;
+  const double ls = use_p ? zpm : zr;
+  const double Z = __shfl_sync(0xffffffffu, incl, 31);
+  const double target = static_cast<double>(u) * Z;
+  double run = incl - ls;
+  int cfound = -1, clast = -1;
+  double before = 0.0;
+#pragma unroll
+  for (int k = 0; k < NPL; ++k) {
+    const double nxt = run + m[k];
+    if (m[k] > 0.0) {
+      clast = lane * NPL + k;
+      if (cfound < 0 && run <= target && target < nxt) {
+        cfound = clast;
+        before = run;
+      }
+    }
+    run = nxt;
+  }
+  const unsigned hit = __ballot_sync(0xffffffffu, cfound >= 0);
+  ChunkPick pk;
+  if (hit) {
+    const int hl = __ffs(hit) - 1;
+    pk.c = __shfl_sync(0xffffffffu, cfound, hl);
+    pk.tin = target - __shfl_sync(0xffffffffu, before, hl);
+  } else {  // rounding left the target past the last mass: the last token with mass
+    int cl = clast;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) cl = max(cl, __shfl_xor_sync(0xffffffffu, cl, o));
+    pk.c = cl;
+    pk.tin = __int_as_float(0x7f800000);
+  }
+  pk.status = status;
+  pk.use_p = use_p;
+  pk.zres = Zres;
+  return pk;
+}
+
+// The token of chunk c at the target tin (measured from the chunk's start), given the chunk's
+// 256 group sums `part` (token order) of the law drawn from (residual, or p when use_p): the
+// group from a scan of the sums, then that group's 8 tokens re-read and recomputed exactly as
+// their sum was, scanned by lane 0. Rounding that leaves the target past the chunk's sums
+// picks its last token with mass. Every lane gets the token.
+template <typename T, int VEC>
+__device__ __forceinline__ int pick_token(const RowSet& rs, float scale, int b, const Decision& d,
+                                          int c, bool use_p, float tin, const float* part,
+                                          int lane) {
+  const int j = d.j;
+  // lane l scans the chunk's groups 8l .. 8l+7 (token order)
+  float gv[8];
+  float lsum = 0.f;
+  int lastg = -1;
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+    gv[e] = part[lane * 8 + e];
+    lsum = __fadd_rn(lsum, gv[e]);
+    if (gv[e] > 0.f) lastg = lane * 8 + e;
+  }
+  float inc = lsum;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const float y = __shfl_up_sync(0xffffffffu, inc, o);
+    if (lane >= o) inc = __fadd_rn(inc, y);
+  }
+  float ex = __shfl_up_sync(0xffffffffu, inc, 1);
+  if (lane == 0) ex = 0.f;
+  int qsel = -1;
+  float gin = 0.f;
+  if (ex <= tin && tin < inc) {
+    float r = ex;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const float nx = __fadd_rn(r, gv[e]);
+      if (qsel < 0 && gv[e] > 0.f && r <= tin && tin < nx) {
+        qsel = lane * 8 + e;
+        gin = __fsub_rn(tin, r);
+      }
+      r = nx;
+    }
+  }
+  const unsigned h = __ballot_sync(0xffffffffu, qsel >= 0);
+  bool last_mode = false;
+  if (h) {
+    const int hl = __ffs(h) - 1;
+    qsel = __shfl_sync(0xffffffffu, qsel, hl);
+    gin = __shfl_sync(0xffffffffu, gin, hl);
+  } else {  // rounding: the chunk's last group with mass, its last token with mass
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) lastg = max(lastg, __shfl_xor_sync(0xffffffffu, lastg, o));
+    qsel = lastg;
+    last_mode = true;
+  }
+  int token = -1;
+  if (qsel >= 0 && lane == 0) {
+    const int K = rs.K, V = rs.V;
+    const bool has_q = j < K;
+    const T* pr = row_ptr<T>(rs, b, j);
+    const T* qr = has_q ? row_ptr<T>(rs, b, K + 1 + j) : pr;
+    const int t0 = c * kCE + qsel * 8;
+    GroupRaw<T, VEC> gp, gq;
+    gp.load(pr, t0, V);
+    if (has_q) gq.load(qr, t0, V);
+    float zp[8], zq[8];
+    gp.values(zp);
+    if (has_q) gq.values(zq);
+    float r = 0.f;
+    int cand = -1, lastv = -1;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const TokenVals v = token_vals(zp[e], has_q ? zq[e] : 0.f, has_q, scale, d);
+      const float val = use_p ? v.p : v.r;
+      const float nx = __fadd_rn(r, val);
+      if (val > 0.f) lastv = t0 + e;
+      if (!last_mode && cand < 0 && val > 0.f && r <= gin && gin < nx) cand = t0 + e;
+      r = nx;
+    }
+    token = cand >= 0 ? cand : lastv;
+  }
+  return __shfl_sync(0xffffffffu, token, 0);
 }
 
 // L2 prefetch of `bytes` bytes (a multiple of 16, 16-byte aligned) from global memory.
@@ -386,7 +550,7 @@ __global__ void __launch_bounds__(kThreads, 4) finish_sample_kernel(const Finish
       const int c = g * p.cpc + lc;
       if (c >= p.nch) break;
       float* pr = s_part + static_cast<size_t>(lc) * 2 * kGroups;
-      const float2 m = chunk_work<T, VEC>(p, b, c, d, lane, pr, pr + kGroups);
+      const float2 m = chunk_work<T, VEC>(p.rs, p.scale, b, c, d, lane, pr, pr + kGroups);
       if (lane < G) cluster.map_shared_rank(s_mass, lane)[c] = m;
     }
   }
@@ -399,80 +563,23 @@ __global__ void __launch_bounds__(kThreads, 4) finish_sample_kernel(const Finish
 
   // ---- which chunk holds the draw (every CTA, the same float64 arithmetic on the same masses)
   const int j = d.j;
-  constexpr int NPL = kMaxChunkCount / 32;
   if (wi == 0) {
-    int status = d.status;
-    bool use_p = j == K;
-    double mr[NPL], mp[NPL];
-    double zr = 0.0, zpm = 0.0;
+    float2 ms[kMassPerLane];
 #pragma unroll
-    for (int k = 0; k < NPL; ++k) {
-      const int c = lane * NPL + k;
-      const float2 m = c < p.nch ? s_mass[c] : make_float2(0.f, 0.f);
-      mr[k] = m.x;
-      mp[k] = m.y;
-      zr += mr[k];
-      zpm += mp[k];
+    for (int k = 0; k < kMassPerLane; ++k) {
+      const int c = lane * kMassPerLane + k;
+      ms[k] = c < p.nch ? s_mass[c] : make_float2(0.f, 0.f);
     }
-    double Zr = zr, Zp = zpm;  // inclusive prefixes over lanes
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const double a = __shfl_up_sync(0xffffffffu, Zr, o), c2 = __shfl_up_sync(0xffffffffu, Zp, o);
-      if (lane >= o) {
-        Zr += a;
-        Zp += c2;
-      }
-    }
-    const double Zres = __shfl_sync(0xffffffffu, Zr, 31);
-    if (!use_p && !(Zres > 0.0)) {  // residual mass rounded to zero: draw from p_j instead
-      use_p = true;
-      status |= DSPARK_SEQ_ZERO_RESIDUAL;
-    }
-    double m[NPL];
-#pragma unroll
-    for (int k = 0; k < NPL; ++k) m[k] = use_p ? mp[k] : mr[k];
-    const double incl = use_p ? Zp : Zr;
-    const double ls = use_p ? zpm : zr;
-    const double Z = __shfl_sync(0xffffffffu, incl, 31);
-    const double target = static_cast<double>(s_u[K]) * Z;
-    double run = incl - ls;
-    int cfound = -1, clast = -1;
-    double before = 0.0;
-#pragma unroll
-    for (int k = 0; k < NPL; ++k) {
-      const double nxt = run + m[k];
-      if (m[k] > 0.0) {
-        clast = lane * NPL + k;
-        if (cfound < 0 && run <= target && target < nxt) {
-          cfound = clast;
-          before = run;
-        }
-      }
-      run = nxt;
-    }
-    const unsigned hit = __ballot_sync(0xffffffffu, cfound >= 0);
-    int c;
-    double tin;
-    if (hit) {
-      const int hl = __ffs(hit) - 1;
-      c = __shfl_sync(0xffffffffu, cfound, hl);
-      tin = target - __shfl_sync(0xffffffffu, before, hl);
-    } else {  // rounding left the target past the last mass: the last token with mass
-      int cl = clast;
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) cl = max(cl, __shfl_xor_sync(0xffffffffu, cl, o));
-      c = cl;
-      tin = __int_as_float(0x7f800000);
-    }
-    const int owner = c >= 0 ? c / p.cpc : 0;
+    const ChunkPick pk = pick_chunk(ms, j == K, s_u[K], d.status, lane);
+    const int owner = pk.c >= 0 ? pk.c / p.cpc : 0;
     if (lane == 0) {
-      s_chunk = owner == g ? c : -2;  // -2: another CTA draws
-      s_use_p = use_p;
-      s_tin = tin;
+      s_chunk = owner == g ? pk.c : -2;  // -2: another CTA draws
+      s_use_p = pk.use_p;
+      s_tin = pk.tin;
       if (owner == g) {
         if (p.out.resid_mass)
-          p.out.resid_mass[b] = j < K ? (use_p ? 0.f : static_cast<float>(Zres)) : 1.f;
-        if (p.out.status) p.out.status[b] = status;
+          p.out.resid_mass[b] = j < K ? (pk.use_p ? 0.f : static_cast<float>(pk.zres)) : 1.f;
+        if (p.out.status) p.out.status[b] = pk.status;
       }
     }
   }
@@ -482,84 +589,12 @@ __global__ void __launch_bounds__(kThreads, 4) finish_sample_kernel(const Finish
   if (wi != 0) return;
   int token = -1;
   if (c >= 0) {
-    // the group holding the target: lane l scans the chunk's groups 8l .. 8l+7 (token order)
     const bool use_p = s_use_p != 0;
-    const float tin = static_cast<float>(s_tin);
     const float* part = s_part + static_cast<size_t>(c - g * p.cpc) * 2 * kGroups +
                         (use_p ? kGroups : 0);
-    float gv[8];
-    float lsum = 0.f;
-    int lastg = -1;
-#pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      gv[e] = part[lane * 8 + e];
-      lsum = __fadd_rn(lsum, gv[e]);
-      if (gv[e] > 0.f) lastg = lane * 8 + e;
-    }
-    float inc = lsum;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const float y = __shfl_up_sync(0xffffffffu, inc, o);
-      if (lane >= o) inc = __fadd_rn(inc, y);
-    }
-    float ex = __shfl_up_sync(0xffffffffu, inc, 1);
-    if (lane == 0) ex = 0.f;
-    int qsel = -1;
-    float gin = 0.f;
-    if (ex <= tin && tin < inc) {
-      float r = ex;
-#pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        const float nx = __fadd_rn(r, gv[e]);
-        if (qsel < 0 && gv[e] > 0.f && r <= tin && tin < nx) {
-          qsel = lane * 8 + e;
-          gin = __fsub_rn(tin, r);
-        }
-        r = nx;
-      }
-    }
-    const unsigned h = __ballot_sync(0xffffffffu, qsel >= 0);
-    bool last_mode = false;
-    if (h) {
-      const int hl = __ffs(h) - 1;
-      qsel = __shfl_sync(0xffffffffu, qsel, hl);
-      gin = __shfl_sync(0xffffffffu, gin, hl);
-    } else {  // rounding: the chunk's last group with mass, its last token with mass
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) lastg = max(lastg, __shfl_xor_sync(0xffffffffu, lastg, o));
-      qsel = lastg;
-      last_mode = true;
-    }
-    if (qsel >= 0) {
-      // the group's 8 tokens, recomputed exactly as their sum was; lane 0 scans them
-      if (lane == 0) {
-        const int K_ = p.rs.K;
-        const bool has_q = j < K_;
-        const T* pr = row_ptr<T>(p.rs, b, j);
-        const T* qr = has_q ? row_ptr<T>(p.rs, b, K_ + 1 + j) : pr;
-        const int t0 = c * kCE + qsel * 8;
-        GroupRaw<T, VEC> gp, gq;
-        gp.load(pr, t0, V);
-        if (has_q) gq.load(qr, t0, V);
-        float zp[8], zq[8];
-        gp.values(zp);
-        if (has_q) gq.values(zq);
-        float r = 0.f;
-        int cand = -1, lastv = -1;
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          const TokenVals v = token_vals(zp[e], has_q ? zq[e] : 0.f, has_q, p.scale, d);
-          const float val = use_p ? v.p : v.r;
-          const float nx = __fadd_rn(r, val);
-          if (val > 0.f) lastv = t0 + e;
-          if (!last_mode && cand < 0 && val > 0.f && r <= gin && gin < nx) cand = t0 + e;
-          r = nx;
-        }
-        token = cand >= 0 ? cand : lastv;
-      }
-    }
+    token = pick_token<T, VEC>(p.rs, p.scale, b, d, c, use_p, static_cast<float>(s_tin), part,
+                               lane);
   }
-  token = __shfl_sync(0xffffffffu, token, 0);
   write_tokens(p, b, j, token, s_x, lane, 32);
 }
 

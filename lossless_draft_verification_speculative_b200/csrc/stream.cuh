@@ -1,9 +1,9 @@
 // Pass 1 of the verify step: every logit row of the block is read from HBM exactly once.
 //
 // The work is split into units (row, chunk): chunk c of a row is its tokens
-// [2048c, min(V, 2048(c+1))). Units are numbered sequence-major (sequence b: P rows 0..K,
-// then for the sampling policy Q rows 0..K-1; within a row, chunks in order); each SM's CTA
-// owns every grid-th unit and hands them to its warps in order. A warp streams a unit with
+// [2048c, min(V, 2048(c+1))). Units are numbered row-major across the batch: a row slot
+// (below), then the sequence, then the chunk; each SM's CTA owns every grid-th unit and hands
+// them to its warps in order. A warp streams a unit with
 // 16-byte
 // loads, several in flight per lane, keeps per-lane running statistics, merges its lanes and
 // writes one record for the unit. A record is a function of the unit's logits alone (not of
@@ -68,8 +68,9 @@ struct StreamParams {
   RowSet rs;
   uint32_t n_units;   // B * rows * nch (< 2^32)
   int nch;            // chunks per row
+  int B;              // sequences
   FastDiv by_nch;     // division by nch
-  FastDiv by_rows;    // division by rows
+  FastDiv by_seqs;    // division by B
 
   float scale;        // log2(e) / T (sampling)
   float2* rec;        // [n_units]: record of unit u at u
@@ -81,6 +82,35 @@ struct StreamParams {
 struct UnitPos {
   int b, i, c;
 };
+
+// Unit u: chunk c = u mod nch, sequence b = (u / nch) mod B, row slot r = u / (nch B). The
+// slots take every sequence's rows in the order P_K (the bonus row), then for i = K-1 down to
+// 0: P_i, then Q_i when sampling. The rows read last, still in L2 when pass 2 re-reads the row
+// pair of a rejection at j, are then the low ones, where rejections concentrate (each draft
+// is accepted with probability below one, so j = 0 is the most likely single outcome).
+__device__ __forceinline__ UnitPos unit_pos(const StreamParams& p, uint32_t u) {
+  UnitPos at;
+  const uint32_t q = p.by_nch.div(u);
+  at.c = static_cast<int>(u - q * static_cast<uint32_t>(p.nch));
+  const uint32_t r = p.by_seqs.div(q);
+  at.b = static_cast<int>(q - r * static_cast<uint32_t>(p.B));
+  const int K = p.rs.K;
+  if (r == 0) {
+    at.i = K;
+  } else if (p.rs.rows == K + 1) {  // greedy: P rows only
+    at.i = K - static_cast<int>(r);
+  } else {
+    const int t = static_cast<int>(r) - 1;
+    const int pair = K - 1 - (t >> 1);
+    at.i = (t & 1) ? K + 1 + pair : pair;
+  }
+  return at;
+}
+
+// Index of a unit's record: rows of a sequence together, chunks in order within a row.
+__device__ __forceinline__ size_t record_index(const StreamParams& p, const UnitPos& at) {
+  return (static_cast<size_t>(at.b) * p.rs.rows + at.i) * p.nch + at.c;
+}
 
 // Sampling: the unit that holds a draft token x_i of a draft row (P row i < K, or Q row i)
 // also writes that token's logit for pass 2, so pass 2 need not fetch it from HBM.
@@ -339,8 +369,8 @@ __device__ __forceinline__ float2 piece_argmax(const T* row, long long o0, long 
 // warp works on the current one, so the atomic's latency is hidden, and the warps that the SM's
 // scheduler favours simply take more units. Every SM holds the same share of the work and its
 // warps finish together; no global atomic, fence or barrier is involved. The whole grid sweeps
-// the units front to back, so the rows read last, still in L2 when pass 2 re-reads a row pair,
-// are those of the last sequences.
+// the units front to back, so the rows read last (row pair 0 of every sequence) are the ones
+// still in L2 when pass 2 runs.
 template <typename T, int VEC, bool kSample>
 __global__ void __launch_bounds__(kStreamThreads, 1) stream_stats_kernel(const StreamParams p) {
   __shared__ unsigned s_next;
@@ -358,11 +388,7 @@ __global__ void __launch_bounds__(kStreamThreads, 1) stream_stats_kernel(const S
   while (m < n_mine) {
     if (lane == 0) nxt = atomicAdd(&s_next, 1u);
     const unsigned u = k + m * G;
-    UnitPos at;
-    const uint32_t r = p.by_nch.div(u);
-    at.c = static_cast<int>(u - r * static_cast<uint32_t>(p.nch));
-    at.b = static_cast<int>(p.by_rows.div(r));
-    at.i = static_cast<int>(r - static_cast<uint32_t>(at.b) * static_cast<uint32_t>(p.rs.rows));
+    const UnitPos at = unit_pos(p, u);
     const T* row = row_ptr<T>(p.rs, at.b, at.i);
     const int o0 = at.c * kCE;
     const int o1 = min(V, o0 + kCE);
@@ -374,7 +400,7 @@ __global__ void __launch_bounds__(kStreamThreads, 1) stream_stats_kernel(const S
     } else {
       rec = piece_argmax<T, VEC>(row, o0, o1, lane);
     }
-    if (lane == 0) p.rec[u] = rec;
+    if (lane == 0) p.rec[record_index(p, at)] = rec;
     m = __shfl_sync(0xffffffffu, nxt, 0);
   }
 }
