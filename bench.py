@@ -43,8 +43,8 @@ def parse_args():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="dsv4_flash_serving")
     ap.add_argument("--e2e-steps", type=int, default=5)
-    ap.add_argument("--cpu-steps", type=int, default=2,
-                    help="full steps of the oracle timed for the CPU baseline")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0,
+                    help="seconds of oracle work timed for the CPU baseline (whole steps)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     return ap.parse_args()
@@ -171,37 +171,40 @@ def run_reference(args, w):
     from oracle import accept_ref as ora
 
     calls = build_calls(w)
-    nseq = 4  # sequences per call per step: a bounded sample of the batch
-    seqs = list(range(nseq))
-    P, Q = wl.logits(w, seqs)
+    # a step is one verified block: one sequence through one call, cycling through the
+    # workload's temperatures and a pool of its sequences, so that any --steps ends in
+    # minutes (about 12 ms of float64 work per block)
+    pool = list(range(min(8, w.B)))
+    P, Q = wl.logits(w, pool)
     Pf, Qf = wl.as_float64(P, w.dtype), wl.as_float64(Q, w.dtype)
-    inputs = [(T, wl.drafts(w, Q, T, seqs), wl.uniforms(w, seqs, T=T).astype(np.float64))
+    inputs = [(T, wl.drafts(w, Q, T, pool), wl.uniforms(w, pool, T=T).astype(np.float64))
               for _, T in calls]
 
-    def step():
-        for T, d, u in inputs:
-            if T == 0:
-                ora.greedy_accept(Pf, d)
-            else:
-                ora.speculative_sample_accept(Pf, Qf, d, T, u)
+    def step(s):
+        T, d, u = inputs[s % len(calls)]
+        b = (s // len(calls)) % len(pool)
+        if T == 0:
+            ora.greedy_accept(Pf[b:b + 1], d[b:b + 1])
+        else:
+            ora.speculative_sample_accept(Pf[b:b + 1], Qf[b:b + 1], d[b:b + 1], T, u[b:b + 1])
 
-    for _ in range(args.warmup):
-        step()
+    for s in range(args.warmup):
+        step(s)
     t0 = time.perf_counter()
-    for _ in range(args.steps):
-        step()
+    for s in range(args.steps):
+        step(s)
     dt = time.perf_counter() - t0
-    blocks = args.steps * len(calls) * nseq
-    value = blocks / dt
-    sample = (f"{nseq} of {w.B} sequences per call, {len(calls)} calls (T={list(w.temperatures)}) "
-              f"per step, float64 NumPy, one process")
+    value = args.steps / dt
+    sample = (f"one block per step: sequence s//{len(calls)} mod {len(pool)} of the first "
+              f"{len(pool)} of {w.B}, call s mod {len(calls)} (T={list(w.temperatures)}); "
+              f"float64 NumPy, one process")
     print(json.dumps({
         "impl": "reference", "metric": METRIC, "value": value, "unit": "blocks/s",
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": dt * 1000 / args.steps, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": w.name, "B": w.B, "K": w.K, "V": w.V,
-                   "temperatures": list(w.temperatures), "sampled_sequences": nseq},
+                   "temperatures": list(w.temperatures), "blocks_per_step": 1},
         "cpu_baseline": {"value": value, "unit": "blocks/s", "cores": 1, "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": value, "unit": "blocks/s", "h2d_bytes_per_step": 0,
@@ -209,8 +212,9 @@ def run_reference(args, w):
     }), flush=True)
 
 
-def cpu_baseline(w, steps):
-    """The oracle timed on the host on `steps` full steps of sequence samples (1 core)."""
+def cpu_baseline(w, seconds):
+    """The oracle timed on the host (1 core): steps of 8 sequences through every call of the
+    workload, repeated until about `seconds` of work have run."""
     from lossless_draft_verification_speculative_b200 import workloads as wl
     from oracle import accept_ref as ora
 
@@ -222,13 +226,15 @@ def cpu_baseline(w, steps):
     inputs = [(T, wl.drafts(w, Q, T, seqs), wl.uniforms(w, seqs, T=T).astype(np.float64))
               for _, T in calls]
     t0 = time.perf_counter()
-    for _ in range(steps):
+    steps, dt = 0, 0.0
+    while steps == 0 or dt < seconds:
         for T, d, u in inputs:
             if T == 0:
                 ora.greedy_accept(Pf, d)
             else:
                 ora.speculative_sample_accept(Pf, Qf, d, T, u)
-    dt = time.perf_counter() - t0
+        steps += 1
+        dt = time.perf_counter() - t0
     blocks = steps * len(calls) * nseq
     return {"value": blocks / dt, "unit": "blocks/s", "cores": 1, "kind": "oracle",
             "sample": f"{steps} x {len(calls)} calls x {nseq} of {w.B} sequences "
@@ -397,7 +403,7 @@ def run_ours(args, w):
     if e2e:
         line["e2e"] = e2e
     if world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(w, args.cpu_steps)
+        line["cpu_baseline"] = cpu_baseline(w, args.cpu_seconds)
     print(json.dumps(line), flush=True)
 
 

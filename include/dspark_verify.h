@@ -105,10 +105,10 @@ size_t dspark_workspace_zero_bytes(int B, int K);
  * Returns DSPARK_OK and fills the fields, or an error for an invalid / unsupported shape.
  * `aligned16` says whether every row start will be 16-byte aligned (vector path).
  * A call runs two kernels on `stream`. Pass 1 reads every logit row once: its units are the
- * (row, chunk) pairs; each SM's CTA owns an equal contiguous range of them, hands them to its
- * warps in order, and each unit gets one statistics record. Pass 2, a programmatic dependent launch, takes
- * the per-sequence decisions and, when sampling, computes the draw's law chunk by chunk and
- * draws the token. */
+ * (row, chunk) pairs, numbered row-major across the batch; the CTA on each SM takes every
+ * grid-th unit and hands them to its warps in order, and each unit gets one statistics
+ * record. Pass 2, a programmatic dependent launch, takes the per-sequence decisions and, when
+ * sampling, computes the draw's law chunk by chunk and draws the token. */
 typedef struct {
   int elems_per_load;              /* 8 (bf16) / 4 (fp32) on the 16-byte path, 1 on the scalar path */
   int loads_in_flight;             /* loads each lane of pass 1 keeps in flight                    */
