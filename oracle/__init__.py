@@ -6,6 +6,7 @@ arm may import this package. It shares no code with the CUDA path.
 
 from .accept_ref import (  # noqa: F401
     STATUS_BAD_DRAFT,
+    STATUS_BAD_PARAM,
     STATUS_NONFINITE,
     STATUS_ZERO_RESIDUAL,
     OracleResult,
@@ -13,6 +14,7 @@ from .accept_ref import (  # noqa: F401
     draw_law,
     greedy_accept,
     inverse_cdf,
+    mixed_accept,
     row_argmax,
     softmax,
     speculative_sample_accept,

@@ -33,6 +33,16 @@ Readings where the pages are silent (each restated in the design notes):
   rounding) falls back to p_j; a draft id outside [0, V) or a row holding NaN or +inf,
   or no finite value at all, makes the whole sequence an error (n = 0, tokens -1).
 
+Mixed serving batches (``mixed_accept``). The mlx-dspark README ("Tuning") truncates the
+block per step through the drafter's confidence head (``--confidence-threshold``) or caps
+it (``--max-draft``), and the ds4 fork the DeepSeek-V4-Flash drafter card names serves
+batches. So each sequence b of a batch may carry its own draft count K_b <= K and its
+own temperature T_b (T_b == 0: greedy). Reading: sequence b is the single-policy step on
+its own truncated block, P rows 0..K_b (row K_b is its bonus row), Q rows 0..K_b-1, drafts
+0..K_b-1 and uniforms u[b, 0..K_b] (u[b, K_b] is its draw); rows, drafts and uniforms past
+those are never read. A draft count outside [0, K] or a negative or non-finite
+temperature makes that sequence an error (STATUS_BAD_PARAM).
+
 Parity pins: every function here is pinned in ``tests/test_oracle_pins.py`` against
 things other than itself (exact enumeration of losslessness, sequential greedy
 decoding, library inverse-CDF draws, closed-form acceptance rates, chi-square).
@@ -48,6 +58,7 @@ import numpy as np
 STATUS_BAD_DRAFT = 1      # a draft id outside [0, V)
 STATUS_NONFINITE = 2      # a row with NaN / +inf, or with no finite value
 STATUS_ZERO_RESIDUAL = 4  # residual mass was 0 after a rejection; drew from p_j instead
+STATUS_BAD_PARAM = 16     # mixed batch: a draft count outside [0, K] or a bad temperature
 
 
 @dataclass
@@ -254,3 +265,55 @@ def speculative_sample_accept(P: np.ndarray, Q: np.ndarray, drafts: np.ndarray, 
         nxt[b] = v
     return OracleResult(n, tokens, nxt, status, p_draft=pd, q_draft=qd, resid_mass=zm,
                         accept_margin=am, cdf_margin=cm)
+
+
+def mixed_accept(P: np.ndarray, Q: Optional[np.ndarray], drafts: np.ndarray,
+                 n_drafts: Optional[np.ndarray], temperatures: np.ndarray,
+                 u: Optional[np.ndarray]) -> OracleResult:
+    """Mixed serving batch: sequence b verifies its first K_b = n_drafts[b] drafts at its
+    own temperature T_b = temperatures[b] (0: greedy).
+
+    P: [B, K+1, V], Q: [B, K, V] (may be None when every T_b is 0), drafts [B, K],
+    n_drafts [B] or None (every K_b = K), temperatures [B], u: [B, K+1] (may be None when
+    every T_b is 0). Sequence b is ``greedy_accept`` or ``speculative_sample_accept`` on
+    P[b, :K_b+1], Q[b, :K_b], drafts[b, :K_b], u[b, :K_b+1]; results are laid out as for K
+    (tokens [B, K+1], -1 past the drawn token; p_draft / q_draft NaN past K_b).
+    """
+    P = np.asarray(P, dtype=np.float64)
+    drafts = np.asarray(drafts)
+    temperatures = np.asarray(temperatures, dtype=np.float64)
+    B, K1, V = P.shape
+    K = K1 - 1
+    nd = np.full(B, K, dtype=np.int64) if n_drafts is None else np.asarray(n_drafts)
+    n = np.zeros(B, dtype=np.int32)
+    tokens = np.full((B, K + 1), -1, dtype=np.int32)
+    nxt = np.full(B, -1, dtype=np.int32)
+    status = np.zeros(B, dtype=np.int32)
+    pd = np.full((B, K), np.nan)
+    qd = np.full((B, K), np.nan)
+    zm = np.full(B, np.nan)
+    am = np.full((B, K), np.inf)
+    cm = np.full(B, np.inf)
+    amax = np.full((B, K + 1), -1, dtype=np.int32)
+    for b in range(B):
+        kb, tb = int(nd[b]), float(temperatures[b])
+        if not (0 <= kb <= K) or not (np.isfinite(tb) and tb >= 0):
+            status[b] = STATUS_BAD_PARAM
+            continue
+        Pb = P[b:b + 1, :kb + 1]
+        db = drafts[b:b + 1, :kb]
+        if tb == 0:
+            r = greedy_accept(Pb, db)
+            amax[b, :kb + 1] = r.argmax[0]
+        else:
+            Qb = np.asarray(Q, dtype=np.float64)[b:b + 1, :kb]
+            ub = np.asarray(u, dtype=np.float64)[b:b + 1, :kb + 1]
+            r = speculative_sample_accept(Pb, Qb, db, tb, ub)
+            pd[b, :kb], qd[b, :kb] = r.p_draft[0], r.q_draft[0]
+            zm[b] = r.resid_mass[0]
+            am[b, :kb] = r.accept_margin[0]
+            cm[b] = r.cdf_margin[0]
+        n[b], nxt[b], status[b] = r.n_accepted[0], r.next_token[0], r.status[0]
+        tokens[b, :kb + 1] = r.tokens[0]
+    return OracleResult(n, tokens, nxt, status, p_draft=pd, q_draft=qd, resid_mass=zm,
+                        accept_margin=am, cdf_margin=cm, argmax=amax)
