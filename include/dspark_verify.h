@@ -44,7 +44,8 @@
  *  - Data errors are reported per sequence on the device, never by a trap: a draft id outside
  *    [0, V), or a row holding NaN or +inf or no finite value, makes that sequence's result
  *    n_accepted = 0, tokens all -1, next_token = -1, with the cause in status[b].
- *  - Limits: 0 <= K <= 32; 1 <= V <= 262144; B * (2K+1) < 2^31.
+ *  - Limits: 0 <= K <= 32; 1 <= V <= 262144; B * (2K+1) < 2^31; row strides ld_p1, ld_pv
+ *    below 2^31 elements (larger ones: DSPARK_ERR_UNSUPPORTED).
  *  - Calls that share a workspace must not overlap on the GPU (same stream, or ordered).
  */
 #ifndef DSPARK_VERIFY_H
@@ -73,6 +74,9 @@ typedef enum { DSPARK_BF16 = 0, DSPARK_F32 = 1 } dspark_dtype_t;
 #define DSPARK_SEQ_ZERO_RESIDUAL 4 /* not an error: residual mass rounded to 0 after a
                                       rejection; the correction was drawn from p_j          */
 #define DSPARK_SEQ_TIMEOUT 8       /* reserved: the kernels have no waits that can give up  */
+#define DSPARK_SEQ_BAD_PARAM 16    /* dspark_mixed_accept: a draft count outside [0, K], or a
+                                      negative or non-finite temperature (or one so small that
+                                      log2(e)/T overflows)                                    */
 
 /* AcceptResult: device buffers, caller-allocated. Required: n_accepted, tokens, next_token.
  * The optional ones (NULL = not written) are diagnostics of the sampling policy. */
@@ -151,6 +155,30 @@ dspark_status_t dspark_speculative_sample_accept(const void* p1, int64_t ld_p1, 
                                                  const float* uniforms, dspark_accept_out_t out,
                                                  void* workspace, size_t workspace_bytes,
                                                  void* stream);
+
+/* A mixed serving batch: each sequence verifies its own number of drafts at its own
+ * temperature, greedy where that temperature is 0. The pages truncate a block per step
+ * through the drafter's confidence head or cap it (mlx-dspark README, "Tuning":
+ * --confidence-threshold, --max-draft), and serve batches (the ds4 batched-serving fork the
+ * DeepSeek-V4-Flash DSpark drafter card names); this is the verify step of such a batch.
+ *  p1, ld_p1, pv, ld_pv, q, drafts as for speculative_sample_accept, for the batch's largest
+ *            block K (q is required when K > 0, even if every sequence is greedy).
+ *  n_drafts  [B] int32 K_b in [0, K], or NULL for K everywhere.
+ *  temperatures [B] float32 T_b: > 0 samples at T_b, == 0 verifies greedily.
+ *  uniforms  [B, K+1] float32 in [0, 1): u[b, i] (i < K_b) tests draft i, u[b, K_b] is the draw.
+ *  Sequence b is the single-policy step on its own block: P rows 0..K_b (row K_b is its
+ *  bonus row), Q rows 0..K_b-1, drafts 0..K_b-1. Rows, drafts and uniforms past those are
+ *  never read (the stream skips the rows: they cost no bandwidth) and may hold anything.
+ *  Results are laid out for K: tokens [B, K+1] with -1 after the drawn token; n_accepted in
+ *  [0, K_b]; p_draft / q_draft / resid_mass are written for sampling sequences only (entries
+ *  past K_b NaN). A K_b outside [0, K] or a bad T_b makes that sequence an error
+ *  (DSPARK_SEQ_BAD_PARAM: n = 0, tokens -1, next -1). */
+dspark_status_t dspark_mixed_accept(const void* p1, int64_t ld_p1, const void* pv, int64_t ld_pv,
+                                    const void* q, dspark_dtype_t dtype, const int32_t* drafts,
+                                    const int32_t* n_drafts, int B, int K, int V,
+                                    const float* temperatures, const float* uniforms,
+                                    dspark_accept_out_t out, void* workspace,
+                                    size_t workspace_bytes, void* stream);
 
 /* speculative_sample_accept without a workspace argument. The pages have no counterpart of
  * this entry point: it exists for callers that cannot allocate device memory where they

@@ -1,13 +1,16 @@
 """DSpark block-draft verify/accept on B200 (sm_100a).
 
 ``greedy_accept`` and ``speculative_sample_accept`` verify a block of K drafted tokens per
-sequence against the base model's [B, K+1, V] logit block and return an ``AcceptResult``.
+sequence against the base model's [B, K+1, V] logit block and return an ``AcceptResult``;
+``mixed_accept`` verifies a serving batch whose sequences have their own draft counts and
+temperatures.
 The work runs in hand-written CUDA kernels behind a C ABI (``include/dspark_verify.h``);
 this package is the thin Python binding over it plus the seeded synthetic workloads.
 """
 
 from .binding import (  # noqa: F401
     SEQ_BAD_DRAFT,
+    SEQ_BAD_PARAM,
     SEQ_NONFINITE,
     SEQ_TIMEOUT,
     SEQ_ZERO_RESIDUAL,
@@ -15,6 +18,7 @@ from .binding import (  # noqa: F401
     DsparkError,
     greedy_accept,
     load_library,
+    mixed_accept,
     plan,
     speculative_sample_accept,
     speculative_sample_accept_static,
@@ -27,6 +31,7 @@ __all__ = [
     "greedy_accept",
     "speculative_sample_accept",
     "speculative_sample_accept_static",
+    "mixed_accept",
     "load_library",
     "plan",
     "workspace_bytes",
@@ -34,4 +39,5 @@ __all__ = [
     "SEQ_NONFINITE",
     "SEQ_ZERO_RESIDUAL",
     "SEQ_TIMEOUT",
+    "SEQ_BAD_PARAM",
 ]

@@ -34,6 +34,7 @@ SEQ_BAD_DRAFT = 1
 SEQ_NONFINITE = 2
 SEQ_ZERO_RESIDUAL = 4
 SEQ_TIMEOUT = 8
+SEQ_BAD_PARAM = 16
 
 
 class DsparkError(RuntimeError):
@@ -105,6 +106,9 @@ def load_library(build_if_missing: bool = True) -> ctypes.CDLL:
     lib.dspark_speculative_sample_accept.argtypes = [vp, i64, vp, i64, vp, i32, vp, i32, i32,
                                                      i32, ctypes.c_float, vp, AcceptOut, vp, sz,
                                                      vp]
+    lib.dspark_mixed_accept.restype = i32
+    lib.dspark_mixed_accept.argtypes = [vp, i64, vp, i64, vp, i32, vp, vp, i32, i32, i32, vp, vp,
+                                        AcceptOut, vp, sz, vp]
     lib.dspark_speculative_sample_accept_static.restype = i32
     lib.dspark_speculative_sample_accept_static.argtypes = [vp, i64, vp, i64, vp, i32, vp, i32,
                                                             i32, i32, ctypes.c_float, vp,
@@ -283,6 +287,50 @@ def speculative_sample_accept(P: Union[torch.Tensor, Tuple[torch.Tensor, torch.T
     return res
 
 
+def mixed_accept(P: Union[torch.Tensor, Tuple[torch.Tensor, torch.Tensor]],
+                 Q: Optional[torch.Tensor], drafts: torch.Tensor, temperatures: torch.Tensor,
+                 uniforms: torch.Tensor, *, n_drafts: Optional[torch.Tensor] = None,
+                 out: Optional[AcceptResult] = None,
+                 workspace: Optional[torch.Tensor] = None) -> AcceptResult:
+    """A mixed serving batch on the GPU: sequence b verifies its first n_drafts[b] drafts
+    (all K when ``n_drafts`` is None) at temperatures[b], greedily where that is 0.
+
+    ``temperatures`` is a float32 [B] tensor and ``n_drafts`` an int32 [B] tensor, both on
+    P's device; u[b, n_drafts[b]] is sequence b's draw. Rows, drafts and uniforms past a
+    sequence's count are never read. A bad count or temperature is reported per sequence
+    (SEQ_BAD_PARAM).
+    """
+    lib = load_library()
+    p1, pv, ld_p1, ld_pv = _split_block(P)
+    if not p1.is_cuda:
+        raise RuntimeError("mixed_accept runs on CUDA tensors only")
+    B, V = p1.shape
+    K = 0 if pv is None else pv.shape[1]
+    drafts = _check_drafts(drafts, B, K, p1.device)
+    if K > 0 and (Q is None or Q.shape != (B, K, V) or not Q.is_contiguous() or
+                  Q.dtype != p1.dtype):
+        raise ValueError("Q must be a contiguous [B, K, V] tensor of P's dtype")
+    if uniforms.dtype != torch.float32 or uniforms.shape != (B, K + 1) or \
+            not uniforms.is_contiguous() or uniforms.device != p1.device:
+        raise ValueError("uniforms must be a contiguous float32 [B, K+1] tensor on P's device")
+    if temperatures.dtype != torch.float32 or temperatures.shape != (B,) or \
+            not temperatures.is_contiguous() or temperatures.device != p1.device:
+        raise ValueError("temperatures must be a contiguous float32 [B] tensor on P's device")
+    if n_drafts is not None and (n_drafts.dtype != torch.int32 or n_drafts.shape != (B,) or
+                                 not n_drafts.is_contiguous() or n_drafts.device != p1.device):
+        raise ValueError("n_drafts must be a contiguous int32 [B] tensor on P's device")
+    res = out if out is not None else _alloc_result(B, K, p1.device, diagnostics=True)
+    nbytes = lib.dspark_workspace_bytes(B, K, V, DTYPE_CODES[p1.dtype])
+    ws = workspace if workspace is not None else _WS.get(p1.device, nbytes, B, K)
+    rc = lib.dspark_mixed_accept(
+        _ptr(p1), ld_p1, _ptr(pv), ld_pv, _ptr(Q), DTYPE_CODES[p1.dtype], _ptr(drafts),
+        _ptr(n_drafts), B, K, V, _ptr(temperatures), _ptr(uniforms), _out_struct(res), _ptr(ws),
+        ws.numel() * ws.element_size(), _stream_handle(p1.device))
+    if rc != DSPARK_OK:
+        raise DsparkError(rc, "dspark_mixed_accept")
+    return res
+
+
 def speculative_sample_accept_static(P: Union[torch.Tensor, Tuple[torch.Tensor, torch.Tensor]],
                                      Q: Optional[torch.Tensor], drafts: torch.Tensor,
                                      temperature: float, uniforms: torch.Tensor, *,
@@ -325,18 +373,23 @@ class PreparedCall:
     """
 
     def __init__(self, policy: str, P, Q, drafts, temperature, uniforms, out: AcceptResult,
-                 workspace: torch.Tensor):
+                 workspace: torch.Tensor, n_drafts: Optional[torch.Tensor] = None):
         self.lib = load_library()
         p1, pv, ld_p1, ld_pv = _split_block(P)
         B, V = p1.shape
         K = 0 if pv is None else pv.shape[1]
-        self.keep = (P, Q, drafts, uniforms, out, workspace, p1, pv)
+        self.keep = (P, Q, drafts, uniforms, out, workspace, p1, pv, temperature, n_drafts)
         dt = DTYPE_CODES[p1.dtype]
         stream = _stream_handle(p1.device)
         nbytes = workspace.numel() * workspace.element_size()
         if policy == "greedy":
             self.fn = self.lib.dspark_greedy_accept
             self.args = (_ptr(p1), ld_p1, _ptr(pv), ld_pv, dt, _ptr(drafts), B, K, V,
+                         _out_struct(out), _ptr(workspace), nbytes, stream)
+        elif policy == "mixed":  # temperature: float32 [B] tensor
+            self.fn = self.lib.dspark_mixed_accept
+            self.args = (_ptr(p1), ld_p1, _ptr(pv), ld_pv, _ptr(Q), dt, _ptr(drafts),
+                         _ptr(n_drafts), B, K, V, _ptr(temperature), _ptr(uniforms),
                          _out_struct(out), _ptr(workspace), nbytes, stream)
         else:
             self.fn = self.lib.dspark_speculative_sample_accept

@@ -1,5 +1,6 @@
 // C ABI of the DSpark block verify/accept step: argument checks, launch planning and the
 // two kernel launches of a call (pass 1 in stream.cuh, pass 2 in finish.cuh).
+#include <climits>
 #include <cmath>
 #include <cstdlib>
 #include <cstring>
@@ -54,9 +55,10 @@ bool make_plan(int V, dspark_dtype_t dt, bool aligned16, Plan* pl) {
 
 size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
-// Workspace: the pass-1 records, one float2 per (row, chunk) unit, then the draft tokens'
-// logits (sampling). Pass 1 writes every record, and the gather of every draft id in [0, V),
-// before pass 2 reads them, so the workspace needs no initialisation.
+// Workspace: the pass-1 records, one float2 per (row, chunk) unit of 2K+1 rows per sequence,
+// then the draft tokens' logits (sampling). Pass 1 writes every record, and the gather of
+// every draft id in [0, V), before pass 2 reads them, so the workspace needs no
+// initialisation.
 struct WsLayout {
   size_t rec, gather, total;
 };
@@ -78,8 +80,7 @@ FastDiv fast_div(uint32_t d) {
   const unsigned __int128 num = static_cast<unsigned __int128>(1) << (32 + s);
   const unsigned __int128 m = (num + d - 1) / d;
   f.m_lo = static_cast<uint32_t>(m & 0xffffffffu);
-  f.m_hi = static_cast<uint32_t>(m >> 32);
-  f.s = s;
+  f.hs = static_cast<uint32_t>(m >> 32) << 8 | s;
   return f;
 }
 
@@ -141,6 +142,8 @@ struct Call {
   int B;
   const int32_t* drafts;
   const float* uniforms;
+  const int32_t* n_drafts;  // mixed batch: [B] or null
+  const float* temps;       // mixed batch: [B]
   float scale;
   dspark_accept_out_t out;
   char* ws;
@@ -148,9 +151,10 @@ struct Call {
 
 // Pass 1 over every (row, chunk) unit (one wave of warps, equal contiguous runs of units),
 // then pass 2 launched as a programmatic dependent of it.
-template <typename T, int VEC, bool kSample>
+template <typename T, int VEC, int kMode>
 dspark_status_t run_call(const Call& c, const Plan& pl, cudaStream_t stream) {
-  const void* k1 = reinterpret_cast<const void*>(&stream_stats_kernel<T, VEC, kSample>);
+  constexpr bool kSample = kMode != kModeGreedy;
+  const void* k1 = reinterpret_cast<const void*>(&stream_stats_kernel<T, VEC, kMode>);
   cudaError_t e = cudaSuccess;
   int ctas = resident_ctas(k1, kStreamThreads, 0, &e);
   if (e != cudaSuccess) return DSPARK_ERR_CUDA;
@@ -162,10 +166,10 @@ dspark_status_t run_call(const Call& c, const Plan& pl, cudaStream_t stream) {
   const long long want = (n_units + kStreamWarps - 1) / kStreamWarps;
   const int grid1 = static_cast<int>(want < ctas ? want : ctas);
 
-  StreamParams sp{};
+  StreamParamsOf<kMode> sp{};
   sp.rs = c.rs;
-  sp.n_units = static_cast<uint32_t>(n_units);
   sp.nch = pl.nch;
+  sp.n_units = static_cast<uint32_t>(n_units);
   sp.B = c.B;
   sp.by_nch = fast_div(static_cast<uint32_t>(pl.nch));
   sp.by_seqs = fast_div(static_cast<uint32_t>(c.B));
@@ -173,21 +177,26 @@ dspark_status_t run_call(const Call& c, const Plan& pl, cudaStream_t stream) {
   sp.rec = reinterpret_cast<float2*>(c.ws + w.rec);
   sp.drafts = c.drafts;
   sp.gather = reinterpret_cast<float*>(c.ws + w.gather);
-  stream_stats_kernel<T, VEC, kSample><<<grid1, kStreamThreads, 0, stream>>>(sp);
+  if constexpr (kMode == kModeMixed) {
+    sp.n_drafts = c.n_drafts;
+    sp.temps = c.temps;
+  }
+  stream_stats_kernel<T, VEC, kMode><<<grid1, kStreamThreads, 0, stream>>>(sp);
   e = cudaGetLastError();
   if (e != cudaSuccess) return DSPARK_ERR_CUDA;
 
-  FinishParams fp{};
+  std::conditional_t<kMode == kModeMixed, FinishParamsMixed, FinishParams> fp{};
   fp.rs = c.rs;
   fp.drafts = c.drafts;
   fp.uniforms = c.uniforms;
-  fp.B = c.B;
-  fp.G = pl.G;
-  fp.cpc = pl.cpc;
   fp.nch = pl.nch;
   fp.scale = c.scale;
   fp.rec = sp.rec;
   fp.gather = sp.gather;
+  if constexpr (kMode == kModeMixed) {
+    fp.n_drafts = c.n_drafts;
+    fp.temps = c.temps;
+  }
   fp.out = c.out;
   cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -204,7 +213,7 @@ dspark_status_t run_call(const Call& c, const Plan& pl, cudaStream_t stream) {
   cfg.attrs = attr;
   cfg.numAttrs = kSample ? 2 : 1;
   if constexpr (kSample)
-    e = cudaLaunchKernelEx(&cfg, finish_sample_kernel<T, VEC>, fp);
+    e = cudaLaunchKernelEx(&cfg, finish_sample_kernel<T, VEC, kMode == kModeMixed>, fp);
   else
     e = cudaLaunchKernelEx(&cfg, finish_greedy_kernel<T>, fp);
   return e == cudaSuccess ? DSPARK_OK : DSPARK_ERR_CUDA;
@@ -224,6 +233,7 @@ dspark_status_t check_common(const void* p1, int64_t ld_p1, const void* pv, int6
   const size_t es = static_cast<size_t>(elem_bytes(dtype));
   if (!aligned(p1, es) || (K > 0 && !aligned(pv, es))) return DSPARK_ERR_UNSUPPORTED;
   if (V > kMaxChunkCount * kCE) return DSPARK_ERR_UNSUPPORTED;
+  if (ld_p1 > INT32_MAX || ld_pv > INT32_MAX) return DSPARK_ERR_UNSUPPORTED;  // 32-bit strides
   return DSPARK_OK;
 }
 
@@ -234,8 +244,8 @@ Call make_call(const void* p1, int64_t ld_p1, const void* pv, int64_t ld_pv, con
   c.rs.p1 = p1;
   c.rs.pv = pv;
   c.rs.q = q;
-  c.rs.ld_p1 = ld_p1;
-  c.rs.ld_pv = ld_pv;
+  c.rs.ld_p1 = static_cast<int32_t>(ld_p1);
+  c.rs.ld_pv = static_cast<int32_t>(ld_pv);
   c.rs.K = K;
   c.rs.V = V;
   c.rs.rows = rows;
@@ -345,8 +355,9 @@ dspark_status_t dspark_greedy_accept(const void* p1, int64_t ld_p1, const void* 
                            workspace, out);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (dtype == DSPARK_BF16)
-    return a16 ? run_call<bf16_t, 8, false>(c, pl, s) : run_call<bf16_t, 1, false>(c, pl, s);
-  return a16 ? run_call<float, 4, false>(c, pl, s) : run_call<float, 1, false>(c, pl, s);
+    return a16 ? run_call<bf16_t, 8, kModeGreedy>(c, pl, s)
+               : run_call<bf16_t, 1, kModeGreedy>(c, pl, s);
+  return a16 ? run_call<float, 4, kModeGreedy>(c, pl, s) : run_call<float, 1, kModeGreedy>(c, pl, s);
 }
 
 dspark_status_t dspark_speculative_sample_accept(const void* p1, int64_t ld_p1, const void* pv,
@@ -378,8 +389,38 @@ dspark_status_t dspark_speculative_sample_accept(const void* p1, int64_t ld_p1, 
                            workspace, out);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (dtype == DSPARK_BF16)
-    return a16 ? run_call<bf16_t, 8, true>(c, pl, s) : run_call<bf16_t, 1, true>(c, pl, s);
-  return a16 ? run_call<float, 4, true>(c, pl, s) : run_call<float, 1, true>(c, pl, s);
+    return a16 ? run_call<bf16_t, 8, kModeSample>(c, pl, s)
+               : run_call<bf16_t, 1, kModeSample>(c, pl, s);
+  return a16 ? run_call<float, 4, kModeSample>(c, pl, s) : run_call<float, 1, kModeSample>(c, pl, s);
+}
+
+dspark_status_t dspark_mixed_accept(const void* p1, int64_t ld_p1, const void* pv, int64_t ld_pv,
+                                    const void* q, dspark_dtype_t dtype, const int32_t* drafts,
+                                    const int32_t* n_drafts, int B, int K, int V,
+                                    const float* temperatures, const float* uniforms,
+                                    dspark_accept_out_t out, void* workspace,
+                                    size_t workspace_bytes, void* stream) {
+  dspark_status_t st = check_common(p1, ld_p1, pv, ld_pv, dtype, drafts, B, K, V, out);
+  if (st != DSPARK_OK || B == 0) return st;
+  if (!temperatures || !uniforms || (K > 0 && !q)) return DSPARK_ERR_INVALID_ARG;
+  const size_t es = static_cast<size_t>(elem_bytes(dtype));
+  if (K > 0 && !aligned(q, es)) return DSPARK_ERR_UNSUPPORTED;
+  const bool a16 = aligned(p1, 16) && (K == 0 || (aligned(pv, 16) && aligned(q, 16))) &&
+                   (ld_p1 * es) % 16 == 0 && (K == 0 || (ld_pv * es) % 16 == 0) &&
+                   (V * es) % 16 == 0;
+  Plan pl;
+  if (!make_plan(V, dtype, a16, &pl)) return DSPARK_ERR_UNSUPPORTED;
+  if (!workspace || workspace_bytes < ws_layout(B, K, pl.nch).total || !aligned(workspace, 256))
+    return DSPARK_ERR_WORKSPACE;
+  Call c = make_call(p1, ld_p1, pv, ld_pv, q, drafts, uniforms, B, K, V, 0.f, 2 * K + 1,
+                     workspace, out);
+  c.n_drafts = n_drafts;
+  c.temps = temperatures;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (dtype == DSPARK_BF16)
+    return a16 ? run_call<bf16_t, 8, kModeMixed>(c, pl, s)
+               : run_call<bf16_t, 1, kModeMixed>(c, pl, s);
+  return a16 ? run_call<float, 4, kModeMixed>(c, pl, s) : run_call<float, 1, kModeMixed>(c, pl, s);
 }
 
 dspark_status_t dspark_speculative_sample_accept_static(const void* p1, int64_t ld_p1,

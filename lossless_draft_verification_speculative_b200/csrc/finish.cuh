@@ -20,22 +20,29 @@
 
 namespace dspark {
 
-constexpr int kErrBits = DSPARK_SEQ_BAD_DRAFT | DSPARK_SEQ_NONFINITE | DSPARK_SEQ_TIMEOUT;
+constexpr int kErrBits =
+    DSPARK_SEQ_BAD_DRAFT | DSPARK_SEQ_NONFINITE | DSPARK_SEQ_TIMEOUT | DSPARK_SEQ_BAD_PARAM;
 constexpr int kMaxRows = 2 * kMaxK + 1;
 constexpr int kMaxFinishCluster = 8;  // CTAs per sampling cluster (portable size)
 
+// Kernel parameters (see StreamParamsMixed on their size). The sampling kernel's cluster size
+// G and chunks per CTA, ceil(n_chunks / G), come from its launch.
 struct FinishParams {
   RowSet rs;
   const int32_t* drafts;    // [B, K]
   const float* uniforms;    // [B, K+1] (sampling)
-  int B;
-  int G;                    // CTAs per sequence = cluster size (sampling)
-  int cpc;                  // chunks per CTA (sampling)
   int nch;                  // chunks per row
   float scale;              // log2(e) / T
   const float2* rec;        // pass-1 records [B * rows, nch]
   const float* gather;      // [B, K, 2]: P_i[x_i], Q_i[x_i] written by pass 1 (sampling)
   dspark_accept_out_t out;
+};
+
+// A mixed batch's per-sequence arrays, kept out of FinishParams for the reason given at
+// StreamParamsMixed.
+struct FinishParamsMixed : FinishParams {
+  const int32_t* n_drafts;  // [B] K_b, or null for K
+  const float* temps;       // [B] T_b
 };
 
 // The pass-1 records of one row, held by one warp: chunk lane + 32k. Missing ones are empty.
@@ -82,19 +89,24 @@ __device__ __forceinline__ float2 reduce_row(const RowRecs& rr) {
   }
 }
 
-// Rows 0..rows-1 of sequence b into s_stat: warp w merges rows w, w + 8, ..., two at a time
-// so that their loads overlap.
-template <bool kSample>
-__device__ __forceinline__ void merge_rows(const FinishParams& p, int b, int rows, int wi,
-                                           int lane, float2* s_stat) {
+// The rows of sequence b into s_stat (row r at s_stat[r]): all of them, or with kFiltered
+// those that `used` selects. Warp w merges rows w, w + 8, ..., two at a time so that their
+// loads overlap.
+template <bool kSample, bool kFiltered>
+__device__ __forceinline__ void merge_rows(const FinishParams& p, int b, const RowFilter& used,
+                                           int wi, int lane, float2* s_stat) {
+  const int rows = p.rs.rows;
   const long long r0 = static_cast<long long>(b) * rows;
   for (int r = wi; r < rows; r += 2 * kWarps) {
     RowRecs a, c;
-    load_row<kSample>(p, r0 + r, lane, a);
-    const bool two = r + kWarps < rows;
+    const bool one = !kFiltered || used(r);
+    const bool two = r + kWarps < rows && (!kFiltered || used(r + kWarps));
+    if (one) load_row<kSample>(p, r0 + r, lane, a);
     if (two) load_row<kSample>(p, r0 + r + kWarps, lane, c);
-    const float2 sa = reduce_row<kSample>(a);
-    if (lane == 0) s_stat[r] = sa;
+    if (one) {
+      const float2 sa = reduce_row<kSample>(a);
+      if (lane == 0) s_stat[r] = sa;
+    }
     if (two) {
       const float2 sc = reduce_row<kSample>(c);
       if (lane == 0) s_stat[r + kWarps] = sc;
@@ -133,34 +145,27 @@ __device__ __forceinline__ void write_tokens(const FinishParams& p, int b, int j
 
 // ------------------------------------------------------------------------------ greedy
 
-template <typename T>
-__global__ void __launch_bounds__(kThreads) finish_greedy_kernel(const FinishParams p) {
-  __shared__ float2 s_arg[kMaxK + 1];
-  __shared__ int s_x[kMaxK];
-  const int lane = threadIdx.x & 31, wi = threadIdx.x >> 5;
-  const int b = blockIdx.x;
-  const int K = p.rs.K, K1 = K + 1;
-  int x = 0;
-  if (wi == 0 && lane < K) {
-    x = p.drafts[static_cast<size_t>(b) * K + lane];
-    s_x[lane] = x;
-  }
-  grid_dependency_wait();
-  merge_rows<false>(p, b, K1, wi, lane, s_arg);
+// Greedy finish of sequence b with nd drafts (every thread of the CTA; its P rows 0..nd are
+// merged): x = drafts[b, lane] in warp 0's lanes below nd, already copied to s_x. kFiltered:
+// the records are laid out for sampling rows (a mixed batch) and rows past nd are skipped.
+template <bool kFiltered>
+__device__ __forceinline__ void greedy_finish(const FinishParams& p, int b, int nd, int x, int wi,
+                                              int lane, float2* s_arg, const int* s_x) {
+  merge_rows<false, kFiltered>(p, b, RowFilter{p.rs.K, nd, false}, wi, lane, s_arg);
   __syncthreads();
   if (wi != 0) return;
   const float ninf = -__int_as_float(0x7f800000);
   bool bad = false;
-  for (int r = lane; r < K1; r += 32) {
+  for (int r = lane; r <= nd; r += 32) {
     const float2 a = s_arg[r];
     // NaN anywhere, a +inf maximum, or nothing above -inf: not a usable row
     bad |= !(a.x > ninf) || !(a.x < -ninf) || __float_as_int(a.y) == INT_MAX;
   }
   int status = __any_sync(0xffffffffu, bad) ? DSPARK_SEQ_NONFINITE : 0;
-  if (__any_sync(0xffffffffu, lane < K && (x < 0 || x >= p.rs.V))) status |= DSPARK_SEQ_BAD_DRAFT;
-  const int arg = lane < K ? __float_as_int(s_arg[lane].y) : -1;
-  const unsigned mis = __ballot_sync(0xffffffffu, lane < K && x != arg);
-  const int j = mis ? __ffs(mis) - 1 : K;
+  if (__any_sync(0xffffffffu, lane < nd && (x < 0 || x >= p.rs.V))) status |= DSPARK_SEQ_BAD_DRAFT;
+  const int arg = lane < nd ? __float_as_int(s_arg[lane].y) : -1;
+  const unsigned mis = __ballot_sync(0xffffffffu, lane < nd && x != arg);
+  const int j = mis ? __ffs(mis) - 1 : nd;
   if (status & kErrBits) {
     write_error(p, b, status, lane, 32);
     return;
@@ -169,11 +174,28 @@ __global__ void __launch_bounds__(kThreads) finish_greedy_kernel(const FinishPar
   if (lane == 0 && p.out.status) p.out.status[b] = 0;
 }
 
+template <typename T>
+__global__ void __launch_bounds__(kThreads) finish_greedy_kernel(const FinishParams p) {
+  __shared__ float2 s_arg[kMaxK + 1];
+  __shared__ int s_x[kMaxK];
+  const int lane = threadIdx.x & 31, wi = threadIdx.x >> 5;
+  const int b = blockIdx.x;
+  const int K = p.rs.K;
+  int x = 0;
+  if (wi == 0 && lane < K) {
+    x = p.drafts[static_cast<size_t>(b) * K + lane];
+    s_x[lane] = x;
+  }
+  grid_dependency_wait();
+  greedy_finish<false>(p, b, K, x, wi, lane, s_arg, s_x);
+}
+
 // ---------------------------------------------------------------------------- sampling
 
 // The row normalisers of the draw's law, and the decision.
 struct Decision {
   int j;
+  int nd;  // the sequence's draft count: j < nd is a rejection, j == nd the bonus
   int status;
   float mp, ip;  // p_j (or p_K): reference and 1 / sum
   float mq, iq;  // q_j: reference and 1 / sum (iq = 0 for the bonus)
@@ -254,7 +276,7 @@ __device__ __forceinline__ float2 chunk_work(const RowSet& rs, float scale, int 
                                              const Decision& d, int lane, float* part_r,
                                              float* part_p) {
   const int K = rs.K, V = rs.V;
-  const bool has_q = d.j < K;
+  const bool has_q = d.j < d.nd;
   const T* pr = row_ptr<T>(rs, b, d.j);
   const T* qr = has_q ? row_ptr<T>(rs, b, K + 1 + d.j) : pr;
   constexpr int kPerLane = kGroups / 32;                      // groups per lane
@@ -419,7 +441,7 @@ __device__ __forceinline__ int pick_token(const RowSet& rs, float scale, int b, 
   int token = -1;
   if (qsel >= 0 && lane == 0) {
     const int K = rs.K, V = rs.V;
-    const bool has_q = j < K;
+    const bool has_q = j < d.nd;
     const T* pr = row_ptr<T>(rs, b, j);
     const T* qr = has_q ? row_ptr<T>(rs, b, K + 1 + j) : pr;
     const int t0 = c * kCE + qsel * 8;
@@ -452,8 +474,9 @@ __device__ __forceinline__ void prefetch_l2(const void* src, uint32_t bytes) {
 
 // Sampling finish. Launched as clusters of G CTAs, one cluster per sequence; CTA g of the
 // cluster owns chunks g*cpc .. g*cpc + cpc - 1 of the draw's law (warp w: local chunks w, w+8).
-template <typename T, int VEC>
-__global__ void __launch_bounds__(kThreads, 4) finish_sample_kernel(const FinishParams p) {
+template <typename T, int VEC, bool kMixed>
+__global__ void __launch_bounds__(kThreads, 4) finish_sample_kernel(
+    const std::conditional_t<kMixed, FinishParamsMixed, FinishParams> p) {
   extern __shared__ float s_part[];  // [cpc][2][kGroups]: group sums (residual, p)
   __shared__ float2 s_stat[kMaxRows];
   __shared__ float2 s_mass[kMaxChunkCount];  // every chunk's (residual, p) mass
@@ -464,18 +487,43 @@ __global__ void __launch_bounds__(kThreads, 4) finish_sample_kernel(const Finish
   __shared__ int s_chunk, s_use_p;
   cg::cluster_group cluster = cg::this_cluster();
   const int tid = threadIdx.x, lane = tid & 31, wi = tid >> 5;
-  const int G = p.G;
+  const int G = static_cast<int>(cluster.num_blocks());
+  const int cpc = (p.nch + G - 1) / G;  // chunks per CTA
   const int b = blockIdx.x / G;
   const int g = static_cast<int>(cluster.block_rank());
   const int K = p.rs.K, K1 = K + 1, V = p.rs.V, rows = p.rs.rows;
+  // the sequence's draft count nd and scale: K and the call's scale, or, in a mixed batch,
+  // its own (a greedy sequence takes the greedy finish in CTA 0; no cluster barrier follows)
+  int nd = K;
+  float scale = p.scale;
+  if constexpr (kMixed) {
+    const SeqMode sm = seq_mode(p.n_drafts, p.temps, b, K);
+    if (!sm.ok) {
+      if (g == 0) write_error(p, b, DSPARK_SEQ_BAD_PARAM, tid, kThreads);
+      return;
+    }
+    nd = sm.kb;
+    scale = sm.scale;
+    if (sm.greedy) {
+      if (g != 0) return;
+      int xg = 0;
+      if (tid < nd) {
+        xg = p.drafts[static_cast<size_t>(b) * K + tid];
+        s_x[tid] = xg;
+      }
+      grid_dependency_wait();
+      greedy_finish<true>(p, b, nd, xg, wi, lane, s_stat, s_x);
+      return;
+    }
+  }
 
   // inputs that pass 1 does not write: drafts, uniforms
   int x = -1;
-  if (tid < K) x = p.drafts[static_cast<size_t>(b) * K + tid];
-  if (tid <= K) s_u[tid] = p.uniforms[static_cast<size_t>(b) * K1 + tid];
+  if (tid < nd) x = p.drafts[static_cast<size_t>(b) * K + tid];
+  if (tid <= nd) s_u[tid] = p.uniforms[static_cast<size_t>(b) * K1 + tid];
   grid_dependency_wait();
   // the draft tokens' logits, gathered by pass 1
-  if (tid < K) {
+  if (tid < nd) {
     s_x[tid] = x;
     float2 zg = make_float2(0.f, 0.f);
     if (x >= 0 && x < V) zg = __ldcg(reinterpret_cast<const float2*>(p.gather) + static_cast<size_t>(b) * K + tid);
@@ -484,31 +532,32 @@ __global__ void __launch_bounds__(kThreads, 4) finish_sample_kernel(const Finish
   }
   __syncthreads();
 
-  // every row's (reference, sum)
-  merge_rows<true>(p, b, rows, wi, lane, s_stat);
+  // the (reference, sum) of every row the sequence uses
+  const RowFilter used{K, nd, true};
+  merge_rows<true, kMixed>(p, b, used, wi, lane, s_stat);
   __syncthreads();
 
   // decisions (warp 0; draft i on lane i)
   if (wi == 0) {
     int status = 0;
     bool bad = false;
-    for (int r = lane; r < rows; r += 32) bad |= !stat_ok(s_stat[r]);
+    for (int r = lane; r < rows; r += 32) bad |= (!kMixed || used(r)) && !stat_ok(s_stat[r]);
     if (__any_sync(0xffffffffu, bad)) status |= DSPARK_SEQ_NONFINITE;
-    const int x = lane < K ? s_x[lane] : 0;
-    const bool bad_draft = lane < K && (x < 0 || x >= V);
+    const int x = lane < nd ? s_x[lane] : 0;
+    const bool bad_draft = lane < nd && (x < 0 || x >= V);
     if (__any_sync(0xffffffffu, bad_draft)) status |= DSPARK_SEQ_BAD_DRAFT;
     const float fnan = __int_as_float(0x7fffffff);
     float px = fnan, qx = fnan;
     bool accept = false;
-    if (lane < K && !bad_draft) {
+    if (lane < nd && !bad_draft) {
       const float2 sp = s_stat[lane], sq = s_stat[K1 + lane];
       // p_i(x_i) = 2^(z*s - M) / S (division within 2 ulp: no IEEE slow path)
-      px = __fdividef(ex2(__fmaf_rn(s_zp[lane], p.scale, -sp.x)), sp.y);
-      qx = __fdividef(ex2(__fmaf_rn(s_zq[lane], p.scale, -sq.x)), sq.y);
+      px = __fdividef(ex2(__fmaf_rn(s_zp[lane], scale, -sp.x)), sp.y);
+      qx = __fdividef(ex2(__fmaf_rn(s_zq[lane], scale, -sq.x)), sq.y);
       accept = __fmul_rn(s_u[lane], qx) < px;
     }
-    const unsigned rej = __ballot_sync(0xffffffffu, lane < K && !accept);
-    const int j = rej ? __ffs(rej) - 1 : K;
+    const unsigned rej = __ballot_sync(0xffffffffu, lane < nd && !accept);
+    const int j = rej ? __ffs(rej) - 1 : nd;
     if (g == 0 && lane < K) {
       if (p.out.p_draft) p.out.p_draft[static_cast<size_t>(b) * K + lane] = px;
       if (p.out.q_draft) p.out.q_draft[static_cast<size_t>(b) * K + lane] = qx;
@@ -517,10 +566,11 @@ __global__ void __launch_bounds__(kThreads, 4) finish_sample_kernel(const Finish
       const float2 sp = s_stat[j];
       Decision d;
       d.j = j;
+      d.nd = nd;
       d.status = status;
       d.mp = sp.x;
       d.ip = __fdividef(1.f, sp.y);
-      if (j < K) {
+      if (j < nd) {
         const float2 sq = s_stat[K1 + j];
         d.mq = sq.x;
         d.iq = __fdividef(1.f, sq.y);
@@ -535,10 +585,10 @@ __global__ void __launch_bounds__(kThreads, 4) finish_sample_kernel(const Finish
   const Decision d = s_dec;
   // this CTA's chunk range of the draw's rows into L2, ahead of the warps' second loads
   if (VEC > 1 && lane == 0 && wi >= kWarps - 2 && !(d.status & kErrBits)) {
-    const int t0 = g * p.cpc * kCE;
-    const int t1 = min(V, t0 + p.cpc * kCE);
+    const int t0 = g * cpc * kCE;
+    const int t1 = min(V, t0 + cpc * kCE);
     const bool q_row = wi == kWarps - 1;
-    if (t0 < t1 && (!q_row || d.j < K)) {
+    if (t0 < t1 && (!q_row || d.j < d.nd)) {
       const uint32_t bytes = static_cast<uint32_t>(t1 - t0) * Elem<T>::kBytes;
       prefetch_l2(row_ptr<T>(p.rs, b, q_row ? K1 + d.j : d.j) + t0, bytes);
     }
@@ -546,11 +596,11 @@ __global__ void __launch_bounds__(kThreads, 4) finish_sample_kernel(const Finish
 
   // this CTA's chunks: group sums into shared memory, chunk masses to every CTA of the cluster
   if (!(d.status & kErrBits)) {
-    for (int lc = wi; lc < p.cpc; lc += kWarps) {
-      const int c = g * p.cpc + lc;
+    for (int lc = wi; lc < cpc; lc += kWarps) {
+      const int c = g * cpc + lc;
       if (c >= p.nch) break;
       float* pr = s_part + static_cast<size_t>(lc) * 2 * kGroups;
-      const float2 m = chunk_work<T, VEC>(p.rs, p.scale, b, c, d, lane, pr, pr + kGroups);
+      const float2 m = chunk_work<T, VEC>(p.rs, scale, b, c, d, lane, pr, pr + kGroups);
       if (lane < G) cluster.map_shared_rank(s_mass, lane)[c] = m;
     }
   }
@@ -570,15 +620,15 @@ __global__ void __launch_bounds__(kThreads, 4) finish_sample_kernel(const Finish
       const int c = lane * kMassPerLane + k;
       ms[k] = c < p.nch ? s_mass[c] : make_float2(0.f, 0.f);
     }
-    const ChunkPick pk = pick_chunk(ms, j == K, s_u[K], d.status, lane);
-    const int owner = pk.c >= 0 ? pk.c / p.cpc : 0;
+    const ChunkPick pk = pick_chunk(ms, j == nd, s_u[nd], d.status, lane);
+    const int owner = pk.c >= 0 ? pk.c / cpc : 0;
     if (lane == 0) {
       s_chunk = owner == g ? pk.c : -2;  // -2: another CTA draws
       s_use_p = pk.use_p;
       s_tin = pk.tin;
       if (owner == g) {
         if (p.out.resid_mass)
-          p.out.resid_mass[b] = j < K ? (pk.use_p ? 0.f : static_cast<float>(pk.zres)) : 1.f;
+          p.out.resid_mass[b] = j < nd ? (pk.use_p ? 0.f : static_cast<float>(pk.zres)) : 1.f;
         if (p.out.status) p.out.status[b] = pk.status;
       }
     }
@@ -590,9 +640,9 @@ __global__ void __launch_bounds__(kThreads, 4) finish_sample_kernel(const Finish
   int token = -1;
   if (c >= 0) {
     const bool use_p = s_use_p != 0;
-    const float* part = s_part + static_cast<size_t>(c - g * p.cpc) * 2 * kGroups +
+    const float* part = s_part + static_cast<size_t>(c - g * cpc) * 2 * kGroups +
                         (use_p ? kGroups : 0);
-    token = pick_token<T, VEC>(p.rs, p.scale, b, d, c, use_p, static_cast<float>(s_tin), part,
+    token = pick_token<T, VEC>(p.rs, scale, b, d, c, use_p, static_cast<float>(s_tin), part,
                                lane);
   }
   write_tokens(p, b, j, token, s_x, lane, 32);

@@ -14,9 +14,14 @@
 // - ref), the online-softmax pair (Milakov & Gimelshein 2018) in base 2; (-inf, 0) for a
 // chunk with no value above -inf; a NaN or +inf anywhere makes the pair non-finite. Greedy:
 // (max, lowest token index of the max) on the raw logits (order is unchanged by 1/T > 0).
+// A mixed batch gives each sequence its own draft count K_b and temperature T_b: its units
+// of rows it does not use (P rows past K_b, Q rows past its drafts, every Q row when T_b is
+// 0) are skipped without a read, and its records are argmax records when T_b is 0, softmax
+// records at scale log2(e) / T_b otherwise.
 #pragma once
 
 #include <climits>
+#include <type_traits>
 
 #include "common.cuh"
 
@@ -30,14 +35,19 @@ constexpr int kBatchVecs = 8;            // loads each lane keeps in flight
 constexpr int kCE = 2048;                // tokens per chunk (pass-1 unit, pass-2 chunk)
 constexpr int kMaxChunkCount = 128;      // chunks per row (V <= 262144)
 
+// What a call computes.
+constexpr int kModeGreedy = 0;  // greedy_accept: argmax records of P rows
+constexpr int kModeSample = 1;  // speculative_sample_accept: softmax records of P and Q rows
+constexpr int kModeMixed = 2;   // a mixed batch: per-sequence draft count and temperature
+
 // The logit rows of one call. Row i of sequence b: P rows i = 0..K (p_1 .. p_{K+1}), then Q
 // rows i = K+1 .. 2K (q_1 .. q_K) when the call samples.
 struct RowSet {
   const void* p1;
   const void* pv;
   const void* q;
-  int64_t ld_p1;
-  int64_t ld_pv;
+  int32_t ld_p1;  // element strides (the host takes these below 2^31)
+  int32_t ld_pv;
   int K;
   int V;
   int rows;  // K + 1 (greedy) or 2K + 1 (sampling)
@@ -55,27 +65,71 @@ __device__ __forceinline__ const T* row_ptr(const RowSet& rs, int b, int i) {
 
 // Unsigned division by a divisor fixed per call, by multiplication: q = floor(n * m / 2^(32+s))
 // with m = ceil(2^(32+s) / d), s = ceil(log2 d), exact for every n < 2^32 (m < 2^33 is kept as
-// m_hi * 2^32 + m_lo). Integer multiplies only: no SFU or conversion instructions.
+// m_hi * 2^32 + m_lo; hs = m_hi << 8 | s). Integer multiplies only: no SFU or conversion
+// instructions. Eight bytes (see StreamParamsMixed on the size of kernel parameters).
 struct FastDiv {
-  uint32_t m_lo, m_hi, s;
+  uint32_t m_lo, hs;
   __device__ __forceinline__ uint32_t div(uint32_t n) const {
-    const uint64_t t = static_cast<uint64_t>(__umulhi(n, m_lo)) + (m_hi ? n : 0u);
-    return static_cast<uint32_t>(t >> s);
+    const uint64_t t = static_cast<uint64_t>(__umulhi(n, m_lo)) + ((hs >> 8) ? n : 0u);
+    return static_cast<uint32_t>(t >> (hs & 0xffu));
   }
 };
 
 struct StreamParams {
   RowSet rs;
-  uint32_t n_units;   // B * rows * nch (< 2^32)
+  uint32_t n_units;   // B * rows * nch (< 2^31)
   int nch;            // chunks per row
   int B;              // sequences
   FastDiv by_nch;     // division by nch
   FastDiv by_seqs;    // division by B
 
   float scale;        // log2(e) / T (sampling)
-  float2* rec;        // [n_units]: record of unit u at u
+  float2* rec;        // [B, rows, nch]: the records, by (sequence, row, chunk)
   const int32_t* drafts;  // [B, K] (sampling)
   float* gather;      // [B, K, 2] (sampling): P_i[x_i], Q_i[x_i] as float
+};
+
+// A mixed batch's parameters add its per-sequence arrays. They are kept out of StreamParams:
+// on this B200 the back-to-back sampling call's time moved by up to a microsecond with the
+// size and layout of the two kernels' parameter structs alone, the arithmetic unchanged (the
+// cause is not known; these structs are the fastest layout measured), so the other modes
+// carry none of the mixed batch's fields.
+struct StreamParamsMixed : StreamParams {
+  const int32_t* n_drafts;  // [B] K_b, or null for K
+  const float* temps;       // [B] T_b
+};
+template <int kMode>
+using StreamParamsOf = std::conditional_t<kMode == kModeMixed, StreamParamsMixed, StreamParams>;
+
+// A sequence of a mixed batch: its draft count K_b, whether its parameters are valid
+// (0 <= K_b <= K, T_b finite and >= 0, log2(e) / T_b finite), whether it is greedy (T_b == 0)
+// and its scale log2(e) / T_b, rounded exactly as the host rounds a call's single scale.
+struct SeqMode {
+  int kb;
+  bool ok;
+  bool greedy;
+  float scale;
+};
+__device__ __forceinline__ SeqMode seq_mode(const int32_t* n_drafts, const float* temps, int b,
+                                            int K) {
+  SeqMode m;
+  m.kb = n_drafts ? __ldg(n_drafts + b) : K;
+  const float T = __ldg(temps + b);
+  m.greedy = T == 0.f;
+  m.scale = T > 0.f ? static_cast<float>(1.4426950408889634 / static_cast<double>(T)) : 0.f;
+  m.ok = m.kb >= 0 && m.kb <= K && T >= 0.f && T <= 3.402823466e38f &&
+         (m.greedy || m.scale <= 3.402823466e38f);
+  return m;
+}
+
+// Which rows of a sequence a call reads: P rows 0..kb (row kb is the bonus row) and, when it
+// samples, the Q rows of its kb drafts. Row r of the block: P rows 0..K, then Q rows.
+struct RowFilter {
+  int K, kb;
+  bool q;
+  __device__ __forceinline__ bool operator()(int r) const {
+    return r <= K ? r <= kb : (q && r - K - 1 < kb);
+  }
 };
 
 // (sequence b, row i, chunk c) of a unit.
@@ -112,13 +166,15 @@ __device__ __forceinline__ size_t record_index(const StreamParams& p, const Unit
   return (static_cast<size_t>(at.b) * p.rs.rows + at.i) * p.nch + at.c;
 }
 
-// Sampling: the unit that holds a draft token x_i of a draft row (P row i < K, or Q row i)
-// also writes that token's logit for pass 2, so pass 2 need not fetch it from HBM.
-// `xd` is drafts[b, draft index of row i] (or -1), loaded before the unit's math.
-template <typename T>
-__device__ __forceinline__ int unit_draft(const StreamParams& p, const UnitPos& at, int lane) {
+// Sampling: the unit that holds a draft token x_i of a draft row (P row i < nd, or Q row i;
+// nd = K, or a mixed batch's K_b) also writes that token's logit for pass 2, so pass 2 need
+// not fetch it from HBM. `xd` is drafts[b, draft index of row i] (or -1), loaded before the
+// unit's math.
+template <typename T, bool kMixed>
+__device__ __forceinline__ int unit_draft(const StreamParams& p, const UnitPos& at, int lane,
+                                          int nd) {
   const int K = p.rs.K;
-  if (lane != 0 || at.i == K) return -1;
+  if (lane != 0 || (kMixed ? (at.i <= K && at.i >= nd) : at.i == K)) return -1;
   const int di = at.i < K ? at.i : at.i - K - 1;
   return __ldg(p.drafts + static_cast<size_t>(at.b) * K + di);
 }
@@ -371,8 +427,9 @@ __device__ __forceinline__ float2 piece_argmax(const T* row, long long o0, long 
 // warps finish together; no global atomic, fence or barrier is involved. The whole grid sweeps
 // the units front to back, so the rows read last (row pair 0 of every sequence) are the ones
 // still in L2 when pass 2 runs.
-template <typename T, int VEC, bool kSample>
-__global__ void __launch_bounds__(kStreamThreads, 1) stream_stats_kernel(const StreamParams p) {
+template <typename T, int VEC, int kMode>
+__global__ void __launch_bounds__(kStreamThreads, 1) stream_stats_kernel(
+    const StreamParamsOf<kMode> p) {
   __shared__ unsigned s_next;
   // the finish kernel may be scheduled as soon as these CTAs retire
   grid_dependents_launch();
@@ -393,14 +450,27 @@ __global__ void __launch_bounds__(kStreamThreads, 1) stream_stats_kernel(const S
     const int o0 = at.c * kCE;
     const int o1 = min(V, o0 + kCE);
     float2 rec;
-    if constexpr (kSample) {
-      const int xd = unit_draft<T>(p, at, lane);
+    bool used = true;
+    if constexpr (kMode == kModeSample) {
+      const int xd = unit_draft<T, false>(p, at, lane, p.rs.K);
       rec = piece_softmax<T, VEC>(row, o0, o1, lane, p.scale);
       unit_gather<T>(p, at, row, xd, o0, o1);
-    } else {
+    } else if constexpr (kMode == kModeGreedy) {
       rec = piece_argmax<T, VEC>(row, o0, o1, lane);
+    } else {
+      const SeqMode sm = seq_mode(p.n_drafts, p.temps, at.b, p.rs.K);
+      used = sm.ok && RowFilter{p.rs.K, sm.kb, !sm.greedy}(at.i);
+      if (used) {
+        if (sm.greedy) {
+          rec = piece_argmax<T, VEC>(row, o0, o1, lane);
+        } else {
+          const int xd = unit_draft<T, true>(p, at, lane, sm.kb);
+          rec = piece_softmax<T, VEC>(row, o0, o1, lane, sm.scale);
+          unit_gather<T>(p, at, row, xd, o0, o1);
+        }
+      }
     }
-    if (lane == 0) p.rec[record_index(p, at)] = rec;
+    if (lane == 0 && used) p.rec[record_index(p, at)] = rec;
     m = __shfl_sync(0xffffffffu, nxt, 0);
   }
 }

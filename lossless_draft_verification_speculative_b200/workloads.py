@@ -211,6 +211,34 @@ def uniforms(w: Workload, seqs: Optional[Sequence[int]] = None, T: float = 1.0,
     return out
 
 
+SEED_MIXED = 3
+
+
+def mixed_params(w: Workload, temperatures: Sequence[float] = (0.0, 0.7, 1.0),
+                 seed: int = SEED_MIXED):
+    """Per-sequence draft counts K_b [B] int32 and temperatures T_b [B] float32 of a mixed
+    serving batch: K_b = K for 40% of the sequences (a full block), else uniform on 0..K-1
+    (a block truncated by a confidence threshold or a cap); T_b uniform on ``temperatures``."""
+    rng = _rng(seed, w.B, w.K)
+    full = rng.random(w.B) < 0.4
+    kb = np.where(full, w.K, rng.integers(0, max(w.K, 1), size=w.B)).astype(np.int32)
+    T = np.asarray(temperatures, dtype=np.float32)[rng.integers(0, len(temperatures), size=w.B)]
+    return kb, T
+
+
+def mixed_inputs(w: Workload, kb: np.ndarray, T: np.ndarray):
+    """Drafts [B, K] and uniforms [B, K+1] of a mixed batch: sequence b's drafts and uniforms
+    are those of a call at its own T_b (entries past K_b are filled but never read)."""
+    d = np.empty((w.B, w.K), dtype=np.int32)
+    u = np.empty((w.B, w.K + 1), dtype=np.float32)
+    for t in np.unique(T):
+        seqs = [int(b) for b in np.flatnonzero(T == t)]
+        _, Q = logits(w, seqs)
+        d[seqs] = drafts(w, Q, float(t), seqs)
+        u[seqs] = uniforms(w, seqs, T=float(t))
+    return d, u
+
+
 def tiny_cycles(w: Workload, cycles: int, T: float = 1.0):
     """The tiny workload's repeated-cycle form: one fixed (P, Q) pair (sequence 0's logits),
     and per cycle fresh drafts and uniforms. Returned batched as B = ``cycles`` sequences

@@ -92,7 +92,16 @@ def _sample(lib, **kw):
                                                 a["out"], a["ws"], a["wsb"], a["s"])
 
 
-@pytest.mark.parametrize("call", [_greedy, _sample])
+def _mixed(lib, **kw):
+    a = dict(p1=FAKE, ld=1024, pv=FAKE, ldv=7 * 1024, q=FAKE, dt=BF16, d=FAKE, nd=FAKE, B=4, K=7,
+             V=1024, T=FAKE, u=FAKE, out=_out(), ws=FAKE, wsb=1 << 30, s=None)
+    a.update(kw)
+    return lib.dspark_mixed_accept(a["p1"], a["ld"], a["pv"], a["ldv"], a["q"], a["dt"], a["d"],
+                                   a["nd"], a["B"], a["K"], a["V"], a["T"], a["u"], a["out"],
+                                   a["ws"], a["wsb"], a["s"])
+
+
+@pytest.mark.parametrize("call", [_greedy, _sample, _mixed])
 def test_invalid_arguments(lib, call):
     INV, UNS, WS = 1, 2, 4
     assert call(lib, B=-1) == INV
@@ -110,6 +119,8 @@ def test_invalid_arguments(lib, call):
     assert call(lib, out=_out(nx=None)) == INV
     assert call(lib, p1=FAKE + 1) == UNS          # not aligned to the element size
     assert call(lib, V=262145, ld=262145, ldv=7 * 262145) == UNS
+    assert call(lib, ld=1 << 31) == UNS           # row strides are 32-bit in the kernels
+    assert call(lib, ldv=1 << 31) == UNS
     assert call(lib, ws=None) == WS
     assert call(lib, wsb=16) == WS
     assert call(lib, ws=FAKE + 16) == WS          # workspace must be 256-byte aligned
@@ -129,3 +140,15 @@ def test_sampling_specific_arguments(lib):
     assert _sample(lib, T=0.0, q=None, u=None, ws=None) == 4
     # K == 0: no draft rows, pv / q / drafts may be NULL; workspace still checked
     assert _sample(lib, K=0, pv=None, q=None, d=None, ldv=0, ws=None) == 4
+
+
+def test_mixed_batch_specific_arguments(lib):
+    INV, UNS = 1, 2
+    assert _mixed(lib, T=None) == INV             # temperatures are required
+    assert _mixed(lib, u=None) == INV
+    assert _mixed(lib, q=None) == INV             # required for K > 0 even if all are greedy
+    assert _mixed(lib, q=FAKE + 1) == UNS
+    # the draft counts may be NULL (every sequence K); the workspace check still applies
+    assert _mixed(lib, nd=None, ws=None) == 4
+    # K == 0: no draft rows; q and drafts may be NULL
+    assert _mixed(lib, K=0, pv=None, q=None, d=None, ldv=0, ws=None) == 4
