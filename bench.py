@@ -341,6 +341,7 @@ def run_ours(args, w):
         b.record()
         torch.cuda.synchronize()
         per_call_us.append(a.elapsed_time(b) * 1000.0 / reps)
+    mixed = time_mixed_batch(w, sets, D, U, workspace, dev, reps)
     value, ms_max = aggregate(ms, args.steps * ncalls * w.B, world, dist, dev)
 
     # results of the last step: committed tokens per verified block
@@ -398,6 +399,9 @@ def run_ours(args, w):
         "committed_token_equivalents_per_s": value * statistics.mean(committed),
         "calls": call_stats,
     }
+    if mixed:
+        mixed["frac_of_peak"] = mixed["GB_per_s"] / peak
+        call_stats["mixed_batch"] = mixed
     if clk:
         line["clocks"] = clk
     if e2e:
@@ -405,6 +409,44 @@ def run_ours(args, w):
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w, args.cpu_seconds)
     print(json.dumps(line), flush=True)
+
+
+def time_mixed_batch(w, sets, D, U, workspace, dev, reps):
+    """A mixed serving batch on the same logits, timed alone (not part of the step): sequence
+    b verifies K_b drafts at T_b (workloads.mixed_params), with the drafts and uniforms of the
+    step's call at T_b. Its bytes are the rows it reads: P rows 0..K_b, and Q rows 0..K_b-1
+    when T_b > 0."""
+    import torch
+
+    from lossless_draft_verification_speculative_b200 import binding as bd
+    from lossless_draft_verification_speculative_b200 import workloads as wl
+
+    kb, Tb = wl.mixed_params(w, w.temperatures)
+    temps = np.asarray(w.temperatures, dtype=np.float64)
+    ti = [int(np.argmin(np.abs(temps - float(t)))) for t in Tb]
+    d = np.stack([D[w.temperatures[i]][b] for b, i in enumerate(ti)]).astype(np.int32)
+    u = np.stack([U[w.temperatures[i]][b] for b, i in enumerate(ti)]).astype(np.float32)
+    es = 2 if w.dtype == "bf16" else 4
+    nbytes = int(sum(es * w.V * ((k + 1) + (k if t > 0 else 0)) for k, t in zip(kb, Tb)))
+    kd, Td = torch.from_numpy(kb).to(dev), torch.from_numpy(Tb).to(dev)
+    dd, ud = torch.from_numpy(d).to(dev), torch.from_numpy(u).to(dev)
+    out = bd._alloc_result(w.B, w.K, dev, diagnostics=True)
+    calls = [bd.PreparedCall("mixed", P, Q, dd, Td, ud, out, workspace, n_drafts=kd)
+             for P, Q in sets]
+    for r in range(8):
+        calls[r % len(calls)]()
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    a.record()
+    for r in range(reps):
+        calls[r % len(calls)]()
+    b.record()
+    torch.cuda.synchronize()
+    us = a.elapsed_time(b) * 1000.0 / reps
+    return {"us_per_call": us, "bytes_read": nbytes, "GB_per_s": nbytes / (us * 1e-6) / 1e9,
+            "mean_drafts": float(kb.mean()), "greedy_sequences": int((Tb == 0).sum()),
+            "committed_tokens_per_block": float((out.n_accepted.double() + 1).mean().item())}
 
 
 def run_e2e(args, w, calls, P, Q, D, U, dev, tdt, outs, workspace, world):
