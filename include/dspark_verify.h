@@ -122,7 +122,8 @@ typedef struct {
   int n_chunks;                    /* chunks per row                                              */
   int greedy_units_per_sequence;   /* pass-1 units of one sequence, greedy: (K+1) * n_chunks      */
   int sampling_units_per_sequence; /* pass-1 units of one sequence, sampling: (2K+1) * n_chunks   */
-  int finish_ctas_per_sequence;    /* pass-2 CTAs per sequence, sampling policy                   */
+  int finish_ctas_per_sequence;    /* pass-2 CTAs per sequence (one cluster), sampling policy:
+                                      min(n_chunks, 16) for B <= 32, else min(n_chunks, 8)       */
 } dspark_plan_t;
 dspark_status_t dspark_plan(int B, int K, int V, dspark_dtype_t dtype, int aligned16,
                             dspark_plan_t* plan);

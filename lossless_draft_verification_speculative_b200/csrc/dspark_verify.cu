@@ -1,5 +1,6 @@
 // C ABI of the DSpark block verify/accept step: argument checks, launch planning and the
 // two kernel launches of a call (pass 1 in stream.cuh, pass 2 in finish.cuh).
+#include <atomic>
 #include <climits>
 #include <cmath>
 #include <cstdlib>
@@ -42,13 +43,14 @@ struct Plan {
   int cpc;  // chunks per pass-2 CTA
 };
 
-bool make_plan(int V, dspark_dtype_t dt, bool aligned16, Plan* pl) {
+bool make_plan(int B, int V, dspark_dtype_t dt, bool aligned16, Plan* pl) {
   const int es = elem_bytes(dt);
   const long long nch = (static_cast<long long>(V) + kCE - 1) / kCE;
   if (nch < 1 || nch > kMaxChunkCount) return false;
   pl->vec = aligned16 ? 16 / es : 1;
   pl->nch = static_cast<int>(nch);
-  pl->G = pl->nch < kMaxFinishCluster ? pl->nch : kMaxFinishCluster;
+  const int gmax = B <= kWideClusterMaxB ? kMaxFinishCluster : kPortableCluster;
+  pl->G = pl->nch < gmax ? pl->nch : gmax;
   pl->cpc = (pl->nch + pl->G - 1) / pl->G;
   return true;
 }
@@ -212,8 +214,21 @@ dspark_status_t run_call(const Call& c, const Plan& pl, cudaStream_t stream) {
   cfg.stream = stream;
   cfg.attrs = attr;
   cfg.numAttrs = kSample ? 2 : 1;
-  if constexpr (kSample)
+  if constexpr (kSample) {
+    if (pl.G > kPortableCluster) {  // a 16-CTA cluster is opt-in, once per kernel and device
+      static std::atomic<bool> wide[kMaxDevices];
+      int dev = 0;
+      if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices)
+        return DSPARK_ERR_CUDA;
+      if (!wide[dev].load(std::memory_order_acquire)) {
+        if (cudaFuncSetAttribute(finish_sample_kernel<T, VEC, kMode == kModeMixed>,
+                                 cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess)
+          return DSPARK_ERR_CUDA;
+        wide[dev].store(true, std::memory_order_release);
+      }
+    }
     e = cudaLaunchKernelEx(&cfg, finish_sample_kernel<T, VEC, kMode == kModeMixed>, fp);
+  }
   else
     e = cudaLaunchKernelEx(&cfg, finish_greedy_kernel<T>, fp);
   return e == cudaSuccess ? DSPARK_OK : DSPARK_ERR_CUDA;
@@ -310,7 +325,7 @@ size_t dspark_workspace_bytes(int B, int K, int V, dspark_dtype_t dtype) {
   if (dtype != DSPARK_BF16 && dtype != DSPARK_F32) return 0;
   if (!shape_ok(B, K, V)) return 0;
   Plan pl;
-  if (!make_plan(V, dtype, false, &pl)) return 0;
+  if (!make_plan(B, V, dtype, false, &pl)) return 0;
   return ws_layout(B, K, pl.nch).total;
 }
 
@@ -325,7 +340,7 @@ dspark_status_t dspark_plan(int B, int K, int V, dspark_dtype_t dtype, int align
   if (!plan || (dtype != DSPARK_BF16 && dtype != DSPARK_F32) || !shape_ok(B, K, V))
     return DSPARK_ERR_INVALID_ARG;
   Plan pl;
-  if (!make_plan(V, dtype, aligned16 != 0, &pl)) return DSPARK_ERR_UNSUPPORTED;
+  if (!make_plan(B, V, dtype, aligned16 != 0, &pl)) return DSPARK_ERR_UNSUPPORTED;
   plan->elems_per_load = pl.vec;
   plan->loads_in_flight = kBatchVecs;
   plan->stream_threads_per_cta = kStreamThreads;
@@ -348,7 +363,7 @@ dspark_status_t dspark_greedy_accept(const void* p1, int64_t ld_p1, const void* 
   const bool a16 = aligned(p1, 16) && (K == 0 || aligned(pv, 16)) && (ld_p1 * es) % 16 == 0 &&
                    (K == 0 || (ld_pv * es) % 16 == 0) && (V * es) % 16 == 0;
   Plan pl;
-  if (!make_plan(V, dtype, a16, &pl)) return DSPARK_ERR_UNSUPPORTED;
+  if (!make_plan(B, V, dtype, a16, &pl)) return DSPARK_ERR_UNSUPPORTED;
   if (!workspace || workspace_bytes < ws_layout(B, K, pl.nch).total || !aligned(workspace, 256))
     return DSPARK_ERR_WORKSPACE;
   const Call c = make_call(p1, ld_p1, pv, ld_pv, nullptr, drafts, nullptr, B, K, V, 0.f, K + 1,
@@ -380,7 +395,7 @@ dspark_status_t dspark_speculative_sample_accept(const void* p1, int64_t ld_p1, 
                    (ld_p1 * es) % 16 == 0 && (K == 0 || (ld_pv * es) % 16 == 0) &&
                    (V * es) % 16 == 0;
   Plan pl;
-  if (!make_plan(V, dtype, a16, &pl)) return DSPARK_ERR_UNSUPPORTED;
+  if (!make_plan(B, V, dtype, a16, &pl)) return DSPARK_ERR_UNSUPPORTED;
   if (!workspace || workspace_bytes < ws_layout(B, K, pl.nch).total || !aligned(workspace, 256))
     return DSPARK_ERR_WORKSPACE;
   const float scale = static_cast<float>(1.4426950408889634 / static_cast<double>(temperature));
@@ -409,7 +424,7 @@ dspark_status_t dspark_mixed_accept(const void* p1, int64_t ld_p1, const void* p
                    (ld_p1 * es) % 16 == 0 && (K == 0 || (ld_pv * es) % 16 == 0) &&
                    (V * es) % 16 == 0;
   Plan pl;
-  if (!make_plan(V, dtype, a16, &pl)) return DSPARK_ERR_UNSUPPORTED;
+  if (!make_plan(B, V, dtype, a16, &pl)) return DSPARK_ERR_UNSUPPORTED;
   if (!workspace || workspace_bytes < ws_layout(B, K, pl.nch).total || !aligned(workspace, 256))
     return DSPARK_ERR_WORKSPACE;
   Call c = make_call(p1, ld_p1, pv, ld_pv, q, drafts, uniforms, B, K, V, 0.f, 2 * K + 1,

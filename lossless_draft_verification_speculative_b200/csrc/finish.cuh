@@ -23,7 +23,12 @@ namespace dspark {
 constexpr int kErrBits =
     DSPARK_SEQ_BAD_DRAFT | DSPARK_SEQ_NONFINITE | DSPARK_SEQ_TIMEOUT | DSPARK_SEQ_BAD_PARAM;
 constexpr int kMaxRows = 2 * kMaxK + 1;
-constexpr int kMaxFinishCluster = 8;  // CTAs per sampling cluster (portable size)
+// CTAs per sampling cluster: 8 (the portable size), or 16 (opt-in) for batches of at most
+// kWideClusterMaxB sequences, whose 16 B CTAs of 4 per SM are still co-resident on 148 SMs and
+// whose warps then take one chunk each instead of two.
+constexpr int kPortableCluster = 8;
+constexpr int kMaxFinishCluster = 16;
+constexpr int kWideClusterMaxB = 32;
 
 // Kernel parameters (see StreamParamsMixed on their size). The sampling kernel's cluster size
 // G and chunks per CTA, ceil(n_chunks / G), come from its launch.
