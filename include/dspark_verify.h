@@ -47,6 +47,12 @@
  *  - Limits: 0 <= K <= 32; 1 <= V <= 262144; B * (2K+1) < 2^31; row strides ld_p1, ld_pv
  *    below 2^31 elements (larger ones: DSPARK_ERR_UNSUPPORTED).
  *  - Calls that share a workspace must not overlap on the GPU (same stream, or ordered).
+ *  - Programmatic dependent launch: a call's first kernel is launched as a programmatic
+ *    dependent of the kernel before it in the stream and waits for that kernel to complete
+ *    before reading any input, and a call's last kernel lets the next kernel in the stream be
+ *    scheduled early. A caller that launches its next kernel with programmatic stream
+ *    serialization must, as always, have it wait (griddepcontrol.wait /
+ *    cudaGridDependencySynchronize) before reading the results.
  */
 #ifndef DSPARK_VERIFY_H
 #define DSPARK_VERIFY_H

@@ -151,8 +151,11 @@ struct Call {
   char* ws;
 };
 
-// Pass 1 over every (row, chunk) unit (one wave of warps, equal contiguous runs of units),
-// then pass 2 launched as a programmatic dependent of it.
+// Pass 1 over every (row, chunk) unit (one CTA per SM, every grid-th unit), then pass 2.
+// Both are programmatic dependent launches: pass 1's CTAs become resident while the previous
+// kernel in the stream drains and wait for it to complete before reading anything (this hides
+// the launch latency between back-to-back calls, about 2 us); pass 2's CTAs load what pass 1
+// does not write and then wait for pass 1.
 template <typename T, int VEC, int kMode>
 dspark_status_t run_call(const Call& c, const Plan& pl, cudaStream_t stream) {
   constexpr bool kSample = kMode != kModeGreedy;
@@ -183,9 +186,20 @@ dspark_status_t run_call(const Call& c, const Plan& pl, cudaStream_t stream) {
     sp.n_drafts = c.n_drafts;
     sp.temps = c.temps;
   }
-  stream_stats_kernel<T, VEC, kMode><<<grid1, kStreamThreads, 0, stream>>>(sp);
-  e = cudaGetLastError();
-  if (e != cudaSuccess) return DSPARK_ERR_CUDA;
+  {
+    cudaLaunchAttribute a1[1];
+    a1[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    a1[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t c1 = {};
+    c1.gridDim = dim3(static_cast<unsigned>(grid1), 1, 1);
+    c1.blockDim = dim3(kStreamThreads, 1, 1);
+    c1.dynamicSmemBytes = 0;
+    c1.stream = stream;
+    c1.attrs = a1;
+    c1.numAttrs = 1;
+    e = cudaLaunchKernelEx(&c1, stream_stats_kernel<T, VEC, kMode>, sp);
+    if (e != cudaSuccess) return DSPARK_ERR_CUDA;
+  }
 
   std::conditional_t<kMode == kModeMixed, FinishParamsMixed, FinishParams> fp{};
   fp.rs = c.rs;

@@ -183,6 +183,8 @@ template <typename T>
 __global__ void __launch_bounds__(kThreads) finish_greedy_kernel(const FinishParams p) {
   __shared__ float2 s_arg[kMaxK + 1];
   __shared__ int s_x[kMaxK];
+  // the next kernel in the stream may be scheduled as these CTAs retire (it waits for them)
+  grid_dependents_launch();
   const int lane = threadIdx.x & 31, wi = threadIdx.x >> 5;
   const int b = blockIdx.x;
   const int K = p.rs.K;
@@ -490,6 +492,8 @@ __global__ void __launch_bounds__(kThreads, 4) finish_sample_kernel(
   __shared__ Decision s_dec;
   __shared__ double s_tin;
   __shared__ int s_chunk, s_use_p;
+  // the next kernel in the stream may be scheduled as these CTAs retire (it waits for them)
+  grid_dependents_launch();
   cg::cluster_group cluster = cg::this_cluster();
   const int tid = threadIdx.x, lane = tid & 31, wi = tid >> 5;
   const int G = static_cast<int>(cluster.num_blocks());

@@ -431,7 +431,11 @@ template <typename T, int VEC, int kMode>
 __global__ void __launch_bounds__(kStreamThreads, 1) stream_stats_kernel(
     const StreamParamsOf<kMode> p) {
   __shared__ unsigned s_next;
-  // the finish kernel may be scheduled as soon as these CTAs retire
+  // Launched as a programmatic dependent of whatever precedes it in the stream, so that its
+  // CTAs are resident as the previous kernel drains: nothing is read before that kernel has
+  // completed and its writes are visible. Only then may the finish kernel be scheduled (it
+  // reads the drafts and uniforms before waiting for this pass).
+  grid_dependency_wait();
   grid_dependents_launch();
   const int lane = threadIdx.x & 31;
   const int wi = threadIdx.x >> 5;
