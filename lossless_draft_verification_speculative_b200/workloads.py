@@ -239,6 +239,40 @@ def mixed_inputs(w: Workload, kb: np.ndarray, T: np.ndarray):
     return d, u
 
 
+SEED_MARKOV = 4
+
+
+def markov_table(V: int, R: int, fmt: str, seed: int = SEED_MARKOV, sd: float = 0.05):
+    """A synthetic Markov-head table markov_w2 of V rows of R values, stored as the GGUF
+    forms the drafter card ships: fmt "f16" -> uint16 [V, R] half-float bits; fmt "q8_0" ->
+    uint8 [V, R/32 * 34] rows of blocks (float16 scale d = max|x| / 127 of the block's 32
+    values, then q = round(x / d) as signed bytes). Values ~ N(0, sd), a few rows 20x wider
+    so that block scales vary."""
+    rng = _rng(seed, V, R)
+    x = rng.normal(0.0, sd, size=(V, R)).astype(np.float32)
+    wide = rng.random(V) < 0.01
+    x[wide] *= 20.0
+    if fmt == "f16":
+        return x.astype(np.float16).view(np.uint16)
+    if fmt != "q8_0":
+        raise ValueError(f"unknown table format {fmt!r}")
+    blocks = x.reshape(V, R // 32, 32)
+    amax = np.abs(blocks).max(axis=2)
+    d = (amax / 127.0).astype(np.float16)
+    d32 = d.astype(np.float32)
+    inv = np.divide(1.0, d32, out=np.zeros_like(d32), where=d32 != 0)
+    q = np.clip(np.rint(blocks * inv[:, :, None]), -127, 127).astype(np.int8)
+    out = np.empty((V, R // 32, 34), dtype=np.uint8)
+    out[:, :, 0:2] = d.view(np.uint8).reshape(V, R // 32, 2)
+    out[:, :, 2:] = q.view(np.uint8)
+    return out.reshape(V, (R // 32) * 34)
+
+
+def markov_states(B: int, R: int, seed: int = SEED_MARKOV) -> np.ndarray:
+    """Rank-R states h [B, R] float32 ~ N(0, 1)."""
+    return _rng(seed, 7, B, R).normal(0.0, 1.0, size=(B, R)).astype(np.float32)
+
+
 def tiny_cycles(w: Workload, cycles: int, T: float = 1.0):
     """The tiny workload's repeated-cycle form: one fixed (P, Q) pair (sequence 0's logits),
     and per cycle fresh drafts and uniforms. Returned batched as B = ``cycles`` sequences
