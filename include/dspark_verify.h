@@ -187,6 +187,23 @@ dspark_status_t dspark_mixed_accept(const void* p1, int64_t ld_p1, const void* p
                                     dspark_accept_out_t out, void* workspace,
                                     size_t workspace_bytes, void* stream);
 
+/* The drafter's Markov-head table mat-vec (the drafter side of the cycle, beside the verify
+ * step): y[b, v] = sum_k W[v, k] h[b, k] over the table markov_w2, V rows of R values. The
+ * DeepSeek-V4-Flash DSpark drafter card ("Files") ships the table in F16 or in GGUF Q8_0 and
+ * says the ds4 engine reads it in full four times per draft block (0.18 ms per call in Q8_0,
+ * 0.63 ms in F16, on a GB10).
+ *  table  device; DSPARK_TABLE_F16: V x R half floats, row-major (row v = vocab entry v);
+ *         DSPARK_TABLE_Q8_0: V rows of R/32 GGUF Q8_0 blocks of 34 bytes (a little-endian
+ *         float16 scale d, then 32 signed bytes q; value d * q[i]). 16-byte aligned.
+ *  R      the Markov rank: 256 (other ranks: DSPARK_ERR_UNSUPPORTED).
+ *  h      device [B, R] float32 states, 16-byte aligned.
+ *  y      device [B, V] float32 results (row b at y + b * V).
+ *  Sums are float32 in a fixed order; batches of more than 4 states read the table once per
+ *  4 states. B == 0 or V == 0 is a no-op. */
+typedef enum { DSPARK_TABLE_F16 = 0, DSPARK_TABLE_Q8_0 = 1 } dspark_table_t;
+dspark_status_t dspark_markov_matvec(const void* table, dspark_table_t type, int V, int R,
+                                     const float* h, int B, float* y, void* stream);
+
 /* speculative_sample_accept without a workspace argument. The pages have no counterpart of
  * this entry point: it exists for callers that cannot allocate device memory where they
  * verify (a serving loop whose KV-cache pool took all free HBM at start-up and left no

@@ -3,7 +3,7 @@
 ``greedy_accept`` and ``speculative_sample_accept`` verify a block of K drafted tokens per
 sequence against the base model's [B, K+1, V] logit block and return an ``AcceptResult``;
 ``mixed_accept`` verifies a serving batch whose sequences have their own draft counts and
-temperatures.
+temperatures; ``markov_matvec`` is the drafter's Markov-head table mat-vec.
 The work runs in hand-written CUDA kernels behind a C ABI (``include/dspark_verify.h``);
 this package is the thin Python binding over it plus the seeded synthetic workloads.
 """
@@ -18,6 +18,7 @@ from .binding import (  # noqa: F401
     DsparkError,
     greedy_accept,
     load_library,
+    markov_matvec,
     mixed_accept,
     plan,
     speculative_sample_accept,
@@ -32,6 +33,7 @@ __all__ = [
     "speculative_sample_accept",
     "speculative_sample_accept_static",
     "mixed_accept",
+    "markov_matvec",
     "load_library",
     "plan",
     "workspace_bytes",

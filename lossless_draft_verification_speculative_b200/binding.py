@@ -109,6 +109,8 @@ def load_library(build_if_missing: bool = True) -> ctypes.CDLL:
     lib.dspark_mixed_accept.restype = i32
     lib.dspark_mixed_accept.argtypes = [vp, i64, vp, i64, vp, i32, vp, vp, i32, i32, i32, vp, vp,
                                         AcceptOut, vp, sz, vp]
+    lib.dspark_markov_matvec.restype = i32
+    lib.dspark_markov_matvec.argtypes = [vp, i32, i32, i32, vp, i32, vp, vp]
     lib.dspark_speculative_sample_accept_static.restype = i32
     lib.dspark_speculative_sample_accept_static.argtypes = [vp, i64, vp, i64, vp, i32, vp, i32,
                                                             i32, i32, ctypes.c_float, vp,
@@ -329,6 +331,40 @@ def mixed_accept(P: Union[torch.Tensor, Tuple[torch.Tensor, torch.Tensor]],
     if rc != DSPARK_OK:
         raise DsparkError(rc, "dspark_mixed_accept")
     return res
+
+
+MARKOV_TABLE_CODES = {"f16": 0, "q8_0": 1}
+
+
+def markov_matvec(table: torch.Tensor, fmt: str, h: torch.Tensor, *,
+                  out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """The drafter's Markov-head table mat-vec on the GPU: y[b, v] = sum_k W[v, k] h[b, k].
+
+    ``table`` holds markov_w2 as the drafter files store it: fmt "f16", a [V, R] float16 (or
+    16-bit integer bits) tensor; fmt "q8_0", a [V, R/32 * 34] uint8 tensor of GGUF Q8_0 rows.
+    ``h`` is a float32 [B, R] tensor on the same device (R = 256). Returns float32 [B, V].
+    """
+    lib = load_library()
+    if fmt not in MARKOV_TABLE_CODES:
+        raise ValueError("fmt must be 'f16' or 'q8_0'")
+    if not table.is_cuda or not table.is_contiguous():
+        raise ValueError("table must be a contiguous CUDA tensor")
+    if h.dtype != torch.float32 or h.dim() != 2 or not h.is_contiguous() or \
+            h.device != table.device:
+        raise ValueError("h must be a contiguous float32 [B, R] tensor on the table's device")
+    B, R = h.shape
+    V = table.shape[0]
+    row_bytes = R * 2 if fmt == "f16" else R // 32 * 34
+    if table.dim() != 2 or table.shape[1] * table.element_size() != row_bytes:
+        raise ValueError(f"table rows must be {row_bytes} bytes for fmt {fmt!r} and R = {R}")
+    y = out if out is not None else torch.empty(B, V, dtype=torch.float32, device=h.device)
+    if y.shape != (B, V) or y.dtype != torch.float32 or not y.is_contiguous():
+        raise ValueError("out must be a contiguous float32 [B, V] tensor")
+    rc = lib.dspark_markov_matvec(_ptr(table), MARKOV_TABLE_CODES[fmt], V, R, _ptr(h), B,
+                                  _ptr(y), _stream_handle(h.device))
+    if rc != DSPARK_OK:
+        raise DsparkError(rc, "dspark_markov_matvec")
+    return y
 
 
 def speculative_sample_accept_static(P: Union[torch.Tensor, Tuple[torch.Tensor, torch.Tensor]],

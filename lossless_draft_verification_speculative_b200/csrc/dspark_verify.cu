@@ -9,6 +9,7 @@
 
 #include "common.cuh"
 #include "finish.cuh"
+#include "markov.cuh"
 #include "stream.cuh"
 
 namespace dspark {
@@ -315,6 +316,29 @@ dspark_status_t static_scratch_address(void** addr) {
   return DSPARK_OK;
 }
 
+// The Markov-head mat-vec for up to kMarkovMaxStates states per launch.
+template <int NB>
+dspark_status_t markov_launch(const void* table, dspark_table_t type, int V, const float* h,
+                              float* y, int ldy, cudaStream_t stream) {
+  const bool q8 = type == DSPARK_TABLE_Q8_0;
+  const void* fn = q8 ? reinterpret_cast<const void*>(&markov_q8_0_kernel<NB>)
+                      : reinterpret_cast<const void*>(&markov_f16_kernel<NB>);
+  cudaError_t e = cudaSuccess;
+  const int ctas = resident_ctas(fn, kMarkovThreads, 0, &e);
+  if (e != cudaSuccess) return DSPARK_ERR_CUDA;
+  if (ctas < 1) return DSPARK_ERR_UNSUPPORTED;
+  const long long rows_per_cta = (kMarkovThreads / 32) * (q8 ? kQ8Rows : (NB <= 2 ? 8 : 4));
+  const long long want = (V + rows_per_cta - 1) / rows_per_cta;
+  const int grid = static_cast<int>(want < ctas ? want : ctas);
+  if (q8)
+    markov_q8_0_kernel<NB><<<grid, kMarkovThreads, 0, stream>>>(
+        static_cast<const uint8_t*>(table), V, h, y, ldy);
+  else
+    markov_f16_kernel<NB><<<grid, kMarkovThreads, 0, stream>>>(
+        static_cast<const uint16_t*>(table), V, h, y, ldy);
+  return cudaGetLastError() == cudaSuccess ? DSPARK_OK : DSPARK_ERR_CUDA;
+}
+
 }  // namespace
 }  // namespace dspark
 
@@ -450,6 +474,31 @@ dspark_status_t dspark_mixed_accept(const void* p1, int64_t ld_p1, const void* p
     return a16 ? run_call<bf16_t, 8, kModeMixed>(c, pl, s)
                : run_call<bf16_t, 1, kModeMixed>(c, pl, s);
   return a16 ? run_call<float, 4, kModeMixed>(c, pl, s) : run_call<float, 1, kModeMixed>(c, pl, s);
+}
+
+dspark_status_t dspark_markov_matvec(const void* table, dspark_table_t type, int V, int R,
+                                     const float* h, int B, float* y, void* stream) {
+  if (type != DSPARK_TABLE_F16 && type != DSPARK_TABLE_Q8_0) return DSPARK_ERR_INVALID_ARG;
+  if (V < 0 || R < 1 || B < 0) return DSPARK_ERR_INVALID_ARG;
+  if (V == 0 || B == 0) return DSPARK_OK;
+  if (!table || !h || !y) return DSPARK_ERR_INVALID_ARG;
+  if (R != kMarkovRank) return DSPARK_ERR_UNSUPPORTED;
+  if (!aligned(table, 16) || !aligned(h, 16) || !aligned(y, 4)) return DSPARK_ERR_UNSUPPORTED;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  for (int b0 = 0; b0 < B; b0 += kMarkovMaxStates) {
+    const int nb = B - b0 < kMarkovMaxStates ? B - b0 : kMarkovMaxStates;
+    const float* hb = h + static_cast<size_t>(b0) * R;
+    float* yb = y + static_cast<size_t>(b0) * V;
+    dspark_status_t st;
+    switch (nb) {
+      case 1: st = markov_launch<1>(table, type, V, hb, yb, V, s); break;
+      case 2: st = markov_launch<2>(table, type, V, hb, yb, V, s); break;
+      case 3: st = markov_launch<3>(table, type, V, hb, yb, V, s); break;
+      default: st = markov_launch<4>(table, type, V, hb, yb, V, s); break;
+    }
+    if (st != DSPARK_OK) return st;
+  }
+  return DSPARK_OK;
 }
 
 dspark_status_t dspark_speculative_sample_accept_static(const void* p1, int64_t ld_p1,

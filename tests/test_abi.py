@@ -156,3 +156,15 @@ def test_mixed_batch_specific_arguments(lib):
     assert _mixed(lib, nd=None, ws=None) == 4
     # K == 0: no draft rows; q and drafts may be NULL
     assert _mixed(lib, K=0, pv=None, q=None, d=None, ldv=0, ws=None) == 4
+
+
+def test_markov_matvec_arguments(lib):
+    INV, UNS = 1, 2
+    mv = lambda t=FAKE, ty=0, V=1000, R=256, h=FAKE, B=1, y=FAKE: (  # noqa: E731
+        lib.dspark_markov_matvec(t, ty, V, R, h, B, y, None))
+    assert mv(ty=2) == INV
+    assert mv(V=-1) == INV and mv(B=-1) == INV and mv(R=0) == INV
+    assert mv(t=None) == INV and mv(h=None) == INV and mv(y=None) == INV
+    assert mv(R=128) == UNS                        # the drafters ship rank 256
+    assert mv(t=FAKE + 8) == UNS and mv(h=FAKE + 4) == UNS and mv(y=FAKE + 2) == UNS
+    assert mv(V=0) == 0 and mv(B=0) == 0           # no-ops
