@@ -330,13 +330,24 @@ dspark_status_t markov_launch(const void* table, dspark_table_t type, int V, con
   const long long rows_per_cta = (kMarkovThreads / 32) * (q8 ? kQ8Rows : (NB <= 2 ? 8 : 4));
   const long long want = (V + rows_per_cta - 1) / rows_per_cta;
   const int grid = static_cast<int>(want < ctas ? want : ctas);
-  if (q8)
-    markov_q8_0_kernel<NB><<<grid, kMarkovThreads, 0, stream>>>(
-        static_cast<const uint8_t*>(table), V, h, y, ldy);
-  else
-    markov_f16_kernel<NB><<<grid, kMarkovThreads, 0, stream>>>(
-        static_cast<const uint16_t*>(table), V, h, y, ldy);
-  return cudaGetLastError() == cudaSuccess ? DSPARK_OK : DSPARK_ERR_CUDA;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(grid), 1, 1);
+  cfg.blockDim = dim3(kMarkovThreads, 1, 1);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = stream;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (q8) {
+    e = cudaLaunchKernelEx(&cfg, markov_q8_0_kernel<NB>, static_cast<const uint8_t*>(table), V,
+                           h, y, ldy);
+  } else {
+    e = cudaLaunchKernelEx(&cfg, markov_f16_kernel<NB>, static_cast<const uint16_t*>(table), V,
+                           h, y, ldy);
+  }
+  return e == cudaSuccess ? DSPARK_OK : DSPARK_ERR_CUDA;
 }
 
 }  // namespace

@@ -6,14 +6,25 @@
 // an HBM stream. One CTA of 8 warps per resident slot walks groups of rows grid-stride; a warp
 // keeps a group's loads in flight together:
 //  - F16: a row is 512 bytes, one 16-byte piece (8 halves) per lane; 8 rows per group (4 with
-//    3 or 4 states). Lane l holds h[b, 8l .. 8l+7] in registers, multiplies its pieces, and
-//    each row's 32 partial sums are added by a butterfly.
+//    3 or 4 states). Lane l holds h[b, 8l .. 8l+7] in registers and multiplies its pieces.
+//    With one state each row's 32 partial sums are added by its own butterfly (8 independent
+//    chains); with more, the group's (row, state) partial sums are added by one transposed
+//    butterfly (each round halves the values a lane carries): 2 states x 8 rows cost 19
+//    shuffles instead of 80. With 3 or 4 states the products run as packed f32x2 FMAs (even
+//    and odd elements in the two halves of the accumulator).
 //  - Q8_0: a row is 8 blocks of 34 bytes (272 bytes, so rows start 16-byte aligned). A group
-//    of 8 consecutive rows (2176 bytes) is copied with 16-byte loads into the warp's shared
-//    buffer; lane l then decodes blocks (row l/8, block l%8) and (row 4 + l/8, block l%8):
+//    of 8 consecutive rows (2176 bytes) is copied by 16-byte asynchronous copies into one of
+//    the warp's two shared buffers, so the next group is in flight while the warp decodes
+//    this one; lane l decodes blocks (row l/8, block l%8) and (row 4 + l/8, block l%8):
 //    d * sum_i q[i] h[b, 32 block + i], and the 8 blocks of a row are added by a butterfly
-//    over the lanes of the row.
-// Sums run in float32 in a fixed order (independent of the launch geometry).
+//    over the lanes of the row. The 32 signed bytes are read as aligned 32-bit words
+//    (funnel-shifted when the block starts 2 bytes into a word) and turned into floats by a
+//    byte permute into the bits of 2^23 + (q + 128) and one subtraction, on the ALU and FMA
+//    pipes rather than the int-to-float converter.
+// Sums run in float32 in a fixed order (independent of the launch geometry). The kernels are
+// programmatic dependent launches: each waits for the kernel before it (which may produce h)
+// before reading anything, then lets the next one be scheduled, so back-to-back calls (the
+// engine reads the table four times per draft block) overlap their launch latency.
 #pragma once
 
 #include <cuda_fp16.h>
@@ -39,11 +50,47 @@ __device__ __forceinline__ void unpack_f16x8(const uint4& w, float* f) {
   }
 }
 
+__host__ __device__ constexpr int pow2_ceil(int x) { return x <= 1 ? 1 : 2 * pow2_ceil((x + 1) / 2); }
+
+// Warp sum of M values per lane (M a power of two <= 32), transposed: in round t (t < log2 M)
+// lanes exchange half of their values with the lane 16 >> t away and keep the sums of the
+// other half, then the last rounds add a single value. Lane l ends with the total over the
+// warp of value index sum_t (bit (4 - t) of l) * (M >> (t + 1)); every lane that shares those
+// bits holds the same total.
+template <int M>
+__device__ __forceinline__ float warp_transpose_sum(float (&v)[M], int lane) {
+  int off = 16;
+#pragma unroll
+  for (int half = M / 2; half >= 1; half /= 2, off >>= 1) {
+    const bool upper = (lane & off) != 0;
+#pragma unroll
+    for (int j = 0; j < half; ++j) {
+      const float keep = upper ? v[j + half] : v[j];
+      const float give = upper ? v[j] : v[j + half];
+      v[j] = __fadd_rn(keep, __shfl_xor_sync(0xffffffffu, give, off));
+    }
+  }
+  float s = v[0];
+#pragma unroll
+  for (; off >= 1; off >>= 1) s = __fadd_rn(s, __shfl_xor_sync(0xffffffffu, s, off));
+  return s;
+}
+template <int M>
+__device__ __forceinline__ int transpose_sum_index(int lane) {
+  int idx = 0, off = 16;
+#pragma unroll
+  for (int half = M / 2; half >= 1; half /= 2, off >>= 1)
+    if (lane & off) idx += half;
+  return idx;
+}
+
 template <int NB>
 __global__ void __launch_bounds__(kMarkovThreads) markov_f16_kernel(const uint16_t* __restrict__ W,
                                                                     int V, const float* h,
                                                                     float* y, int ldy) {
   constexpr int ROWS = NB <= 2 ? 8 : 4;
+  grid_dependency_wait();  // h comes from the kernel before (programmatic launch)
+  grid_dependents_launch();
   const int lane = threadIdx.x & 31;
   const int gw = blockIdx.x * (kMarkovThreads / 32) + (threadIdx.x >> 5);
   const int nw = gridDim.x * (kMarkovThreads / 32);
@@ -62,75 +109,152 @@ __global__ void __launch_bounds__(kMarkovThreads) markov_f16_kernel(const uint16
     for (int r = 0; r < ROWS; ++r)
       w[r] = v0 + r < V ? ld_stream16(W + (v0 + r) * kMarkovRank + 8 * lane)
                         : make_uint4(0, 0, 0, 0);
+    if constexpr (NB == 1) {
+      // one state: a butterfly per row, the rows' chains independent of one another
 #pragma unroll
-    for (int r = 0; r < ROWS; ++r) {
-      float f[8];
-      unpack_f16x8(w[r], f);
+      for (int r = 0; r < ROWS; ++r) {
+        float f[8];
+        unpack_f16x8(w[r], f);
+        float acc = __fmul_rn(f[0], hr[0][0]);
 #pragma unroll
-      for (int b = 0; b < NB; ++b) {
-        float acc = __fmul_rn(f[0], hr[b][0]);
-#pragma unroll
-        for (int e = 1; e < 8; ++e) acc = __fmaf_rn(f[e], hr[b][e], acc);
+        for (int e = 1; e < 8; ++e) acc = __fmaf_rn(f[e], hr[0][e], acc);
         acc = warp_sum(acc);
-        if (lane == 0 && v0 + r < V) y[static_cast<long long>(b) * ldy + v0 + r] = acc;
+        if (lane == 0 && v0 + r < V) y[v0 + r] = acc;
+      }
+    } else {
+      constexpr int M = pow2_ceil(ROWS * NB);
+      float part[M];
+#pragma unroll
+      for (int m = ROWS * NB; m < M; ++m) part[m] = 0.f;
+#pragma unroll
+      for (int r = 0; r < ROWS; ++r) {
+        float f[8];
+        unpack_f16x8(w[r], f);
+#pragma unroll
+        for (int b = 0; b < NB; ++b) {
+          if constexpr (NB == 2) {  // (3 or 4 states: packed pairs, fewer instructions)
+            float acc = __fmul_rn(f[0], hr[b][0]);
+#pragma unroll
+            for (int e = 1; e < 8; ++e) acc = __fmaf_rn(f[e], hr[b][e], acc);
+            part[r * NB + b] = acc;
+            continue;
+          }
+          // even and odd elements in the two halves of a packed accumulator
+          uint64_t acc = fma2(pk2(f[0], f[1]), pk2(hr[b][0], hr[b][1]), 0ull);
+#pragma unroll
+          for (int e = 2; e < 8; e += 2)
+            acc = fma2(pk2(f[e], f[e + 1]), pk2(hr[b][e], hr[b][e + 1]), acc);
+          float lo, hi;
+          upk2(acc, lo, hi);
+          part[r * NB + b] = __fadd_rn(lo, hi);
+        }
+      }
+      const float tot = warp_transpose_sum<M>(part, lane);
+      const int idx = transpose_sum_index<M>(lane);
+      if ((lane & (32 / M - 1)) == 0 && idx < ROWS * NB) {
+        const int r = idx / NB, b = idx % NB;
+        if (v0 + r < V) y[static_cast<long long>(b) * ldy + v0 + r] = tot;
       }
     }
   }
 }
 
+// Four signed bytes (a 32-bit word) -> 4 floats, exactly: each byte, biased by 128, goes into
+// the low mantissa bits of 2^23 (a byte permute), and 2^23 + 128 is subtracted.
+__device__ __forceinline__ void s8x4_to_float(uint32_t x, float* f) {
+  const uint32_t u = x ^ 0x80808080u;
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+    f[i] = __fsub_rn(__uint_as_float(__byte_perm(u, 0x4B000000u, 0x7540u | i)), 8388736.f);
+}
+
+// 16 bytes global -> shared without registers (bypassing L1); n = 0 zero-fills.
+__device__ __forceinline__ void cp_async16(void* dst, const void* src, int n) {
+  const uint32_t d = static_cast<uint32_t>(__cvta_generic_to_shared(dst));
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(d), "l"(src), "r"(n)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+// A warp's groups are double-buffered: the copy of its next group is in flight while it
+// decodes the current one. 5 CTAs (40 warps) per SM, 4 with 3 or 4 states (their sums need
+// more than 51 registers).
 template <int NB>
-__global__ void __launch_bounds__(kMarkovThreads) markov_q8_0_kernel(const uint8_t* __restrict__ W,
-                                                                     int V, const float* h,
-                                                                     float* y, int ldy) {
-  __shared__ __align__(16) uint8_t s_rows[kMarkovThreads / 32][kQ8Rows * kQ8RowBytes];
-  // the states, block by block with a stride of 33 floats, so that the 8 lanes of a row (one
-  // per block) read 8 different banks
-  __shared__ float s_h[NB][8 * 33];
-  for (int i = threadIdx.x; i < NB * kMarkovRank; i += kMarkovThreads) {
-    const int b = i / kMarkovRank, k = i % kMarkovRank;
-    s_h[b][(k >> 5) * 33 + (k & 31)] = h[i];
-  }
-  __syncthreads();
+__global__ void __launch_bounds__(kMarkovThreads, NB <= 2 ? 5 : 4) markov_q8_0_kernel(
+    const uint8_t* __restrict__ W, int V, const float* h, float* y, int ldy) {
+  constexpr int kGroupBytes = kQ8Rows * kQ8RowBytes;  // 2176
+  constexpr int kPieces = kGroupBytes / 16;           // 136 16-byte pieces per group
+  __shared__ __align__(16) uint8_t s_rows[kMarkovThreads / 32][2][kGroupBytes];
+  // the states, block by block with a stride of 36 floats (16-byte rows whose four-word reads
+  // by the 8 lanes of a row, one per block, hit 32 different banks)
+  constexpr int kHS = 36;
+  __shared__ __align__(16) float s_h[NB][8 * kHS];
   const int lane = threadIdx.x & 31, wi = threadIdx.x >> 5;
+  const int blk = lane & 7;
   const int gw = blockIdx.x * (kMarkovThreads / 32) + wi;
   const int nw = gridDim.x * (kMarkovThreads / 32);
-  uint8_t* buf = s_rows[wi];
-  constexpr int kPieces = kQ8Rows * kQ8RowBytes / 16;   // 136 16-byte pieces per group
-  const int blk = lane & 7;
-  for (long long v0 = static_cast<long long>(gw) * kQ8Rows; v0 < V;
-       v0 += static_cast<long long>(nw) * kQ8Rows) {
+  const long long stride = static_cast<long long>(nw) * kQ8Rows;
+  // copy of the group at row v0 into buffer st (rows past V zero-filled), as one commit group
+  auto fetch = [&](long long v0, int st) {
     const long long nbytes = (V - v0 < kQ8Rows ? V - v0 : kQ8Rows) * kQ8RowBytes;
     const uint8_t* src = W + v0 * kQ8RowBytes;
-    uint4 piece[(kPieces + 31) / 32];
 #pragma unroll
     for (int k = 0; k < (kPieces + 31) / 32; ++k) {
       const int c = lane + 32 * k;
-      piece[k] = c < kPieces && 16LL * c < nbytes ? ld_stream16(src + 16 * c)
-                                                 : make_uint4(0, 0, 0, 0);
+      if (c < kPieces) {
+        const bool in = 16LL * c < nbytes;
+        cp_async16(&s_rows[wi][st][16 * c], in ? src + 16 * c : W, in ? 16 : 0);
+      }
     }
-#pragma unroll
-    for (int k = 0; k < (kPieces + 31) / 32; ++k) {
-      const int c = lane + 32 * k;
-      if (c < kPieces) *reinterpret_cast<uint4*>(buf + 16 * c) = piece[k];
+    cp_async_commit();
+  };
+  grid_dependency_wait();  // h comes from the kernel before (programmatic launch)
+  grid_dependents_launch();
+  long long v0 = static_cast<long long>(gw) * kQ8Rows;
+  if (v0 < V) fetch(v0, 0);
+  for (int i = threadIdx.x; i < NB * kMarkovRank; i += kMarkovThreads) {
+    const int b = i / kMarkovRank, k = i % kMarkovRank;
+    s_h[b][(k >> 5) * kHS + (k & 31)] = h[i];
+  }
+  __syncthreads();
+  for (int st = 0; v0 < V; v0 += stride, st ^= 1) {
+    if (v0 + stride < V) {
+      fetch(v0 + stride, st ^ 1);
+      cp_async_wait<1>();
+    } else {
+      cp_async_wait<0>();
     }
-    __syncwarp();
+    __syncwarp();  // every lane's copies of this group have landed
+    const uint8_t* buf = s_rows[wi][st];
 #pragma unroll
     for (int half = 0; half < 2; ++half) {
       const int row = half * 4 + (lane >> 3);
-      const uint8_t* blockp = buf + row * kQ8RowBytes + blk * 34;
-      const float d = __half2float(*reinterpret_cast<const __half*>(blockp));
+      const int qoff = row * kQ8RowBytes + blk * 34 + 2;  // first signed byte of the block
+      const float d = __half2float(*reinterpret_cast<const __half*>(buf + qoff - 2));
+      const uint32_t* wp = reinterpret_cast<const uint32_t*>(buf + (qoff & ~3));
+      const uint32_t sh = (qoff & 3) * 8;  // 0 or 16
       float acc[NB];
 #pragma unroll
       for (int b = 0; b < NB; ++b) acc[b] = 0.f;
+      uint32_t lo = wp[0];
 #pragma unroll
-      for (int i = 0; i < 32; i += 2) {
-        const uint16_t two = *reinterpret_cast<const uint16_t*>(blockp + 2 + i);
-        const float q0 = static_cast<float>(static_cast<int8_t>(two & 0xff));
-        const float q1 = static_cast<float>(static_cast<int8_t>(two >> 8));
+      for (int k = 0; k < 8; ++k) {
+        // a block 2 bytes into a word ends 2 bytes into a 9th
+        const uint32_t hi = (k < 7 || sh) ? wp[k + 1] : 0u;
+        float q[4];
+        s8x4_to_float(__funnelshift_r(lo, hi, sh), q);
+        lo = hi;
 #pragma unroll
         for (int b = 0; b < NB; ++b) {
-          acc[b] = __fmaf_rn(q0, s_h[b][33 * blk + i], acc[b]);
-          acc[b] = __fmaf_rn(q1, s_h[b][33 * blk + i + 1], acc[b]);
+          const float4 a = *reinterpret_cast<const float4*>(&s_h[b][blk * kHS + 4 * k]);
+          acc[b] = __fmaf_rn(q[0], a.x, acc[b]);
+          acc[b] = __fmaf_rn(q[1], a.y, acc[b]);
+          acc[b] = __fmaf_rn(q[2], a.z, acc[b]);
+          acc[b] = __fmaf_rn(q[3], a.w, acc[b]);
         }
       }
 #pragma unroll
@@ -141,7 +265,7 @@ __global__ void __launch_bounds__(kMarkovThreads) markov_q8_0_kernel(const uint8
         if (blk == 0 && v0 + row < V) y[static_cast<long long>(b) * ldy + v0 + row] = s;
       }
     }
-    __syncwarp();  // the buffer is refilled by the next group
+    __syncwarp();  // the buffer is refilled two groups on
   }
 }
 

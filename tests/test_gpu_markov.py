@@ -54,3 +54,4 @@ def test_one_hot_state_reads_a_column():
     y = bd.markov_matvec(torch.from_numpy(raw).to(DEV), "q8_0", torch.from_numpy(H).to(DEV))
     torch.cuda.synchronize()
     assert np.array_equal(y.cpu().numpy()[0].astype(np.float64), mk.q8_0_table(raw, R)[:, 77])
+

@@ -76,3 +76,4 @@ def test_synthetic_q8_0_table_within_the_quantiser_bound():
     d = np.abs(got).reshape(V, R // 32, 32).max(axis=2) / 127.0
     err = np.abs(got - ref).reshape(V, R // 32, 32)
     assert np.all(err <= (d[:, :, None] * 0.5 * 1.01 + np.abs(ref).reshape(V, R // 32, 32) * 2e-3))
+
