@@ -358,6 +358,7 @@ def run_ours(args, w):
         dist.destroy_process_group()
     if rank != 0:
         return
+    markov = time_markov_matvec(dev)
 
     peaks = measured_peaks()
     peak = peaks["hbm_gbs"] if peaks else FALLBACK_HBM_GBS
@@ -402,6 +403,10 @@ def run_ours(args, w):
     if mixed:
         mixed["frac_of_peak"] = mixed["GB_per_s"] / peak
         call_stats["mixed_batch"] = mixed
+    if markov:
+        for m in markov.values():
+            m["frac_of_peak"] = m["GB_per_s"] / peak
+        call_stats["markov_matvec"] = markov
     if clk:
         line["clocks"] = clk
     if e2e:
@@ -447,6 +452,56 @@ def time_mixed_batch(w, sets, D, U, workspace, dev, reps):
     return {"us_per_call": us, "bytes_read": nbytes, "GB_per_s": nbytes / (us * 1e-6) / 1e9,
             "mean_drafts": float(kb.mean()), "greedy_sequences": int((Tb == 0).sum()),
             "committed_tokens_per_block": float((out.n_accepted.double() + 1).mean().item())}
+
+
+MARKOV_V, MARKOV_R = 129280, 256  # the DSpark drafters' vocabulary and Markov rank
+
+
+def time_markov_matvec(dev, n=50, replays=5):
+    """The drafter's Markov-head table mat-vec (y = W h over a V x 256 table), timed alone (not
+    part of the step): n calls on rotating copies of the table (more than L2 in total)
+    captured in one CUDA graph, events around its replays. Bytes: the table, read once per
+    call (the states and outputs are under 0.1% of it)."""
+    import torch
+
+    from lossless_draft_verification_speculative_b200 import binding as bd
+    from lossless_draft_verification_speculative_b200 import workloads as wl
+
+    res = {}
+    stream = torch.cuda.Stream(device=dev)
+    for fmt in ("f16", "q8_0"):
+        raw = wl.markov_table(MARKOV_V, MARKOV_R, fmt)
+        t0 = torch.from_numpy(raw.view(np.int16) if fmt == "f16" else raw).to(dev)
+        nbytes = t0.numel() * t0.element_size()
+        copies = -(-200_000_000 // nbytes)
+        tabs = [t0] + [t0.clone() for _ in range(copies - 1)]
+        for B in (1, 4):
+            h = torch.from_numpy(wl.markov_states(B, MARKOV_R)).to(dev)
+            y = torch.empty(B, MARKOV_V, device=dev)
+            with torch.cuda.stream(stream):
+                for i in range(8):
+                    bd.markov_matvec(tabs[i % copies], fmt, h, out=y)
+            torch.cuda.synchronize(dev)
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                for i in range(n):
+                    bd.markov_matvec(tabs[i % copies], fmt, h, out=y)
+            for _ in range(3):
+                g.replay()
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            torch.cuda.synchronize(dev)
+            a.record()
+            for _ in range(replays):
+                g.replay()
+            b.record()
+            torch.cuda.synchronize(dev)
+            us = a.elapsed_time(b) * 1000.0 / (replays * n)
+            res[f"{fmt}_B{B}"] = {"us_per_call": us, "table_bytes": nbytes,
+                                  "GB_per_s": nbytes / (us * 1e-6) / 1e9}
+            del g
+        del tabs, t0
+    return res
 
 
 def run_e2e(args, w, calls, P, Q, D, U, dev, tdt, outs, workspace, world):
