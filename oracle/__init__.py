@@ -12,6 +12,7 @@ from .accept_ref import (  # noqa: F401
     OracleResult,
     cdf_interval,
     draw_law,
+    early_exit_accept,
     greedy_accept,
     inverse_cdf,
     mixed_accept,

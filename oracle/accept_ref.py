@@ -43,6 +43,17 @@ its own truncated block, P rows 0..K_b (row K_b is its bonus row), Q rows 0..K_b
 those are never read. A draft count outside [0, K] or a negative or non-finite
 temperature makes that sequence an error (STATUS_BAD_PARAM).
 
+Early exit (``early_exit_accept``). The same step, reading each sequence's rows in draft
+order and stopping at its first rejection; the pages state that acceptance runs between 52%
+and 91% (the DeepSeek-V4-Flash drafter card), so most blocks end early. Reading: a
+sequence's drafts are inputs and are all checked (a bad id: STATUS_BAD_DRAFT, nothing read);
+then for i = 0..K-1 the rows P_i (and Q_i when sampling) are read, a bad one ends the
+sequence with STATUS_NONFINITE, and draft i is tested; the walk stops at the first failed
+test j. Only when every draft passes is P_K read (bad: STATUS_NONFINITE). Rows after j are
+never read, so whatever they hold cannot change the result: on blocks whose rows are all
+usable it equals ``speculative_sample_accept`` (``greedy_accept`` at T == 0), with p_draft /
+q_draft NaN past j.
+
 Parity pins: every function here is pinned in ``tests/test_oracle_pins.py`` against
 things other than itself (exact enumeration of losslessness, sequential greedy
 decoding, library inverse-CDF draws, closed-form acceptance rates, chi-square).
@@ -317,3 +328,87 @@ def mixed_accept(P: np.ndarray, Q: Optional[np.ndarray], drafts: np.ndarray,
         tokens[b, :kb + 1] = r.tokens[0]
     return OracleResult(n, tokens, nxt, status, p_draft=pd, q_draft=qd, resid_mass=zm,
                         accept_margin=am, cdf_margin=cm, argmax=amax)
+
+
+def early_exit_accept(P: np.ndarray, Q: Optional[np.ndarray], drafts: np.ndarray, T: float,
+                      u: Optional[np.ndarray]) -> OracleResult:
+    """The verify step read row by row, stopping each sequence at its first rejection.
+
+    P: [B, K+1, V], Q: [B, K, V] float64 logits (Q and u may be None when T == 0); drafts
+    [B, K]; u: [B, K+1]. Sequence b walks i = 0..K-1: P_i (and Q_i) must be usable rows, then
+    draft x_i is tested (T == 0: x_i == argmax P_i; else u_i q_i(x_i) < p_i(x_i)); the first
+    failure is j. Every draft accepted: P_K must be usable and j = K. The token is argmax P_j
+    (T == 0) or the inverse CDF at u_K of max(p_j - q_j, 0) (p_j if that has no mass) or of
+    p_K. Rows after j are not looked at.
+    """
+    greedy = T == 0
+    if not greedy and not (T > 0 and np.isfinite(T)):
+        raise ValueError("temperature must be finite and >= 0")
+    P = np.asarray(P, dtype=np.float64)
+    drafts = np.asarray(drafts)
+    B, K1, V = P.shape
+    K = K1 - 1
+    if not greedy:
+        Q = np.asarray(Q, dtype=np.float64)
+        u = np.asarray(u, dtype=np.float64)
+    n = np.zeros(B, dtype=np.int32)
+    tokens = np.full((B, K + 1), -1, dtype=np.int32)
+    nxt = np.full(B, -1, dtype=np.int32)
+    status = np.zeros(B, dtype=np.int32)
+    pd = np.full((B, K), np.nan)
+    qd = np.full((B, K), np.nan)
+    zm = np.full(B, np.nan)
+    am = np.full((B, K), np.inf)
+    cm = np.full(B, np.inf)
+    amax = np.full((B, K + 1), -1, dtype=np.int32)
+    for b in range(B):
+        if K and (np.any(drafts[b] < 0) or np.any(drafts[b] >= V)):
+            status[b] = STATUS_BAD_DRAFT
+            continue
+        j, bad = K, False
+        for i in range(K):
+            if _row_is_bad(P[b, i]) or (not greedy and _row_is_bad(Q[b, i])):
+                bad = True
+                break
+            x = int(drafts[b, i])
+            if greedy:
+                amax[b, i] = row_argmax(P[b, i])
+                if x != amax[b, i]:
+                    j = i
+                    break
+            else:
+                p, q = softmax(P[b, i], T), softmax(Q[b, i], T)
+                pd[b, i], qd[b, i] = p[x], q[x]
+                if q[x] > 0:
+                    am[b, i] = abs(u[b, i] - p[x] / q[x])
+                if not (u[b, i] * q[x] < p[x]):
+                    j = i
+                    break
+        if not bad and j == K and _row_is_bad(P[b, K]):
+            bad = True
+        if bad:
+            status[b] = STATUS_NONFINITE
+            pd[b], qd[b], am[b] = np.nan, np.nan, np.inf
+            continue
+        st = 0
+        if greedy:
+            v = amax[b, j] = row_argmax(P[b, j])
+        else:
+            w = softmax(P[b, j], T)
+            zm[b] = 1.0
+            if j < K:
+                r = np.maximum(w - softmax(Q[b, j], T), 0.0)
+                if r.sum() > 0:
+                    w, zm[b] = r, r.sum()
+                else:
+                    st, zm[b] = STATUS_ZERO_RESIDUAL, 0.0
+            v, cm[b] = inverse_cdf(w, float(u[b, K]))
+        status[b] = st
+        n[b] = j
+        tokens[b, :j] = drafts[b, :j]
+        tokens[b, j] = v
+        nxt[b] = v
+    return OracleResult(n, tokens, nxt, status, p_draft=None if greedy else pd,
+                        q_draft=None if greedy else qd, resid_mass=None if greedy else zm,
+                        accept_margin=None if greedy else am, cdf_margin=None if greedy else cm,
+                        argmax=amax)
