@@ -47,6 +47,8 @@ def parse_args():
                     help="seconds of oracle work timed for the CPU baseline (whole steps)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-stress", action="store_true",
+                    help="skip the early-exit timing on the B=256, K=15, V=262144 workload")
     return ap.parse_args()
 
 
@@ -359,6 +361,9 @@ def run_ours(args, w):
     if rank != 0:
         return
     markov = time_markov_matvec(dev)
+    early = time_early_exit_serving(w, sets, Dd, Ud, workspace, dev, reps, per_call_us, calls)
+    if not args.no_stress:
+        early.update(time_early_exit_stress(dev))
 
     peaks = measured_peaks()
     peak = peaks["hbm_gbs"] if peaks else FALLBACK_HBM_GBS
@@ -407,6 +412,7 @@ def run_ours(args, w):
         for m in markov.values():
             m["frac_of_peak"] = m["GB_per_s"] / peak
         call_stats["markov_matvec"] = markov
+    call_stats["early_exit"] = early
     if clk:
         line["clocks"] = clk
     if e2e:
@@ -452,6 +458,100 @@ def time_mixed_batch(w, sets, D, U, workspace, dev, reps):
     return {"us_per_call": us, "bytes_read": nbytes, "GB_per_s": nbytes / (us * 1e-6) / 1e9,
             "mean_drafts": float(kb.mean()), "greedy_sequences": int((Tb == 0).sum()),
             "committed_tokens_per_block": float((out.n_accepted.double() + 1).mean().item())}
+
+
+def early_exit_bytes(n_accepted, K, V, elem_bytes, sample):
+    """Bytes the early-exit call streams: wave w (pairs [2^w - 1, 2^(w+1) - 1) cut at K, the
+    last adding the bonus row) reads its rows of every sequence that accepted all drafts
+    before it, i.e. whose accepted count is at least the wave's first pair."""
+    waves, w = [], 0
+    while True:
+        lo, hi = min(2 ** w - 1, K), min(2 ** (w + 1) - 1, K)
+        waves.append((lo, hi))
+        if hi >= K:
+            break
+        w += 1
+    n = np.asarray(n_accepted)
+    rows = 0
+    for i, (lo, hi) in enumerate(waves):
+        per = (hi - lo) * (2 if sample else 1) + (1 if i == len(waves) - 1 else 0)
+        rows += per * int((n >= lo).sum())
+    return rows * V * elem_bytes
+
+
+def _time_calls(fns, reps, warm=3):
+    import torch
+
+    for r in range(warm):
+        fns[r % len(fns)]()
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    a.record()
+    for r in range(reps):
+        fns[r % len(fns)]()
+    b.record()
+    torch.cuda.synchronize()
+    return a.elapsed_time(b) * 1000.0 / reps
+
+
+def time_early_exit_serving(w, sets, Dd, Ud, workspace, dev, reps, per_call_us, calls):
+    """early_exit_accept on the step's inputs (outside the step), beside the full call of the
+    same temperature: back-to-back calls on the rotating input sets. Bytes are those the
+    waves stream (``early_exit_bytes``), from the call's own accepted counts."""
+    from lossless_draft_verification_speculative_b200 import binding as bd
+
+    res = {}
+    for c, (kind, T) in enumerate(calls):
+        out = bd._alloc_result(w.B, w.K, dev, diagnostics=True)
+        fns = [bd.PreparedCall("early_exit", P, Q, Dd[T], T, Ud[T], out, workspace)
+               for P, Q in sets]
+        us = _time_calls(fns, reps)
+        nb = early_exit_bytes(out.n_accepted.cpu().numpy(), w.K, w.V, w.elem_bytes, T > 0)
+        res[f"{w.name}_T{T}"] = {"us_per_call": us, "full_call_us": per_call_us[c],
+                                 "bytes_streamed": nb, "GB_per_s": nb / (us * 1e-6) / 1e9,
+                                 "mean_accepted": float(out.n_accepted.double().mean().item())}
+    return res
+
+
+def time_early_exit_stress(dev, reps=20):
+    """The B=256, K=15, V=262144 workload (4.2 GB per sampling call, far above L2): the full
+    call and early_exit_accept at each of its temperatures, back to back on one input set."""
+    import torch
+
+    from lossless_draft_verification_speculative_b200 import binding as bd
+    from lossless_draft_verification_speculative_b200 import workloads as wl
+
+    w = wl.WORKLOADS["stress"]
+    P, Q, D = wl.generate(w, w.temperatures, processes=min(16, os.cpu_count() or 1))
+    Pd = torch.from_numpy(P.view(np.int16)).to(dev).view(torch.bfloat16)
+    Qd = torch.from_numpy(Q.view(np.int16)).to(dev).view(torch.bfloat16)
+    del P, Q
+    ws = bd.new_workspace(bd.workspace_bytes(w.B, w.K, w.V, torch.bfloat16), dev)
+    res = {}
+    for T in w.temperatures:
+        dd = torch.from_numpy(D[T]).to(dev)
+        ud = torch.from_numpy(wl.uniforms(w, T=T)).to(dev)
+        out_f = bd._alloc_result(w.B, w.K, dev, diagnostics=True)
+        out_e = bd._alloc_result(w.B, w.K, dev, diagnostics=True)
+        full = bd.PreparedCall("greedy" if T == 0 else "sample", Pd, Qd, dd, T, ud, out_f, ws)
+        early = bd.PreparedCall("early_exit", Pd, Qd, dd, T, ud, out_e, ws)
+        us_f = _time_calls([full], reps)
+        us_e = _time_calls([early], reps)
+        n = out_e.n_accepted.cpu().numpy()
+        same = bool(torch.equal(out_f.tokens, out_e.tokens))
+        full_bytes = w.greedy_bytes() if T == 0 else w.sampling_bytes()
+        nb = early_exit_bytes(n, w.K, w.V, w.elem_bytes, T > 0)
+        res[f"stress_T{T}"] = {"us_per_call": us_e, "full_call_us": us_f,
+                               "full_call_bytes": full_bytes, "bytes_streamed": nb,
+                               "GB_per_s": nb / (us_e * 1e-6) / 1e9,
+                               "full_call_GB_per_s": full_bytes / (us_f * 1e-6) / 1e9,
+                               "blocks_per_s": w.B / (us_e * 1e-6),
+                               "full_call_blocks_per_s": w.B / (us_f * 1e-6),
+                               "mean_accepted": float(n.mean()), "same_tokens": same}
+    del Pd, Qd, ws
+    torch.cuda.empty_cache()
+    return res
 
 
 MARKOV_V, MARKOV_R = 129280, 256  # the DSpark drafters' vocabulary and Markov rank

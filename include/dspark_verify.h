@@ -104,6 +104,7 @@ int dspark_version(void);
 
 /* Bytes of device workspace the verify calls need for this shape (valid for both policies).
  * Returns 0 when the shape is invalid or unsupported.
+ * The size covers every policy, dspark_early_exit_accept included.
  * A workspace needs no initialisation: a call writes every word of it that it reads.
  * dspark_workspace_zero_bytes returns the size of the prefix that must be zero before a call,
  * which is 0 for this library (kept so that callers can clear generically). One workspace
@@ -186,6 +187,30 @@ dspark_status_t dspark_mixed_accept(const void* p1, int64_t ld_p1, const void* p
                                     const float* temperatures, const float* uniforms,
                                     dspark_accept_out_t out, void* workspace,
                                     size_t workspace_bytes, void* stream);
+
+/* Early exit: the verify step reading each sequence's rows in draft order and stopping at
+ * its first rejection (greedy: its first mismatch). The pages report acceptance between 52%
+ * and 91% (DeepSeek-V4-Flash DSpark drafter card), so most blocks end early, and the rows
+ * after a sequence's first rejection j cannot change its result; the large blocks (B=256,
+ * K=15, V=262144 reads 4.2 GB in full) then read a fraction of their bytes.
+ *  Arguments as for speculative_sample_accept (T == 0: greedy; q and uniforms may then be
+ *  NULL), with the same workspace.
+ *  The pairs (P_i, Q_i) are read in waves of 1, 2, 4, ... pairs (the last wave adds the
+ *  bonus row P_K); each wave reads only the sequences that accepted every earlier draft. A
+ *  call launches two kernels per wave (ceil(log2(K+1)) waves, one when K == 0) and, when
+ *  sampling, the finish.
+ *  Results: on blocks whose rows are all usable, identical to speculative_sample_accept /
+ *  greedy_accept (same records, decisions and draw). Rows after the stop are never read, so
+ *  a NaN or inf there is not reported; a bad row at or before the stop, or a bad bonus row
+ *  after a full accept, gives DSPARK_SEQ_NONFINITE; a bad draft id gives
+ *  DSPARK_SEQ_BAD_DRAFT alone (nothing is read). p_draft / q_draft are written up to the stop
+ *  and NaN after it. */
+dspark_status_t dspark_early_exit_accept(const void* p1, int64_t ld_p1, const void* pv,
+                                        int64_t ld_pv, const void* q, dspark_dtype_t dtype,
+                                        const int32_t* drafts, int B, int K, int V,
+                                        float temperature, const float* uniforms,
+                                        dspark_accept_out_t out, void* workspace,
+                                        size_t workspace_bytes, void* stream);
 
 /* The drafter's Markov-head table mat-vec (the drafter side of the cycle, beside the verify
  * step): y[b, v] = sum_k W[v, k] h[b, k] over the table markov_w2, V rows of R values. The

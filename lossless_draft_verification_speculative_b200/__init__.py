@@ -3,7 +3,8 @@
 ``greedy_accept`` and ``speculative_sample_accept`` verify a block of K drafted tokens per
 sequence against the base model's [B, K+1, V] logit block and return an ``AcceptResult``;
 ``mixed_accept`` verifies a serving batch whose sequences have their own draft counts and
-temperatures; ``markov_matvec`` is the drafter's Markov-head table mat-vec.
+temperatures; ``early_exit_accept`` reads each sequence's rows only up to its first
+rejection; ``markov_matvec`` is the drafter's Markov-head table mat-vec.
 The work runs in hand-written CUDA kernels behind a C ABI (``include/dspark_verify.h``);
 this package is the thin Python binding over it plus the seeded synthetic workloads.
 """
@@ -16,6 +17,7 @@ from .binding import (  # noqa: F401
     SEQ_ZERO_RESIDUAL,
     AcceptResult,
     DsparkError,
+    early_exit_accept,
     greedy_accept,
     load_library,
     markov_matvec,
@@ -33,6 +35,7 @@ __all__ = [
     "speculative_sample_accept",
     "speculative_sample_accept_static",
     "mixed_accept",
+    "early_exit_accept",
     "markov_matvec",
     "load_library",
     "plan",

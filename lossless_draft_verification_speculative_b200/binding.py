@@ -109,6 +109,9 @@ def load_library(build_if_missing: bool = True) -> ctypes.CDLL:
     lib.dspark_mixed_accept.restype = i32
     lib.dspark_mixed_accept.argtypes = [vp, i64, vp, i64, vp, i32, vp, vp, i32, i32, i32, vp, vp,
                                         AcceptOut, vp, sz, vp]
+    lib.dspark_early_exit_accept.restype = i32
+    lib.dspark_early_exit_accept.argtypes = [vp, i64, vp, i64, vp, i32, vp, i32, i32, i32,
+                                             ctypes.c_float, vp, AcceptOut, vp, sz, vp]
     lib.dspark_markov_matvec.restype = i32
     lib.dspark_markov_matvec.argtypes = [vp, i32, i32, i32, vp, i32, vp, vp]
     lib.dspark_speculative_sample_accept_static.restype = i32
@@ -333,6 +336,42 @@ def mixed_accept(P: Union[torch.Tensor, Tuple[torch.Tensor, torch.Tensor]],
     return res
 
 
+def early_exit_accept(P: Union[torch.Tensor, Tuple[torch.Tensor, torch.Tensor]],
+                      Q: Optional[torch.Tensor], drafts: torch.Tensor, temperature: float,
+                      uniforms: Optional[torch.Tensor], *, out: Optional[AcceptResult] = None,
+                      workspace: Optional[torch.Tensor] = None) -> AcceptResult:
+    """The verify step with early exit: each sequence's rows are read in draft order, in
+    waves, until its first rejection (T == 0: its first greedy mismatch; Q and uniforms may
+    then be None). Identical results to ``speculative_sample_accept`` on blocks whose rows
+    are all usable; rows after a sequence's stop are never read."""
+    lib = load_library()
+    p1, pv, ld_p1, ld_pv = _split_block(P)
+    if not p1.is_cuda:
+        raise RuntimeError("early_exit_accept runs on CUDA tensors only")
+    B, V = p1.shape
+    K = 0 if pv is None else pv.shape[1]
+    drafts = _check_drafts(drafts, B, K, p1.device)
+    if temperature > 0:
+        if K > 0 and (Q is None or Q.shape != (B, K, V) or not Q.is_contiguous() or
+                      Q.dtype != p1.dtype):
+            raise ValueError("Q must be a contiguous [B, K, V] tensor of P's dtype")
+        if uniforms is None or uniforms.dtype != torch.float32 or \
+                uniforms.shape != (B, K + 1) or not uniforms.is_contiguous() or \
+                uniforms.device != p1.device:
+            raise ValueError("uniforms must be a contiguous float32 [B, K+1] tensor on P's "
+                             "device")
+    res = out if out is not None else _alloc_result(B, K, p1.device, diagnostics=True)
+    nbytes = lib.dspark_workspace_bytes(B, K, V, DTYPE_CODES[p1.dtype])
+    ws = workspace if workspace is not None else _WS.get(p1.device, nbytes, B, K)
+    rc = lib.dspark_early_exit_accept(
+        _ptr(p1), ld_p1, _ptr(pv), ld_pv, _ptr(Q), DTYPE_CODES[p1.dtype], _ptr(drafts), B, K,
+        V, float(temperature), _ptr(uniforms), _out_struct(res), _ptr(ws),
+        ws.numel() * ws.element_size(), _stream_handle(p1.device))
+    if rc != DSPARK_OK:
+        raise DsparkError(rc, "dspark_early_exit_accept")
+    return res
+
+
 MARKOV_TABLE_CODES = {"f16": 0, "q8_0": 1}
 
 
@@ -422,6 +461,11 @@ class PreparedCall:
             self.fn = self.lib.dspark_greedy_accept
             self.args = (_ptr(p1), ld_p1, _ptr(pv), ld_pv, dt, _ptr(drafts), B, K, V,
                          _out_struct(out), _ptr(workspace), nbytes, stream)
+        elif policy == "early_exit":
+            self.fn = self.lib.dspark_early_exit_accept
+            self.args = (_ptr(p1), ld_p1, _ptr(pv), ld_pv, _ptr(Q), dt, _ptr(drafts), B, K, V,
+                         float(temperature), _ptr(uniforms), _out_struct(out), _ptr(workspace),
+                         nbytes, stream)
         elif policy == "mixed":  # temperature: float32 [B] tensor
             self.fn = self.lib.dspark_mixed_accept
             self.args = (_ptr(p1), ld_p1, _ptr(pv), ld_pv, _ptr(Q), dt, _ptr(drafts),

@@ -21,7 +21,7 @@ INCLUDE = os.path.join(ROOT, "include")
 LIB_DIR = os.path.join(PKG_DIR, "_lib")
 LIB_PATH = os.path.join(LIB_DIR, "libdspark_verify.so")
 SOURCES = ["dspark_verify.cu"]
-HEADERS = ["common.cuh", "stream.cuh", "finish.cuh", "markov.cuh"]
+HEADERS = ["common.cuh", "stream.cuh", "finish.cuh", "early_exit.cuh", "markov.cuh"]
 
 
 def nvcc_path() -> str:

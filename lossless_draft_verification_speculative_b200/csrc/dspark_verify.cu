@@ -8,6 +8,7 @@
 #include <mutex>
 
 #include "common.cuh"
+#include "early_exit.cuh"
 #include "finish.cuh"
 #include "markov.cuh"
 #include "stream.cuh"
@@ -59,11 +60,12 @@ bool make_plan(int B, int V, dspark_dtype_t dt, bool aligned16, Plan* pl) {
 size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
 // Workspace: the pass-1 records, one float2 per (row, chunk) unit of 2K+1 rows per sequence,
-// then the draft tokens' logits (sampling). Pass 1 writes every record, and the gather of
-// every draft id in [0, V), before pass 2 reads them, so the workspace needs no
-// initialisation.
+// then the draft tokens' logits (sampling), then what the early-exit waves keep: each
+// sequence's decision, two lists of alive sequences and the per-wave alive counts. Pass 1
+// writes every record, and the gather of every draft id in [0, V), before pass 2 reads them;
+// the first early-exit wave zeroes the counts; so the workspace needs no initialisation.
 struct WsLayout {
-  size_t rec, gather, total;
+  size_t rec, gather, dec, alive, cnt, total;
 };
 
 WsLayout ws_layout(long long B, long long K, int nch) {
@@ -71,8 +73,20 @@ WsLayout ws_layout(long long B, long long K, int nch) {
   WsLayout w{};
   w.rec = 0;
   w.gather = align256(sizeof(float2) * static_cast<size_t>(B * rows * nch));
-  w.total = w.gather + align256(sizeof(float2) * static_cast<size_t>(B * K));
+  w.dec = w.gather + align256(sizeof(float2) * static_cast<size_t>(B * K));
+  w.alive = w.dec + align256(sizeof(Decision) * static_cast<size_t>(B));
+  w.cnt = w.alive + align256(sizeof(int) * 2 * static_cast<size_t>(B));
+  w.total = w.cnt + align256(sizeof(int) * kMaxWaves);
   return w;
+}
+
+// Early-exit waves for K drafts: pairs [2^w - 1, 2^(w+1) - 1) cut at K, the last one ending at K.
+int n_waves(int K) {
+  int w = 0, lo = 0, hi = 0;
+  for (;; ++w) {
+    wave_range(w, K, lo, hi);
+    if (hi >= K) return w + 1;
+  }
 }
 
 // Constants of FastDiv for divisor d >= 1 (see stream.cuh).
@@ -160,6 +174,7 @@ struct Call {
 template <typename T, int VEC, int kMode>
 dspark_status_t run_call(const Call& c, const Plan& pl, cudaStream_t stream) {
   constexpr bool kSample = kMode != kModeGreedy;
+  constexpr int kFin = kMode == kModeMixed ? kFinMixed : kFinUniform;
   const void* k1 = reinterpret_cast<const void*>(&stream_stats_kernel<T, VEC, kMode>);
   cudaError_t e = cudaSuccess;
   int ctas = resident_ctas(k1, kStreamThreads, 0, &e);
@@ -236,17 +251,134 @@ dspark_status_t run_call(const Call& c, const Plan& pl, cudaStream_t stream) {
       if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices)
         return DSPARK_ERR_CUDA;
       if (!wide[dev].load(std::memory_order_acquire)) {
-        if (cudaFuncSetAttribute(finish_sample_kernel<T, VEC, kMode == kModeMixed>,
+        if (cudaFuncSetAttribute(finish_sample_kernel<T, VEC, kFin>,
                                  cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess)
           return DSPARK_ERR_CUDA;
         wide[dev].store(true, std::memory_order_release);
       }
     }
-    e = cudaLaunchKernelEx(&cfg, finish_sample_kernel<T, VEC, kMode == kModeMixed>, fp);
+    e = cudaLaunchKernelEx(&cfg, finish_sample_kernel<T, VEC, kFin>, fp);
   }
   else
     e = cudaLaunchKernelEx(&cfg, finish_greedy_kernel<T>, fp);
   return e == cudaSuccess ? DSPARK_OK : DSPARK_ERR_CUDA;
+}
+
+// Early exit (early_exit.cuh): per wave, pass 1 over the alive sequences' rows of the wave and
+// the wave's decisions; then, when sampling, the finish from the stored decisions. Every
+// launch is a programmatic dependent of the one before.
+template <typename T, int VEC, bool kSample>
+dspark_status_t run_early_exit(const Call& c, const Plan& pl, cudaStream_t stream) {
+  const void* k1 = reinterpret_cast<const void*>(&ee_stream_kernel<T, VEC, kSample>);
+  cudaError_t e = cudaSuccess;
+  int ctas = resident_ctas(k1, kStreamThreads, 0, &e);
+  if (e != cudaSuccess) return DSPARK_ERR_CUDA;
+  if (ctas < 1) return DSPARK_ERR_UNSUPPORTED;
+  if (max_ctas_override() && max_ctas_override() < ctas) ctas = max_ctas_override();
+  const long long total_units = static_cast<long long>(c.B) * c.rs.rows * pl.nch;
+  if (total_units >= (1LL << 31)) return DSPARK_ERR_UNSUPPORTED;
+  const WsLayout w = ws_layout(c.B, c.rs.K, pl.nch);
+  const int K = c.rs.K;
+  const int W = n_waves(K);
+  int* alive[2] = {reinterpret_cast<int*>(c.ws + w.alive),
+                   reinterpret_cast<int*>(c.ws + w.alive) + c.B};
+  int* cnt = reinterpret_cast<int*>(c.ws + w.cnt);
+  Decision* dec = reinterpret_cast<Decision*>(c.ws + w.dec);
+
+  cudaLaunchAttribute pdl[1];
+  pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  pdl[0].val.programmaticStreamSerializationAllowed = 1;
+  for (int wv = 0; wv < W; ++wv) {
+    WaveArgs wa{};
+    wave_range(wv, K, wa.lo, wa.hi);
+    wa.last = wv == W - 1;
+    wa.wave = wv;
+    wa.alive = alive[wv & 1];
+    wa.alive_next = alive[(wv + 1) & 1];
+    wa.cnt = cnt;
+
+    EeStreamParams sp{};
+    sp.rs = c.rs;
+    sp.nch = pl.nch;
+    sp.B = c.B;
+    sp.scale = c.scale;
+    sp.rec = reinterpret_cast<float2*>(c.ws + w.rec);
+    sp.drafts = c.drafts;
+    sp.gather = reinterpret_cast<float*>(c.ws + w.gather);
+    sp.wv = wa;
+    const long long slots = static_cast<long long>(wa.hi - wa.lo) * (kSample ? 2 : 1) + wa.last;
+    const long long want = (static_cast<long long>(c.B) * slots * pl.nch + kStreamWarps - 1) /
+                           kStreamWarps;  // units of a wave in which every sequence is alive
+    cudaLaunchConfig_t c1 = {};
+    c1.gridDim = dim3(static_cast<unsigned>(want < ctas ? want : ctas), 1, 1);
+    c1.blockDim = dim3(kStreamThreads, 1, 1);
+    c1.stream = stream;
+    c1.attrs = pdl;
+    c1.numAttrs = 1;
+    e = cudaLaunchKernelEx(&c1, ee_stream_kernel<T, VEC, kSample>, sp);
+    if (e != cudaSuccess) return DSPARK_ERR_CUDA;
+
+    EeDecideParams dp{};
+    dp.rs = c.rs;
+    dp.drafts = c.drafts;
+    dp.uniforms = c.uniforms;
+    dp.nch = pl.nch;
+    dp.scale = c.scale;
+    dp.rec = sp.rec;
+    dp.gather = sp.gather;
+    dp.out = c.out;
+    dp.wv = wa;
+    dp.dec = dec;
+    cudaLaunchConfig_t c2 = {};
+    c2.gridDim = dim3(static_cast<unsigned>(c.B), 1, 1);
+    c2.blockDim = dim3(kThreads, 1, 1);
+    c2.stream = stream;
+    c2.attrs = pdl;
+    c2.numAttrs = 1;
+    e = cudaLaunchKernelEx(&c2, ee_decide_kernel<kSample>, dp);
+    if (e != cudaSuccess) return DSPARK_ERR_CUDA;
+  }
+  if constexpr (!kSample) {
+    return DSPARK_OK;
+  } else {
+    FinishParamsEarlyExit fp{};
+    fp.rs = c.rs;
+    fp.drafts = c.drafts;
+    fp.uniforms = c.uniforms;
+    fp.nch = pl.nch;
+    fp.scale = c.scale;
+    fp.rec = reinterpret_cast<float2*>(c.ws + w.rec);
+    fp.gather = reinterpret_cast<float*>(c.ws + w.gather);
+    fp.out = c.out;
+    fp.dec = dec;
+    cudaLaunchAttribute attr[2];
+    attr[0] = pdl[0];
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = static_cast<unsigned>(pl.G);
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(static_cast<long long>(c.B) * pl.G), 1, 1);
+    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.dynamicSmemBytes = static_cast<size_t>(pl.cpc) * 2 * kGroups * sizeof(float);
+    cfg.stream = stream;
+    cfg.attrs = attr;
+    cfg.numAttrs = 2;
+    if (pl.G > kPortableCluster) {  // a 16-CTA cluster is opt-in, once per kernel and device
+      static std::atomic<bool> wide[kMaxDevices];
+      int dev = 0;
+      if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices)
+        return DSPARK_ERR_CUDA;
+      if (!wide[dev].load(std::memory_order_acquire)) {
+        if (cudaFuncSetAttribute(finish_sample_kernel<T, VEC, kFinEarlyExit>,
+                                 cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess)
+          return DSPARK_ERR_CUDA;
+        wide[dev].store(true, std::memory_order_release);
+      }
+    }
+    e = cudaLaunchKernelEx(&cfg, finish_sample_kernel<T, VEC, kFinEarlyExit>, fp);
+    return e == cudaSuccess ? DSPARK_OK : DSPARK_ERR_CUDA;
+  }
 }
 
 bool out_ok(const dspark_accept_out_t& o) { return o.n_accepted && o.tokens && o.next_token; }
@@ -485,6 +617,48 @@ dspark_status_t dspark_mixed_accept(const void* p1, int64_t ld_p1, const void* p
     return a16 ? run_call<bf16_t, 8, kModeMixed>(c, pl, s)
                : run_call<bf16_t, 1, kModeMixed>(c, pl, s);
   return a16 ? run_call<float, 4, kModeMixed>(c, pl, s) : run_call<float, 1, kModeMixed>(c, pl, s);
+}
+
+dspark_status_t dspark_early_exit_accept(const void* p1, int64_t ld_p1, const void* pv,
+                                        int64_t ld_pv, const void* q, dspark_dtype_t dtype,
+                                        const int32_t* drafts, int B, int K, int V,
+                                        float temperature, const float* uniforms,
+                                        dspark_accept_out_t out, void* workspace,
+                                        size_t workspace_bytes, void* stream) {
+  if (!(temperature >= 0.f) || !std::isfinite(temperature)) return DSPARK_ERR_INVALID_ARG;
+  dspark_status_t st = check_common(p1, ld_p1, pv, ld_pv, dtype, drafts, B, K, V, out);
+  if (st != DSPARK_OK || B == 0) return st;
+  const bool sample = temperature > 0.f;
+  const size_t es = static_cast<size_t>(elem_bytes(dtype));
+  if (sample) {
+    if (!uniforms || (K > 0 && !q)) return DSPARK_ERR_INVALID_ARG;
+    if (K > 0 && !aligned(q, es)) return DSPARK_ERR_UNSUPPORTED;
+  }
+  const bool a16 = aligned(p1, 16) && (K == 0 || (aligned(pv, 16) && (!sample || aligned(q, 16)))) &&
+                   (ld_p1 * es) % 16 == 0 && (K == 0 || (ld_pv * es) % 16 == 0) &&
+                   (V * es) % 16 == 0;
+  Plan pl;
+  if (!make_plan(B, V, dtype, a16, &pl)) return DSPARK_ERR_UNSUPPORTED;
+  if (!workspace || workspace_bytes < ws_layout(B, K, pl.nch).total || !aligned(workspace, 256))
+    return DSPARK_ERR_WORKSPACE;
+  float scale = 0.f;
+  if (sample) {
+    scale = static_cast<float>(1.4426950408889634 / static_cast<double>(temperature));
+    if (!std::isfinite(scale)) return DSPARK_ERR_INVALID_ARG;
+  }
+  // the record layout of a full call: 2K+1 rows per sequence when sampling, K+1 for greedy
+  const Call c = make_call(p1, ld_p1, pv, ld_pv, sample ? q : nullptr, drafts,
+                           sample ? uniforms : nullptr, B, K, V, scale,
+                           sample ? 2 * K + 1 : K + 1, workspace, out);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (dtype == DSPARK_BF16) {
+    if (sample)
+      return a16 ? run_early_exit<bf16_t, 8, true>(c, pl, s) : run_early_exit<bf16_t, 1, true>(c, pl, s);
+    return a16 ? run_early_exit<bf16_t, 8, false>(c, pl, s) : run_early_exit<bf16_t, 1, false>(c, pl, s);
+  }
+  if (sample)
+    return a16 ? run_early_exit<float, 4, true>(c, pl, s) : run_early_exit<float, 1, true>(c, pl, s);
+  return a16 ? run_early_exit<float, 4, false>(c, pl, s) : run_early_exit<float, 1, false>(c, pl, s);
 }
 
 dspark_status_t dspark_markov_matvec(const void* table, dspark_table_t type, int V, int R,

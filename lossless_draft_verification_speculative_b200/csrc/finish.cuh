@@ -97,8 +97,8 @@ __device__ __forceinline__ float2 reduce_row(const RowRecs& rr) {
 // The rows of sequence b into s_stat (row r at s_stat[r]): all of them, or with kFiltered
 // those that `used` selects. Warp w merges rows w, w + 8, ..., two at a time so that their
 // loads overlap.
-template <bool kSample, bool kFiltered>
-__device__ __forceinline__ void merge_rows(const FinishParams& p, int b, const RowFilter& used,
+template <bool kSample, bool kFiltered, class Filter = RowFilter>
+__device__ __forceinline__ void merge_rows(const FinishParams& p, int b, const Filter& used,
                                            int wi, int lane, float2* s_stat) {
   const int rows = p.rs.rows;
   const long long r0 = static_cast<long long>(b) * rows;
@@ -479,11 +479,26 @@ __device__ __forceinline__ void prefetch_l2(const void* src, uint32_t bytes) {
   asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
 }
 
+// What the sampling finish starts from: the pass-1 records of a uniform call or of a mixed
+// batch (it merges them and takes the decisions), or the decisions that the early-exit waves
+// stored (early_exit.cuh).
+constexpr int kFinUniform = 0;
+constexpr int kFinMixed = 1;
+constexpr int kFinEarlyExit = 2;
+
+struct FinishParamsEarlyExit : FinishParams {
+  const Decision* dec;  // [B], written by the wave that ended each sequence
+};
+template <int kFin>
+using FinishParamsOf = std::conditional_t<
+    kFin == kFinMixed, FinishParamsMixed,
+    std::conditional_t<kFin == kFinEarlyExit, FinishParamsEarlyExit, FinishParams>>;
+
 // Sampling finish. Launched as clusters of G CTAs, one cluster per sequence; CTA g of the
 // cluster owns chunks g*cpc .. g*cpc + cpc - 1 of the draw's law (warp w: local chunks w, w+8).
-template <typename T, int VEC, bool kMixed>
-__global__ void __launch_bounds__(kThreads, 4) finish_sample_kernel(
-    const std::conditional_t<kMixed, FinishParamsMixed, FinishParams> p) {
+template <typename T, int VEC, int kFin>
+__global__ void __launch_bounds__(kThreads, 4) finish_sample_kernel(const FinishParamsOf<kFin> p) {
+  constexpr bool kMixed = kFin == kFinMixed;
   extern __shared__ float s_part[];  // [cpc][2][kGroups]: group sums (residual, p)
   __shared__ float2 s_stat[kMaxRows];
   __shared__ float2 s_mass[kMaxChunkCount];  // every chunk's (residual, p) mass
@@ -531,63 +546,69 @@ __global__ void __launch_bounds__(kThreads, 4) finish_sample_kernel(
   if (tid < nd) x = p.drafts[static_cast<size_t>(b) * K + tid];
   if (tid <= nd) s_u[tid] = p.uniforms[static_cast<size_t>(b) * K1 + tid];
   grid_dependency_wait();
-  // the draft tokens' logits, gathered by pass 1
-  if (tid < nd) {
-    s_x[tid] = x;
-    float2 zg = make_float2(0.f, 0.f);
-    if (x >= 0 && x < V) zg = __ldcg(reinterpret_cast<const float2*>(p.gather) + static_cast<size_t>(b) * K + tid);
-    s_zp[tid] = zg.x;
-    s_zq[tid] = zg.y;
-  }
-  __syncthreads();
-
-  // the (reference, sum) of every row the sequence uses
-  const RowFilter used{K, nd, true};
-  merge_rows<true, kMixed>(p, b, used, wi, lane, s_stat);
-  __syncthreads();
-
-  // decisions (warp 0; draft i on lane i)
-  if (wi == 0) {
-    int status = 0;
-    bool bad = false;
-    for (int r = lane; r < rows; r += 32) bad |= (!kMixed || used(r)) && !stat_ok(s_stat[r]);
-    if (__any_sync(0xffffffffu, bad)) status |= DSPARK_SEQ_NONFINITE;
-    const int x = lane < nd ? s_x[lane] : 0;
-    const bool bad_draft = lane < nd && (x < 0 || x >= V);
-    if (__any_sync(0xffffffffu, bad_draft)) status |= DSPARK_SEQ_BAD_DRAFT;
-    const float fnan = __int_as_float(0x7fffffff);
-    float px = fnan, qx = fnan;
-    bool accept = false;
-    if (lane < nd && !bad_draft) {
-      const float2 sp = s_stat[lane], sq = s_stat[K1 + lane];
-      // p_i(x_i) = 2^(z*s - M) / S (division within 2 ulp: no IEEE slow path)
-      px = __fdividef(ex2(__fmaf_rn(s_zp[lane], scale, -sp.x)), sp.y);
-      qx = __fdividef(ex2(__fmaf_rn(s_zq[lane], scale, -sq.x)), sq.y);
-      accept = __fmul_rn(s_u[lane], qx) < px;
+  if constexpr (kFin == kFinEarlyExit) {
+    if (tid < nd) s_x[tid] = x;
+    if (tid == 0) s_dec = p.dec[b];
+  } else {
+    // the draft tokens' logits, gathered by pass 1
+    if (tid < nd) {
+      s_x[tid] = x;
+      float2 zg = make_float2(0.f, 0.f);
+      if (x >= 0 && x < V)
+        zg = __ldcg(reinterpret_cast<const float2*>(p.gather) + static_cast<size_t>(b) * K + tid);
+      s_zp[tid] = zg.x;
+      s_zq[tid] = zg.y;
     }
-    const unsigned rej = __ballot_sync(0xffffffffu, lane < nd && !accept);
-    const int j = rej ? __ffs(rej) - 1 : nd;
-    if (g == 0 && lane < K) {
-      if (p.out.p_draft) p.out.p_draft[static_cast<size_t>(b) * K + lane] = px;
-      if (p.out.q_draft) p.out.q_draft[static_cast<size_t>(b) * K + lane] = qx;
-    }
-    if (lane == 0) {
-      const float2 sp = s_stat[j];
-      Decision d;
-      d.j = j;
-      d.nd = nd;
-      d.status = status;
-      d.mp = sp.x;
-      d.ip = __fdividef(1.f, sp.y);
-      if (j < nd) {
-        const float2 sq = s_stat[K1 + j];
-        d.mq = sq.x;
-        d.iq = __fdividef(1.f, sq.y);
-      } else {
-        d.mq = 0.f;
-        d.iq = 0.f;
+    __syncthreads();
+
+    // the (reference, sum) of every row the sequence uses
+    const RowFilter used{K, nd, true};
+    merge_rows<true, kMixed>(p, b, used, wi, lane, s_stat);
+    __syncthreads();
+
+    // decisions (warp 0; draft i on lane i)
+    if (wi == 0) {
+      int status = 0;
+      bool bad = false;
+      for (int r = lane; r < rows; r += 32) bad |= (!kMixed || used(r)) && !stat_ok(s_stat[r]);
+      if (__any_sync(0xffffffffu, bad)) status |= DSPARK_SEQ_NONFINITE;
+      const int x = lane < nd ? s_x[lane] : 0;
+      const bool bad_draft = lane < nd && (x < 0 || x >= V);
+      if (__any_sync(0xffffffffu, bad_draft)) status |= DSPARK_SEQ_BAD_DRAFT;
+      const float fnan = __int_as_float(0x7fffffff);
+      float px = fnan, qx = fnan;
+      bool accept = false;
+      if (lane < nd && !bad_draft) {
+        const float2 sp = s_stat[lane], sq = s_stat[K1 + lane];
+        // p_i(x_i) = 2^(z*s - M) / S (division within 2 ulp: no IEEE slow path)
+        px = __fdividef(ex2(__fmaf_rn(s_zp[lane], scale, -sp.x)), sp.y);
+        qx = __fdividef(ex2(__fmaf_rn(s_zq[lane], scale, -sq.x)), sq.y);
+        accept = __fmul_rn(s_u[lane], qx) < px;
       }
-      s_dec = d;
+      const unsigned rej = __ballot_sync(0xffffffffu, lane < nd && !accept);
+      const int j = rej ? __ffs(rej) - 1 : nd;
+      if (g == 0 && lane < K) {
+        if (p.out.p_draft) p.out.p_draft[static_cast<size_t>(b) * K + lane] = px;
+        if (p.out.q_draft) p.out.q_draft[static_cast<size_t>(b) * K + lane] = qx;
+      }
+      if (lane == 0) {
+        const float2 sp = s_stat[j];
+        Decision d;
+        d.j = j;
+        d.nd = nd;
+        d.status = status;
+        d.mp = sp.x;
+        d.ip = __fdividef(1.f, sp.y);
+        if (j < nd) {
+          const float2 sq = s_stat[K1 + j];
+          d.mq = sq.x;
+          d.iq = __fdividef(1.f, sq.y);
+        } else {
+          d.mq = 0.f;
+          d.iq = 0.f;
+        }
+        s_dec = d;
+      }
     }
   }
   __syncthreads();

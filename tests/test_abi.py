@@ -105,7 +105,16 @@ def _mixed(lib, **kw):
                                    a["ws"], a["wsb"], a["s"])
 
 
-@pytest.mark.parametrize("call", [_greedy, _sample, _mixed])
+def _early_exit(lib, **kw):
+    a = dict(p1=FAKE, ld=1024, pv=FAKE, ldv=7 * 1024, q=FAKE, dt=BF16, d=FAKE, B=4, K=7, V=1024,
+             T=1.0, u=FAKE, out=_out(), ws=FAKE, wsb=1 << 30, s=None)
+    a.update(kw)
+    return lib.dspark_early_exit_accept(a["p1"], a["ld"], a["pv"], a["ldv"], a["q"], a["dt"],
+                                        a["d"], a["B"], a["K"], a["V"], a["T"], a["u"],
+                                        a["out"], a["ws"], a["wsb"], a["s"])
+
+
+@pytest.mark.parametrize("call", [_greedy, _sample, _mixed, _early_exit])
 def test_invalid_arguments(lib, call):
     INV, UNS, WS = 1, 2, 4
     assert call(lib, B=-1) == INV
@@ -168,3 +177,18 @@ def test_markov_matvec_arguments(lib):
     assert mv(R=128) == UNS                        # the drafters ship rank 256
     assert mv(t=FAKE + 8) == UNS and mv(h=FAKE + 4) == UNS and mv(y=FAKE + 2) == UNS
     assert mv(V=0) == 0 and mv(B=0) == 0           # no-ops
+
+
+def test_early_exit_specific_arguments(lib):
+    INV, UNS, WS = 1, 2, 4
+    assert _early_exit(lib, T=-0.5) == INV
+    assert _early_exit(lib, T=float("nan")) == INV
+    assert _early_exit(lib, T=1e-45) == INV
+    assert _early_exit(lib, q=None) == INV
+    assert _early_exit(lib, u=None) == INV
+    assert _early_exit(lib, q=FAKE + 1) == UNS
+    # T == 0 verifies greedily: q and uniforms may be NULL; the workspace check still applies
+    assert _early_exit(lib, T=0.0, q=None, u=None, ws=None) == WS
+    assert _early_exit(lib, K=0, pv=None, q=None, d=None, ldv=0, ws=None) == WS
+    # the one workspace size serves every policy
+    assert _early_exit(lib, wsb=lib.dspark_workspace_bytes(4, 7, 1024, BF16) - 1) == WS

@@ -124,6 +124,61 @@ def test_stress_full_size(stress, T):
             assert j == w.K or d[b, j] != am[b, j]
 
 
+def _early_exit(P, Q, d, u, T, dtype):
+    dd = torch.from_numpy(np.ascontiguousarray(d, dtype=np.int32)).to(DEV)
+    ud = torch.from_numpy(np.ascontiguousarray(u, dtype=np.float32)).to(DEV)
+    r = bd.early_exit_accept(to_dev(P, dtype), to_dev(Q, dtype) if T > 0 else None, dd, T,
+                             ud if T > 0 else None)
+    torch.cuda.synchronize()
+    return {k: v.cpu().numpy() for k, v in vars(r).items() if v is not None}
+
+
+def _ee_same_as_full(e, f, T, K):
+    for key in ("n_accepted", "tokens", "next_token", "status"):
+        assert np.array_equal(e[key], f[key]), key
+    if T > 0:
+        assert np.array_equal(e["resid_mass"], f["resid_mass"])
+        for b in range(e["n_accepted"].shape[0]):
+            t = min(int(f["n_accepted"][b]) + 1, K)
+            assert np.array_equal(e["p_draft"][b, :t], f["p_draft"][b, :t])
+            assert np.all(np.isnan(e["p_draft"][b, t:]))
+
+
+@pytest.mark.parametrize("T", [0.0, 0.7, 1.0])
+def test_dsv4_flash_serving_early_exit(dsv4, T):
+    """Early exit on the serving workload: identical to the full call, and to the oracle."""
+    w, P, Q, D = dsv4
+    d, u = D[T], wl.uniforms(w, T=T)
+    e = _early_exit(P, Q, d, u, T, w.dtype)
+    _ee_same_as_full(e, run_gpu(P, Q, d, u, T, w.dtype), T, w.K)
+    Pf = wl.as_float64(P, w.dtype)
+    o = ora.early_exit_accept(Pf, wl.as_float64(Q, w.dtype) if T else None, d, T,
+                              u.astype(np.float64) if T else None)
+    if T == 0:
+        compare_greedy(e, o)
+    else:
+        assert compare_sampling(e, o, f"ee dsv4 T={T}", (P, Q, u, T, w.dtype)) <= w.B // 4
+
+
+@pytest.mark.parametrize("T", [0.0, 0.6, 1.0])
+def test_stress_full_size_early_exit(stress, T):
+    """B256 K15 V262144 with early exit: identical to the full call on every sequence, and to
+    the oracle on sampled sequences."""
+    w, P, Q, D = stress
+    d, u = D[T], wl.uniforms(w, T=T)
+    e = _early_exit(P, Q, d, u, T, w.dtype)
+    _ee_same_as_full(e, run_gpu(P, Q, d, u, T, w.dtype), T, w.K)
+    s = STRESS_SAMPLE
+    Pf = wl.as_float64(P[s], w.dtype)
+    o = ora.early_exit_accept(Pf, wl.as_float64(Q[s], w.dtype) if T else None, d[s], T,
+                              u[s].astype(np.float64) if T else None)
+    es = {k: v[s] for k, v in e.items()}
+    if T == 0:
+        compare_greedy(es, o)
+    else:
+        compare_sampling(es, o, f"ee stress T={T}", (P[s], Q[s], u[s], T, w.dtype))
+
+
 # --------------------------------------------------------------------- conventions
 
 def test_block_convention_separate_buffers():
