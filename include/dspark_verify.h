@@ -164,6 +164,17 @@ dspark_status_t dspark_speculative_sample_accept(const void* p1, int64_t ld_p1, 
                                                  void* workspace, size_t workspace_bytes,
                                                  void* stream);
 
+/* Pass 1 of speculative_sample_accept alone: the stream of every P and Q row and its
+ * statistics records, written to the workspace, with no decision and no output. It is the
+ * call's dominant kernel; this entry point lets a benchmark time that kernel on its own (a
+ * full call launches it and then the finish, which events on the stream cannot separate).
+ * Arguments as for speculative_sample_accept; T must be > 0 (T == 0 has no sampling pass:
+ * INVALID_ARG). Returns after enqueueing one kernel on `stream`. */
+dspark_status_t dspark_sample_pass1(const void* p1, int64_t ld_p1, const void* pv, int64_t ld_pv,
+                                   const void* q, dspark_dtype_t dtype, const int32_t* drafts,
+                                   int B, int K, int V, float temperature, void* workspace,
+                                   size_t workspace_bytes, void* stream);
+
 /* A mixed serving batch: each sequence verifies its own number of drafts at its own
  * temperature, greedy where that temperature is 0. The pages truncate a block per step
  * through the drafter's confidence head or cap it (mlx-dspark README, "Tuning":

@@ -109,6 +109,9 @@ def load_library(build_if_missing: bool = True) -> ctypes.CDLL:
     lib.dspark_mixed_accept.restype = i32
     lib.dspark_mixed_accept.argtypes = [vp, i64, vp, i64, vp, i32, vp, vp, i32, i32, i32, vp, vp,
                                         AcceptOut, vp, sz, vp]
+    lib.dspark_sample_pass1.restype = i32
+    lib.dspark_sample_pass1.argtypes = [vp, i64, vp, i64, vp, i32, vp, i32, i32, i32,
+                                        ctypes.c_float, vp, sz, vp]
     lib.dspark_early_exit_accept.restype = i32
     lib.dspark_early_exit_accept.argtypes = [vp, i64, vp, i64, vp, i32, vp, i32, i32, i32,
                                              ctypes.c_float, vp, AcceptOut, vp, sz, vp]
@@ -461,6 +464,10 @@ class PreparedCall:
             self.fn = self.lib.dspark_greedy_accept
             self.args = (_ptr(p1), ld_p1, _ptr(pv), ld_pv, dt, _ptr(drafts), B, K, V,
                          _out_struct(out), _ptr(workspace), nbytes, stream)
+        elif policy == "sample_pass1":  # the sampling call's pass 1 alone (timing)
+            self.fn = self.lib.dspark_sample_pass1
+            self.args = (_ptr(p1), ld_p1, _ptr(pv), ld_pv, _ptr(Q), dt, _ptr(drafts), B, K, V,
+                         float(temperature), _ptr(workspace), nbytes, stream)
         elif policy == "early_exit":
             self.fn = self.lib.dspark_early_exit_accept
             self.args = (_ptr(p1), ld_p1, _ptr(pv), ld_pv, _ptr(Q), dt, _ptr(drafts), B, K, V,

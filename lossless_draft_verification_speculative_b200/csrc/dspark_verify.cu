@@ -172,7 +172,8 @@ struct Call {
 // the launch latency between back-to-back calls, about 2 us); pass 2's CTAs load what pass 1
 // does not write and then wait for pass 1.
 template <typename T, int VEC, int kMode>
-dspark_status_t run_call(const Call& c, const Plan& pl, cudaStream_t stream) {
+dspark_status_t run_call(const Call& c, const Plan& pl, cudaStream_t stream,
+                         bool pass1_only = false) {
   constexpr bool kSample = kMode != kModeGreedy;
   constexpr int kFin = kMode == kModeMixed ? kFinMixed : kFinUniform;
   const void* k1 = reinterpret_cast<const void*>(&stream_stats_kernel<T, VEC, kMode>);
@@ -216,6 +217,7 @@ dspark_status_t run_call(const Call& c, const Plan& pl, cudaStream_t stream) {
     e = cudaLaunchKernelEx(&c1, stream_stats_kernel<T, VEC, kMode>, sp);
     if (e != cudaSuccess) return DSPARK_ERR_CUDA;
   }
+  if (pass1_only) return DSPARK_OK;
 
   std::conditional_t<kMode == kModeMixed, FinishParamsMixed, FinishParams> fp{};
   fp.rs = c.rs;
@@ -588,6 +590,40 @@ dspark_status_t dspark_speculative_sample_accept(const void* p1, int64_t ld_p1, 
     return a16 ? run_call<bf16_t, 8, kModeSample>(c, pl, s)
                : run_call<bf16_t, 1, kModeSample>(c, pl, s);
   return a16 ? run_call<float, 4, kModeSample>(c, pl, s) : run_call<float, 1, kModeSample>(c, pl, s);
+}
+
+dspark_status_t dspark_sample_pass1(const void* p1, int64_t ld_p1, const void* pv, int64_t ld_pv,
+                                   const void* q, dspark_dtype_t dtype, const int32_t* drafts,
+                                   int B, int K, int V, float temperature, void* workspace,
+                                   size_t workspace_bytes, void* stream) {
+  if (!(temperature > 0.f) || !std::isfinite(temperature)) return DSPARK_ERR_INVALID_ARG;
+  if (dtype != DSPARK_BF16 && dtype != DSPARK_F32) return DSPARK_ERR_INVALID_ARG;
+  if (!shape_ok(B, K, V)) return DSPARK_ERR_INVALID_ARG;
+  if (B == 0) return DSPARK_OK;
+  if (!p1 || (K > 0 && (!pv || !drafts || !q))) return DSPARK_ERR_INVALID_ARG;
+  if (ld_p1 < V || (K > 0 && ld_pv < static_cast<int64_t>(K) * V)) return DSPARK_ERR_INVALID_ARG;
+  const size_t es = static_cast<size_t>(elem_bytes(dtype));
+  if (!aligned(p1, es) || (K > 0 && (!aligned(pv, es) || !aligned(q, es))))
+    return DSPARK_ERR_UNSUPPORTED;
+  if (V > kMaxChunkCount * kCE || ld_p1 > INT32_MAX || ld_pv > INT32_MAX)
+    return DSPARK_ERR_UNSUPPORTED;
+  const bool a16 = aligned(p1, 16) && (K == 0 || (aligned(pv, 16) && aligned(q, 16))) &&
+                   (ld_p1 * es) % 16 == 0 && (K == 0 || (ld_pv * es) % 16 == 0) &&
+                   (V * es) % 16 == 0;
+  Plan pl;
+  if (!make_plan(B, V, dtype, a16, &pl)) return DSPARK_ERR_UNSUPPORTED;
+  if (!workspace || workspace_bytes < ws_layout(B, K, pl.nch).total || !aligned(workspace, 256))
+    return DSPARK_ERR_WORKSPACE;
+  const float scale = static_cast<float>(1.4426950408889634 / static_cast<double>(temperature));
+  if (!std::isfinite(scale)) return DSPARK_ERR_INVALID_ARG;
+  const Call c = make_call(p1, ld_p1, pv, ld_pv, q, drafts, nullptr, B, K, V, scale, 2 * K + 1,
+                           workspace, dspark_accept_out_t{});
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (dtype == DSPARK_BF16)
+    return a16 ? run_call<bf16_t, 8, kModeSample>(c, pl, s, true)
+               : run_call<bf16_t, 1, kModeSample>(c, pl, s, true);
+  return a16 ? run_call<float, 4, kModeSample>(c, pl, s, true)
+             : run_call<float, 1, kModeSample>(c, pl, s, true);
 }
 
 dspark_status_t dspark_mixed_accept(const void* p1, int64_t ld_p1, const void* pv, int64_t ld_pv,

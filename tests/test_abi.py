@@ -192,3 +192,23 @@ def test_early_exit_specific_arguments(lib):
     assert _early_exit(lib, K=0, pv=None, q=None, d=None, ldv=0, ws=None) == WS
     # the one workspace size serves every policy
     assert _early_exit(lib, wsb=lib.dspark_workspace_bytes(4, 7, 1024, BF16) - 1) == WS
+
+
+def test_sample_pass1_arguments(lib):
+    INV, UNS, WS = 1, 2, 4
+
+    def p1(**kw):
+        a = dict(p1=FAKE, ld=1024, pv=FAKE, ldv=7 * 1024, q=FAKE, dt=BF16, d=FAKE, B=4, K=7,
+                 V=1024, T=1.0, ws=FAKE, wsb=1 << 30, s=None)
+        a.update(kw)
+        return lib.dspark_sample_pass1(a["p1"], a["ld"], a["pv"], a["ldv"], a["q"], a["dt"],
+                                       a["d"], a["B"], a["K"], a["V"], a["T"], a["ws"], a["wsb"],
+                                       a["s"])
+    assert p1(T=0.0) == INV                       # no sampling pass at T == 0
+    assert p1(T=float("nan")) == INV
+    assert p1(q=None) == INV
+    assert p1(B=-1) == INV
+    assert p1(ld=1000) == INV
+    assert p1(q=FAKE + 1) == UNS
+    assert p1(ws=None) == WS
+    assert p1(B=0) == 0

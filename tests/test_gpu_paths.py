@@ -90,3 +90,30 @@ def test_calls_of_alternating_sizes():
         ws = bd.new_workspace(bd.workspace_bytes(B, 3, V, torch.bfloat16), DEV)
         compare_sampling(_run(P, Q, d, u, 1.0, "bf16", ws), run_oracle(P, Q, d, u, 1.0, "bf16"),
                          f"alt B={B} V={V}", (P, Q, u, 1.0, "bf16"))
+
+
+@pytest.mark.parametrize("V,dtype", [(129280, "bf16"), (5001, "f32")])
+def test_pass1_alone_writes_the_full_calls_records(V, dtype):
+    """dspark_sample_pass1 (the benchmark's timing of the dominant kernel) launches the same
+    pass 1 as a full sampling call: the records and gathered logits in the workspace match
+    bit for bit."""
+    w = wl.Workload("p1", B=16, K=7, V=V, dtype=dtype, kind="mixed_sigma",
+                    params={"sd": 3.0, "sigmas": (0.25, 1.0, 4.0)})
+    P, Q = wl.logits(w)
+    T = 0.7
+    d, u = wl.drafts(w, Q, T), wl.uniforms(w, T=T)
+    Pd, Qd = to_dev(P, dtype), to_dev(Q, dtype)
+    dd = torch.from_numpy(d).to(DEV)
+    ud = torch.from_numpy(u).to(DEV)
+    tdt = torch.bfloat16 if dtype == "bf16" else torch.float32
+    nb = bd.workspace_bytes(w.B, w.K, w.V, tdt)
+    ws_full, ws_p1 = bd.new_workspace(nb, DEV), bd.new_workspace(nb, DEV)
+    bd.speculative_sample_accept(Pd, Qd, dd, T, ud, workspace=ws_full)
+    out = bd._alloc_result(w.B, w.K, DEV, diagnostics=True)
+    bd.PreparedCall("sample_pass1", Pd, Qd, dd, T, ud, out, ws_p1)()
+    torch.cuda.synchronize()
+    nch = -(-V // 2048)
+    rec = w.B * (2 * w.K + 1) * nch * 8
+    gat0 = -(-rec // 256) * 256
+    assert torch.equal(ws_full[:rec], ws_p1[:rec])
+    assert torch.equal(ws_full[gat0:gat0 + w.B * w.K * 8], ws_p1[gat0:gat0 + w.B * w.K * 8])
