@@ -369,6 +369,7 @@ def run_ours(args, w):
     if rank != 0:
         return
     markov = time_markov_matvec(dev)
+    small = time_small_batches(dev)
     early = time_early_exit_serving(w, sets, Dd, Ud, workspace, dev, reps, per_call_us, calls)
     if not args.no_stress:
         early.update(time_early_exit_stress(dev))
@@ -428,6 +429,9 @@ def run_ours(args, w):
             m["frac_of_peak"] = m["GB_per_s"] / peak
         call_stats["markov_matvec"] = markov
     call_stats["early_exit"] = early
+    for m in small.values():
+        m["frac_of_peak"] = m["GB_per_s"] / peak
+    call_stats["small_batches"] = small
     if clk:
         line["clocks"] = clk
     if e2e:
@@ -508,6 +512,41 @@ def _time_calls(fns, reps, warm=3):
     b.record()
     torch.cuda.synchronize()
     return a.elapsed_time(b) * 1000.0 / reps
+
+
+def time_small_batches(dev, reps=300):
+    """The two small verify workloads, timed alone (not part of the step): Qwen3-4B-shaped
+    B=1, K=7, V=151936 and Gemma-4-12B-shaped B=8, K=7, V=262144, greedy and sampling at T=1,
+    back-to-back calls on rotating copies of the inputs (more than L2 in all), so their
+    latency floors (two dependent launches and the finish's chain) show beside the bytes."""
+    import torch
+
+    from lossless_draft_verification_speculative_b200 import binding as bd
+    from lossless_draft_verification_speculative_b200 import workloads as wl
+
+    res = {}
+    for name in ("qwen3_4b_block7", "gemma4_12b_block7"):
+        w = wl.WORKLOADS[name]
+        P, Q = wl.logits(w)
+        Pd = torch.from_numpy(P.view(np.int16)).to(dev).view(torch.bfloat16)
+        Qd = torch.from_numpy(Q.view(np.int16)).to(dev).view(torch.bfloat16)
+        copies = max(2, -(-200_000_000 // (Pd.numel() * 2 + Qd.numel() * 2)))
+        sets = [(Pd, Qd)] + [(Pd.clone(), Qd.clone()) for _ in range(copies - 1)]
+        ws = bd.new_workspace(bd.workspace_bytes(w.B, w.K, w.V, torch.bfloat16), dev)
+        for T in (0.0, 1.0):
+            dd = torch.from_numpy(wl.drafts(w, Q, T)).to(dev)
+            ud = torch.from_numpy(wl.uniforms(w, T=T)).to(dev)
+            out = bd._alloc_result(w.B, w.K, dev, diagnostics=True)
+            kind = "greedy" if T == 0 else "sample"
+            fns = [bd.PreparedCall(kind, p, q, dd, T, ud, out, ws) for p, q in sets]
+            us = _time_calls(fns, reps, warm=len(fns))
+            nb = w.greedy_bytes() if T == 0 else w.sampling_bytes()
+            res[f"{name}_T{T}"] = {"us_per_call": us, "algorithmic_bytes": nb,
+                                   "GB_per_s": nb / (us * 1e-6) / 1e9,
+                                   "rotating_copies": copies}
+        del sets, Pd, Qd, ws
+    torch.cuda.empty_cache()
+    return res
 
 
 def time_early_exit_serving(w, sets, Dd, Ud, workspace, dev, reps, per_call_us, calls):
