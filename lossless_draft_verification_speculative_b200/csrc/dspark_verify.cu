@@ -461,7 +461,7 @@ dspark_status_t markov_launch(const void* table, dspark_table_t type, int V, con
   const int ctas = resident_ctas(fn, kMarkovThreads, 0, &e);
   if (e != cudaSuccess) return DSPARK_ERR_CUDA;
   if (ctas < 1) return DSPARK_ERR_UNSUPPORTED;
-  const long long rows_per_cta = (kMarkovThreads / 32) * (q8 ? kQ8Rows : (NB <= 2 ? 8 : 4));
+  const long long rows_per_cta = (kMarkovThreads / 32) * (q8 ? kQ8Rows : (NB == 1 ? 8 : 4));
   const long long want = (V + rows_per_cta - 1) / rows_per_cta;
   const int grid = static_cast<int>(want < ctas ? want : ctas);
   cudaLaunchAttribute attr[1];

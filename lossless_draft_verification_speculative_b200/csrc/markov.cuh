@@ -6,11 +6,11 @@
 // an HBM stream. One CTA of 8 warps per resident slot walks groups of rows grid-stride; a warp
 // keeps a group's loads in flight together:
 //  - F16: a row is 512 bytes, one 16-byte piece (8 halves) per lane; 8 rows per group (4 with
-//    3 or 4 states). Lane l holds h[b, 8l .. 8l+7] in registers and multiplies its pieces.
+//    several states: with 2 states, 8 rows took 15.1 us per 129280-row call and 4 rows 12.7). Lane l holds h[b, 8l .. 8l+7] in registers and multiplies its pieces.
 //    With one state each row's 32 partial sums are added by its own butterfly (8 independent
 //    chains); with more, the group's (row, state) partial sums are added by one transposed
-//    butterfly (each round halves the values a lane carries): 2 states x 8 rows cost 19
-//    shuffles instead of 80. With 3 or 4 states the products run as packed f32x2 FMAs (even
+//    butterfly (each round halves the values a lane carries): 2 states x 4 rows cost 9
+//    shuffles instead of 40. With 3 or 4 states the products run as packed f32x2 FMAs (even
 //    and odd elements in the two halves of the accumulator).
 //  - Q8_0: a row is 8 blocks of 34 bytes (272 bytes, so rows start 16-byte aligned). A group
 //    of 8 consecutive rows (2176 bytes) is copied by 16-byte asynchronous copies into one of
@@ -88,7 +88,7 @@ template <int NB>
 __global__ void __launch_bounds__(kMarkovThreads) markov_f16_kernel(const uint16_t* __restrict__ W,
                                                                     int V, const float* h,
                                                                     float* y, int ldy) {
-  constexpr int ROWS = NB <= 2 ? 8 : 4;
+  constexpr int ROWS = NB == 1 ? 8 : 4;
   grid_dependency_wait();  // h comes from the kernel before (programmatic launch)
   grid_dependents_launch();
   const int lane = threadIdx.x & 31;
