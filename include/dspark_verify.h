@@ -99,7 +99,8 @@ typedef struct {
 /* Human-readable name of a dspark_status_t value. Never NULL. */
 const char* dspark_status_string(int status);
 
-/* Library ABI version (bumped on any incompatible change). */
+/* Library ABI version (bumped on any incompatible change; 4: the workspace grew by the
+ * early-exit waves' state, so a size taken from an older library is too small). */
 int dspark_version(void);
 
 /* Bytes of device workspace the verify calls need for this shape (valid for both policies).

@@ -16,7 +16,7 @@
 namespace dspark {
 namespace {
 
-constexpr int kAbiVersion = 3;
+constexpr int kAbiVersion = 4;  // 4: the workspace also holds the early-exit waves' state
 constexpr int kMaxDevices = 64;
 
 // Tuning switch, read at every call: DSPARK_MAX_CTAS caps the pass-1 CTAs (0 = one per SM).
