@@ -166,6 +166,42 @@ struct Call {
   char* ws;
 };
 
+// The sampling finish: one cluster of pl.G CTAs per sequence, each with pl.cpc chunks of group
+// sums in dynamic shared memory, as a programmatic dependent of the kernel before it. A
+// 16-CTA cluster is opt-in, once per kernel instantiation and device.
+template <typename T, int VEC, int kFin>
+dspark_status_t launch_finish_sample(const FinishParamsOf<kFin>& fp, const Plan& pl, int B,
+                                     cudaStream_t stream) {
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  attr[1].id = cudaLaunchAttributeClusterDimension;
+  attr[1].val.clusterDim.x = static_cast<unsigned>(pl.G);
+  attr[1].val.clusterDim.y = 1;
+  attr[1].val.clusterDim.z = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(static_cast<long long>(B) * pl.G), 1, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = static_cast<size_t>(pl.cpc) * 2 * kGroups * sizeof(float);
+  cfg.stream = stream;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  if (pl.G > kPortableCluster) {
+    static std::atomic<bool> wide[kMaxDevices];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return DSPARK_ERR_CUDA;
+    if (!wide[dev].load(std::memory_order_acquire)) {
+      if (cudaFuncSetAttribute(finish_sample_kernel<T, VEC, kFin>,
+                               cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess)
+        return DSPARK_ERR_CUDA;
+      wide[dev].store(true, std::memory_order_release);
+    }
+  }
+  return cudaLaunchKernelEx(&cfg, finish_sample_kernel<T, VEC, kFin>, fp) == cudaSuccess
+             ? DSPARK_OK
+             : DSPARK_ERR_CUDA;
+}
+
 // Pass 1 over every (row, chunk) unit (one CTA per SM, every grid-th unit), then pass 2.
 // Both are programmatic dependent launches: pass 1's CTAs become resident while the previous
 // kernel in the stream drains and wait for it to complete before reading anything (this hides
@@ -219,7 +255,7 @@ dspark_status_t run_call(const Call& c, const Plan& pl, cudaStream_t stream,
   }
   if (pass1_only) return DSPARK_OK;
 
-  std::conditional_t<kMode == kModeMixed, FinishParamsMixed, FinishParams> fp{};
+  FinishParamsOf<kFin> fp{};
   fp.rs = c.rs;
   fp.drafts = c.drafts;
   fp.uniforms = c.uniforms;
@@ -232,38 +268,21 @@ dspark_status_t run_call(const Call& c, const Plan& pl, cudaStream_t stream,
     fp.temps = c.temps;
   }
   fp.out = c.out;
-  cudaLaunchAttribute attr[2];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  attr[1].id = cudaLaunchAttributeClusterDimension;
-  attr[1].val.clusterDim.x = static_cast<unsigned>(pl.G);
-  attr[1].val.clusterDim.y = 1;
-  attr[1].val.clusterDim.z = 1;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(static_cast<unsigned>(kSample ? static_cast<long long>(c.B) * pl.G : c.B), 1, 1);
-  cfg.blockDim = dim3(kThreads, 1, 1);
-  cfg.dynamicSmemBytes = kSample ? static_cast<size_t>(pl.cpc) * 2 * kGroups * sizeof(float) : 0;
-  cfg.stream = stream;
-  cfg.attrs = attr;
-  cfg.numAttrs = kSample ? 2 : 1;
   if constexpr (kSample) {
-    if (pl.G > kPortableCluster) {  // a 16-CTA cluster is opt-in, once per kernel and device
-      static std::atomic<bool> wide[kMaxDevices];
-      int dev = 0;
-      if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices)
-        return DSPARK_ERR_CUDA;
-      if (!wide[dev].load(std::memory_order_acquire)) {
-        if (cudaFuncSetAttribute(finish_sample_kernel<T, VEC, kFin>,
-                                 cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess)
-          return DSPARK_ERR_CUDA;
-        wide[dev].store(true, std::memory_order_release);
-      }
-    }
-    e = cudaLaunchKernelEx(&cfg, finish_sample_kernel<T, VEC, kFin>, fp);
-  }
-  else
+    return launch_finish_sample<T, VEC, kFin>(fp, pl, c.B, stream);
+  } else {
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(c.B), 1, 1);
+    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.stream = stream;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
     e = cudaLaunchKernelEx(&cfg, finish_greedy_kernel<T>, fp);
-  return e == cudaSuccess ? DSPARK_OK : DSPARK_ERR_CUDA;
+    return e == cudaSuccess ? DSPARK_OK : DSPARK_ERR_CUDA;
+  }
 }
 
 // Early exit (early_exit.cuh): per wave, pass 1 over the alive sequences' rows of the wave and
@@ -353,33 +372,7 @@ dspark_status_t run_early_exit(const Call& c, const Plan& pl, cudaStream_t strea
     fp.gather = reinterpret_cast<float*>(c.ws + w.gather);
     fp.out = c.out;
     fp.dec = dec;
-    cudaLaunchAttribute attr[2];
-    attr[0] = pdl[0];
-    attr[1].id = cudaLaunchAttributeClusterDimension;
-    attr[1].val.clusterDim.x = static_cast<unsigned>(pl.G);
-    attr[1].val.clusterDim.y = 1;
-    attr[1].val.clusterDim.z = 1;
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(static_cast<unsigned>(static_cast<long long>(c.B) * pl.G), 1, 1);
-    cfg.blockDim = dim3(kThreads, 1, 1);
-    cfg.dynamicSmemBytes = static_cast<size_t>(pl.cpc) * 2 * kGroups * sizeof(float);
-    cfg.stream = stream;
-    cfg.attrs = attr;
-    cfg.numAttrs = 2;
-    if (pl.G > kPortableCluster) {  // a 16-CTA cluster is opt-in, once per kernel and device
-      static std::atomic<bool> wide[kMaxDevices];
-      int dev = 0;
-      if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices)
-        return DSPARK_ERR_CUDA;
-      if (!wide[dev].load(std::memory_order_acquire)) {
-        if (cudaFuncSetAttribute(finish_sample_kernel<T, VEC, kFinEarlyExit>,
-                                 cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess)
-          return DSPARK_ERR_CUDA;
-        wide[dev].store(true, std::memory_order_release);
-      }
-    }
-    e = cudaLaunchKernelEx(&cfg, finish_sample_kernel<T, VEC, kFinEarlyExit>, fp);
-    return e == cudaSuccess ? DSPARK_OK : DSPARK_ERR_CUDA;
+    return launch_finish_sample<T, VEC, kFinEarlyExit>(fp, pl, c.B, stream);
   }
 }
 
