@@ -29,6 +29,11 @@
  *    target's (the adapter.py docstring's "lossless accept policy"; the DeepSeek-V4-Flash
  *    DSpark drafter card's "lossless by construction").
  *
+ * Beside these: dspark_mixed_accept (a serving batch with per-sequence draft counts and
+ * temperatures), dspark_early_exit_accept (rows read only up to each sequence's first
+ * rejection), dspark_markov_matvec (the drafter's Markov-head table mat-vec), and
+ * dspark_sample_pass1 (the sampling call's stream kernel alone, for timing it).
+ *
  * Conventions common to every entry point
  * ---------------------------------------
  *  - Every buffer pointer is a DEVICE pointer owned by the caller. The library allocates no
