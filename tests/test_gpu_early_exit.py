@@ -7,7 +7,6 @@ every output up to the stop is bit-identical. Rows after a sequence's stop are n
 poisoning them changes nothing.
 """
 
-import os
 
 import numpy as np
 import pytest

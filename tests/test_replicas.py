@@ -7,7 +7,6 @@ rank's time."""
 import os
 import sys
 
-import numpy as np
 import pytest
 import torch.distributed as dist
 import torch.multiprocessing as mp

@@ -5,7 +5,6 @@ whether it runs first in a fresh process (its first call looks up the scratch ad
 after every other test. Shapes beyond the fixed scratch are rejected before any CUDA work.
 """
 
-import ctypes
 
 import numpy as np
 import pytest
