@@ -368,11 +368,16 @@ def run_ours(args, w):
         dist.destroy_process_group()
     if rank != 0:
         return
-    markov = time_markov_matvec(dev)
-    small = time_small_batches(dev)
-    early = time_early_exit_serving(w, sets, Dd, Ud, workspace, dev, reps, per_call_us, calls)
-    if not args.no_stress:
-        early.update(time_early_exit_stress(dev))
+    # single-GPU characterisations beside the step, on the one-GPU line only (a scaling run
+    # holds every GPU while rank 0 would run them)
+    markov, small, early = {}, {}, {}
+    if world == 1:
+        markov = time_markov_matvec(dev)
+        small = time_small_batches(dev)
+        early = time_early_exit_serving(w, sets, Dd, Ud, workspace, dev, reps, per_call_us,
+                                        calls)
+        if not args.no_stress:
+            early.update(time_early_exit_stress(dev))
 
     peaks = measured_peaks()
     peak = peaks["hbm_gbs"] if peaks else FALLBACK_HBM_GBS
@@ -428,10 +433,12 @@ def run_ours(args, w):
         for m in markov.values():
             m["frac_of_peak"] = m["GB_per_s"] / peak
         call_stats["markov_matvec"] = markov
-    call_stats["early_exit"] = early
+    if early:
+        call_stats["early_exit"] = early
     for m in small.values():
         m["frac_of_peak"] = m["GB_per_s"] / peak
-    call_stats["small_batches"] = small
+    if small:
+        call_stats["small_batches"] = small
     if clk:
         line["clocks"] = clk
     if e2e:
