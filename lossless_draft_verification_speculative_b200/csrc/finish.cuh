@@ -3,9 +3,10 @@
 // Greedy: one CTA per sequence merges the pass-1 argmax records of its K+1 rows (a warp per
 // row), compares the drafts with the row argmaxes and writes the AcceptResult.
 //
-// Sampling: one thread-block cluster of G = min(8, n_chunks) CTAs per sequence. Every CTA
-// merges the 2K+1 rows' softmax records and takes the accept decisions (the same inputs and
-// arithmetic in each, so the same j). It then computes, one 2048-token chunk per warp, the
+// Sampling: one thread-block cluster of G = min(8, n_chunks) CTAs per sequence (min(16,
+// n_chunks) for batches of at most 32). Every CTA merges the 2K+1 rows' softmax records and
+// takes the accept decisions (the same inputs and arithmetic in each, so the same j); after
+// the early-exit waves it loads the decision they stored instead. It then computes, one 2048-token chunk per warp, the
 // mass of the draw's law: r = max(p_j - q_j, 0) after a rejection (j < K), p_K for the bonus
 // (j = K), keeping the sums of every 8-token group in shared memory and sending each chunk's
 // mass to every CTA of the cluster (distributed shared memory). After one cluster barrier all
