@@ -25,7 +25,7 @@
 
 namespace dspark {
 
-constexpr int kMaxWaves = 8;  // waves for K <= 32: 1 + 2 + 4 + 8 + 16 + 1
+constexpr int kMaxWaves = 8;  // K <= 32 takes 6 waves, of 1, 2, 4, 8, 16 and 1 pairs
 
 // Pairs [lo, hi) of wave w.
 __host__ __device__ __forceinline__ void wave_range(int w, int K, int& lo, int& hi) {
