@@ -107,3 +107,52 @@ def test_bad_draft_id_reads_nothing():
     for T in (0.0, 1.0):
         a = ora.early_exit_accept(P, Q, d, T, u)
         assert list(a.status) == [0, ora.STATUS_BAD_DRAFT, ora.STATUS_BAD_DRAFT, 0]
+
+
+def test_exact_enumeration_is_lossless():
+    """V = 4, K = 2, probabilities in eighths: over every draft pair x ~ q_1 x q_2 and every
+    cell of the three uniforms between consecutive members of the Farey sequence F_8 (all
+    decision and CDF boundaries lie there), the tokens early_exit_accept emits, continued
+    with p_{n+2}.. where it stops early, follow p_1 x p_2 x p_3 exactly."""
+    import itertools
+    from fractions import Fraction
+
+    F8 = lambda *xs: [Fraction(x, 8) for x in xs]  # noqa: E731
+    # both residuals keep two tokens (max(p_1 - q_1, 0) = (2, 0, 1, 0)/8, max(p_2 - q_2, 0) =
+    # (0, 2, 1, 0)/8), so the draw's uniform decides the token and a draw with the wrong
+    # uniform changes the law
+    Pp = [F8(3, 2, 2, 1), F8(1, 3, 2, 2), F8(1, 2, 3, 2)]
+    Qp = [F8(1, 3, 1, 3), F8(2, 1, 1, 4)]
+    V, K = 4, 2
+    with np.errstate(divide="ignore"):
+        zP = np.log(np.array([[float(x) for x in r] for r in Pp]))
+        zQ = np.log(np.array([[float(x) for x in r] for r in Qp]))
+    F = sorted({Fraction(a, b) for b in range(1, 9) for a in range(b + 1)})
+    cells = [((F[k] + F[k + 1]) / 2, F[k + 1] - F[k]) for k in range(len(F) - 1)]
+    runs = [(x, us) for x in itertools.product(range(V), repeat=K)
+            if Qp[0][x[0]] * Qp[1][x[1]] > 0
+            for us in itertools.product(cells, repeat=K + 1)]
+    n = len(runs)
+    d = np.array([x for x, _ in runs])
+    u = np.array([[float(c[0]) for c in us] for _, us in runs])
+    res = ora.early_exit_accept(np.repeat(zP[None], n, 0), np.repeat(zQ[None], n, 0), d, 1.0, u)
+    assert np.all(res.status == 0)
+    law = {}
+    for r, (x, us) in enumerate(runs):
+        w = Qp[0][x[0]] * Qp[1][x[1]]
+        for c in us:
+            w *= c[1]
+        nb = int(res.n_accepted[r])
+        emitted = tuple(int(t) for t in res.tokens[r, : nb + 1])
+        for tail in itertools.product(range(V), repeat=K - nb):
+            ww = w
+            for m, t in enumerate(tail):
+                ww *= Pp[nb + 1 + m][t]
+            if ww:
+                law[emitted + tail] = law.get(emitted + tail, Fraction(0)) + ww
+    want = {}
+    for s in itertools.product(range(V), repeat=K + 1):
+        w = Pp[0][s[0]] * Pp[1][s[1]] * Pp[2][s[2]]
+        if w:
+            want[s] = w
+    assert law == want
