@@ -257,7 +257,11 @@ dspark_status_t dspark_markov_matvec(const void* table, dspark_table_t type, int
  *    holds e.g. B = 64, K = 7, V = 129280 bf16, about 0.5 MB; not B = 256, K = 15, V = 262144).
  *  Set-up: the first call on a device, with that device current, looks up the array's device
  *    address (cudaGetSymbolAddress) and keeps it; make that first call before any stream
- *    capture on that device. A failed look-up returns DSPARK_ERR_CUDA.
+ *    capture on that device. A failed look-up returns DSPARK_ERR_CUDA. The call runs on the
+ *    CURRENT device: make the device that holds the buffers current first. The kept address
+ *    belongs to the device's primary context as it was at the first call; after a
+ *    cudaDeviceReset of that device the library must be reloaded before this entry is used
+ *    again.
  *  The array needs no clearing: each call writes every word of it that it reads.
  *  All calls on one device share the array: calls that overlap on the GPU race and give
  *    wrong results. Order them (one stream, or events). */

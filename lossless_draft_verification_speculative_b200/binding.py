@@ -253,7 +253,8 @@ def greedy_accept(P: Union[torch.Tensor, Tuple[torch.Tensor, torch.Tensor]],
     B, V = p1.shape
     K = 0 if pv is None else pv.shape[1]
     drafts = _check_drafts(drafts, B, K, p1.device)
-    res = out if out is not None else _alloc_result(B, K, p1.device, diagnostics=False)
+    res = _check_out(out, B, K, p1.device) if out is not None else \
+        _alloc_result(B, K, p1.device, diagnostics=False)
     nbytes = lib.dspark_workspace_bytes(B, K, V, DTYPE_CODES[p1.dtype])
     ws = workspace if workspace is not None else _WS.get(p1.device, nbytes, B, K)
     rc = lib.dspark_greedy_accept(_ptr(p1), ld_p1, _ptr(pv), ld_pv, DTYPE_CODES[p1.dtype],
@@ -277,13 +278,10 @@ def speculative_sample_accept(P: Union[torch.Tensor, Tuple[torch.Tensor, torch.T
     B, V = p1.shape
     K = 0 if pv is None else pv.shape[1]
     drafts = _check_drafts(drafts, B, K, p1.device)
-    if Q is not None and K > 0:
-        if Q.shape != (B, K, V) or not Q.is_contiguous() or Q.dtype != p1.dtype:
-            raise ValueError("Q must be a contiguous [B, K, V] tensor of P's dtype")
-    if uniforms.dtype != torch.float32 or uniforms.shape != (B, K + 1) or \
-            not uniforms.is_contiguous() or uniforms.device != p1.device:
-        raise ValueError("uniforms must be a contiguous float32 [B, K+1] tensor on P's device")
-    res = out if out is not None else _alloc_result(B, K, p1.device, diagnostics=True)
+    if float(temperature) > 0:
+        _check_sampling(Q, uniforms, p1, B, K, V)
+    res = _check_out(out, B, K, p1.device) if out is not None else \
+        _alloc_result(B, K, p1.device, diagnostics=True)
     nbytes = lib.dspark_workspace_bytes(B, K, V, DTYPE_CODES[p1.dtype])
     ws = workspace if workspace is not None else _WS.get(p1.device, nbytes, B, K)
     rc = lib.dspark_speculative_sample_accept(
@@ -327,7 +325,8 @@ def mixed_accept(P: Union[torch.Tensor, Tuple[torch.Tensor, torch.Tensor]],
     if n_drafts is not None and (n_drafts.dtype != torch.int32 or n_drafts.shape != (B,) or
                                  not n_drafts.is_contiguous() or n_drafts.device != p1.device):
         raise ValueError("n_drafts must be a contiguous int32 [B] tensor on P's device")
-    res = out if out is not None else _alloc_result(B, K, p1.device, diagnostics=True)
+    res = _check_out(out, B, K, p1.device) if out is not None else \
+        _alloc_result(B, K, p1.device, diagnostics=True)
     nbytes = lib.dspark_workspace_bytes(B, K, V, DTYPE_CODES[p1.dtype])
     ws = workspace if workspace is not None else _WS.get(p1.device, nbytes, B, K)
     rc = lib.dspark_mixed_accept(
@@ -363,7 +362,8 @@ def early_exit_accept(P: Union[torch.Tensor, Tuple[torch.Tensor, torch.Tensor]],
                 uniforms.device != p1.device:
             raise ValueError("uniforms must be a contiguous float32 [B, K+1] tensor on P's "
                              "device")
-    res = out if out is not None else _alloc_result(B, K, p1.device, diagnostics=True)
+    res = _check_out(out, B, K, p1.device) if out is not None else \
+        _alloc_result(B, K, p1.device, diagnostics=True)
     nbytes = lib.dspark_workspace_bytes(B, K, V, DTYPE_CODES[p1.dtype])
     ws = workspace if workspace is not None else _WS.get(p1.device, nbytes, B, K)
     rc = lib.dspark_early_exit_accept(
@@ -421,16 +421,62 @@ def speculative_sample_accept_static(P: Union[torch.Tensor, Tuple[torch.Tensor, 
     """
     lib = load_library()
     p1, pv, ld_p1, ld_pv = _split_block(P)
-    if not p1.is_cuda:
-        raise RuntimeError("speculative_sample_accept_static runs on CUDA tensors only")
     B, V = p1.shape
     K = 0 if pv is None else pv.shape[1]
+    # every layout check before anything reaches the library: it checks pointers for null,
+    # not the sizes behind them
     drafts = _check_drafts(drafts, B, K, p1.device)
-    rc = lib.dspark_speculative_sample_accept_static(
-        _ptr(p1), ld_p1, _ptr(pv), ld_pv, _ptr(Q), DTYPE_CODES[p1.dtype], _ptr(drafts), B, K,
-        V, float(temperature), _ptr(uniforms), _out_struct(out), _stream_handle(p1.device))
+    if float(temperature) > 0:
+        _check_sampling(Q, uniforms, p1, B, K, V)
+    if out is None:
+        raise ValueError("out is required: the call allocates nothing")
+    _check_out(out, B, K, p1.device)
+    if not p1.is_cuda:
+        raise RuntimeError("speculative_sample_accept_static runs on CUDA tensors only")
+    # the library resolves its scratch on the current device: make it P's
+    with torch.cuda.device(p1.device):
+        rc = lib.dspark_speculative_sample_accept_static(
+            _ptr(p1), ld_p1, _ptr(pv), ld_pv, _ptr(Q), DTYPE_CODES[p1.dtype], _ptr(drafts), B,
+            K, V, float(temperature), _ptr(uniforms), _out_struct(out),
+            _stream_handle(p1.device))
     if rc != DSPARK_OK:
         raise DsparkError(rc, "dspark_speculative_sample_accept_static")
+    return out
+
+
+def _check_sampling(Q: Optional[torch.Tensor], uniforms: torch.Tensor, p1: torch.Tensor, B: int,
+                    K: int, V: int) -> None:
+    """Q [B, K, V] contiguous in P's dtype on P's device (K > 0), uniforms float32 [B, K+1]."""
+    if K > 0:
+        if Q is None or Q.shape != (B, K, V) or not Q.is_contiguous() or Q.dtype != p1.dtype \
+                or Q.device != p1.device:
+            raise ValueError("Q must be a contiguous [B, K, V] tensor of P's dtype and device")
+    if uniforms is None or uniforms.dtype != torch.float32 or uniforms.shape != (B, K + 1) or \
+            not uniforms.is_contiguous() or uniforms.device != p1.device:
+        raise ValueError("uniforms must be a contiguous float32 [B, K+1] tensor on P's device")
+
+
+_OUT_SHAPES = {"n_accepted": (torch.int32, 1), "tokens": (torch.int32, 2),
+               "next_token": (torch.int32, 1), "status": (torch.int32, 1),
+               "p_draft": (torch.float32, 2), "q_draft": (torch.float32, 2),
+               "resid_mass": (torch.float32, 1)}
+
+
+def _check_out(out: AcceptResult, B: int, K: int, device) -> AcceptResult:
+    """A caller-supplied result: every tensor it holds is contiguous, on P's device, of its
+    field's dtype and shape (the kernels write B, B x (K+1) or B x K elements there)."""
+    shapes = {1: (B,), 2: (B, K)}
+    for name, (dtype, rank) in _OUT_SHAPES.items():
+        t = getattr(out, name)
+        if t is None:
+            if name in ("n_accepted", "tokens", "next_token"):
+                raise ValueError(f"out.{name} is required")
+            continue
+        shape = (B, K + 1) if name == "tokens" else shapes[rank]
+        if t.dtype != dtype or tuple(t.shape) != shape or not t.is_contiguous() or \
+                t.device != device:
+            raise ValueError(f"out.{name} must be a contiguous {dtype} tensor of shape "
+                             f"{list(shape)} on P's device")
     return out
 
 

@@ -90,10 +90,10 @@ struct StreamParams {
 };
 
 // A mixed batch's parameters add its per-sequence arrays. They are kept out of StreamParams:
-// on this B200 the back-to-back sampling call's time moved by up to a microsecond with the
-// size and layout of the two kernels' parameter structs alone, the arithmetic unchanged (the
-// cause is not known; these structs are the fastest layout measured), so the other modes
-// carry none of the mixed batch's fields.
+// the back-to-back sampling call's time moved by up to a microsecond with the size and layout
+// of the two kernels' parameter structs alone, the arithmetic unchanged (the cause is not
+// known; these structs are the fastest layout measured), so the other modes carry none of
+// the mixed batch's fields.
 struct StreamParamsMixed : StreamParams {
   const int32_t* n_drafts;  // [B] K_b, or null for K
   const float* temps;       // [B] T_b

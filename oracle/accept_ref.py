@@ -24,7 +24,7 @@ What it computes, and where that comes from:
   draft is accepted draw the bonus token from p_{K+1}. Greedy: accept while the draft
   equals the base argmax, then emit the argmax of the first mismatching (or bonus) row.
 
-Readings where the pages are silent (each restated in the design notes):
+Readings where the pages are silent:
   temperature divides both P and Q logits; T == 0 means greedy; u[b, i] tests draft i
   and u[b, K] is the single draw for the resample or bonus token; accept iff
   u * q(x) < p(x) (strict; q == 0 < p accepts); the inverse CDF runs in ascending token
