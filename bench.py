@@ -215,8 +215,53 @@ def run_reference(args, w):
     }), flush=True)
 
 
-def cpu_baseline(w, seconds):
-    """The oracle timed on the host (1 core): steps of 8 sequences through every call of the
+def cpu_baseline(w, seconds, outs=None):
+    """The oracle timed on the host cores, and the bench's own results checked against it.
+
+    Timings: on all host cores (one spawn-started process per core, at most one per sequence,
+    each verifying its sequences through every call of the step over and over for `seconds`),
+    and on one core (steps of 8 sequences through every call, repeated for `seconds`).
+    Parity: with ``outs`` (the GPU results of the step's calls, rank 0's batch) every
+    sequence of every call is compared with the oracle: greedy bit for bit, sampling decisions
+    and tokens identical except where the oracle's uniform lies within 1e-6 of a boundary."""
+    from oracle import parallel as par
+
+    pool = par.timed_all_cores(w.name, w.temperatures, seconds)
+    one = cpu_baseline_one_core(w, seconds)
+    res = {"value": pool["value"], "unit": "blocks/s", "cores": pool["cores"], "kind": "oracle",
+           "sample": f"{pool['blocks']} verified blocks ({w.B} sequences x {len(w.temperatures)} "
+                     f"calls, repeated) in {pool['seconds']:.1f} s of float64 NumPy on "
+                     f"{pool['cores']} processes, one per host core",
+           "host_cores": par.host_cores(), "single_core": one}
+    near = oracle_parity(w, outs) if outs is not None else None
+    return res, near
+
+
+def oracle_parity(w, outs):
+    """Every sequence of the step's calls against the oracle (all host cores)."""
+    from oracle import parallel as par
+
+    calls = build_calls(w)
+    per = {}
+    total = {"sequences": 0, "near_boundary": 0, "differ": 0, "differ_outside_band": 0}
+    for c, (kind, T) in enumerate(calls):
+        o = par.run(w.name, T, seqs=range(w.B))
+        n_g = outs[c].n_accepted.cpu().numpy()
+        t_g = outs[c].tokens.cpu().numpy()
+        same = (n_g == o["n_accepted"]) & np.all(t_g == o["tokens"], axis=1)
+        near = o["near"] if kind == "sample" else np.zeros(w.B, bool)
+        st = {"sequences": int(w.B), "near_boundary": int(near.sum()),
+              "differ": int((~same).sum()), "differ_outside_band": int((~same & ~near).sum())}
+        per[f"{kind}_T{T}"] = st
+        for k in total:
+            total[k] += st[k]
+    total["calls"] = per
+    total["eps"] = 1e-6
+    return total
+
+
+def cpu_baseline_one_core(w, seconds):
+    """The oracle timed on one host core: steps of 8 sequences through every call of the
     workload, repeated until about `seconds` of work have run."""
     from lossless_draft_verification_speculative_b200 import workloads as wl
     from oracle import accept_ref as ora
@@ -444,7 +489,9 @@ def run_ours(args, w):
     if e2e:
         line["e2e"] = e2e
     if world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(w, args.cpu_seconds)
+        line["cpu_baseline"], near = cpu_baseline(w, args.cpu_seconds, outs)
+        if near is not None:
+            line["near_boundary"] = near
     print(json.dumps(line), flush=True)
 
 

@@ -16,8 +16,7 @@ Every sequence b draws from its own generator ``default_rng([seed, b, ...])``, s
 subset of sequences can be regenerated on its own (the oracle checks sampled
 sequences of the large workloads without materialising the whole batch twice).
 
-Readings of the workload descriptions (each is listed with its reason in the design
-notes): "N(0, s)" names a standard deviation; values are generated in float32 and
+Readings of the workload descriptions: "N(0, s)" names a standard deviation; values are generated in float32 and
 rounded to bf16 with round-to-nearest-even; drafts are drawn from the *rounded* Q
 that the verifier will see.
 """

@@ -16,6 +16,10 @@ BOUNDARY_EPS = 1e-6     # decisions may differ only where u is this close to a b
 RESID_ATOL = 2e-6
 ERR_BITS = bd.SEQ_BAD_DRAFT | bd.SEQ_NONFINITE
 
+# (label, sequences compared, near-boundary sequences, of which the GPU result differed):
+# every sampling comparison of the run, printed in the session summary (conftest.py)
+NEAR_LOG = []
+
 
 def to_dev(arr, dtype):
     arr = np.ascontiguousarray(arr)
@@ -24,9 +28,10 @@ def to_dev(arr, dtype):
     return torch.from_numpy(arr.astype(np.float32)).to(DEV)
 
 
-def run_gpu(P, Q, d, u, T, dtype, block=None):
-    """One verify call through the binding. P: [B, K+1, V] stored logits (or a (p1, pv) pair
-    of device tensors via ``block``). Returns host numpy arrays."""
+def run_gpu(P, Q, d, u, T, dtype, block=None, Q_dev=None):
+    """One verify call through the binding. P: [B, K+1, V] stored logits (or a device block /
+    (p1, pv) pair via ``block``; ``Q_dev``: Q already on the device). Returns host numpy
+    arrays."""
     Pd = block if block is not None else to_dev(P, dtype)
     K = d.shape[1]
     dd = torch.from_numpy(np.ascontiguousarray(d, dtype=np.int32)).to(DEV)
@@ -34,7 +39,7 @@ def run_gpu(P, Q, d, u, T, dtype, block=None):
     if T == 0:
         r = bd.greedy_accept(Pd, dd)
     else:
-        Qd = to_dev(Q, dtype) if K > 0 else None
+        Qd = Q_dev if Q_dev is not None else (to_dev(Q, dtype) if K > 0 else None)
         r = bd.speculative_sample_accept(Pd, Qd, dd, T, ud)
     torch.cuda.synchronize()
     return {k: v.cpu().numpy() for k, v in vars(r).items() if v is not None}
@@ -71,6 +76,8 @@ def compare_sampling(g, o, label="", inputs=None):
     assert np.all(g["n_accepted"][err] == 0) and np.all(g["next_token"][err] == -1)
     K = g["tokens"].shape[1] - 1
     near = 0
+    flagged = int(np.count_nonzero(o.near_boundary(BOUNDARY_EPS)[ok])) \
+        if o.accept_margin is not None else 0
     for b in np.flatnonzero(ok):
         jg, jo = int(g["n_accepted"][b]), int(o.n_accepted[b])
         if jg != jo:
@@ -98,4 +105,5 @@ def compare_sampling(g, o, label="", inputs=None):
             ((o.status & bd.SEQ_ZERO_RESIDUAL) == 0)
         np.testing.assert_allclose(g["resid_mass"][rej].astype(np.float64), o.resid_mass[rej],
                                    rtol=PROB_RTOL, atol=RESID_ATOL, err_msg=label + "resid_mass")
+    NEAR_LOG.append((label, int(np.count_nonzero(ok)), flagged, near))
     return near

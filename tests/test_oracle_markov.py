@@ -88,3 +88,21 @@ def test_table_sizes_match_the_card():
     q8 = wl.markov_table(8, R, "q8_0").shape[1] * V
     assert q8 == V * (R // 32) * mk.Q8_0_BLOCK_BYTES
     assert round((f16 - q8) / 1e6) == 31
+
+
+def _matrix(text):
+    return np.asarray([[float(x) for x in row.split()] for row in text.split(";")])
+
+
+def test_abs_products_worked_by_hand():
+    """The error scale that sets the GPU test's tolerance, on a 2 x 2 case worked by hand
+    (tests/golden/abs_products_2x2.txt): a transposed operand or a dropped absolute value
+    changes the result."""
+    kv = {}
+    for line in open(os.path.join(os.path.dirname(__file__), "golden", "abs_products_2x2.txt")):
+        if line.strip() and not line.startswith("#"):
+            k, v = line.split(":", 1)
+            kv[k.strip()] = _matrix(v)
+    got = mk.abs_products(kv["W"], kv["h"])
+    assert np.array_equal(got, kv["abs_products"])
+    assert not np.array_equal(mk.markov_matvec(kv["W"], kv["h"]), kv["abs_products"])

@@ -8,7 +8,6 @@ its benchmark.py greedy loop), library inverse-CDF draws, the closed-form accept
 rate of speculative sampling, a chi-square goodness of fit, and hand-worked examples.
 """
 
-import itertools
 import os
 from fractions import Fraction
 
@@ -17,104 +16,14 @@ import pytest
 from scipy import special, stats
 
 from oracle import accept_ref as ora
+
+import enumeration as en
 from lossless_draft_verification_speculative_b200 import workloads as wl
 
 GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
 
 
 # ---------------------------------------------------------------- helpers
-
-def _logits_of(probs, T=1.0):
-    """Logits whose softmax at temperature T is exactly the given probabilities (0 -> -inf)."""
-    p = np.asarray([float(x) for x in probs])
-    with np.errstate(divide="ignore"):
-        return np.log(p) * T
-
-
-def _farey(n):
-    """All fractions a/b in [0, 1] with b <= n, sorted (the Farey sequence F_n)."""
-    s = {Fraction(a, b) for b in range(1, n + 1) for a in range(0, b + 1)}
-    return sorted(s)
-
-
-_ENUM_CACHE = {}
-
-
-def _enumerate_emitted(Pp, Qp, T, denom, draft_law=None):
-    """Exact distribution of the first K+1 emitted tokens for prefix-independent rows.
-
-    Pp: K+1 rows of rational probabilities, Qp: K rows (the q the verifier is given).
-    Every draft tuple is weighted by prod draft_law_i(x_i) (default: q itself); every
-    uniform coordinate is swept over the intervals between consecutive members of the
-    Farey sequence F_denom. All probabilities have denominators dividing ``denom``, so
-    every ratio p/q and every normalised CDF point of any residual lies in F_denom: the
-    oracle's output is constant on each interval and its midpoint decides it. Tokens the
-    cycle does not emit are continued with p_{n+2}..p_{K+1}, as a prefix-independent
-    target would produce them.
-    """
-    law = Qp if draft_law is None else draft_law
-    K = len(Qp)
-    V = len(Pp[0])
-    zP = np.stack([_logits_of(r, T) for r in Pp])[None]
-    zQ = np.stack([_logits_of(r, T) for r in Qp])[None]
-    F = _farey(denom)
-    cells = [((F[k] + F[k + 1]) / 2, F[k + 1] - F[k]) for k in range(len(F) - 1)]
-    ucells = list(itertools.product(cells, repeat=K + 1))
-    u_one = np.asarray([[float(c[0]) for c in us] for us in ucells], dtype=np.float64)
-    w_one = []
-    for us in ucells:
-        w = Fraction(1)
-        for c in us:
-            w *= c[1]
-        w_one.append(w)
-    drafts_all = [x for x in itertools.product(range(V), repeat=K)
-                  if all(Qp[i][x[i]] > 0 or law[i][x[i]] > 0 for i in range(K))]
-    nu = len(ucells)
-    key = (repr(Pp), repr(Qp), T, denom, tuple(drafts_all))
-    if key not in _ENUM_CACHE:
-        n = nu * len(drafts_all)
-        d = np.repeat(np.asarray(drafts_all, dtype=np.int64), nu, axis=0)
-        u = np.tile(u_one, (len(drafts_all), 1))
-        _ENUM_CACHE[key] = ora.speculative_sample_accept(
-            np.repeat(zP, n, axis=0), np.repeat(zQ, n, axis=0), d, T, u)
-    res = _ENUM_CACHE[key]
-    emitted_w = {}
-    for a, x in enumerate(drafts_all):
-        wx = Fraction(1)
-        for i in range(K):
-            wx *= law[i][x[i]]
-        if not wx:
-            continue
-        acc = {}
-        for k in range(nu):
-            row = a * nu + k
-            nb = int(res.n_accepted[row])
-            key = tuple(int(t) for t in res.tokens[row, : nb + 1])
-            acc[key] = acc.get(key, Fraction(0)) + w_one[k]
-        for key, w in acc.items():
-            emitted_w[key] = emitted_w.get(key, Fraction(0)) + wx * w
-    dist = {}
-    for emitted, w in emitted_w.items():
-        nb = len(emitted) - 1
-        for tail in itertools.product(range(V), repeat=K - nb):
-            ww = w
-            for m, t in enumerate(tail):
-                ww *= Pp[nb + 1 + m][t]
-            if ww:
-                dist[emitted + tail] = dist.get(emitted + tail, Fraction(0)) + ww
-    return dist
-
-
-def _product_dist(Pp):
-    out = {}
-    for s in itertools.product(range(len(Pp[0])), repeat=len(Pp)):
-        w = Fraction(1)
-        for r, t in enumerate(s):
-            w *= Pp[r][t]
-        if w:
-            out[s] = w
-    return out
-
 
 F8 = lambda *xs: [Fraction(x, 8) for x in xs]  # noqa: E731
 
@@ -125,8 +34,8 @@ def test_enumeration_lossless_exact():
     """V=4, K=2: the joint law of the K+1 emitted tokens equals p_1 x p_2 x p_3 exactly."""
     Pp = [F8(4, 2, 1, 1), F8(1, 1, 2, 4), F8(2, 2, 3, 1)]
     Qp = [F8(2, 3, 2, 1), F8(4, 2, 1, 1)]
-    got = _enumerate_emitted(Pp, Qp, 1.0, 8)
-    assert got == _product_dist(Pp)
+    got, _ = en.enumerate_emitted(Pp, Qp, 1.0, 8)
+    assert got == en.product_dist(Pp)
 
 
 @pytest.mark.parametrize("T", [0.5, 2.0])
@@ -135,16 +44,16 @@ def test_enumeration_lossless_exact_tempered(T):
     F4 = lambda *xs: [Fraction(x, 4) for x in xs]  # noqa: E731
     Pp = [F4(2, 1, 1, 0), F4(0, 1, 1, 2), F4(1, 1, 1, 1)]
     Qp = [F4(1, 1, 1, 1), F4(2, 2, 0, 0)]
-    got = _enumerate_emitted(Pp, Qp, T, 4)
-    assert got == _product_dist(Pp)
+    got, _ = en.enumerate_emitted(Pp, Qp, T, 4)
+    assert got == en.product_dist(Pp)
 
 
 def test_enumeration_lossless_with_masked_tokens():
     """Zero-probability tokens (logit -inf) in p and in q: still exactly lossless."""
     Pp = [F8(0, 4, 4, 0), F8(1, 0, 3, 4), F8(0, 0, 0, 8)]
     Qp = [F8(2, 2, 2, 2), F8(0, 4, 0, 4)]
-    got = _enumerate_emitted(Pp, Qp, 1.0, 8)
-    assert got == _product_dist(Pp)
+    got, _ = en.enumerate_emitted(Pp, Qp, 1.0, 8)
+    assert got == en.product_dist(Pp)
 
 
 def test_enumeration_detects_a_wrong_rule():
@@ -156,10 +65,10 @@ def test_enumeration_detects_a_wrong_rule():
     Pp = [F8(4, 2, 1, 1), F8(1, 1, 2, 4), F8(2, 2, 3, 1)]
     Qp_true = [F8(2, 3, 2, 1), F8(4, 2, 1, 1)]
     Qp_fake = [F8(2, 2, 2, 2), F8(2, 2, 2, 2)]
-    got = _enumerate_emitted(Pp, Qp_true, 1.0, 8)
-    bad = _enumerate_emitted(Pp, Qp_true, 1.0, 8, draft_law=Qp_fake)
-    assert got == _product_dist(Pp)
-    assert bad != _product_dist(Pp)
+    got, _ = en.enumerate_emitted(Pp, Qp_true, 1.0, 8)
+    bad, _ = en.enumerate_emitted(Pp, Qp_true, 1.0, 8, draft_law=Qp_fake)
+    assert got == en.product_dist(Pp)
+    assert bad != en.product_dist(Pp)
 
 
 # ---------------------------------------------------------- greedy
@@ -307,7 +216,7 @@ def test_temperature_scaling_identity():
 def test_softmax_matches_chosen_probabilities():
     probs = [Fraction(1, 2), Fraction(1, 4), Fraction(1, 8), Fraction(1, 8), Fraction(0)]
     for T in (0.5, 1.0, 3.0):
-        p = ora.softmax(_logits_of(probs, T), T)
+        p = ora.softmax(en.logits_of(probs, T), T)
         np.testing.assert_allclose(p, [float(x) for x in probs], rtol=1e-15, atol=0)
 
 
@@ -413,14 +322,14 @@ def test_golden_hand_worked_examples():
         K = int(c["K"])
         Pp = [_fr_row(c[f"p{r + 1}"]) for r in range(K + 1)]
         T = float(c.get("T", "1"))
-        zP = np.stack([_logits_of(r, T) for r in Pp])[None]
+        zP = np.stack([en.logits_of(r, T) for r in Pp])[None]
         d = np.asarray([[int(t) for t in c["drafts"].split()]])
         u = np.asarray([[float(t) for t in c["u"].split()]])
         if c["policy"] == "greedy":
             res = ora.greedy_accept(zP, d)
         else:
             Qp = [_fr_row(c[f"q{i + 1}"]) for i in range(K)]
-            zQ = np.stack([_logits_of(r, T) for r in Qp])[None]
+            zQ = np.stack([en.logits_of(r, T) for r in Qp])[None]
             res = ora.speculative_sample_accept(zP, zQ, d, T, u)
         assert int(res.n_accepted[0]) == int(c["n_accepted"]), c
         assert [int(t) for t in res.tokens[0]] == [int(t) for t in c["tokens"].split()], c
@@ -432,8 +341,8 @@ def test_near_boundary_flag():
     """A uniform placed 1e-9 from the accept boundary is flagged; 1e-3 away is not."""
     Pp = [F8(4, 2, 1, 1), F8(2, 2, 2, 2)]
     Qp = [F8(2, 2, 2, 2)]
-    zP = np.stack([_logits_of(r) for r in Pp])[None]
-    zQ = np.stack([_logits_of(r) for r in Qp])[None]
+    zP = np.stack([en.logits_of(r) for r in Pp])[None]
+    zQ = np.stack([en.logits_of(r) for r in Qp])[None]
     d = np.asarray([[2]])  # ratio (1/8)/(2/8) = 0.5
     near = ora.speculative_sample_accept(zP, zQ, d, 1.0, np.asarray([[0.5 - 1e-9, 0.3]]))
     far = ora.speculative_sample_accept(zP, zQ, d, 1.0, np.asarray([[0.499, 0.3]]))
