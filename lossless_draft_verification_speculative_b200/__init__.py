@@ -4,7 +4,9 @@
 sequence against the base model's [B, K+1, V] logit block and return an ``AcceptResult``;
 ``mixed_accept`` verifies a serving batch whose sequences have their own draft counts and
 temperatures; ``early_exit_accept`` reads each sequence's rows only up to its first
-rejection; ``markov_matvec`` is the drafter's Markov-head table mat-vec.
+rejection; ``markov_matvec`` is the drafter's Markov-head table mat-vec; ``YieldQuench`` is
+the host-side policy that turns speculation off for requests whose acceptance does not pay
+for the verify (``include/dspark_policy.h``).
 The work runs in hand-written CUDA kernels behind a C ABI (``include/dspark_verify.h``);
 this package is the thin Python binding over it plus the seeded synthetic workloads.
 """
@@ -16,6 +18,7 @@ from .binding import (  # noqa: F401
     SEQ_TIMEOUT,
     SEQ_ZERO_RESIDUAL,
     AcceptResult,
+    YieldQuench,
     DsparkError,
     early_exit_accept,
     greedy_accept,
@@ -31,6 +34,7 @@ from .binding import (  # noqa: F401
 __all__ = [
     "AcceptResult",
     "DsparkError",
+    "YieldQuench",
     "greedy_accept",
     "speculative_sample_accept",
     "speculative_sample_accept_static",

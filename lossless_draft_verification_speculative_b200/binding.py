@@ -62,15 +62,33 @@ class Plan(ctypes.Structure):
         "greedy_units_per_sequence", "sampling_units_per_sequence", "finish_ctas_per_sequence")]
 
 
+QUENCH_MAX_WINDOW = 64  # DSPARK_QUENCH_MAX_WINDOW of include/dspark_policy.h
+SPEC_ON, SPEC_OFF_YIELD, SPEC_OFF_KV = 0, 1, 2
+
+
+class QuenchConfig(ctypes.Structure):
+    _fields_ = [("break_even", ctypes.c_double), ("warmup", ctypes.c_int32),
+                ("window", ctypes.c_int32), ("kv_limit", ctypes.c_int64)]
+
+
+class QuenchState(ctypes.Structure):
+    _fields_ = [("state", ctypes.c_int32), ("cycles", ctypes.c_int32),
+                ("committed", ctypes.c_int64), ("window_sum", ctypes.c_int32),
+                ("ring", ctypes.c_int32 * QUENCH_MAX_WINDOW)]
+
+
 _LIB = None
 
 
 def header_functions() -> list:
-    """Names of every function declared in include/dspark_verify.h."""
-    path = os.path.join(build_lib.INCLUDE, "dspark_verify.h")
-    text = open(path).read()
-    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-    return sorted(set(re.findall(r"\b(dspark_[a-z0-9_]+)\s*\(", text)))
+    """Names of every function declared in the headers under include/."""
+    names = set()
+    for h in sorted(os.listdir(build_lib.INCLUDE)):
+        if h.endswith(".h"):
+            text = open(os.path.join(build_lib.INCLUDE, h)).read()
+            text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+            names |= set(re.findall(r"\b(dspark_[a-z0-9_]+)\s*\(", text))
+    return sorted(names)
 
 
 def library_path() -> str:
@@ -117,6 +135,10 @@ def load_library(build_if_missing: bool = True) -> ctypes.CDLL:
                                              ctypes.c_float, vp, AcceptOut, vp, sz, vp]
     lib.dspark_markov_matvec.restype = i32
     lib.dspark_markov_matvec.argtypes = [vp, i32, i32, i32, vp, i32, vp, vp]
+    lib.dspark_quench_reset.restype = i32
+    lib.dspark_quench_reset.argtypes = [vp, i32]
+    lib.dspark_quench_update.restype = i32
+    lib.dspark_quench_update.argtypes = [ctypes.POINTER(QuenchConfig), vp, i32, vp, vp, vp]
     lib.dspark_speculative_sample_accept_static.restype = i32
     lib.dspark_speculative_sample_accept_static.argtypes = [vp, i64, vp, i64, vp, i32, vp, i32,
                                                             i32, i32, ctypes.c_float, vp,
@@ -535,3 +557,53 @@ class PreparedCall:
         rc = self.fn(*self.args)
         if rc != DSPARK_OK:
             raise DsparkError(rc, self.name)
+
+
+class YieldQuench:
+    """The yield-quench speculation policy over a batch of requests (include/dspark_policy.h).
+
+    After each verify step, ``update`` takes every request's ``n_accepted`` (a negative value:
+    not verified this step) and, optionally, its context depth, and returns which requests
+    should keep drafting: a request stops for good once the mean committed tokens of its last
+    ``window`` cycles fall below ``break_even`` (after ``warmup`` cycles), or once its context
+    exceeds ``kv_limit`` tokens (the DeepSeek-V4-Flash DSpark drafter card's 64k gate). The
+    controller runs in the C library on host arrays.
+    """
+
+    def __init__(self, n_requests: int, break_even: float, warmup: int = 8, window: int = 16,
+                 kv_limit: int = 65536):
+        self.lib = load_library()
+        self.config = QuenchConfig(float(break_even), int(warmup), int(window), int(kv_limit))
+        self.n = int(n_requests)
+        self.states = (QuenchState * max(1, self.n))()
+        rc = self.lib.dspark_quench_reset(ctypes.cast(self.states, ctypes.c_void_p), self.n)
+        if rc != DSPARK_OK:
+            raise DsparkError(rc, "dspark_quench_reset")
+
+    def update(self, n_accepted, kv_depth=None):
+        import numpy as np
+
+        na = np.ascontiguousarray(
+            n_accepted.cpu().numpy() if isinstance(n_accepted, torch.Tensor) else n_accepted,
+            dtype=np.int32)
+        if na.shape != (self.n,):
+            raise ValueError(f"n_accepted must have shape [{self.n}]")
+        kv = None
+        if kv_depth is not None:
+            kv = np.ascontiguousarray(
+                kv_depth.cpu().numpy() if isinstance(kv_depth, torch.Tensor) else kv_depth,
+                dtype=np.int64)
+            if kv.shape != (self.n,):
+                raise ValueError(f"kv_depth must have shape [{self.n}]")
+        out = np.zeros(self.n, dtype=np.int32)
+        rc = self.lib.dspark_quench_update(
+            ctypes.byref(self.config), ctypes.cast(self.states, ctypes.c_void_p), self.n,
+            na.ctypes.data, None if kv is None else kv.ctypes.data, out.ctypes.data)
+        if rc != DSPARK_OK:
+            raise DsparkError(rc, "dspark_quench_update")
+        return out.astype(bool)
+
+    def state(self, b: int) -> dict:
+        s = self.states[b]
+        return {"state": s.state, "cycles": s.cycles, "committed": s.committed,
+                "window_sum": s.window_sum}

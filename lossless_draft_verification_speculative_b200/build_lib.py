@@ -2,7 +2,8 @@
 
     python -m lossless_draft_verification_speculative_b200.build_lib
 
-compiles ``csrc/dspark_verify.cu`` with nvcc (``-gencode arch=compute_100a,code=sm_100a``),
+compiles ``csrc/dspark_verify.cu`` (the kernels and their C ABI) and ``csrc/policy.cc`` (the
+host-side speculation policy) with nvcc (``-gencode arch=compute_100a,code=sm_100a``),
 links the CUDA runtime statically and writes the library next to this file, under
 ``_lib/``. The Python binding loads it from there.
 """
@@ -20,7 +21,7 @@ CSRC = os.path.join(PKG_DIR, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB_DIR = os.path.join(PKG_DIR, "_lib")
 LIB_PATH = os.path.join(LIB_DIR, "libdspark_verify.so")
-SOURCES = ["dspark_verify.cu"]
+SOURCES = ["dspark_verify.cu", "policy.cc"]
 HEADERS = ["common.cuh", "stream.cuh", "finish.cuh", "early_exit.cuh", "markov.cuh"]
 
 
@@ -33,7 +34,7 @@ def nvcc_path() -> str:
 
 def _inputs():
     files = [os.path.join(CSRC, s) for s in SOURCES + HEADERS]
-    files.append(os.path.join(INCLUDE, "dspark_verify.h"))
+    files += [os.path.join(INCLUDE, h) for h in ("dspark_verify.h", "dspark_policy.h")]
     files.append(os.path.abspath(__file__))
     return files
 
