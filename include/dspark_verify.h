@@ -130,13 +130,14 @@ typedef struct {
   int elems_per_load;              /* 8 (bf16) / 4 (fp32) on the 16-byte path, 1 on the scalar path */
   int loads_in_flight;             /* loads each lane of pass 1 keeps in flight                    */
   int stream_threads_per_cta;      /* pass 1: one CTA of this many threads per SM                  */
-  int threads_per_cta;             /* pass 2                                                      */
+  int threads_per_cta;             /* pass 2 of the greedy policy, early-exit decisions           */
   int chunk_elems;                 /* tokens per chunk (pass-1 unit, pass-2 chunk)                */
   int n_chunks;                    /* chunks per row                                              */
   int greedy_units_per_sequence;   /* pass-1 units of one sequence, greedy: (K+1) * n_chunks      */
   int sampling_units_per_sequence; /* pass-1 units of one sequence, sampling: (2K+1) * n_chunks   */
   int finish_ctas_per_sequence;    /* pass-2 CTAs per sequence (one cluster), sampling policy:
-                                      min(n_chunks, 16) for B <= 32, else min(n_chunks, 8)       */
+                                      ceil(n_chunks / 32), one chunk per warp                    */
+  int finish_threads_per_cta;      /* pass-2 CTA size of the sampling policy (32 warps)           */
 } dspark_plan_t;
 dspark_status_t dspark_plan(int B, int K, int V, dspark_dtype_t dtype, int aligned16,
                             dspark_plan_t* plan);

@@ -59,7 +59,8 @@ class Plan(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int) for n in (
         "elems_per_load", "loads_in_flight", "stream_threads_per_cta", "threads_per_cta",
         "chunk_elems", "n_chunks",
-        "greedy_units_per_sequence", "sampling_units_per_sequence", "finish_ctas_per_sequence")]
+        "greedy_units_per_sequence", "sampling_units_per_sequence", "finish_ctas_per_sequence",
+        "finish_threads_per_cta")]
 
 
 QUENCH_MAX_WINDOW = 64  # DSPARK_QUENCH_MAX_WINDOW of include/dspark_policy.h

@@ -16,7 +16,7 @@
 namespace dspark {
 namespace {
 
-constexpr int kAbiVersion = 4;  // 4: the workspace also holds the early-exit waves' state
+constexpr int kAbiVersion = 5;  // 5: dspark_plan_t gained finish_threads_per_cta
 constexpr int kMaxDevices = 64;
 
 // Tuning switch, read at every call: DSPARK_MAX_CTAS caps the pass-1 CTAs (0 = one per SM).
@@ -51,8 +51,8 @@ bool make_plan(int B, int V, dspark_dtype_t dt, bool aligned16, Plan* pl) {
   if (nch < 1 || nch > kMaxChunkCount) return false;
   pl->vec = aligned16 ? 16 / es : 1;
   pl->nch = static_cast<int>(nch);
-  const int gmax = B <= kWideClusterMaxB ? kMaxFinishCluster : kPortableCluster;
-  pl->G = pl->nch < gmax ? pl->nch : gmax;
+  // sampling finish: one chunk per warp of 32-warp CTAs, G = ceil(nch / 32) <= 4 per cluster
+  pl->G = (pl->nch + kFinWarps - 1) / kFinWarps;
   pl->cpc = (pl->nch + pl->G - 1) / pl->G;
   return true;
 }
@@ -166,12 +166,13 @@ struct Call {
   char* ws;
 };
 
-// The sampling finish: one cluster of pl.G CTAs per sequence, each with pl.cpc chunks of group
-// sums in dynamic shared memory, as a programmatic dependent of the kernel before it. A
-// 16-CTA cluster is opt-in, once per kernel instantiation and device.
+// The sampling finish: one cluster of pl.G CTAs of 32 warps per sequence, each with pl.cpc
+// chunks of group sums in dynamic shared memory, as a programmatic dependent of the kernel
+// before it.
 template <typename T, int VEC, int kFin>
 dspark_status_t launch_finish_sample(const FinishParamsOf<kFin>& fp, const Plan& pl, int B,
                                      cudaStream_t stream) {
+  constexpr int kW = kFinWarps;
   cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
@@ -181,23 +182,26 @@ dspark_status_t launch_finish_sample(const FinishParamsOf<kFin>& fp, const Plan&
   attr[1].val.clusterDim.z = 1;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(static_cast<long long>(B) * pl.G), 1, 1);
-  cfg.blockDim = dim3(kThreads, 1, 1);
-  cfg.dynamicSmemBytes = static_cast<size_t>(pl.cpc) * 2 * kGroups * sizeof(float);
+  cfg.blockDim = dim3(kW * 32, 1, 1);
+  cfg.dynamicSmemBytes = static_cast<size_t>(pl.cpc) * kGroups * sizeof(float);
   cfg.stream = stream;
   cfg.attrs = attr;
   cfg.numAttrs = 2;
-  if (pl.G > kPortableCluster) {
-    static std::atomic<bool> wide[kMaxDevices];
+  {
+    // once per kernel instantiation and device: room for the group sums of up to 32 chunks
+    static std::atomic<bool> ready[kMaxDevices];
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return DSPARK_ERR_CUDA;
-    if (!wide[dev].load(std::memory_order_acquire)) {
-      if (cudaFuncSetAttribute(finish_sample_kernel<T, VEC, kFin>,
-                               cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess)
+    if (!ready[dev].load(std::memory_order_acquire)) {
+      if (cudaFuncSetAttribute(finish_sample_kernel<T, VEC, kFin, kW>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(kFinMaxCpc * kGroups * sizeof(float))) !=
+          cudaSuccess)
         return DSPARK_ERR_CUDA;
-      wide[dev].store(true, std::memory_order_release);
+      ready[dev].store(true, std::memory_order_release);
     }
   }
-  return cudaLaunchKernelEx(&cfg, finish_sample_kernel<T, VEC, kFin>, fp) == cudaSuccess
+  return cudaLaunchKernelEx(&cfg, finish_sample_kernel<T, VEC, kFin, kW>, fp) == cudaSuccess
              ? DSPARK_OK
              : DSPARK_ERR_CUDA;
 }
@@ -526,6 +530,7 @@ dspark_status_t dspark_plan(int B, int K, int V, dspark_dtype_t dtype, int align
   plan->greedy_units_per_sequence = (K + 1) * pl.nch;
   plan->sampling_units_per_sequence = (2 * K + 1) * pl.nch;
   plan->finish_ctas_per_sequence = pl.G;
+  plan->finish_threads_per_cta = kFinWarps * 32;
   return DSPARK_OK;
 }
 

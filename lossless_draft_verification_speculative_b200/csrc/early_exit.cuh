@@ -156,7 +156,7 @@ __global__ void __launch_bounds__(kThreads) ee_decide_kernel(const EeDecideParam
   if (static_cast<int>(blockIdx.x) >= n_alive) return;
   const int b = wv.wave == 0 ? static_cast<int>(blockIdx.x) : __ldcg(wv.alive + blockIdx.x);
   const WaveRows rows{K, wv.lo, wv.hi, wv.last != 0, kSample};
-  merge_rows<kSample, true, WaveRows>(p, b, rows, wi, lane, s_stat);
+  merge_rows<kSample, true, kWarps, WaveRows>(p, b, rows, wi, lane, s_stat);
   __syncthreads();
   if (wi != 0) return;
 

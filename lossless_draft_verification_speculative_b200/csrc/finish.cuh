@@ -3,18 +3,21 @@
 // Greedy: one CTA per sequence merges the pass-1 argmax records of its K+1 rows (a warp per
 // row), compares the drafts with the row argmaxes and writes the AcceptResult.
 //
-// Sampling: one thread-block cluster of G = min(8, n_chunks) CTAs per sequence (min(16,
-// n_chunks) for batches of at most 32). Every CTA merges the 2K+1 rows' softmax records and
-// takes the accept decisions (the same inputs and arithmetic in each, so the same j); after
-// the early-exit waves it loads the decision they stored instead. It then computes, one 2048-token chunk per warp, the
-// mass of the draw's law: r = max(p_j - q_j, 0) after a rejection (j < K), p_K for the bonus
-// (j = K), keeping the sums of every 8-token group in shared memory and sending each chunk's
-// mass to every CTA of the cluster (distributed shared memory). After one cluster barrier all
-// CTAs locate the chunk that holds the draw (float64 prefix over the chunk masses); its owner
-// finds the group from its group sums, re-reads that group's 8 tokens and scans them.
+// Sampling: one thread-block cluster of G = ceil(n_chunks / 32) CTAs of 32 warps per sequence
+// (2 for V = 129280, at most 4), one CTA per SM. Small clusters of whole-SM CTAs are placed at
+// once: with 8-CTA clusters of 8-warp CTAs the GPU left a cluster unplaced until others had
+// finished (the clusters must fit in a GPC). Every CTA merges the 2K+1 rows' softmax records
+// and takes the accept decisions (the same inputs and arithmetic in each, so the same j);
+// after the early-exit waves it loads the decision they stored instead. Each warp then
+// computes one 2048-token chunk of the draw's law, r = max(p_j - q_j, 0) after a rejection
+// (j < K), p_K for the bonus (j = K), keeping the sums of every 8-token group in shared
+// memory and sending the chunk's mass to every CTA of the cluster (distributed shared memory).
+// After one cluster barrier every CTA locates the chunk that holds the draw (float64 prefix
+// over the chunk masses); its owner finds the group from its group sums, re-reads that
+// group's 8 tokens and scans them.
 //
-// Both kernels start with the loads that do not depend on pass 1 (drafts, uniforms, the
-// draft-token logits) and then wait for pass 1 to complete (programmatic dependent launch).
+// Both kernels start with the loads that do not depend on pass 1 (drafts, uniforms) and then
+// wait for pass 1 to complete (programmatic dependent launch).
 #pragma once
 
 #include "stream.cuh"
@@ -24,12 +27,8 @@ namespace dspark {
 constexpr int kErrBits =
     DSPARK_SEQ_BAD_DRAFT | DSPARK_SEQ_NONFINITE | DSPARK_SEQ_TIMEOUT | DSPARK_SEQ_BAD_PARAM;
 constexpr int kMaxRows = 2 * kMaxK + 1;
-// CTAs per sampling cluster: 8 (the portable size), or 16 (opt-in) for batches of at most
-// kWideClusterMaxB sequences, whose 16 B CTAs of 4 per SM are still co-resident on 148 SMs and
-// whose warps then take one chunk each instead of two.
-constexpr int kPortableCluster = 8;
-constexpr int kMaxFinishCluster = 16;
-constexpr int kWideClusterMaxB = 32;
+constexpr int kFinWarps = 32;   // warps per sampling-finish CTA: one chunk each
+constexpr int kFinMaxCpc = 32;  // chunks per finish CTA at most
 
 // Kernel parameters (see StreamParamsMixed on their size). The sampling kernel's cluster size
 // G and chunks per CTA, ceil(n_chunks / G), come from its launch.
@@ -96,26 +95,26 @@ __device__ __forceinline__ float2 reduce_row(const RowRecs& rr) {
 }
 
 // The rows of sequence b into s_stat (row r at s_stat[r]): all of them, or with kFiltered
-// those that `used` selects. Warp w merges rows w, w + 8, ..., two at a time so that their
-// loads overlap.
-template <bool kSample, bool kFiltered, class Filter = RowFilter>
+// those that `used` selects. Warp w of kW merges rows w, w + kW, ..., two at a time so that
+// their loads overlap.
+template <bool kSample, bool kFiltered, int kW = kWarps, class Filter = RowFilter>
 __device__ __forceinline__ void merge_rows(const FinishParams& p, int b, const Filter& used,
                                            int wi, int lane, float2* s_stat) {
   const int rows = p.rs.rows;
   const long long r0 = static_cast<long long>(b) * rows;
-  for (int r = wi; r < rows; r += 2 * kWarps) {
+  for (int r = wi; r < rows; r += 2 * kW) {
     RowRecs a, c;
     const bool one = !kFiltered || used(r);
-    const bool two = r + kWarps < rows && (!kFiltered || used(r + kWarps));
+    const bool two = r + kW < rows && (!kFiltered || used(r + kW));
     if (one) load_row<kSample>(p, r0 + r, lane, a);
-    if (two) load_row<kSample>(p, r0 + r + kWarps, lane, c);
+    if (two) load_row<kSample>(p, r0 + r + kW, lane, c);
     if (one) {
       const float2 sa = reduce_row<kSample>(a);
       if (lane == 0) s_stat[r] = sa;
     }
     if (two) {
       const float2 sc = reduce_row<kSample>(c);
-      if (lane == 0) s_stat[r + kWarps] = sc;
+      if (lane == 0) s_stat[r + kW] = sc;
     }
   }
 }
@@ -154,10 +153,10 @@ __device__ __forceinline__ void write_tokens(const FinishParams& p, int b, int j
 // Greedy finish of sequence b with nd drafts (every thread of the CTA; its P rows 0..nd are
 // merged): x = drafts[b, lane] in warp 0's lanes below nd, already copied to s_x. kFiltered:
 // the records are laid out for sampling rows (a mixed batch) and rows past nd are skipped.
-template <bool kFiltered>
+template <bool kFiltered, int kW = kWarps>
 __device__ __forceinline__ void greedy_finish(const FinishParams& p, int b, int nd, int x, int wi,
                                               int lane, float2* s_arg, const int* s_x) {
-  merge_rows<false, kFiltered>(p, b, RowFilter{p.rs.K, nd, false}, wi, lane, s_arg);
+  merge_rows<false, kFiltered, kW>(p, b, RowFilter{p.rs.K, nd, false}, wi, lane, s_arg);
   __syncthreads();
   if (wi != 0) return;
   const float ninf = -__int_as_float(0x7f800000);
@@ -209,21 +208,35 @@ struct Decision {
   float mq, iq;  // q_j: reference and 1 / sum (iq = 0 for the bonus)
 };
 
-// Per-token values of the draw's law. The group sums, the chunk masses and the draw's scan all
-// come from exactly this arithmetic, so the scan reproduces the sums it located.
-//   p value:        p_j(v) = 2^(z_p[v]*s - m_p) / S_p
-//   residual value: max(p_j(v) - q_j(v), 0)
-struct TokenVals {
-  float r;  // residual (equals p on the bonus row)
-  float p;
-};
-__device__ __forceinline__ TokenVals token_vals(float zp, float zq, bool has_q, float s,
-                                                const Decision& d) {
-  const float ep = ex2(__fmaf_rn(zp, s, -d.mp));
-  const float pv = __fmul_rn(ep, d.ip);
-  if (!has_q) return {pv, pv};
-  const float eq = ex2(__fmaf_rn(zq, s, -d.mq));
-  return {fmaxf(__fmaf_rn(ep, d.ip, -__fmul_rn(eq, d.iq)), 0.f), pv};
+// The values of the draw's law at a group's 8 tokens, in token order. The group sums, the chunk
+// masses and the draw's scan all come from exactly these values, so the scan reproduces the
+// sums it located:
+//   p value:        p_j(v) = 2^(z_p[v]*s - m_p) * (1 / S_p)
+//   residual value: max(p_j(v) - q_j(v), 0), rounded as fma(e_p, 1/S_p, -(e_q * (1/S_q)))
+// (the residual equals p on the bonus row, which has no q). Pairs of tokens share one packed
+// f32x2 instruction where the arithmetic allows; each half rounds like the scalar operation.
+template <bool kResid>
+__device__ __forceinline__ void law_values(const float* zp, const float* zq, float s,
+                                           const Decision& d, float* out) {
+  const uint64_t s2 = pk2(s, s);
+  const uint64_t nmp = pk2(-d.mp, -d.mp), ip = pk2(d.ip, d.ip);
+#pragma unroll
+  for (int e = 0; e < 8; e += 2) {
+    float a0, a1;
+    upk2(fma2(pk2(zp[e], zp[e + 1]), s2, nmp), a0, a1);
+    const uint64_t ep = pk2(ex2(a0), ex2(a1));
+    if constexpr (kResid) {
+      float c0, c1;
+      upk2(fma2(pk2(zq[e], zq[e + 1]), s2, pk2(-d.mq, -d.mq)), c0, c1);
+      const uint64_t neq = mul2(pk2(ex2(c0), ex2(c1)), pk2(-d.iq, -d.iq));
+      float r0, r1;
+      upk2(fma2(ep, ip, neq), r0, r1);
+      out[e] = fmaxf(r0, 0.f);
+      out[e + 1] = fmaxf(r1, 0.f);
+    } else {
+      upk2(mul2(ep, ip), out[e], out[e + 1]);
+    }
+  }
 }
 
 // A group: 8 consecutive tokens 8q .. 8q+7 of a chunk (q = 0..255). Lane l of a warp handles
@@ -259,37 +272,40 @@ struct GroupRaw {
   }
 };
 
-// Sums over a group's 8 tokens in token order.
-template <typename T, int VEC>
-__device__ __forceinline__ TokenVals group_sums(const GroupRaw<T, VEC>& gp,
-                                                const GroupRaw<T, VEC>& gq, bool has_q, float s,
-                                                const Decision& d) {
+// The law's values at a group's 8 tokens (residual when kResid, else p), in token order.
+template <typename T, int VEC, bool kResid>
+__device__ __forceinline__ void group_values(const GroupRaw<T, VEC>& gp, const GroupRaw<T, VEC>& gq,
+                                             float s, const Decision& d, float* v) {
   float zp[8], zq[8];
   gp.values(zp);
-  if (has_q) gq.values(zq);
-  TokenVals acc{0.f, 0.f};
+  if constexpr (kResid) gq.values(zq);
+  law_values<kResid>(zp, zq, s, d, v);
+}
+
+// Sum of a group's 8 law values in token order.
+template <typename T, int VEC, bool kResid>
+__device__ __forceinline__ float group_sum(const GroupRaw<T, VEC>& gp, const GroupRaw<T, VEC>& gq,
+                                           float s, const Decision& d) {
+  float v[8];
+  group_values<T, VEC, kResid>(gp, gq, s, d, v);
+  float acc = 0.f;
 #pragma unroll
-  for (int e = 0; e < 8; ++e) {
-    const TokenVals v = token_vals(zp[e], has_q ? zq[e] : 0.f, has_q, s, d);
-    acc.r = __fadd_rn(acc.r, v.r);
-    acc.p = __fadd_rn(acc.p, v.p);
-  }
+  for (int e = 0; e < 8; ++e) acc = __fadd_rn(acc, v[e]);
   return acc;
 }
 
-// Chunk c of the draw's law, one warp: the 256 group sums into part_r / part_p (token order;
-// either may be null) and the chunk's (residual mass, p mass) on every lane.
-template <typename T, int VEC>
-__device__ __forceinline__ float2 chunk_work(const RowSet& rs, float scale, int b, int c,
-                                             const Decision& d, int lane, float* part_r,
-                                             float* part_p) {
+// Chunk c of the draw's law (kResid: the residual of row pair j, else p of row j), one warp:
+// the 256 group sums into part (token order) and the chunk's mass on every lane. Out of line:
+// its registers are allocated apart from the kernel's (the finish has several call sites).
+template <typename T, int VEC, bool kResid>
+__device__ __forceinline__ float chunk_work(const RowSet& rs, float scale, int b, int c,
+                                            const Decision& d, int lane, float* part) {
   const int K = rs.K, V = rs.V;
-  const bool has_q = d.j < d.nd;
   const T* pr = row_ptr<T>(rs, b, d.j);
-  const T* qr = has_q ? row_ptr<T>(rs, b, K + 1 + d.j) : pr;
+  const T* qr = kResid ? row_ptr<T>(rs, b, K + 1 + d.j) : pr;
   constexpr int kPerLane = kGroups / 32;                      // groups per lane
   constexpr int kRound = VEC == 8 ? 4 : (VEC == 4 ? 2 : 1);  // groups in flight per row
-  float lr = 0.f, lp = 0.f;
+  float acc = 0.f;
 #pragma unroll
   for (int k0 = 0; k0 < kPerLane; k0 += kRound) {
     GroupRaw<T, VEC> gp[kRound], gq[kRound];
@@ -297,19 +313,16 @@ __device__ __forceinline__ float2 chunk_work(const RowSet& rs, float scale, int 
     for (int k = 0; k < kRound; ++k) {
       const int t0 = c * kCE + ((k0 + k) * 32 + lane) * 8;
       gp[k].load(pr, t0, V);
-      if (has_q) gq[k].load(qr, t0, V);
+      if constexpr (kResid) gq[k].load(qr, t0, V);
     }
 #pragma unroll
     for (int k = 0; k < kRound; ++k) {
-      const TokenVals gsum = group_sums<T, VEC>(gp[k], gq[k], has_q, scale, d);
-      const int q = (k0 + k) * 32 + lane;
-      if (part_r) part_r[q] = gsum.r;
-      if (part_p) part_p[q] = gsum.p;
-      lr = __fadd_rn(lr, gsum.r);
-      lp = __fadd_rn(lp, gsum.p);
+      const float gsum = group_sum<T, VEC, kResid>(gp[k], gq[k], scale, d);
+      part[(k0 + k) * 32 + lane] = gsum;
+      acc = __fadd_rn(acc, gsum);
     }
   }
-  return make_float2(warp_sum(lr), warp_sum(lp));
+  return warp_sum(acc);
 }
 
 // Where the draw falls among the chunks of its row: float64 prefix over the chunk masses
@@ -317,47 +330,30 @@ __device__ __forceinline__ float2 chunk_work(const RowSet& rs, float scale, int 
 // row), target u*Z, first chunk whose inclusive prefix passes it. Every lane gets the result.
 constexpr int kMassPerLane = kMaxChunkCount / 32;
 struct ChunkPick {
-  int c;        // chunk that holds the draw; -1 when no chunk has mass
-  int status;   // the decision's status, plus DSPARK_SEQ_ZERO_RESIDUAL when that applies
-  bool use_p;   // draw from p_j itself: the bonus row, or a residual that rounded to zero
-  double tin;   // the target measured from the chunk's start (+inf: past the last mass)
-  double zres;  // the residual mass (rejection rows)
+  int c;       // chunk that holds the draw; -1 when no chunk has mass
+  double tin;  // the target measured from the chunk's start (+inf: past the last mass)
+  double z;    // the law's total mass
 };
 
-__device__ __forceinline__ ChunkPick pick_chunk(const float2 (&ms)[kMassPerLane], bool bonus,
-                                                float u, int status, int lane) {
+__device__ __forceinline__ ChunkPick pick_chunk(const float (&ms)[kMassPerLane], float u,
+                                                int lane) {
   constexpr int NPL = kMassPerLane;
-  bool use_p = bonus;
-  double mr[NPL], mp[NPL];
-  double zr = 0.0, zpm = 0.0;
+  double m[NPL];
+  double ls = 0.0;
 #pragma unroll
   for (int k = 0; k < NPL; ++k) {
-    mr[k] = ms[k].x;
-    mp[k] = ms[k].y;
-    zr += mr[k];
-    zpm += mp[k];
+    m[k] = ms[k];
+    ls += m[k];
   }
-  double Zr = zr, Zp = zpm;  // inclusive prefixes over lanes
+  double incl = ls;  // inclusive prefix over lanes
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
-    const double a = __shfl_up_sync(0xffffffffu, Zr, o), c2 = __shfl_up_sync(0xffffffffu, Zp, o);
-    if (lane >= o) {
-      Zr += a;
-      Zp += c2;
-    }
+    const double a = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += a;
   }
-  const double Zres = __shfl_sync(0xffffffffu, Zr, 31);
-  if (!use_p && !(Zres > 0.0)) {  // residual mass rounded to zero: draw from p_j instead
-    use_p = true;
-    status |= DSPARK_SEQ_ZERO_RESIDUAL;
-  }
-  double m[NPL];
-#pragma unroll
-  for (int k = 0; k < NPL; ++k) m[k] = use_p ? mp[k] : mr[k];
-  const double incl = use_p ? Zp : Zr;
-  const double ls = use_p ? zpm : zr;
-  const double Z = __shfl_sync(0xffffffffu, incl, 31);
-  const double target = static_cast<double>(u) * Z;
+  ChunkPick pk;
+  pk.z = __shfl_sync(0xffffffffu, incl, 31);
+  const double target = static_cast<double>(u) * pk.z;
   double run = incl - ls;
   int cfound = -1, clast = -1;
   double before = 0.0;
@@ -374,7 +370,6 @@ __device__ __forceinline__ ChunkPick pick_chunk(const float2 (&ms)[kMassPerLane]
     run = nxt;
   }
   const unsigned hit = __ballot_sync(0xffffffffu, cfound >= 0);
-  ChunkPick pk;
   if (hit) {
     const int hl = __ffs(hit) - 1;
     pk.c = __shfl_sync(0xffffffffu, cfound, hl);
@@ -386,21 +381,17 @@ __device__ __forceinline__ ChunkPick pick_chunk(const float2 (&ms)[kMassPerLane]
     pk.c = cl;
     pk.tin = __int_as_float(0x7f800000);
   }
-  pk.status = status;
-  pk.use_p = use_p;
-  pk.zres = Zres;
   return pk;
 }
 
 // The token of chunk c at the target tin (measured from the chunk's start), given the chunk's
-// 256 group sums `part` (token order) of the law drawn from (residual, or p when use_p): the
-// group from a scan of the sums, then that group's 8 tokens re-read and recomputed exactly as
-// their sum was, scanned by lane 0. Rounding that leaves the target past the chunk's sums
-// picks its last token with mass. Every lane gets the token.
-template <typename T, int VEC>
+// 256 group sums `part` (token order) of the law (kResid: residual, else p): the group from a
+// scan of the sums, then that group's 8 tokens re-read and recomputed exactly as their sum
+// was, scanned by lane 0. Rounding that leaves the target past the chunk's sums picks its last
+// token with mass. Every lane gets the token.
+template <typename T, int VEC, bool kResid>
 __device__ __forceinline__ int pick_token(const RowSet& rs, float scale, int b, const Decision& d,
-                                          int c, bool use_p, float tin, const float* part,
-                                          int lane) {
+                                          int c, float tin, const float* part, int lane) {
   const int j = d.j;
   // lane l scans the chunk's groups 8l .. 8l+7 (token order)
   float gv[8];
@@ -449,25 +440,21 @@ __device__ __forceinline__ int pick_token(const RowSet& rs, float scale, int b, 
   int token = -1;
   if (qsel >= 0 && lane == 0) {
     const int K = rs.K, V = rs.V;
-    const bool has_q = j < d.nd;
     const T* pr = row_ptr<T>(rs, b, j);
-    const T* qr = has_q ? row_ptr<T>(rs, b, K + 1 + j) : pr;
+    const T* qr = kResid ? row_ptr<T>(rs, b, K + 1 + j) : pr;
     const int t0 = c * kCE + qsel * 8;
     GroupRaw<T, VEC> gp, gq;
     gp.load(pr, t0, V);
-    if (has_q) gq.load(qr, t0, V);
-    float zp[8], zq[8];
-    gp.values(zp);
-    if (has_q) gq.values(zq);
+    if constexpr (kResid) gq.load(qr, t0, V);
+    float v[8];
+    group_values<T, VEC, kResid>(gp, gq, scale, d, v);
     float r = 0.f;
     int cand = -1, lastv = -1;
 #pragma unroll
     for (int e = 0; e < 8; ++e) {
-      const TokenVals v = token_vals(zp[e], has_q ? zq[e] : 0.f, has_q, scale, d);
-      const float val = use_p ? v.p : v.r;
-      const float nx = __fadd_rn(r, val);
-      if (val > 0.f) lastv = t0 + e;
-      if (!last_mode && cand < 0 && val > 0.f && r <= gin && gin < nx) cand = t0 + e;
+      const float nx = __fadd_rn(r, v[e]);
+      if (v[e] > 0.f) lastv = t0 + e;
+      if (!last_mode && cand < 0 && v[e] > 0.f && r <= gin && gin < nx) cand = t0 + e;
       r = nx;
     }
     token = cand >= 0 ? cand : lastv;
@@ -495,19 +482,22 @@ using FinishParamsOf = std::conditional_t<
     kFin == kFinMixed, FinishParamsMixed,
     std::conditional_t<kFin == kFinEarlyExit, FinishParamsEarlyExit, FinishParams>>;
 
-// Sampling finish. Launched as clusters of G CTAs, one cluster per sequence; CTA g of the
-// cluster owns chunks g*cpc .. g*cpc + cpc - 1 of the draw's law (warp w: local chunks w, w+8).
-template <typename T, int VEC, int kFin>
-__global__ void __launch_bounds__(kThreads, 4) finish_sample_kernel(const FinishParamsOf<kFin> p) {
+// Sampling finish. Launched as clusters of G CTAs of kW warps, one cluster per sequence; CTA g
+// of the cluster owns chunks g*cpc .. g*cpc + cpc - 1 of the draw's law (warp w: local chunks
+// w, w + kW, ...).
+template <typename T, int VEC, int kFin, int kW>
+__global__ void __launch_bounds__(kW * 32, kW <= 8 ? 4 : 1)
+    finish_sample_kernel(const FinishParamsOf<kFin> p) {
   constexpr bool kMixed = kFin == kFinMixed;
-  extern __shared__ float s_part[];  // [cpc][2][kGroups]: group sums (residual, p)
+  constexpr int kT = kW * 32;
+  extern __shared__ float s_part[];  // [cpc][kGroups]: group sums of the draw's law
   __shared__ float2 s_stat[kMaxRows];
-  __shared__ float2 s_mass[kMaxChunkCount];  // every chunk's (residual, p) mass
-  __shared__ float s_zp[kMaxK], s_zq[kMaxK], s_u[kMaxK + 1];
+  __shared__ float s_mass[kMaxChunkCount];  // every chunk's mass of the draw's law
+  __shared__ float s_u[kMaxK + 1];
   __shared__ int s_x[kMaxK];
   __shared__ Decision s_dec;
-  __shared__ double s_tin;
-  __shared__ int s_chunk, s_use_p;
+  __shared__ double s_tin, s_z;
+  __shared__ int s_chunk;
   // the next kernel in the stream may be scheduled as these CTAs retire (it waits for them)
   grid_dependents_launch();
   cg::cluster_group cluster = cg::this_cluster();
@@ -524,7 +514,7 @@ __global__ void __launch_bounds__(kThreads, 4) finish_sample_kernel(const Finish
   if constexpr (kMixed) {
     const SeqMode sm = seq_mode(p.n_drafts, p.temps, b, K);
     if (!sm.ok) {
-      if (g == 0) write_error(p, b, DSPARK_SEQ_BAD_PARAM, tid, kThreads);
+      if (g == 0) write_error(p, b, DSPARK_SEQ_BAD_PARAM, tid, kT);
       return;
     }
     nd = sm.kb;
@@ -537,7 +527,7 @@ __global__ void __launch_bounds__(kThreads, 4) finish_sample_kernel(const Finish
         s_x[tid] = xg;
       }
       grid_dependency_wait();
-      greedy_finish<true>(p, b, nd, xg, wi, lane, s_stat, s_x);
+      greedy_finish<true, kW>(p, b, nd, xg, wi, lane, s_stat, s_x);
       return;
     }
   }
@@ -551,20 +541,18 @@ __global__ void __launch_bounds__(kThreads, 4) finish_sample_kernel(const Finish
     if (tid < nd) s_x[tid] = x;
     if (tid == 0) s_dec = p.dec[b];
   } else {
-    // the draft tokens' logits, gathered by pass 1
+    // the draft tokens' logits, gathered by pass 1: warp 0 keeps draft i's on lane i, its load
+    // in flight with the records' below
+    float2 zg = make_float2(0.f, 0.f);
     if (tid < nd) {
       s_x[tid] = x;
-      float2 zg = make_float2(0.f, 0.f);
       if (x >= 0 && x < V)
         zg = __ldcg(reinterpret_cast<const float2*>(p.gather) + static_cast<size_t>(b) * K + tid);
-      s_zp[tid] = zg.x;
-      s_zq[tid] = zg.y;
     }
-    __syncthreads();
 
     // the (reference, sum) of every row the sequence uses
     const RowFilter used{K, nd, true};
-    merge_rows<true, kMixed>(p, b, used, wi, lane, s_stat);
+    merge_rows<true, kMixed, kW>(p, b, used, wi, lane, s_stat);
     __syncthreads();
 
     // decisions (warp 0; draft i on lane i)
@@ -582,8 +570,8 @@ __global__ void __launch_bounds__(kThreads, 4) finish_sample_kernel(const Finish
       if (lane < nd && !bad_draft) {
         const float2 sp = s_stat[lane], sq = s_stat[K1 + lane];
         // p_i(x_i) = 2^(z*s - M) / S (division within 2 ulp: no IEEE slow path)
-        px = __fdividef(ex2(__fmaf_rn(s_zp[lane], scale, -sp.x)), sp.y);
-        qx = __fdividef(ex2(__fmaf_rn(s_zq[lane], scale, -sq.x)), sq.y);
+        px = __fdividef(ex2(__fmaf_rn(zg.x, scale, -sp.x)), sp.y);
+        qx = __fdividef(ex2(__fmaf_rn(zg.y, scale, -sq.x)), sq.y);
         accept = __fmul_rn(s_u[lane], qx) < px;
       }
       const unsigned rej = __ballot_sync(0xffffffffu, lane < nd && !accept);
@@ -615,66 +603,86 @@ __global__ void __launch_bounds__(kThreads, 4) finish_sample_kernel(const Finish
   __syncthreads();
   const Decision d = s_dec;
   // this CTA's chunk range of the draw's rows into L2, ahead of the warps' second loads
-  if (VEC > 1 && lane == 0 && wi >= kWarps - 2 && !(d.status & kErrBits)) {
+  if (VEC > 1 && lane == 0 && wi >= kW - 2 && !(d.status & kErrBits)) {
     const int t0 = g * cpc * kCE;
     const int t1 = min(V, t0 + cpc * kCE);
-    const bool q_row = wi == kWarps - 1;
+    const bool q_row = wi == kW - 1;
     if (t0 < t1 && (!q_row || d.j < d.nd)) {
       const uint32_t bytes = static_cast<uint32_t>(t1 - t0) * Elem<T>::kBytes;
       prefetch_l2(row_ptr<T>(p.rs, b, q_row ? K1 + d.j : d.j) + t0, bytes);
     }
   }
 
-  // this CTA's chunks: group sums into shared memory, chunk masses to every CTA of the cluster
+  // this CTA's chunks of the draw's law (the residual after a rejection, p_K for the bonus):
+  // group sums into shared memory, chunk masses to every CTA of the cluster
+  const bool resid = d.j < d.nd;
   if (!(d.status & kErrBits)) {
-    for (int lc = wi; lc < cpc; lc += kWarps) {
+    for (int lc = wi; lc < cpc; lc += kW) {
       const int c = g * cpc + lc;
       if (c >= p.nch) break;
-      float* pr = s_part + static_cast<size_t>(lc) * 2 * kGroups;
-      const float2 m = chunk_work<T, VEC>(p.rs, scale, b, c, d, lane, pr, pr + kGroups);
+      float* pr = s_part + static_cast<size_t>(lc) * kGroups;
+      const float m = resid ? chunk_work<T, VEC, true>(p.rs, scale, b, c, d, lane, pr)
+                            : chunk_work<T, VEC, false>(p.rs, scale, b, c, d, lane, pr);
       if (lane < G) cluster.map_shared_rank(s_mass, lane)[c] = m;
     }
   }
   cluster.sync();  // every chunk mass has landed in every CTA; group sums are visible CTA-wide
 
   if (d.status & kErrBits) {
-    if (g == 0) write_error(p, b, d.status, tid, kThreads);
+    if (g == 0) write_error(p, b, d.status, tid, kT);
     return;
   }
 
   // ---- which chunk holds the draw (every CTA, the same float64 arithmetic on the same masses)
   const int j = d.j;
-  if (wi == 0) {
-    float2 ms[kMassPerLane];
+  int status = d.status;
+  bool use_p = !resid;
+  for (int pass = 0; pass < 2; ++pass) {
+    if (wi == 0) {
+      float ms[kMassPerLane];
 #pragma unroll
-    for (int k = 0; k < kMassPerLane; ++k) {
-      const int c = lane * kMassPerLane + k;
-      ms[k] = c < p.nch ? s_mass[c] : make_float2(0.f, 0.f);
-    }
-    const ChunkPick pk = pick_chunk(ms, j == nd, s_u[nd], d.status, lane);
-    const int owner = pk.c >= 0 ? pk.c / cpc : 0;
-    if (lane == 0) {
-      s_chunk = owner == g ? pk.c : -2;  // -2: another CTA draws
-      s_use_p = pk.use_p;
-      s_tin = pk.tin;
-      if (owner == g) {
-        if (p.out.resid_mass)
-          p.out.resid_mass[b] = j < nd ? (pk.use_p ? 0.f : static_cast<float>(pk.zres)) : 1.f;
-        if (p.out.status) p.out.status[b] = pk.status;
+      for (int k = 0; k < kMassPerLane; ++k) {
+        const int c = lane * kMassPerLane + k;
+        ms[k] = c < p.nch ? s_mass[c] : 0.f;
+      }
+      const ChunkPick pk = pick_chunk(ms, s_u[nd], lane);
+      if (lane == 0) {
+        s_chunk = pk.c;
+        s_tin = pk.tin;
+        s_z = pk.z;
       }
     }
+    __syncthreads();
+    if (use_p || s_z > 0.0) break;
+    // a residual whose every value rounded to zero (impossible in exact arithmetic after a
+    // rejection): draw from p_j instead. Every CTA of the cluster sees the same masses and
+    // takes this branch; the masses are rewritten only after every CTA has read them.
+    use_p = true;
+    status |= DSPARK_SEQ_ZERO_RESIDUAL;
+    cluster.sync();
+    for (int lc = wi; lc < cpc; lc += kW) {
+      const int c = g * cpc + lc;
+      if (c >= p.nch) break;
+      const float m = chunk_work<T, VEC, false>(p.rs, scale, b, c, d, lane,
+                                                s_part + static_cast<size_t>(lc) * kGroups);
+      if (lane < G) cluster.map_shared_rank(s_mass, lane)[c] = m;
+    }
+    cluster.sync();
   }
-  __syncthreads();
   const int c = s_chunk;
-  if (c == -2) return;
+  const int owner = c >= 0 ? c / cpc : 0;
+  if (owner != g) return;  // another CTA draws
   if (wi != 0) return;
+  if (lane == 0) {
+    if (p.out.resid_mass) p.out.resid_mass[b] = resid ? (use_p ? 0.f : static_cast<float>(s_z)) : 1.f;
+    if (p.out.status) p.out.status[b] = status;
+  }
   int token = -1;
   if (c >= 0) {
-    const bool use_p = s_use_p != 0;
-    const float* part = s_part + static_cast<size_t>(c - g * cpc) * 2 * kGroups +
-                        (use_p ? kGroups : 0);
-    token = pick_token<T, VEC>(p.rs, scale, b, d, c, use_p, static_cast<float>(s_tin), part,
-                               lane);
+    const float* part = s_part + static_cast<size_t>(c - g * cpc) * kGroups;
+    const float tin = static_cast<float>(s_tin);
+    token = use_p ? pick_token<T, VEC, false>(p.rs, scale, b, d, c, tin, part, lane)
+                  : pick_token<T, VEC, true>(p.rs, scale, b, d, c, tin, part, lane);
   }
   write_tokens(p, b, j, token, s_x, lane, 32);
 }

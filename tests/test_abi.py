@@ -58,12 +58,12 @@ def test_plans_cover_every_workload_shape(lib):
         # pass-1 units: one per (row, chunk); K+1 rows (greedy), 2K+1 rows (sampling)
         assert p.greedy_units_per_sequence == 8 * p.n_chunks
         assert p.sampling_units_per_sequence == 15 * p.n_chunks
-        # one pass-2 cluster per sequence: up to 16 CTAs for batches of at most 32 sequences,
-        # else up to 8 (the portable cluster size)
-        assert p.finish_ctas_per_sequence == min(16, p.n_chunks)
+        # one pass-2 cluster per sequence of 32-warp CTAs, one chunk per warp, whatever B
+        assert p.finish_threads_per_cta == 1024
+        assert p.finish_ctas_per_sequence == -(-p.n_chunks // 32) <= 4
         q = binding.Plan()
         assert lib.dspark_plan(64, 7, V, BF16, 1, ctypes.byref(q)) == 0
-        assert q.finish_ctas_per_sequence == min(8, q.n_chunks)
+        assert q.finish_ctas_per_sequence == p.finish_ctas_per_sequence
         assert lib.dspark_plan(4, 7, V, BF16, 0, ctypes.byref(p)) == 0
         assert p.elems_per_load == 1
         assert lib.dspark_plan(4, 7, V, F32, 1, ctypes.byref(p)) == 0
