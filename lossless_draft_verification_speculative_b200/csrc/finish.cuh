@@ -495,9 +495,7 @@ __global__ void __launch_bounds__(kW * 32, kW <= 8 ? 4 : 1)
   __shared__ float s_mass[kMaxChunkCount];  // every chunk's mass of the draw's law
   __shared__ float s_u[kMaxK + 1];
   __shared__ int s_x[kMaxK];
-  __shared__ Decision s_dec;
-  __shared__ double s_tin, s_z;
-  __shared__ int s_chunk;
+  __shared__ float2 s_zg[kMaxK];
   // the next kernel in the stream may be scheduled as these CTAs retire (it waits for them)
   grid_dependents_launch();
   cg::cluster_group cluster = cg::this_cluster();
@@ -537,12 +535,13 @@ __global__ void __launch_bounds__(kW * 32, kW <= 8 ? 4 : 1)
   if (tid < nd) x = p.drafts[static_cast<size_t>(b) * K + tid];
   if (tid <= nd) s_u[tid] = p.uniforms[static_cast<size_t>(b) * K1 + tid];
   grid_dependency_wait();
+  Decision d;
   if constexpr (kFin == kFinEarlyExit) {
     if (tid < nd) s_x[tid] = x;
-    if (tid == 0) s_dec = p.dec[b];
+    d = p.dec[b];  // every warp reads the stored decision itself
+    __syncthreads();
   } else {
-    // the draft tokens' logits, gathered by pass 1: warp 0 keeps draft i's on lane i, its load
-    // in flight with the records' below
+    // the draft tokens' logits, gathered by pass 1, in flight with the records' below
     float2 zg = make_float2(0.f, 0.f);
     if (tid < nd) {
       s_x[tid] = x;
@@ -553,55 +552,49 @@ __global__ void __launch_bounds__(kW * 32, kW <= 8 ? 4 : 1)
     // the (reference, sum) of every row the sequence uses
     const RowFilter used{K, nd, true};
     merge_rows<true, kMixed, kW>(p, b, used, wi, lane, s_stat);
+    if (tid < nd) s_zg[tid] = zg;
     __syncthreads();
 
-    // decisions (warp 0; draft i on lane i)
-    if (wi == 0) {
-      int status = 0;
-      bool bad = false;
-      for (int r = lane; r < rows; r += 32) bad |= (!kMixed || used(r)) && !stat_ok(s_stat[r]);
-      if (__any_sync(0xffffffffu, bad)) status |= DSPARK_SEQ_NONFINITE;
-      const int x = lane < nd ? s_x[lane] : 0;
-      const bool bad_draft = lane < nd && (x < 0 || x >= V);
-      if (__any_sync(0xffffffffu, bad_draft)) status |= DSPARK_SEQ_BAD_DRAFT;
-      const float fnan = __int_as_float(0x7fffffff);
-      float px = fnan, qx = fnan;
-      bool accept = false;
-      if (lane < nd && !bad_draft) {
-        const float2 sp = s_stat[lane], sq = s_stat[K1 + lane];
-        // p_i(x_i) = 2^(z*s - M) / S (division within 2 ulp: no IEEE slow path)
-        px = __fdividef(ex2(__fmaf_rn(zg.x, scale, -sp.x)), sp.y);
-        qx = __fdividef(ex2(__fmaf_rn(zg.y, scale, -sq.x)), sq.y);
-        accept = __fmul_rn(s_u[lane], qx) < px;
-      }
-      const unsigned rej = __ballot_sync(0xffffffffu, lane < nd && !accept);
-      const int j = rej ? __ffs(rej) - 1 : nd;
-      if (g == 0 && lane < K) {
-        if (p.out.p_draft) p.out.p_draft[static_cast<size_t>(b) * K + lane] = px;
-        if (p.out.q_draft) p.out.q_draft[static_cast<size_t>(b) * K + lane] = qx;
-      }
-      if (lane == 0) {
-        const float2 sp = s_stat[j];
-        Decision d;
-        d.j = j;
-        d.nd = nd;
-        d.status = status;
-        d.mp = sp.x;
-        d.ip = __fdividef(1.f, sp.y);
-        if (j < nd) {
-          const float2 sq = s_stat[K1 + j];
-          d.mq = sq.x;
-          d.iq = __fdividef(1.f, sq.y);
-        } else {
-          d.mq = 0.f;
-          d.iq = 0.f;
-        }
-        s_dec = d;
-      }
+    // decisions, by every warp (the same inputs and arithmetic, so the same j everywhere):
+    // draft i on lane i
+    int status = 0;
+    bool bad = false;
+    for (int r = lane; r < rows; r += 32) bad |= (!kMixed || used(r)) && !stat_ok(s_stat[r]);
+    if (__any_sync(0xffffffffu, bad)) status |= DSPARK_SEQ_NONFINITE;
+    const int xl = lane < nd ? s_x[lane] : 0;
+    const bool bad_draft = lane < nd && (xl < 0 || xl >= V);
+    if (__any_sync(0xffffffffu, bad_draft)) status |= DSPARK_SEQ_BAD_DRAFT;
+    const float fnan = __int_as_float(0x7fffffff);
+    float px = fnan, qx = fnan;
+    bool accept = false;
+    if (lane < nd && !bad_draft) {
+      const float2 sp = s_stat[lane], sq = s_stat[K1 + lane], zg = s_zg[lane];
+      // p_i(x_i) = 2^(z*s - M) / S (division within 2 ulp: no IEEE slow path)
+      px = __fdividef(ex2(__fmaf_rn(zg.x, scale, -sp.x)), sp.y);
+      qx = __fdividef(ex2(__fmaf_rn(zg.y, scale, -sq.x)), sq.y);
+      accept = __fmul_rn(s_u[lane], qx) < px;
+    }
+    const unsigned rej = __ballot_sync(0xffffffffu, lane < nd && !accept);
+    const int j = rej ? __ffs(rej) - 1 : nd;
+    if (g == 0 && wi == 0 && lane < K) {
+      if (p.out.p_draft) p.out.p_draft[static_cast<size_t>(b) * K + lane] = px;
+      if (p.out.q_draft) p.out.q_draft[static_cast<size_t>(b) * K + lane] = qx;
+    }
+    const float2 sp = s_stat[j];
+    d.j = j;
+    d.nd = nd;
+    d.status = status;
+    d.mp = sp.x;
+    d.ip = __fdividef(1.f, sp.y);
+    if (j < nd) {
+      const float2 sq = s_stat[K1 + j];
+      d.mq = sq.x;
+      d.iq = __fdividef(1.f, sq.y);
+    } else {
+      d.mq = 0.f;
+      d.iq = 0.f;
     }
   }
-  __syncthreads();
-  const Decision d = s_dec;
   // this CTA's chunk range of the draw's rows into L2, ahead of the warps' second loads
   if (VEC > 1 && lane == 0 && wi >= kW - 2 && !(d.status & kErrBits)) {
     const int t0 = g * cpc * kCE;
@@ -633,54 +626,51 @@ __global__ void __launch_bounds__(kW * 32, kW <= 8 ? 4 : 1)
     return;
   }
 
-  // ---- which chunk holds the draw (every CTA, the same float64 arithmetic on the same masses)
+  // ---- which chunk holds the draw (warp 0 of every CTA, the same float64 arithmetic on the
+  // same masses)
   const int j = d.j;
   int status = d.status;
   bool use_p = !resid;
-  for (int pass = 0; pass < 2; ++pass) {
-    if (wi == 0) {
-      float ms[kMassPerLane];
-#pragma unroll
-      for (int k = 0; k < kMassPerLane; ++k) {
-        const int c = lane * kMassPerLane + k;
-        ms[k] = c < p.nch ? s_mass[c] : 0.f;
-      }
-      const ChunkPick pk = pick_chunk(ms, s_u[nd], lane);
-      if (lane == 0) {
-        s_chunk = pk.c;
-        s_tin = pk.tin;
-        s_z = pk.z;
-      }
-    }
-    __syncthreads();
-    if (use_p || s_z > 0.0) break;
+  if (resid) {
     // a residual whose every value rounded to zero (impossible in exact arithmetic after a
-    // rejection): draw from p_j instead. Every CTA of the cluster sees the same masses and
-    // takes this branch; the masses are rewritten only after every CTA has read them.
-    use_p = true;
-    status |= DSPARK_SEQ_ZERO_RESIDUAL;
-    cluster.sync();
-    for (int lc = wi; lc < cpc; lc += kW) {
-      const int c = g * cpc + lc;
-      if (c >= p.nch) break;
-      const float m = chunk_work<T, VEC, false>(p.rs, scale, b, c, d, lane,
-                                                s_part + static_cast<size_t>(lc) * kGroups);
-      if (lane < G) cluster.map_shared_rank(s_mass, lane)[c] = m;
+    // rejection): draw from p_j instead. Every warp of the cluster sees the same masses and
+    // takes this branch together; the masses are rewritten only after every CTA read them.
+    bool any = false;
+    for (int c = lane; c < p.nch; c += 32) any |= s_mass[c] > 0.f;
+    if (!__any_sync(0xffffffffu, any)) {
+      use_p = true;
+      status |= DSPARK_SEQ_ZERO_RESIDUAL;
+      cluster.sync();
+      for (int lc = wi; lc < cpc; lc += kW) {
+        const int c = g * cpc + lc;
+        if (c >= p.nch) break;
+        const float m = chunk_work<T, VEC, false>(p.rs, scale, b, c, d, lane,
+                                                  s_part + static_cast<size_t>(lc) * kGroups);
+        if (lane < G) cluster.map_shared_rank(s_mass, lane)[c] = m;
+      }
+      cluster.sync();
     }
-    cluster.sync();
   }
-  const int c = s_chunk;
+  if (wi != 0) return;
+  float ms[kMassPerLane];
+#pragma unroll
+  for (int k = 0; k < kMassPerLane; ++k) {
+    const int c = lane * kMassPerLane + k;
+    ms[k] = c < p.nch ? s_mass[c] : 0.f;
+  }
+  const ChunkPick pk = pick_chunk(ms, s_u[nd], lane);
+  const int c = pk.c;
   const int owner = c >= 0 ? c / cpc : 0;
   if (owner != g) return;  // another CTA draws
-  if (wi != 0) return;
   if (lane == 0) {
-    if (p.out.resid_mass) p.out.resid_mass[b] = resid ? (use_p ? 0.f : static_cast<float>(s_z)) : 1.f;
+    if (p.out.resid_mass)
+      p.out.resid_mass[b] = resid ? (use_p ? 0.f : static_cast<float>(pk.z)) : 1.f;
     if (p.out.status) p.out.status[b] = status;
   }
   int token = -1;
   if (c >= 0) {
     const float* part = s_part + static_cast<size_t>(c - g * cpc) * kGroups;
-    const float tin = static_cast<float>(s_tin);
+    const float tin = static_cast<float>(pk.tin);
     token = use_p ? pick_token<T, VEC, false>(p.rs, scale, b, d, c, tin, part, lane)
                   : pick_token<T, VEC, true>(p.rs, scale, b, d, c, tin, part, lane);
   }
