@@ -533,18 +533,30 @@ def time_mixed_batch(w, sets, D, U, workspace, dev, reps):
             "committed_tokens_per_block": float((out.n_accepted.double() + 1).mean().item())}
 
 
-def early_exit_bytes(n_accepted, K, V, elem_bytes, sample):
-    """Bytes the early-exit call streams: wave w (pairs [2^w - 1, 2^(w+1) - 1) cut at K, the
-    last adding the bonus row) reads its rows of every sequence that accepted all drafts
-    before it, i.e. whose accepted count is at least the wave's first pair."""
-    waves, w = [], 0
+EE_BIG_PAIR_BYTES = 64 << 20  # the library's kEeBigPairBytes (early_exit.cuh)
+
+
+def early_exit_waves(B, K, V, elem_bytes, sample):
+    """The pairs [lo, hi) of each early-exit wave, as the library schedules them: waves of 1, 2,
+    4, ... pairs when one row pair of the whole batch is at least 64 MB, else 2, 8, 32, ...,
+    cut at K."""
+    pair = B * V * elem_bytes * (2 if sample else 1)
+    first, growth = (1, 2) if pair >= EE_BIG_PAIR_BYTES else (2, 4)
+    waves, a, n = [], 0, first
     while True:
-        lo, hi = min(2 ** w - 1, K), min(2 ** (w + 1) - 1, K)
+        lo, hi = min(a, K), min(a + n, K)
         waves.append((lo, hi))
         if hi >= K:
-            break
-        w += 1
+            return waves
+        a, n = a + n, n * growth
+
+
+def early_exit_bytes(n_accepted, K, V, elem_bytes, sample):
+    """Bytes the early-exit call streams: each wave (``early_exit_waves``, the last adding the
+    bonus row) reads its rows of every sequence that accepted all drafts before it, i.e. whose
+    accepted count is at least the wave's first pair."""
     n = np.asarray(n_accepted)
+    waves = early_exit_waves(n.size, K, V, elem_bytes, sample)
     rows = 0
     for i, (lo, hi) in enumerate(waves):
         per = (hi - lo) * (2 if sample else 1) + (1 if i == len(waves) - 1 else 0)

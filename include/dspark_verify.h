@@ -213,9 +213,11 @@ dspark_status_t dspark_mixed_accept(const void* p1, int64_t ld_p1, const void* p
  * K=15, V=262144 reads 4.2 GB in full) then read a fraction of their bytes.
  *  Arguments as for speculative_sample_accept (T == 0: greedy; q and uniforms may then be
  *  NULL), with the same workspace.
- *  The pairs (P_i, Q_i) are read in waves of 1, 2, 4, ... pairs (the last wave adds the
- *  bonus row P_K); each wave reads only the sequences that accepted every earlier draft. A
- *  call launches two kernels per wave (ceil(log2(K+1)) waves, one when K == 0) and, when
+ *  The pairs (P_i, Q_i) are read in waves (the last wave adds the bonus row P_K); each wave
+ *  reads only the sequences that accepted every earlier draft. When one row pair of the whole
+ *  batch (B * V elements of P, and of Q when sampling) takes at least 64 MiB the waves are 1,
+ *  2, 4, ... pairs, else 2, 8, 32, ... pairs (a wave costs about 5 us beyond its bytes, which
+ *  a smaller pair does not hide), cut at K. A call launches two kernels per wave and, when
  *  sampling, the finish.
  *  Results: on blocks whose rows are all usable, identical to speculative_sample_accept /
  *  greedy_accept (same records, decisions and draw). Rows after the stop are never read, so

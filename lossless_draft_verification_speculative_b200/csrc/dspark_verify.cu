@@ -41,6 +41,7 @@ bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) %
 struct Plan {
   int vec;  // elements per load: 16-byte vectors (8 bf16 / 4 fp32) or 1
   int nch;  // 2048-token chunks per row
+  int fw;   // warps per sampling-finish CTA: 16 (small batches) or 32
   int G;    // pass-2 CTAs per sequence (one cluster), sampling
   int cpc;  // chunks per pass-2 CTA
 };
@@ -51,8 +52,17 @@ bool make_plan(int B, int V, dspark_dtype_t dt, bool aligned16, Plan* pl) {
   if (nch < 1 || nch > kMaxChunkCount) return false;
   pl->vec = aligned16 ? 16 / es : 1;
   pl->nch = static_cast<int>(nch);
-  // sampling finish: one chunk per warp of 32-warp CTAs, G = ceil(nch / 32) <= 4 per cluster
-  pl->G = (pl->nch + kFinWarps - 1) / kFinWarps;
+  // sampling finish, one CTA per SM and one chunk per warp: CTAs of 16 warps (G = ceil(nch /
+  // 16) <= 8 per cluster, each warp's chunk in one load round) while the batch's clusters fit
+  // on the SMs of a B200, else 32 warps (G = ceil(nch / 32) <= 4)
+  const int g16 = (pl->nch + kFinWarpsSmall - 1) / kFinWarpsSmall;
+  if (static_cast<long long>(B) * g16 <= kPlanSMs) {
+    pl->fw = kFinWarpsSmall;
+    pl->G = g16;
+  } else {
+    pl->fw = kFinWarps;
+    pl->G = (pl->nch + kFinWarps - 1) / kFinWarps;
+  }
   pl->cpc = (pl->nch + pl->G - 1) / pl->G;
   return true;
 }
@@ -81,10 +91,10 @@ WsLayout ws_layout(long long B, long long K, int nch) {
 }
 
 // Early-exit waves for K drafts: pairs [2^w - 1, 2^(w+1) - 1) cut at K, the last one ending at K.
-int n_waves(int K) {
+int n_waves(const WaveSchedule& ws, int K) {
   int w = 0, lo = 0, hi = 0;
   for (;; ++w) {
-    wave_range(w, K, lo, hi);
+    wave_range(ws, w, K, lo, hi);
     if (hi >= K) return w + 1;
   }
 }
@@ -166,13 +176,12 @@ struct Call {
   char* ws;
 };
 
-// The sampling finish: one cluster of pl.G CTAs of 32 warps per sequence, each with pl.cpc
+// The sampling finish: one cluster of pl.G CTAs of kW warps per sequence, each with pl.cpc
 // chunks of group sums in dynamic shared memory, as a programmatic dependent of the kernel
 // before it.
-template <typename T, int VEC, int kFin>
-dspark_status_t launch_finish_sample(const FinishParamsOf<kFin>& fp, const Plan& pl, int B,
-                                     cudaStream_t stream) {
-  constexpr int kW = kFinWarps;
+template <typename T, int VEC, int kFin, int kW>
+dspark_status_t launch_finish_sample_w(const FinishParamsOf<kFin>& fp, const Plan& pl, int B,
+                                       cudaStream_t stream) {
   cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
@@ -204,6 +213,14 @@ dspark_status_t launch_finish_sample(const FinishParamsOf<kFin>& fp, const Plan&
   return cudaLaunchKernelEx(&cfg, finish_sample_kernel<T, VEC, kFin, kW>, fp) == cudaSuccess
              ? DSPARK_OK
              : DSPARK_ERR_CUDA;
+}
+
+template <typename T, int VEC, int kFin>
+dspark_status_t launch_finish_sample(const FinishParamsOf<kFin>& fp, const Plan& pl, int B,
+                                     cudaStream_t stream) {
+  return pl.fw == kFinWarpsSmall
+             ? launch_finish_sample_w<T, VEC, kFin, kFinWarpsSmall>(fp, pl, B, stream)
+             : launch_finish_sample_w<T, VEC, kFin, kFinWarps>(fp, pl, B, stream);
 }
 
 // Pass 1 over every (row, chunk) unit (one CTA per SM, every grid-th unit), then pass 2.
@@ -304,7 +321,8 @@ dspark_status_t run_early_exit(const Call& c, const Plan& pl, cudaStream_t strea
   if (total_units >= (1LL << 31)) return DSPARK_ERR_UNSUPPORTED;
   const WsLayout w = ws_layout(c.B, c.rs.K, pl.nch);
   const int K = c.rs.K;
-  const int W = n_waves(K);
+  const WaveSchedule sched = wave_schedule(c.B, c.rs.V, static_cast<int>(sizeof(T)), kSample);
+  const int W = n_waves(sched, K);
   int* alive[2] = {reinterpret_cast<int*>(c.ws + w.alive),
                    reinterpret_cast<int*>(c.ws + w.alive) + c.B};
   int* cnt = reinterpret_cast<int*>(c.ws + w.cnt);
@@ -315,7 +333,7 @@ dspark_status_t run_early_exit(const Call& c, const Plan& pl, cudaStream_t strea
   pdl[0].val.programmaticStreamSerializationAllowed = 1;
   for (int wv = 0; wv < W; ++wv) {
     WaveArgs wa{};
-    wave_range(wv, K, wa.lo, wa.hi);
+    wave_range(sched, wv, K, wa.lo, wa.hi);
     wa.last = wv == W - 1;
     wa.wave = wv;
     wa.alive = alive[wv & 1];
@@ -530,7 +548,7 @@ dspark_status_t dspark_plan(int B, int K, int V, dspark_dtype_t dtype, int align
   plan->greedy_units_per_sequence = (K + 1) * pl.nch;
   plan->sampling_units_per_sequence = (2 * K + 1) * pl.nch;
   plan->finish_ctas_per_sequence = pl.G;
-  plan->finish_threads_per_cta = kFinWarps * 32;
+  plan->finish_threads_per_cta = pl.fw * 32;
   return DSPARK_OK;
 }
 

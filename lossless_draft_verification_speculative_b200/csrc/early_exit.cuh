@@ -4,8 +4,8 @@
 // A draft is accepted with probability below one (the DeepSeek-V4-Flash DSpark drafter card
 // reports acceptance between 52% and 91%), so most blocks end well before row K, and the rows
 // after a sequence's first rejection j cannot change its result. The pairs (P_i, Q_i) are
-// taken in waves of 1, 2, 4, ... pairs (wave w: pairs [2^w - 1, 2^(w+1) - 1), cut at K), the
-// last wave adding the bonus row P_K. A wave is two launches:
+// taken in waves (wave_schedule below: 1, 2, 4, ... pairs for large batches, 2, 8, 32, ...
+// for the others, cut at K), the last wave adding the bonus row P_K. A wave is two launches:
 //  - ee_stream_kernel: pass 1 (stream.cuh) over the units of the wave's rows of the
 //    sequences still alive, in the same record layout as a full call (so a record, a
 //    function of its unit's logits alone, is bit-identical to the full call's);
@@ -25,14 +25,31 @@
 
 namespace dspark {
 
-constexpr int kMaxWaves = 8;  // K <= 32 takes 6 waves, of 1, 2, 4, 8, 16 and 1 pairs
+constexpr int kMaxWaves = 8;  // K <= 32 takes at most 6 waves, of 1, 2, 4, 8, 16 and 1 pairs
+
+// The wave schedule: waves of `first`, first * growth, ... pairs, cut at K. A wave has a fixed
+// cost (the stream's ramp and tail, the decisions' launch and merge: about 5 us), so when a
+// row pair of the whole batch is smaller than kEeBigPairBytes (the stream of one pair would
+// not hide it) the waves are 2, 8, 32, ... pairs; larger batches take 1, 2, 4, ... pairs.
+// (B=64, K=7, V=129280: 2 waves, [0, 2) and [2, 7); B=256, K=15, V=262144: 4 waves.)
+struct WaveSchedule {
+  int first, growth;
+};
+constexpr long long kEeBigPairBytes = 64ll << 20;
+inline WaveSchedule wave_schedule(long long B, long long V, int elem_bytes, bool sample) {
+  const long long pair = B * V * elem_bytes * (sample ? 2 : 1);
+  return pair >= kEeBigPairBytes ? WaveSchedule{1, 2} : WaveSchedule{2, 4};
+}
 
 // Pairs [lo, hi) of wave w.
-__host__ __device__ __forceinline__ void wave_range(int w, int K, int& lo, int& hi) {
-  lo = (1 << w) - 1;
-  hi = (1 << (w + 1)) - 1;
-  lo = lo < K ? lo : K;
-  hi = hi < K ? hi : K;
+inline void wave_range(const WaveSchedule& ws, int w, int K, int& lo, int& hi) {
+  long long a = 0, n = ws.first;
+  for (int i = 0; i < w && a < K; ++i) {
+    a += n;
+    n *= ws.growth;
+  }
+  lo = static_cast<int>(a < K ? a : K);
+  hi = static_cast<int>(a + n < K ? a + n : K);
 }
 
 // The wave's rows: P_i (and Q_i when sampling) for pairs i in [lo, hi), and P_K in the last.

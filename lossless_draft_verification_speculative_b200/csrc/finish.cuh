@@ -4,8 +4,10 @@
 // row), compares the drafts with the row argmaxes and writes the AcceptResult.
 //
 // Sampling: one thread-block cluster of G = ceil(n_chunks / 32) CTAs of 32 warps per sequence
-// (2 for V = 129280, at most 4), one CTA per SM. Small clusters of whole-SM CTAs are placed at
-// once: with 8-CTA clusters of 8-warp CTAs the GPU left a cluster unplaced until others had
+// (2 for V = 129280, at most 4), one CTA per SM; batches whose clusters of 16-warp CTAs
+// (ceil(n_chunks / 16) per sequence) fit on the SMs take those, which spread a sequence's
+// chunks over twice the SMs and load each chunk in one round. Small clusters of whole-SM CTAs
+// are placed at once: with 8-CTA clusters of 8-warp CTAs the GPU left a cluster unplaced until others had
 // finished (the clusters must fit in a GPC). Every CTA merges the 2K+1 rows' softmax records
 // and takes the accept decisions (the same inputs and arithmetic in each, so the same j);
 // after the early-exit waves it loads the decision they stored instead. Each warp then
@@ -27,8 +29,10 @@ namespace dspark {
 constexpr int kErrBits =
     DSPARK_SEQ_BAD_DRAFT | DSPARK_SEQ_NONFINITE | DSPARK_SEQ_TIMEOUT | DSPARK_SEQ_BAD_PARAM;
 constexpr int kMaxRows = 2 * kMaxK + 1;
-constexpr int kFinWarps = 32;   // warps per sampling-finish CTA: one chunk each
-constexpr int kFinMaxCpc = 32;  // chunks per finish CTA at most
+constexpr int kFinWarps = 32;       // warps per sampling-finish CTA: one chunk each
+constexpr int kFinWarpsSmall = 16;  // the same for small batches, 128 registers per thread
+constexpr int kFinMaxCpc = 32;      // chunks per finish CTA at most
+constexpr int kPlanSMs = 148;       // SMs of a B200: the small-batch layout while B * G fits
 
 // Kernel parameters (see StreamParamsMixed on their size). The sampling kernel's cluster size
 // G and chunks per CTA, ceil(n_chunks / G), come from its launch.
@@ -297,14 +301,15 @@ __device__ __forceinline__ float group_sum(const GroupRaw<T, VEC>& gp, const Gro
 // Chunk c of the draw's law (kResid: the residual of row pair j, else p of row j), one warp:
 // the 256 group sums into part (token order) and the chunk's mass on every lane. Out of line:
 // its registers are allocated apart from the kernel's (the finish has several call sites).
-template <typename T, int VEC, bool kResid>
+template <typename T, int VEC, bool kResid, bool kWide = false>
 __device__ __forceinline__ float chunk_work(const RowSet& rs, float scale, int b, int c,
                                             const Decision& d, int lane, float* part) {
   const int K = rs.K, V = rs.V;
   const T* pr = row_ptr<T>(rs, b, d.j);
   const T* qr = kResid ? row_ptr<T>(rs, b, K + 1 + d.j) : pr;
-  constexpr int kPerLane = kGroups / 32;                      // groups per lane
-  constexpr int kRound = VEC == 8 ? 4 : (VEC == 4 ? 2 : 1);  // groups in flight per row
+  constexpr int kPerLane = kGroups / 32;  // groups per lane
+  // groups in flight per row: all 8 (one round) with 128 registers per thread on bf16 rows
+  constexpr int kRound = VEC == 8 ? (kWide ? 8 : 4) : (VEC == 4 ? 2 : 1);
   float acc = 0.f;
 #pragma unroll
   for (int k0 = 0; k0 < kPerLane; k0 += kRound) {
@@ -486,10 +491,10 @@ using FinishParamsOf = std::conditional_t<
 // of the cluster owns chunks g*cpc .. g*cpc + cpc - 1 of the draw's law (warp w: local chunks
 // w, w + kW, ...).
 template <typename T, int VEC, int kFin, int kW>
-__global__ void __launch_bounds__(kW * 32, kW <= 8 ? 4 : 1)
-    finish_sample_kernel(const FinishParamsOf<kFin> p) {
+__global__ void __launch_bounds__(kW * 32, 1) finish_sample_kernel(const FinishParamsOf<kFin> p) {
   constexpr bool kMixed = kFin == kFinMixed;
   constexpr int kT = kW * 32;
+  constexpr bool kWide = kW <= kFinWarpsSmall;  // 128 registers per thread
   extern __shared__ float s_part[];  // [cpc][kGroups]: group sums of the draw's law
   __shared__ float2 s_stat[kMaxRows];
   __shared__ float s_mass[kMaxChunkCount];  // every chunk's mass of the draw's law
@@ -614,8 +619,8 @@ __global__ void __launch_bounds__(kW * 32, kW <= 8 ? 4 : 1)
       const int c = g * cpc + lc;
       if (c >= p.nch) break;
       float* pr = s_part + static_cast<size_t>(lc) * kGroups;
-      const float m = resid ? chunk_work<T, VEC, true>(p.rs, scale, b, c, d, lane, pr)
-                            : chunk_work<T, VEC, false>(p.rs, scale, b, c, d, lane, pr);
+      const float m = resid ? chunk_work<T, VEC, true, kWide>(p.rs, scale, b, c, d, lane, pr)
+                            : chunk_work<T, VEC, false, kWide>(p.rs, scale, b, c, d, lane, pr);
       if (lane < G) cluster.map_shared_rank(s_mass, lane)[c] = m;
     }
   }

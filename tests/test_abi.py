@@ -58,12 +58,17 @@ def test_plans_cover_every_workload_shape(lib):
         # pass-1 units: one per (row, chunk); K+1 rows (greedy), 2K+1 rows (sampling)
         assert p.greedy_units_per_sequence == 8 * p.n_chunks
         assert p.sampling_units_per_sequence == 15 * p.n_chunks
-        # one pass-2 cluster per sequence of 32-warp CTAs, one chunk per warp, whatever B
-        assert p.finish_threads_per_cta == 1024
-        assert p.finish_ctas_per_sequence == -(-p.n_chunks // 32) <= 4
-        q = binding.Plan()
-        assert lib.dspark_plan(64, 7, V, BF16, 1, ctypes.byref(q)) == 0
-        assert q.finish_ctas_per_sequence == p.finish_ctas_per_sequence
+        # one pass-2 cluster per sequence, one chunk per warp: 16-warp CTAs while the batch's
+        # clusters fit on 148 SMs, else 32-warp CTAs
+        for B in (4, 64, 200):
+            q = binding.Plan()
+            assert lib.dspark_plan(B, 7, V, BF16, 1, ctypes.byref(q)) == 0
+            g16 = -(-q.n_chunks // 16)
+            if B * g16 <= 148:
+                assert q.finish_threads_per_cta == 512 and q.finish_ctas_per_sequence == g16 <= 8
+            else:
+                assert q.finish_threads_per_cta == 1024
+                assert q.finish_ctas_per_sequence == -(-q.n_chunks // 32) <= 4
         assert lib.dspark_plan(4, 7, V, BF16, 0, ctypes.byref(p)) == 0
         assert p.elems_per_load == 1
         assert lib.dspark_plan(4, 7, V, F32, 1, ctypes.byref(p)) == 0
