@@ -243,11 +243,22 @@ dspark_status_t dspark_early_exit_accept(const void* p1, int64_t ld_p1, const vo
  *  R      the Markov rank: 256 (other ranks: DSPARK_ERR_UNSUPPORTED).
  *  h      device [B, R] float32 states, 16-byte aligned.
  *  y      device [B, V] float32 results (row b at y + b * V).
- *  Sums are float32 in a fixed order; batches of more than 4 states read the table once per
- *  4 states. B == 0 or V == 0 is a no-op. */
+ *  F16: float32 sums in a fixed order on the CUDA cores, the table read once per 4 states.
+ *  Q8_0, B <= 2: float32 sums in a fixed order on the CUDA cores, one read of the table.
+ *  Q8_0, B > 2: on the tensor cores (tcgen05), the table read once per 64 states. Each state is
+ *    scaled by a power of two and split into float16 parts hi + lo (within 2^-23 of its
+ *    largest |h|); each block's 32 products q * part are exact and summed in float32 by the
+ *    tensor cores, then scaled by d and the 8 blocks added by float32 FMAs in a fixed order.
+ *  A non-finite state value gives non-finite results. B == 0 or V == 0 is a no-op. */
 typedef enum { DSPARK_TABLE_F16 = 0, DSPARK_TABLE_Q8_0 = 1 } dspark_table_t;
 dspark_status_t dspark_markov_matvec(const void* table, dspark_table_t type, int V, int R,
                                      const float* h, int B, float* y, void* stream);
+
+/* The number of waits inside the library's pipelined kernels (the Q8_0 mat-vec) that ran out
+ * (about a second each) on the current device since the library was loaded: 0 unless a kernel
+ * gave up; a kernel that gives up frees its resources and leaves its outputs incomplete.
+ * Synchronous (waits for the device). DSPARK_ERR_INVALID_ARG for a NULL count. */
+dspark_status_t dspark_pipeline_timeouts(unsigned long long* count);
 
 /* speculative_sample_accept without a workspace argument. The pages have no counterpart of
  * this entry point: it exists for callers that cannot allocate device memory where they

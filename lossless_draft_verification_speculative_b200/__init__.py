@@ -25,6 +25,7 @@ from .binding import (  # noqa: F401
     load_library,
     markov_matvec,
     mixed_accept,
+    pipeline_timeouts,
     plan,
     speculative_sample_accept,
     speculative_sample_accept_static,
@@ -41,6 +42,7 @@ __all__ = [
     "mixed_accept",
     "early_exit_accept",
     "markov_matvec",
+    "pipeline_timeouts",
     "load_library",
     "plan",
     "workspace_bytes",

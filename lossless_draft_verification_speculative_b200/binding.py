@@ -136,6 +136,8 @@ def load_library(build_if_missing: bool = True) -> ctypes.CDLL:
                                              ctypes.c_float, vp, AcceptOut, vp, sz, vp]
     lib.dspark_markov_matvec.restype = i32
     lib.dspark_markov_matvec.argtypes = [vp, i32, i32, i32, vp, i32, vp, vp]
+    lib.dspark_pipeline_timeouts.restype = i32
+    lib.dspark_pipeline_timeouts.argtypes = [ctypes.POINTER(ctypes.c_ulonglong)]
     lib.dspark_quench_reset.restype = i32
     lib.dspark_quench_reset.argtypes = [vp, i32]
     lib.dspark_quench_update.restype = i32
@@ -430,6 +432,18 @@ def markov_matvec(table: torch.Tensor, fmt: str, h: torch.Tensor, *,
     if rc != DSPARK_OK:
         raise DsparkError(rc, "dspark_markov_matvec")
     return y
+
+
+def pipeline_timeouts(device=None) -> int:
+    """Waits inside the library's pipelined kernels that ran out on ``device`` (default: the
+    current CUDA device) since the library was loaded; 0 unless a kernel gave up."""
+    lib = load_library()
+    n = ctypes.c_ulonglong(0)
+    with torch.cuda.device(device if device is not None else torch.cuda.current_device()):
+        rc = lib.dspark_pipeline_timeouts(ctypes.byref(n))
+    if rc != DSPARK_OK:
+        raise DsparkError(rc, "dspark_pipeline_timeouts")
+    return int(n.value)
 
 
 def speculative_sample_accept_static(P: Union[torch.Tensor, Tuple[torch.Tensor, torch.Tensor]],

@@ -22,7 +22,8 @@ INCLUDE = os.path.join(ROOT, "include")
 LIB_DIR = os.path.join(PKG_DIR, "_lib")
 LIB_PATH = os.path.join(LIB_DIR, "libdspark_verify.so")
 SOURCES = ["dspark_verify.cu", "policy.cc"]
-HEADERS = ["common.cuh", "stream.cuh", "finish.cuh", "early_exit.cuh", "markov.cuh"]
+HEADERS = ["common.cuh", "stream.cuh", "finish.cuh", "early_exit.cuh", "markov.cuh",
+           "markov_mma.cuh"]
 
 
 def nvcc_path() -> str:

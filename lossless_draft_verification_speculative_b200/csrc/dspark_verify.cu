@@ -11,12 +11,13 @@
 #include "early_exit.cuh"
 #include "finish.cuh"
 #include "markov.cuh"
+#include "markov_mma.cuh"
 #include "stream.cuh"
 
 namespace dspark {
 namespace {
 
-constexpr int kAbiVersion = 5;  // 5: dspark_plan_t gained finish_threads_per_cta
+constexpr int kAbiVersion = 6;  // 6: dspark_pipeline_timeouts
 constexpr int kMaxDevices = 64;
 
 // Tuning switch, read at every call: DSPARK_MAX_CTAS caps the pass-1 CTAs (0 = one per SM).
@@ -499,6 +500,39 @@ dspark_status_t markov_launch(const void* table, dspark_table_t type, int V, con
   return e == cudaSuccess ? DSPARK_OK : DSPARK_ERR_CUDA;
 }
 
+// Batches of up to this many states take the CUDA-core Q8_0 kernel (one launch, faster there:
+// 9.5 against 15.5 us per 129280-row call at one state, on par at four); larger ones the
+// tensor-core kernel, 64 states per launch.
+constexpr int kMarkovCudaCoreStates = 2;
+
+// The Q8_0 mat-vec on the tensor cores for nb <= N states (N = 16, 32, 48 or 64): one CTA per
+// SM over the 128-row tiles.
+template <int N>
+dspark_status_t markov_mma_launch(const void* table, int V, const float* h, int nb, float* y,
+                                  int ldy, cudaStream_t stream) {
+  const void* fn = reinterpret_cast<const void*>(&markov_q8_0_mma_kernel<N>);
+  const size_t smem = static_cast<size_t>(mma_q8_smem(N).total);
+  cudaError_t e = cudaSuccess;
+  const int ctas = resident_ctas(fn, kMmaThreads, smem, &e);
+  if (e != cudaSuccess) return DSPARK_ERR_CUDA;
+  if (ctas < 1) return DSPARK_ERR_UNSUPPORTED;
+  const int n_tiles = (V + kMmaRows - 1) / kMmaRows;
+  const int grid = n_tiles < ctas ? n_tiles : ctas;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(grid), 1, 1);
+  cfg.blockDim = dim3(kMmaThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, markov_q8_0_mma_kernel<N>, static_cast<const uint8_t*>(table), V,
+                         h, nb, y, ldy);
+  return e == cudaSuccess ? DSPARK_OK : DSPARK_ERR_CUDA;
+}
+
 }  // namespace
 }  // namespace dspark
 
@@ -722,6 +756,24 @@ dspark_status_t dspark_markov_matvec(const void* table, dspark_table_t type, int
   if (R != kMarkovRank) return DSPARK_ERR_UNSUPPORTED;
   if (!aligned(table, 16) || !aligned(h, 16) || !aligned(y, 4)) return DSPARK_ERR_UNSUPPORTED;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (type == DSPARK_TABLE_Q8_0 && B > kMarkovCudaCoreStates) {
+    for (int b0 = 0; b0 < B; b0 += kMmaMaxStates) {
+      const int nb = B - b0 < kMmaMaxStates ? B - b0 : kMmaMaxStates;
+      const float* hb = h + static_cast<size_t>(b0) * R;
+      float* yb = y + static_cast<size_t>(b0) * V;
+      dspark_status_t st;
+      if (nb <= 16)
+        st = markov_mma_launch<16>(table, V, hb, nb, yb, V, s);
+      else if (nb <= 32)
+        st = markov_mma_launch<32>(table, V, hb, nb, yb, V, s);
+      else if (nb <= 48)
+        st = markov_mma_launch<48>(table, V, hb, nb, yb, V, s);
+      else
+        st = markov_mma_launch<64>(table, V, hb, nb, yb, V, s);
+      if (st != DSPARK_OK) return st;
+    }
+    return DSPARK_OK;
+  }
   for (int b0 = 0; b0 < B; b0 += kMarkovMaxStates) {
     const int nb = B - b0 < kMarkovMaxStates ? B - b0 : kMarkovMaxStates;
     const float* hb = h + static_cast<size_t>(b0) * R;
@@ -736,6 +788,13 @@ dspark_status_t dspark_markov_matvec(const void* table, dspark_table_t type, int
     if (st != DSPARK_OK) return st;
   }
   return DSPARK_OK;
+}
+
+dspark_status_t dspark_pipeline_timeouts(unsigned long long* count) {
+  if (!count) return DSPARK_ERR_INVALID_ARG;
+  return cudaMemcpyFromSymbol(count, g_pipeline_timeouts, sizeof(*count)) == cudaSuccess
+             ? DSPARK_OK
+             : DSPARK_ERR_CUDA;
 }
 
 dspark_status_t dspark_speculative_sample_accept_static(const void* p1, int64_t ld_p1,

@@ -1,0 +1,516 @@
+// The Markov-head mat-vec y[b, v] = sum_k W[v, k] h[b, k] over a GGUF Q8_0 table, on the
+// fifth-generation tensor cores (tcgen05), for 1 to 64 states per launch with one read of the
+// table (the DeepSeek-V4-Flash DSpark drafter card, "Files": markov_w2 in Q8_0, 8 blocks of
+// 34 bytes per row of R = 256; the engine reads it four times per draft block).
+//
+// Exact operands. A Q8_0 value is d q with q a signed byte, exact in float16; the block scale
+// d is per (row, block of 32), so each block gets its own float32 accumulators and d is
+// applied afterwards. Each state h_b is scaled by a power of two 2^e_b (m_b 2^e_b in
+// [2^14, 2^15), m_b = max_k |h[b, k]|) and split into float16 parts hi + lo, which represent it
+// to within 2^-23 m_b (|h 2^e - hi| <= 8, so lo rounds at 2^-9 or finer); every product
+// q * part is exact in float32. The parts are the two halves of the MMA's N: B row b is hi_b,
+// row N + b is lo_b. Per tile of 128 rows and block j:
+//   D_j[r, b] + D_j[r, N + b] = sum_{k in block j} q[r, k] (hi[b, k] + lo[b, k])  (tensor cores)
+//   y[b, r] = 2^-e_b sum_j d[r, j] (D_j[r, b] + D_j[r, N + b])             (CUDA cores, f32)
+//
+// One CTA per SM (persistent over tiles t = blockIdx.x + i gridDim.x), 14 warps. A work item
+// is half a tile (4 blocks, K = 128); item i of the CTA is half i % 2 of its tile i / 2.
+//  - warp 0, one lane: copies each tile's 128 rows x 272 bytes (contiguous in the table) into
+//    a shared staging ring with one bulk asynchronous copy (cp.async.bulk, mbarrier
+//    completion); warp 0 also allocates and frees the tensor memory.
+//  - warp 1, one lane: per item, per block, 2 MMAs (K = 16 each) of M = 128, N = 2 x 16..64
+//    into the block's accumulators, then one commit.
+//  - warps 2-5 and 6-9, two teams of 128 threads (thread = tile row), team T converting the
+//    items of half T into A slab T: the q bytes to float16 in the 128-byte-swizzled K-major
+//    layout, the scales d to float32 beside the slab.
+//  - warps 10-13, 128 threads (thread = tile row = TMEM lane; lane quarter = warp % 4): per
+//    item, read the accumulators from tensor memory (tcgen05.ld), add hi + lo, multiply by d
+//    and accumulate; after the second half write y. Their release of the item frees both its
+//    accumulator slot and its A slab (the MMAs that read the slab are complete by then).
+// Rings: 2-3 staging buffers (a tile each), 2 A slabs (32 KB), 1-4 accumulator slots in tensor
+// memory (8 N columns each). Every mbarrier wait is bounded (about a second); a wait that runs
+// out sets an abort flag that ends every role's loop, counts the event in a device counter
+// (dspark_pipeline_timeouts), lets the copies and MMAs in flight finish (again bounded) and
+// frees the tensor memory before the CTA exits.
+#pragma once
+
+#include <cuda_fp16.h>
+
+#include "common.cuh"
+#include "markov.cuh"
+
+namespace dspark {
+
+constexpr int kMmaRows = 128;          // tile rows (MMA M)
+constexpr int kMmaMaxStates = 64;      // states per launch (MMA N = 2 x 64 at most)
+constexpr int kMmaThreads = 448;       // 14 warps
+constexpr int kMmaTeam = 128;          // threads of a converter team or of the epilogue
+constexpr int kQ8RowBytesT = 272;      // 8 blocks x 34 bytes
+constexpr int kMmaRawBytes = kMmaRows * kQ8RowBytesT;  // 34816, a staging buffer
+constexpr int kMmaSlabBytes = kMmaRows * 128 * 2;      // 32768: 128 rows x 128 halves
+constexpr int kMmaTmemCols = 512;
+
+__device__ unsigned long long g_pipeline_timeouts = 0;
+
+// ---------------------------------------------------------------- mbarrier / async helpers
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ void mbar_init(uint32_t bar, int count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Wait for the phase of the given parity to complete, for at most about a second (2^31 SM
+// clocks); false (and the CTA's abort flag set) when it runs out or another role aborted.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort) {
+  if (mbar_try(bar, parity)) return true;
+  const long long t0 = clock64();
+  while (true) {
+    if (mbar_try(bar, parity)) return true;
+    if (*abort) return false;
+    if (clock64() - t0 > (1ll << 31)) {
+      *abort = 1;
+      atomicAdd(&g_pipeline_timeouts, 1ull);
+      return false;
+    }
+  }
+}
+
+__device__ __forceinline__ void bulk_copy_g2s(uint32_t dst, const void* src, uint32_t bytes,
+                                              uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::
+          "r"(dst),
+      "l"(src), "r"(bytes), "r"(bar)
+      : "memory");
+}
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// ---------------------------------------------------------------- tcgen05 helpers
+
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+// Shared-memory matrix descriptor of a K-major operand in the 128-byte swizzle layout: rows of
+// 128 bytes, 8-row groups 1024 bytes apart (the group stride), the 16-byte chunk c of row r
+// stored at chunk c ^ (r % 8); the group base is 1024-byte aligned. A K step of 16 halves
+// (32 bytes) inside the 128-byte row advances the start address by 32.
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
+  return static_cast<uint64_t>((saddr >> 4) & 0x3FFFu) | (1ull << 16) |  // leading offset (unused)
+         (64ull << 32) |                                                // group stride 1024 B
+         (1ull << 46) |                                                 // descriptor version
+         (2ull << 61);                                                  // 128-byte swizzle
+}
+
+// Instruction descriptor: kind::f16, A and B float16, K-major, D float32, M = 128, N.
+__host__ __device__ constexpr uint32_t mma_idesc_f16(int n) {
+  return (1u << 4) | (static_cast<uint32_t>(n >> 3) << 17) | (static_cast<uint32_t>(128 >> 4) << 24);
+}
+
+__device__ __forceinline__ void mma_f16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                        uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+__device__ __forceinline__ void mma_commit(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::
+                   "r"(bar)
+               : "memory");
+}
+
+// 16 consecutive float32 columns of this warp's 32 TMEM lanes (one row per lane).
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float* v) {
+  uint32_t r[16];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr)
+      : "memory");
+#pragma unroll
+  for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+}
+// 8 consecutive float32 columns of this warp's 32 TMEM lanes.
+__device__ __forceinline__ void tmem_ld8(uint32_t taddr, float* v) {
+  uint32_t r[8];
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]),
+                 "=r"(r[6]), "=r"(r[7])
+               : "r"(taddr)
+               : "memory");
+#pragma unroll
+  for (int i = 0; i < 8; ++i) v[i] = __uint_as_float(r[i]);
+}
+__device__ __forceinline__ void tmem_ld_wait() {
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+// ---------------------------------------------------------------- the kernel
+
+struct MmaQ8Smem {
+  // offsets (bytes) from the 1024-aligned dynamic shared-memory base
+  int b_off, slab_off, d_off, raw_off, bar_off, total;
+};
+
+__host__ __device__ constexpr int mma_raw_stages(int n) { return n <= 48 ? 3 : 2; }
+// accumulator slots in the 512 TMEM columns: 8 N columns each (4 blocks x hi, lo), at most 4
+__host__ __device__ constexpr int mma_tmem_slots(int n) { return 512 / (8 * n) < 4 ? 512 / (8 * n) : 4; }
+
+__host__ __device__ inline MmaQ8Smem mma_q8_smem(int n) {
+  MmaQ8Smem s{};
+  s.b_off = 0;                                     // 4 atoms x 2n rows x 128 B
+  s.slab_off = s.b_off + 4 * 2 * n * 128;          // 2 x 32 KB
+  s.d_off = s.slab_off + 2 * kMmaSlabBytes;        // 2 x 4 blocks x 128 rows float
+  s.raw_off = s.d_off + 2 * 4 * kMmaRows * 4;
+  s.bar_off = s.raw_off + mma_raw_stages(n) * kMmaRawBytes;
+  s.total = s.bar_off + 1024 + 1024;  // barriers, flags, exponents; slack to align the base
+  return s;
+}
+
+// Converts this thread's row of work item (tile, half HF) from the staging buffer into the A
+// slab: 4 blocks, each 2 scale bytes then 32 signed bytes. The 144 bytes that cover the half
+// are read as 9 aligned 16-byte words; pairs of q bytes (even offsets, never split across a
+// word) become float16x2 through a byte permute into 0x64 bytes (1024 + (q + 128)) and an exact
+// subtraction of 1152. The scales go to d[bl * 128 + r].
+template <int HF>
+__device__ __forceinline__ void q8_convert_row(const uint8_t* raw_row, uint8_t* slab, float* d,
+                                               int r) {
+  uint32_t w[36];
+#pragma unroll
+  for (int c = 0; c < 9; ++c) {
+    const uint4 v = *reinterpret_cast<const uint4*>(raw_row + 128 * HF + 16 * c);
+    w[4 * c] = v.x; w[4 * c + 1] = v.y; w[4 * c + 2] = v.z; w[4 * c + 3] = v.w;
+  }
+  const __half2 bias = __halves2half2(__ushort_as_half(0x6480), __ushort_as_half(0x6480));
+#pragma unroll
+  for (int bl = 0; bl < 4; ++bl) {
+    constexpr int kBase = 8 * HF;   // (136 HF) - (128 HF): the half's first byte in w
+    const int s = kBase + 34 * bl;  // the block's first byte (the scale), even
+    d[bl * kMmaRows + r] = __half2float(__ushort_as_half(
+        static_cast<unsigned short>((w[s >> 2] >> (8 * (s & 3))) & 0xffffu)));
+    uint32_t h2[16];
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      const int o = s + 2 + 2 * j;  // even: the pair sits in one word
+      const uint32_t x = w[o >> 2] ^ 0x80808080u;
+      const uint32_t sel = (o & 3) == 0 ? 0x4140u : 0x4342u;
+      const uint32_t p = __byte_perm(x, 0x64646464u, sel);
+      const __half2 v = __hsub2(*reinterpret_cast<const __half2*>(&p), bias);
+      h2[j] = *reinterpret_cast<const uint32_t*>(&v);
+    }
+    // block bl = K [32 bl, 32 bl + 32) of the slab: atom bl / 2, chunks 4 (bl % 2) .. + 3
+    uint8_t* atom = slab + (bl >> 1) * (kMmaRows * 128) + r * 128;
+#pragma unroll
+    for (int m = 0; m < 4; ++m) {
+      const int c = 4 * (bl & 1) + m;
+      *reinterpret_cast<uint4*>(atom + ((c ^ (r & 7)) << 4)) =
+          make_uint4(h2[4 * m], h2[4 * m + 1], h2[4 * m + 2], h2[4 * m + 3]);
+    }
+  }
+}
+
+// 2^e as a float for -126 <= e <= 127 (exact).
+__device__ __forceinline__ float pow2f(int e) { return __int_as_float((e + 127) << 23); }
+
+// floor(log2 m) for a finite m > 0 (subnormals included).
+__device__ __forceinline__ int ilog2f(float m) {
+  const uint32_t u = __float_as_uint(m);
+  const int be = static_cast<int>(u >> 23);
+  return be != 0 ? be - 127 : -149 + (31 - __clz(static_cast<int>(u & 0x7fffffu)));
+}
+
+template <int N>
+__global__ void __launch_bounds__(kMmaThreads, 1)
+    markov_q8_0_mma_kernel(const uint8_t* __restrict__ W, int V, const float* h, int nb,
+                           float* y, int ldy) {
+  constexpr int kRaw = mma_raw_stages(N);
+  constexpr int kSlots = mma_tmem_slots(N);
+  constexpr int kStatesPerWarp = (N + 12) / 13;  // the split is done by warps 1-13
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                           ~static_cast<uintptr_t>(1023));
+  const MmaQ8Smem L = mma_q8_smem(N);
+  uint8_t* s_b = sm + L.b_off;
+  uint8_t* s_slab = sm + L.slab_off;
+  float* s_d = reinterpret_cast<float*>(sm + L.d_off);
+  uint8_t* s_raw = sm + L.raw_off;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + L.bar_off);
+  uint64_t* raw_full = bars;        // [3] producer (expect_tx) + the copy's bytes
+  uint64_t* raw_empty = bars + 3;   // [3] both converter teams (256)
+  uint64_t* slab_full = bars + 6;   // [2] a converter team (128)
+  uint64_t* slab_free = bars + 8;   // [2] the epilogue (128)
+  uint64_t* acc_full = bars + 10;   // [4] MMA commit
+  uint64_t* acc_empty = bars + 14;  // [4] the epilogue (128)
+  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(bars + 18);
+  volatile int* s_abort = reinterpret_cast<volatile int*>(bars + 19);
+  float* s_scale = reinterpret_cast<float*>(bars + 20);  // [2][64]: 2^-e_b as two factors
+
+  const int tid = threadIdx.x, wi = tid >> 5, lane = tid & 31;
+  const int n_tiles = (V + kMmaRows - 1) / kMmaRows;
+  const int my_tiles = blockIdx.x < n_tiles ? (n_tiles - 1 - blockIdx.x) / gridDim.x + 1 : 0;
+  const int n_items = 2 * my_tiles;
+
+  if (tid == 0) {
+    for (int i = 0; i < 3; ++i) {
+      mbar_init(smem_u32(&raw_full[i]), 1);
+      mbar_init(smem_u32(&raw_empty[i]), 2 * kMmaTeam);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(smem_u32(&slab_full[i]), kMmaTeam);
+      mbar_init(smem_u32(&slab_free[i]), kMmaTeam);
+    }
+    for (int i = 0; i < 4; ++i) {
+      mbar_init(smem_u32(&acc_full[i]), 1);
+      mbar_init(smem_u32(&acc_empty[i]), kMmaTeam);
+    }
+    *s_abort = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (wi == 0) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(s_tmem)),
+                 "r"(kMmaTmemCols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    tc_fence_before();
+  }
+  __syncthreads();  // barriers initialised, tensor memory allocated
+
+  grid_dependency_wait();  // h comes from the kernel before (programmatic launch)
+  grid_dependents_launch();
+
+  if (wi == 0) {
+    // ---- producer: one bulk copy per tile (the first ones overlap the split below)
+    if (lane == 0) {
+      int armed = 0;
+      for (int j = 0; j < my_tiles; ++j) {
+        const int st = j % kRaw;
+        if (!mbar_wait(smem_u32(&raw_empty[st]), ((j / kRaw) & 1) ^ 1, s_abort)) break;
+        const long long t = blockIdx.x + static_cast<long long>(j) * gridDim.x;
+        const int rows = V - t * kMmaRows < kMmaRows ? static_cast<int>(V - t * kMmaRows) : kMmaRows;
+        const uint32_t bytes = static_cast<uint32_t>(rows * kQ8RowBytesT);
+        mbar_arrive_tx(smem_u32(&raw_full[st]), bytes);
+        bulk_copy_g2s(smem_u32(s_raw + st * kMmaRawBytes), W + t * kMmaRows * kQ8RowBytesT,
+                      bytes, smem_u32(&raw_full[st]));
+        armed = j + 1;
+      }
+      if (*s_abort) {
+        // let the copies in flight land before the CTA's shared memory goes away
+        for (int j = armed - kRaw < 0 ? 0 : armed - kRaw; j < armed; ++j) {
+          const uint32_t bar = smem_u32(&raw_full[j % kRaw]);
+          const long long t0 = clock64();
+          while (!mbar_try(bar, (j / kRaw) & 1) && clock64() - t0 < (1ll << 31)) {
+          }
+        }
+      }
+    }
+  } else {
+    // ---- warps 1-13: the B operand. State b (rows nb..N-1 zero) scaled by 2^e_b and split
+    // into float16 hi (B row b) and lo (B row N + b), 128-byte-swizzled K-major: atom k / 64,
+    // row n, 16-byte chunk (k % 64) / 8 stored at chunk ((k % 64) / 8) ^ (n % 8), element k % 8.
+    const int w1 = wi - 1;
+    float hv[kStatesPerWarp][8];
+#pragma unroll
+    for (int u = 0; u < kStatesPerWarp; ++u) {
+      const int b = w1 + 13 * u;
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+        hv[u][j] = b < nb ? __ldg(h + b * kMarkovRank + lane + 32 * j) : 0.f;
+    }
+#pragma unroll
+    for (int u = 0; u < kStatesPerWarp; ++u) {
+      const int b = w1 + 13 * u;
+      if (b >= N) break;
+      float m = 0.f;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) m = max_nan(m, fabsf(hv[u][j]));  // NaN anywhere: m NaN
+      m = warp_max_nan(m);
+      int e = 0;
+      if (m > 0.f && m <= 3.402823466e38f) e = 14 - ilog2f(m);  // m 2^e in [2^14, 2^15)
+      // 2^e in two exact factors (e in [-114, 163]); 2^-e likewise
+      const int e1 = e > 127 ? 127 : e, e2 = e - e1;
+      const float f1 = pow2f(e1), f2 = pow2f(e2);
+      if (lane == 0) {
+        const int g1 = -e < -126 ? -126 : -e;
+        s_scale[b] = pow2f(g1);
+        s_scale[64 + b] = pow2f(-e - g1);
+      }
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const int k = lane + 32 * j;
+        const float x = __fmul_rn(__fmul_rn(hv[u][j], f1), f2);
+        const __half hi = __float2half_rn(x);
+        // (a non-finite x keeps lo = 0: its products are those of x itself)
+        const __half lo =
+            is_finite(x) ? __float2half_rn(__fsub_rn(x, __half2float(hi))) : __float2half_rn(0.f);
+        const int off_hi = (k >> 6) * (2 * N * 128) + b * 128 +
+                           ((((k & 63) >> 3) ^ (b & 7)) << 4) + (k & 7) * 2;
+        const int off_lo = (k >> 6) * (2 * N * 128) + (N + b) * 128 +
+                           ((((k & 63) >> 3) ^ ((N + b) & 7)) << 4) + (k & 7) * 2;
+        *reinterpret_cast<__half*>(s_b + off_hi) = hi;
+        *reinterpret_cast<__half*>(s_b + off_lo) = lo;
+      }
+    }
+    fence_proxy_async_smem();
+    asm volatile("bar.sync 1, %0;" ::"n"(kMmaThreads - 32) : "memory");  // warps 1-13
+    const uint32_t tbase = *s_tmem;
+    tc_fence_after();
+
+    if (wi == 1) {
+      // ---- MMA issuer
+      if (lane == 0) {
+        constexpr uint32_t idesc = mma_idesc_f16(2 * N);
+        const uint32_t b0 = smem_u32(s_b);
+        int issued = 0;
+        for (int i = 0; i < n_items; ++i) {
+          const int sl = i & 1, ts = i % kSlots;
+          if (!mbar_wait(smem_u32(&slab_full[sl]), (i >> 1) & 1, s_abort)) break;
+          if (!mbar_wait(smem_u32(&acc_empty[ts]), ((i / kSlots) & 1) ^ 1, s_abort)) break;
+          tc_fence_after();
+          const uint32_t a0 = smem_u32(s_slab + sl * kMmaSlabBytes);
+#pragma unroll
+          for (int bl = 0; bl < 4; ++bl) {
+            const uint32_t d_tmem = tbase + ts * (8 * N) + bl * (2 * N);
+#pragma unroll
+            for (int w = 0; w < 2; ++w) {
+              const uint32_t in_atom = 64 * (bl & 1) + 32 * w;  // bytes into the 128-byte row
+              const uint64_t ad = sw128_desc(a0 + (bl >> 1) * (kMmaRows * 128) + in_atom);
+              const uint32_t katom = 2 * sl + (bl >> 1);
+              const uint64_t bd = sw128_desc(b0 + katom * (2 * N * 128) + in_atom);
+              mma_f16(d_tmem, ad, bd, idesc, w != 0);
+            }
+          }
+          mma_commit(smem_u32(&acc_full[ts]));
+          issued = i + 1;
+        }
+        if (*s_abort && issued > 0) {
+          // the last commit completes once every MMA issued before it has
+          const int i = issued - 1;
+          const uint32_t bar = smem_u32(&acc_full[i % kSlots]);
+          const long long t0 = clock64();
+          while (!mbar_try(bar, (i / kSlots) & 1) && clock64() - t0 < (1ll << 31)) {
+          }
+        }
+      }
+    } else if (wi < 10) {
+      // ---- converter team T = half T of every tile
+      const int T = wi >= 6;
+      const int r = 32 * ((wi - 2) & 3) + lane;  // tile row
+      uint8_t* slab = s_slab + T * kMmaSlabBytes;
+      float* d = s_d + T * 4 * kMmaRows;
+      for (int j = 0; j < my_tiles; ++j) {
+        const int st = j % kRaw;
+        bool ok = mbar_wait(smem_u32(&raw_full[st]), (j / kRaw) & 1, s_abort);
+        ok = ok && mbar_wait(smem_u32(&slab_free[T]), (j & 1) ^ 1, s_abort);
+        if (!__all_sync(0xffffffffu, ok)) break;
+        const uint8_t* raw_row = s_raw + st * kMmaRawBytes + r * kQ8RowBytesT;
+        if (T == 0)
+          q8_convert_row<0>(raw_row, slab, d, r);
+        else
+          q8_convert_row<1>(raw_row, slab, d, r);
+        fence_proxy_async_smem();
+        mbar_arrive(smem_u32(&slab_full[T]));
+        mbar_arrive(smem_u32(&raw_empty[st]));
+      }
+    } else {
+      // ---- epilogue: thread = tile row = TMEM lane
+      const int q = wi & 3;
+      const int r = 32 * q + lane;
+      bool live = true;
+      for (int j = 0; j < my_tiles && live; ++j) {
+        float acc[N];
+#pragma unroll
+        for (int c = 0; c < N; ++c) acc[c] = 0.f;
+        for (int sl = 0; sl < 2; ++sl) {
+          const int i = 2 * j + sl, ts = i % kSlots;
+          // (the wait on slab_full, long complete, orders the team's scale writes before the
+          // reads below)
+          bool ok = mbar_wait(smem_u32(&acc_full[ts]), (i / kSlots) & 1, s_abort);
+          ok = ok && mbar_wait(smem_u32(&slab_full[sl]), j & 1, s_abort);
+          if (!__all_sync(0xffffffffu, ok)) {
+            live = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t ta = tbase + (static_cast<uint32_t>(32 * q) << 16) + ts * (8 * N);
+          const float* d = s_d + sl * 4 * kMmaRows;
+#pragma unroll
+          for (int bl = 0; bl < 4; ++bl) {
+            const float dv = d[bl * kMmaRows + r];
+            // (columns in chunks of 16, or 8 at N >= 48 to stay within the registers)
+            constexpr int kC = N >= 48 ? 8 : 16;
+#pragma unroll
+            for (int c = 0; c < N; c += kC) {
+              float vh[kC], vl[kC];
+              if constexpr (kC == 16) {
+                tmem_ld16(ta + bl * (2 * N) + c, vh);
+                tmem_ld16(ta + bl * (2 * N) + N + c, vl);
+              } else {
+                tmem_ld8(ta + bl * (2 * N) + c, vh);
+                tmem_ld8(ta + bl * (2 * N) + N + c, vl);
+              }
+              tmem_ld_wait();
+#pragma unroll
+              for (int k = 0; k < kC; ++k)
+                acc[c + k] = __fmaf_rn(dv, __fadd_rn(vh[k], vl[k]), acc[c + k]);
+            }
+          }
+          tc_fence_before();
+          mbar_arrive(smem_u32(&acc_empty[ts]));
+          mbar_arrive(smem_u32(&slab_free[sl]));
+        }
+        if (!live) break;
+        const long long t = blockIdx.x + static_cast<long long>(j) * gridDim.x;
+        const long long row = t * kMmaRows + r;
+        if (row < V) {
+#pragma unroll
+          for (int c = 0; c < N; ++c)
+            if (c < nb)
+              y[static_cast<long long>(c) * ldy + row] =
+                  __fmul_rn(__fmul_rn(acc[c], s_scale[c]), s_scale[64 + c]);
+        }
+      }
+    }
+  }
+
+  __syncthreads();
+  if (wi == 0) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(*s_tmem),
+                 "r"(kMmaTmemCols)
+                 : "memory");
+  }
+}
+
+}  // namespace dspark

@@ -1,9 +1,14 @@
 """The Markov-head table mat-vec on the GPU against the float64 oracle.
 
-Tolerance, from the arithmetic: each output is a float32 sum of R = 256 products (8 per
-lane, then a butterfly; or 32 per Q8_0 block, a scale multiply, then 8 blocks), so its error
-is below (R + 8) * 2^-24 * sum_k |W[v, k] h[b, k]|; the tests allow twice R * 2^-24 times that
-sum, plus 1e-30.
+Tolerance, from the arithmetic. F16: each output is a float32 sum of R = 256 products (8 per
+lane, then a butterfly), so its error is below (R + 8) * 2^-24 * sum_k |W[v, k] h[b, k]|; the
+tests allow twice R * 2^-24 times that sum, plus 1e-30. Q8_0 (tensor cores): the state, scaled
+by a power of two, is split into float16 hi + lo within 2^-23 of its largest |h|; each block's
+64 products q * part are exact and summed in float32 (at most a few roundings of 2^-24 per
+MMA step of 16 products), then scaled by d and the 8 blocks added by float32 FMAs. The same
+2 R 2^-24 sum |W h| covers the sums; the tests add 2^-22 max_k |h[b, k]| sum_k |W[v, k]| for
+the split. (One or two Q8_0 states take the CUDA-core kernel, float32 sums like F16; the added
+term only loosens their bound.)
 """
 
 import numpy as np
@@ -29,8 +34,13 @@ def _check(V, B, fmt, seed=4):
     W = mk.f16_table(raw) if fmt == "f16" else mk.q8_0_table(raw, R)
     ref = mk.markov_matvec(W, H)
     bound = 2 * R * 2.0 ** -24 * mk.abs_products(W, H) + 1e-30
+    if fmt == "q8_0":
+        hmax = np.abs(H.astype(np.float64)).max(axis=1)                  # [B]
+        wsum = np.abs(W).sum(axis=1)                                      # [V]
+        bound = bound + 2.0 ** -22 * hmax[:, None] * wsum[None, :]
     err = np.abs(y.cpu().numpy().astype(np.float64) - ref)
     assert np.all(err <= bound), (fmt, V, B, float((err / bound).max()))
+    assert bd.pipeline_timeouts() == 0
 
 
 @pytest.mark.parametrize("fmt", ["f16", "q8_0"])
@@ -39,10 +49,22 @@ def test_serving_vocab(fmt, B):
     _check(129280, B, fmt)
 
 
+@pytest.mark.parametrize("B", [3, 16, 17, 48, 64, 65, 130])
+def test_q8_0_many_states(B):
+    """One read of the table per 64 states on the tensor cores (N = 16, 32, 48, 64 and splits)."""
+    _check(129280, B, "q8_0", seed=7)
+
+
 @pytest.mark.parametrize("fmt", ["f16", "q8_0"])
-@pytest.mark.parametrize("V", [1, 7, 8, 9, 63, 65, 1000, 262144])
+@pytest.mark.parametrize("V", [1, 7, 8, 9, 63, 65, 127, 128, 129, 1000, 262144])
 def test_ragged_vocab(fmt, V):
     _check(V, 2, fmt, seed=5)
+
+
+@pytest.mark.parametrize("V", [1, 127, 128, 129, 1000, 18943, 262144])
+def test_ragged_vocab_tensor_cores(V):
+    """Partial last tiles and grids smaller than the SM count on the tensor-core path."""
+    _check(V, 5, "q8_0", seed=9)
 
 
 def test_one_hot_state_reads_a_column():
@@ -55,3 +77,31 @@ def test_one_hot_state_reads_a_column():
     torch.cuda.synchronize()
     assert np.array_equal(y.cpu().numpy()[0].astype(np.float64), mk.q8_0_table(raw, R)[:, 77])
 
+
+
+def test_q8_0_state_scales():
+    """States of very different magnitudes (each is scaled by its own power of two), a zero
+    state and one with a single nonzero entry, in one launch."""
+    V = 5000
+    raw = wl.markov_table(V, R, "q8_0", seed=8)
+    H = wl.markov_states(6, R, seed=8).astype(np.float64)
+    H[0] *= 1e-30
+    H[1] *= 1e20
+    H[2] = 0.0
+    H[3] = 0.0
+    H[3, 200] = -3.0
+    H[4] *= 2.0 ** -140  # subnormal float32 states
+    H = H.astype(np.float32)
+    y = bd.markov_matvec(torch.from_numpy(raw).to(DEV), "q8_0", torch.from_numpy(H).to(DEV))
+    torch.cuda.synchronize()
+    W = mk.q8_0_table(raw, R)
+    ref = mk.markov_matvec(W, H)
+    bound = 2 * R * 2.0 ** -24 * mk.abs_products(W, H) + \
+        2.0 ** -22 * np.abs(H.astype(np.float64)).max(axis=1)[:, None] * np.abs(W).sum(axis=1)[None, :]
+    err = np.abs(y.cpu().numpy().astype(np.float64) - ref)
+    # subnormal results are flushed by nothing here, but the bound is relative: allow the
+    # smallest float32 subnormal on top
+    assert np.all(err <= bound + 2.0 ** -149)
+    assert np.all(y.cpu().numpy()[2] == 0.0)
+    assert np.array_equal(y.cpu().numpy()[3].astype(np.float64), W[:, 200] * -3.0)
+    assert bd.pipeline_timeouts() == 0
