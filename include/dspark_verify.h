@@ -244,8 +244,10 @@ dspark_status_t dspark_early_exit_accept(const void* p1, int64_t ld_p1, const vo
  *  h      device [B, R] float32 states, 16-byte aligned.
  *  y      device [B, V] float32 results (row b at y + b * V).
  *  F16: float32 sums in a fixed order on the CUDA cores, the table read once per 4 states.
- *  Q8_0, B <= 2: float32 sums in a fixed order on the CUDA cores, one read of the table.
- *  Q8_0, B > 2: on the tensor cores (tcgen05), the table read once per 64 states. Each state is
+ *  Q8_0, B <= 4: on the CUDA cores, one read of the table: exact integer dot products of each
+ *    block's bytes with three signed-byte digit planes of the state (within 2^-22 of the
+ *    block's largest |h|), combined and scaled by d in float32.
+ *  Q8_0, B > 4: on the tensor cores (tcgen05), the table read once per 64 states. Each state is
  *    scaled by a power of two and split into float16 parts hi + lo (within 2^-23 of its
  *    largest |h|); each block's 32 products q * part are exact and summed in float32 by the
  *    tensor cores, then scaled by d and the 8 blocks added by float32 FMAs in a fixed order.

@@ -500,10 +500,9 @@ dspark_status_t markov_launch(const void* table, dspark_table_t type, int V, con
   return e == cudaSuccess ? DSPARK_OK : DSPARK_ERR_CUDA;
 }
 
-// Batches of up to this many states take the CUDA-core Q8_0 kernel (one launch, faster there:
-// 9.5 against 15.5 us per 129280-row call at one state, on par at four); larger ones the
-// tensor-core kernel, 64 states per launch.
-constexpr int kMarkovCudaCoreStates = 2;
+// Batches of up to this many states take the CUDA-core Q8_0 kernel (one launch; faster there);
+// larger ones the tensor-core kernel, 64 states per launch.
+constexpr int kMarkovCudaCoreStates = 4;
 
 // The Q8_0 mat-vec on the tensor cores for nb <= N states (N = 16, 32, 48 or 64): one CTA per
 // SM over the 128-row tiles.

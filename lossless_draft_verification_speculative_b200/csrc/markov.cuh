@@ -12,16 +12,15 @@
 //    butterfly (each round halves the values a lane carries): 2 states x 4 rows cost 9
 //    shuffles instead of 40. With 3 or 4 states the products run as packed f32x2 FMAs (even
 //    and odd elements in the two halves of the accumulator).
-//  - Q8_0: a row is 8 blocks of 34 bytes (272 bytes, so rows start 16-byte aligned). A group
-//    of 8 consecutive rows (2176 bytes) is copied by 16-byte asynchronous copies into one of
-//    the warp's two shared buffers, so the next group is in flight while the warp decodes
-//    this one; lane l decodes blocks (row l/8, block l%8) and (row 4 + l/8, block l%8):
-//    d * sum_i q[i] h[b, 32 block + i], and the 8 blocks of a row are added by a butterfly
-//    over the lanes of the row. The 32 signed bytes are read as aligned 32-bit words
-//    (funnel-shifted when the block starts 2 bytes into a word) and turned into floats by a
-//    byte permute into the bits of 2^23 + (q + 128) and one subtraction, on the ALU and FMA
-//    pipes rather than the int-to-float converter.
-// Sums run in float32 in a fixed order (independent of the launch geometry). The kernels are
+//  - Q8_0 (1 to 4 states; more take the tensor-core kernel): a row is 8 blocks of 34 bytes
+//    (272 bytes, so rows start 16-byte aligned). A group of 8 consecutive rows (2176 bytes) is
+//    copied by 16-byte asynchronous copies into one of the warp's two shared buffers, so the
+//    next group is in flight while the warp decodes this one; lane l decodes blocks (row l/8,
+//    block l%8) and (row 4 + l/8, block l%8): d * sum_i q[i] h[b, 32 block + i] as exact
+//    integer dot products (__dp4a) of the signed bytes with three signed-byte digit planes of
+//    the state (below), and the 8 blocks of a row are added by a butterfly over the lanes of
+//    the row.
+// Sums run in a fixed order (independent of the launch geometry). The kernels are
 // programmatic dependent launches: each waits for the kernel before it (which may produce h)
 // before reading anything, then lets the next one be scheduled, so back-to-back calls (the
 // engine reads the table four times per draft block) overlap their launch latency.
@@ -159,15 +158,6 @@ __global__ void __launch_bounds__(kMarkovThreads) markov_f16_kernel(const uint16
   }
 }
 
-// Four signed bytes (a 32-bit word) -> 4 floats, exactly: each byte, biased by 128, goes into
-// the low mantissa bits of 2^23 (a byte permute), and 2^23 + 128 is subtracted.
-__device__ __forceinline__ void s8x4_to_float(uint32_t x, float* f) {
-  const uint32_t u = x ^ 0x80808080u;
-#pragma unroll
-  for (int i = 0; i < 4; ++i)
-    f[i] = __fsub_rn(__uint_as_float(__byte_perm(u, 0x4B000000u, 0x7540u | i)), 8388736.f);
-}
-
 // 16 bytes global -> shared without registers (bypassing L1); n = 0 zero-fills.
 __device__ __forceinline__ void cp_async16(void* dst, const void* src, int n) {
   const uint32_t d = static_cast<uint32_t>(__cvta_generic_to_shared(dst));
@@ -180,19 +170,76 @@ __device__ __forceinline__ void cp_async_wait() {
   asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
+// The states as signed-byte digits, for the Q8_0 products on the integer dot-product unit
+// (__dp4a): per state b and table block j (32 values), a power-of-two scale s = 2^x (the
+// smallest with max_i |h_i| / s <= 127 over the block; 2^0 for an all-zero block) and three
+// digit planes with
+//   h_i = s (a_i + (b_i + (c_i + e_i) / 254) / 254),   |a_i|, |b_i|, |c_i| <= 127, |e_i| <= 1/2,
+// each digit the nearest integer to the scaled remainder. Then sum_i q_i h_i =
+// s (A + (B + C / 254) / 254) + err with A = sum_i q_i a_i etc. exact 32-bit dot products of
+// signed bytes (|A| <= 32 * 128 * 127 < 2^22) and |err| <= s / (2 * 254^2) sum_i |q_i|
+// < 2^-22 max_i |h_i| sum_i |q_i| (s < 2 max_i |h_i| / 127); the rest is float32 rounding of
+// the combination. Layout per state: [plane][block][12 words], 8 words of digits and 4 of
+// padding, so that the 8 lanes of a row, one per block, read their 16-byte words from 8
+// disjoint groups of 4 banks.
+constexpr int kQ8Planes = 3;
+constexpr int kQ8Blocks = kMarkovRank / 32;  // 8
+constexpr int kQ8DigWords = 12;              // per (plane, block), 8 used
+constexpr int kQ8StateWords = kQ8Planes * kQ8Blocks * kQ8DigWords;
+
+// x * 2^k exactly (when the result is a normal float), for -252 <= k <= 254.
+__device__ __forceinline__ float mul_pow2(float x, int k) {
+  const int k1 = k > 127 ? 127 : (k < -126 ? -126 : k);
+  return __fmul_rn(__fmul_rn(x, __int_as_float((k1 + 127) << 23)),
+                   __int_as_float((k - k1 + 127) << 23));
+}
+
+// One warp: the digits of state b's block j (lane i holds element i) into dig (the state's
+// words) and the block's exponent x into ex[j].
+__device__ __forceinline__ void q8_state_digits(float hv, int j, int lane, int8_t* dig, int* ex) {
+  const float ah = fabsf(hv);
+  const uint32_t mb = __reduce_max_sync(0xffffffffu, __float_as_uint(ah));  // |h| bits are ordered
+  const float m = __uint_as_float(mb);
+  int x = 0;
+  if (m > 0.f && m <= 3.402823466e38f) {
+    // floor(log2 m) from the bits (subnormals included); s = 2^(that - 6), or twice that when
+    // m / s would exceed 127
+    const int be = static_cast<int>(mb >> 23);
+    const int lg = be != 0 ? be - 127 : -149 + (31 - __clz(static_cast<int>(mb & 0x7fffffu)));
+    x = lg - 6;
+    if (mul_pow2(m, -x) > 127.f) x += 1;
+  }
+  const float v = mul_pow2(hv, -x);  // exact: |v| <= 127
+  const float a = rintf(v);
+  const float r1 = __fmul_rn(__fsub_rn(v, a), 254.f);  // exact: |v - a| <= 1/2
+  const float b = rintf(r1);
+  const float c = rintf(__fmul_rn(__fsub_rn(r1, b), 254.f));
+  // (a non-finite state value leaves its digits undefined; its exponent marks the block)
+  dig[((0 * kQ8Blocks + j) * kQ8DigWords) * 4 + lane] = static_cast<int8_t>(a);
+  dig[((1 * kQ8Blocks + j) * kQ8DigWords) * 4 + lane] = static_cast<int8_t>(b);
+  dig[((2 * kQ8Blocks + j) * kQ8DigWords) * 4 + lane] = static_cast<int8_t>(c);
+  if (lane == 0) ex[j] = m <= 3.402823466e38f ? x : 1024;  // 1024: non-finite
+}
+
+// |x| < 2^22 as a float, exactly, without the int-to-float converter.
+__device__ __forceinline__ float small_int_to_float(int x) {
+  return __fsub_rn(__int_as_float(x + 0x4B400000), 12582912.f);
+}
+
 // A warp's groups are double-buffered: the copy of its next group is in flight while it
-// decodes the current one. 5 CTAs (40 warps) per SM, 4 with 3 or 4 states (their sums need
-// more than 51 registers).
+// decodes the current one. Lane l takes blocks (row l/8, block l%8) and (row 4 + l/8, block
+// l%8): for each state, three integer dot-product chains over the block's 32 signed bytes
+// (read as aligned 32-bit words, funnel-shifted when the block starts 2 bytes into a word)
+// against the state's digit planes, then s (A + (B + C / 254) / 254) times the block scale d;
+// the 8 blocks of a row are added by a butterfly over the lanes of the row.
 template <int NB>
-__global__ void __launch_bounds__(kMarkovThreads, NB <= 2 ? 5 : 4) markov_q8_0_kernel(
+__global__ void __launch_bounds__(kMarkovThreads, NB <= 2 ? 4 : 3) markov_q8_0_kernel(
     const uint8_t* __restrict__ W, int V, const float* h, float* y, int ldy) {
   constexpr int kGroupBytes = kQ8Rows * kQ8RowBytes;  // 2176
   constexpr int kPieces = kGroupBytes / 16;           // 136 16-byte pieces per group
   __shared__ __align__(16) uint8_t s_rows[kMarkovThreads / 32][2][kGroupBytes];
-  // the states, block by block with a stride of 36 floats (16-byte rows whose four-word reads
-  // by the 8 lanes of a row, one per block, hit 32 different banks)
-  constexpr int kHS = 36;
-  __shared__ __align__(16) float s_h[NB][8 * kHS];
+  __shared__ __align__(16) int8_t s_dig[NB][kQ8StateWords * 4];
+  __shared__ int s_ex[NB][kQ8Blocks];
   const int lane = threadIdx.x & 31, wi = threadIdx.x >> 5;
   const int blk = lane & 7;
   const int gw = blockIdx.x * (kMarkovThreads / 32) + wi;
@@ -216,11 +263,15 @@ __global__ void __launch_bounds__(kMarkovThreads, NB <= 2 ? 5 : 4) markov_q8_0_k
   grid_dependents_launch();
   long long v0 = static_cast<long long>(gw) * kQ8Rows;
   if (v0 < V) fetch(v0, 0);
-  for (int i = threadIdx.x; i < NB * kMarkovRank; i += kMarkovThreads) {
-    const int b = i / kMarkovRank, k = i % kMarkovRank;
-    s_h[b][(k >> 5) * kHS + (k & 31)] = h[i];
+  // the states' digits: warp w takes (state, block) pairs w, w + 8, ...
+  for (int t = wi; t < NB * kQ8Blocks; t += kMarkovThreads / 32) {
+    const int b = t / kQ8Blocks, j = t % kQ8Blocks;
+    q8_state_digits(h[b * kMarkovRank + j * 32 + lane], j, lane, s_dig[b], s_ex[b]);
   }
   __syncthreads();
+  int xb[NB];  // this lane's block exponent per state
+#pragma unroll
+  for (int b = 0; b < NB; ++b) xb[b] = s_ex[b][blk];
   for (int st = 0; v0 < V; v0 += stride, st ^= 1) {
     if (v0 + stride < V) {
       fetch(v0 + stride, st ^ 1);
@@ -237,29 +288,36 @@ __global__ void __launch_bounds__(kMarkovThreads, NB <= 2 ? 5 : 4) markov_q8_0_k
       const float d = __half2float(*reinterpret_cast<const __half*>(buf + qoff - 2));
       const uint32_t* wp = reinterpret_cast<const uint32_t*>(buf + (qoff & ~3));
       const uint32_t sh = (qoff & 3) * 8;  // 0 or 16
-      float acc[NB];
-#pragma unroll
-      for (int b = 0; b < NB; ++b) acc[b] = 0.f;
+      int q[8];
       uint32_t lo = wp[0];
 #pragma unroll
       for (int k = 0; k < 8; ++k) {
         // a block 2 bytes into a word ends 2 bytes into a 9th
         const uint32_t hi = (k < 7 || sh) ? wp[k + 1] : 0u;
-        float q[4];
-        s8x4_to_float(__funnelshift_r(lo, hi, sh), q);
+        q[k] = static_cast<int>(__funnelshift_r(lo, hi, sh));
         lo = hi;
-#pragma unroll
-        for (int b = 0; b < NB; ++b) {
-          const float4 a = *reinterpret_cast<const float4*>(&s_h[b][blk * kHS + 4 * k]);
-          acc[b] = __fmaf_rn(q[0], a.x, acc[b]);
-          acc[b] = __fmaf_rn(q[1], a.y, acc[b]);
-          acc[b] = __fmaf_rn(q[2], a.z, acc[b]);
-          acc[b] = __fmaf_rn(q[3], a.w, acc[b]);
-        }
       }
 #pragma unroll
       for (int b = 0; b < NB; ++b) {
-        float s = __fmul_rn(d, acc[b]);
+        int acc[kQ8Planes];
+#pragma unroll
+        for (int pl = 0; pl < kQ8Planes; ++pl) {
+          const int4* dg = reinterpret_cast<const int4*>(s_dig[b]) +
+                           (pl * kQ8Blocks + blk) * (kQ8DigWords / 4);
+          const int4 g0 = dg[0], g1 = dg[1];
+          int a = __dp4a(q[0], g0.x, 0);
+          a = __dp4a(q[1], g0.y, a);
+          a = __dp4a(q[2], g0.z, a);
+          a = __dp4a(q[3], g0.w, a);
+          a = __dp4a(q[4], g1.x, a);
+          a = __dp4a(q[5], g1.y, a);
+          a = __dp4a(q[6], g1.z, a);
+          acc[pl] = __dp4a(q[7], g1.w, a);
+        }
+        float f = __fmaf_rn(small_int_to_float(acc[2]), 1.f / 254.f, small_int_to_float(acc[1]));
+        f = __fmaf_rn(f, 1.f / 254.f, small_int_to_float(acc[0]));
+        // d s f; a non-finite state block gives NaN
+        float s = xb[b] == 1024 ? __int_as_float(0x7fc00000) : mul_pow2(__fmul_rn(d, f), xb[b]);
 #pragma unroll
         for (int o = 1; o < 8; o <<= 1) s = __fadd_rn(s, __shfl_xor_sync(0xffffffffu, s, o));
         if (blk == 0 && v0 + row < V) y[static_cast<long long>(b) * ldy + v0 + row] = s;

@@ -14,24 +14,26 @@
 //   y[b, r] = 2^-e_b sum_j d[r, j] (D_j[r, b] + D_j[r, N + b])             (CUDA cores, f32)
 //
 // One CTA per SM (persistent over tiles t = blockIdx.x + i gridDim.x), 14 warps. A work item
-// is half a tile (4 blocks, K = 128); item i of the CTA is half i % 2 of its tile i / 2.
+// is a quarter tile (2 blocks, K = 64: one 128-byte swizzle atom); item i of the CTA is quarter
+// i % 4 of its tile i / 4.
 //  - warp 0, one lane: copies each tile's 128 rows x 272 bytes (contiguous in the table) into
 //    a shared staging ring with one bulk asynchronous copy (cp.async.bulk, mbarrier
 //    completion); warp 0 also allocates and frees the tensor memory.
 //  - warp 1, one lane: per item, per block, 2 MMAs (K = 16 each) of M = 128, N = 2 x 16..64
-//    into the block's accumulators, then one commit.
-//  - warps 2-5 and 6-9, two teams of 128 threads (thread = tile row), team T converting the
-//    items of half T into A slab T: the q bytes to float16 in the 128-byte-swizzled K-major
-//    layout, the scales d to float32 beside the slab.
+//    into the block's accumulators, then two commits: the item's A slab is free, its
+//    accumulators are ready.
+//  - warps 2-5 and 6-9, two teams of 128 threads (thread = tile row), team T converting
+//    quarters T and T + 2 of every tile into A slabs T and T + 2 (each team double-buffered):
+//    the q bytes to float16 in the 128-byte-swizzled K-major layout, the scales d to float32
+//    in a ring of 8 items.
 //  - warps 10-13, 128 threads (thread = tile row = TMEM lane; lane quarter = warp % 4): per
 //    item, read the accumulators from tensor memory (tcgen05.ld), add hi + lo, multiply by d
-//    and accumulate; after the second half write y. Their release of the item frees both its
-//    accumulator slot and its A slab (the MMAs that read the slab are complete by then).
-// Rings: 2-3 staging buffers (a tile each), 2 A slabs (32 KB), 1-4 accumulator slots in tensor
-// memory (8 N columns each). Every mbarrier wait is bounded (about a second); a wait that runs
-// out sets an abort flag that ends every role's loop, counts the event in a device counter
-// (dspark_pipeline_timeouts), lets the copies and MMAs in flight finish (again bounded) and
-// frees the tensor memory before the CTA exits.
+//    and accumulate; after the fourth quarter write y.
+// Rings: 2-3 staging buffers (a tile each), 4 A slabs (16 KB), 8 scale sets, 2-8 accumulator
+// slots in tensor memory (4 N columns each). Every mbarrier wait is bounded (about a second);
+// a wait that runs out sets an abort flag that ends every role's loop, counts the event in a
+// device counter (dspark_pipeline_timeouts), lets the copies and MMAs in flight finish (again
+// bounded) and frees the tensor memory before the CTA exits.
 #pragma once
 
 #include <cuda_fp16.h>
@@ -47,7 +49,7 @@ constexpr int kMmaThreads = 448;       // 14 warps
 constexpr int kMmaTeam = 128;          // threads of a converter team or of the epilogue
 constexpr int kQ8RowBytesT = 272;      // 8 blocks x 34 bytes
 constexpr int kMmaRawBytes = kMmaRows * kQ8RowBytesT;  // 34816, a staging buffer
-constexpr int kMmaSlabBytes = kMmaRows * 128 * 2;      // 32768: 128 rows x 128 halves
+constexpr int kMmaSlabBytes = kMmaRows * 128;          // 16384: 128 rows x 64 halves
 constexpr int kMmaTmemCols = 512;
 
 __device__ unsigned long long g_pipeline_timeouts = 0;
@@ -183,40 +185,43 @@ struct MmaQ8Smem {
   int b_off, slab_off, d_off, raw_off, bar_off, total;
 };
 
+constexpr int kMmaSlabs = 4;   // one per quarter
+constexpr int kMmaDRing = 8;   // scale sets (items) in flight
+
 __host__ __device__ constexpr int mma_raw_stages(int n) { return n <= 48 ? 3 : 2; }
-// accumulator slots in the 512 TMEM columns: 8 N columns each (4 blocks x hi, lo), at most 4
-__host__ __device__ constexpr int mma_tmem_slots(int n) { return 512 / (8 * n) < 4 ? 512 / (8 * n) : 4; }
+// accumulator slots in the 512 TMEM columns: 4 N columns each (2 blocks x hi, lo), at most 8
+__host__ __device__ constexpr int mma_tmem_slots(int n) { return 512 / (4 * n) < 8 ? 512 / (4 * n) : 8; }
 
 __host__ __device__ inline MmaQ8Smem mma_q8_smem(int n) {
   MmaQ8Smem s{};
   s.b_off = 0;                                     // 4 atoms x 2n rows x 128 B
-  s.slab_off = s.b_off + 4 * 2 * n * 128;          // 2 x 32 KB
-  s.d_off = s.slab_off + 2 * kMmaSlabBytes;        // 2 x 4 blocks x 128 rows float
-  s.raw_off = s.d_off + 2 * 4 * kMmaRows * 4;
+  s.slab_off = s.b_off + 4 * 2 * n * 128;          // 4 x 16 KB
+  s.d_off = s.slab_off + kMmaSlabs * kMmaSlabBytes;  // 8 x 2 blocks x 128 rows float
+  s.raw_off = s.d_off + kMmaDRing * 2 * kMmaRows * 4;
   s.bar_off = s.raw_off + mma_raw_stages(n) * kMmaRawBytes;
-  s.total = s.bar_off + 1024 + 1024;  // barriers, flags, exponents; slack to align the base
+  s.total = s.bar_off + 1024 + 1024;  // barriers, flags, scales; slack to align the base
   return s;
 }
 
-// Converts this thread's row of work item (tile, half HF) from the staging buffer into the A
-// slab: 4 blocks, each 2 scale bytes then 32 signed bytes. The 144 bytes that cover the half
-// are read as 9 aligned 16-byte words; pairs of q bytes (even offsets, never split across a
-// word) become float16x2 through a byte permute into 0x64 bytes (1024 + (q + 128)) and an exact
-// subtraction of 1152. The scales go to d[bl * 128 + r].
-template <int HF>
-__device__ __forceinline__ void q8_convert_row(const uint8_t* raw_row, uint8_t* slab, float* d,
-                                               int r) {
-  uint32_t w[36];
+// Converts this thread's row of quarter QQ (blocks 2 QQ and 2 QQ + 1: raw bytes [68 QQ,
+// 68 QQ + 68)) from the staging buffer into the A slab (one swizzle atom). The 80 bytes from
+// the 16-byte boundary below 68 QQ are read as 5 aligned 16-byte words; pairs of q bytes (even
+// offsets, never split across a word) become float16x2 through a byte permute into 0x64 bytes
+// (1024 + (q + 128)) and an exact subtraction of 1152. The scales go to d[bl * 128 + r].
+template <int QQ>
+__device__ __forceinline__ void q8_convert_quarter(const uint8_t* raw_row, uint8_t* slab,
+                                                   float* d, int r) {
+  constexpr int kStart = (68 * QQ) & ~15;
+  uint32_t w[20];
 #pragma unroll
-  for (int c = 0; c < 9; ++c) {
-    const uint4 v = *reinterpret_cast<const uint4*>(raw_row + 128 * HF + 16 * c);
+  for (int c = 0; c < 5; ++c) {
+    const uint4 v = *reinterpret_cast<const uint4*>(raw_row + kStart + 16 * c);
     w[4 * c] = v.x; w[4 * c + 1] = v.y; w[4 * c + 2] = v.z; w[4 * c + 3] = v.w;
   }
   const __half2 bias = __halves2half2(__ushort_as_half(0x6480), __ushort_as_half(0x6480));
 #pragma unroll
-  for (int bl = 0; bl < 4; ++bl) {
-    constexpr int kBase = 8 * HF;   // (136 HF) - (128 HF): the half's first byte in w
-    const int s = kBase + 34 * bl;  // the block's first byte (the scale), even
+  for (int bl = 0; bl < 2; ++bl) {
+    const int s = 68 * QQ - kStart + 34 * bl;  // the block's first byte (the scale), even
     d[bl * kMmaRows + r] = __half2float(__ushort_as_half(
         static_cast<unsigned short>((w[s >> 2] >> (8 * (s & 3))) & 0xffffu)));
     uint32_t h2[16];
@@ -229,12 +234,12 @@ __device__ __forceinline__ void q8_convert_row(const uint8_t* raw_row, uint8_t* 
       const __half2 v = __hsub2(*reinterpret_cast<const __half2*>(&p), bias);
       h2[j] = *reinterpret_cast<const uint32_t*>(&v);
     }
-    // block bl = K [32 bl, 32 bl + 32) of the slab: atom bl / 2, chunks 4 (bl % 2) .. + 3
-    uint8_t* atom = slab + (bl >> 1) * (kMmaRows * 128) + r * 128;
+    // block bl = K [32 bl, 32 bl + 32) of the atom: 16-byte chunks 4 bl .. 4 bl + 3
+    uint8_t* row = slab + r * 128;
 #pragma unroll
     for (int m = 0; m < 4; ++m) {
-      const int c = 4 * (bl & 1) + m;
-      *reinterpret_cast<uint4*>(atom + ((c ^ (r & 7)) << 4)) =
+      const int c = 4 * bl + m;
+      *reinterpret_cast<uint4*>(row + ((c ^ (r & 7)) << 4)) =
           make_uint4(h2[4 * m], h2[4 * m + 1], h2[4 * m + 2], h2[4 * m + 3]);
     }
   }
@@ -268,29 +273,33 @@ __global__ void __launch_bounds__(kMmaThreads, 1)
   uint64_t* bars = reinterpret_cast<uint64_t*>(sm + L.bar_off);
   uint64_t* raw_full = bars;        // [3] producer (expect_tx) + the copy's bytes
   uint64_t* raw_empty = bars + 3;   // [3] both converter teams (256)
-  uint64_t* slab_full = bars + 6;   // [2] a converter team (128)
-  uint64_t* slab_free = bars + 8;   // [2] the epilogue (128)
-  uint64_t* acc_full = bars + 10;   // [4] MMA commit
-  uint64_t* acc_empty = bars + 14;  // [4] the epilogue (128)
-  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(bars + 18);
-  volatile int* s_abort = reinterpret_cast<volatile int*>(bars + 19);
-  float* s_scale = reinterpret_cast<float*>(bars + 20);  // [2][64]: 2^-e_b as two factors
+  uint64_t* slab_full = bars + 6;   // [4] a converter team (128)
+  uint64_t* slab_free = bars + 10;  // [4] MMA commit
+  uint64_t* d_full = bars + 14;     // [8] a converter team (128)
+  uint64_t* d_free = bars + 22;     // [8] the epilogue (128)
+  uint64_t* acc_full = bars + 30;   // [8] MMA commit
+  uint64_t* acc_empty = bars + 38;  // [8] the epilogue (128)
+  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(bars + 46);
+  volatile int* s_abort = reinterpret_cast<volatile int*>(bars + 47);
+  float* s_scale = reinterpret_cast<float*>(bars + 48);  // [2][64]: 2^-e_b as two factors
 
   const int tid = threadIdx.x, wi = tid >> 5, lane = tid & 31;
   const int n_tiles = (V + kMmaRows - 1) / kMmaRows;
   const int my_tiles = blockIdx.x < n_tiles ? (n_tiles - 1 - blockIdx.x) / gridDim.x + 1 : 0;
-  const int n_items = 2 * my_tiles;
+  const int n_items = 4 * my_tiles;
 
   if (tid == 0) {
     for (int i = 0; i < 3; ++i) {
       mbar_init(smem_u32(&raw_full[i]), 1);
       mbar_init(smem_u32(&raw_empty[i]), 2 * kMmaTeam);
     }
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < kMmaSlabs; ++i) {
       mbar_init(smem_u32(&slab_full[i]), kMmaTeam);
-      mbar_init(smem_u32(&slab_free[i]), kMmaTeam);
+      mbar_init(smem_u32(&slab_free[i]), 1);
     }
-    for (int i = 0; i < 4; ++i) {
+    for (int i = 0; i < 8; ++i) {
+      mbar_init(smem_u32(&d_full[i]), kMmaTeam);
+      mbar_init(smem_u32(&d_free[i]), kMmaTeam);
       mbar_init(smem_u32(&acc_full[i]), 1);
       mbar_init(smem_u32(&acc_empty[i]), kMmaTeam);
     }
@@ -394,23 +403,23 @@ __global__ void __launch_bounds__(kMmaThreads, 1)
         const uint32_t b0 = smem_u32(s_b);
         int issued = 0;
         for (int i = 0; i < n_items; ++i) {
-          const int sl = i & 1, ts = i % kSlots;
-          if (!mbar_wait(smem_u32(&slab_full[sl]), (i >> 1) & 1, s_abort)) break;
+          const int qq = i & 3, ts = i % kSlots;
+          if (!mbar_wait(smem_u32(&slab_full[qq]), (i >> 2) & 1, s_abort)) break;
           if (!mbar_wait(smem_u32(&acc_empty[ts]), ((i / kSlots) & 1) ^ 1, s_abort)) break;
           tc_fence_after();
-          const uint32_t a0 = smem_u32(s_slab + sl * kMmaSlabBytes);
+          const uint32_t a0 = smem_u32(s_slab + qq * kMmaSlabBytes);
 #pragma unroll
-          for (int bl = 0; bl < 4; ++bl) {
-            const uint32_t d_tmem = tbase + ts * (8 * N) + bl * (2 * N);
+          for (int bl = 0; bl < 2; ++bl) {
+            const uint32_t d_tmem = tbase + ts * (4 * N) + bl * (2 * N);
 #pragma unroll
             for (int w = 0; w < 2; ++w) {
-              const uint32_t in_atom = 64 * (bl & 1) + 32 * w;  // bytes into the 128-byte row
-              const uint64_t ad = sw128_desc(a0 + (bl >> 1) * (kMmaRows * 128) + in_atom);
-              const uint32_t katom = 2 * sl + (bl >> 1);
-              const uint64_t bd = sw128_desc(b0 + katom * (2 * N * 128) + in_atom);
+              const uint32_t in_atom = 64 * bl + 32 * w;  // bytes into the 128-byte row
+              const uint64_t ad = sw128_desc(a0 + in_atom);
+              const uint64_t bd = sw128_desc(b0 + qq * (2 * N * 128) + in_atom);
               mma_f16(d_tmem, ad, bd, idesc, w != 0);
             }
           }
+          mma_commit(smem_u32(&slab_free[qq]));
           mma_commit(smem_u32(&acc_full[ts]));
           issued = i + 1;
         }
@@ -424,24 +433,38 @@ __global__ void __launch_bounds__(kMmaThreads, 1)
         }
       }
     } else if (wi < 10) {
-      // ---- converter team T = half T of every tile
+      // ---- converter team T: quarters T and T + 2 of every tile
       const int T = wi >= 6;
       const int r = 32 * ((wi - 2) & 3) + lane;  // tile row
-      uint8_t* slab = s_slab + T * kMmaSlabBytes;
-      float* d = s_d + T * 4 * kMmaRows;
-      for (int j = 0; j < my_tiles; ++j) {
+      bool live = true;
+      for (int j = 0; j < my_tiles && live; ++j) {
         const int st = j % kRaw;
-        bool ok = mbar_wait(smem_u32(&raw_full[st]), (j / kRaw) & 1, s_abort);
-        ok = ok && mbar_wait(smem_u32(&slab_free[T]), (j & 1) ^ 1, s_abort);
-        if (!__all_sync(0xffffffffu, ok)) break;
         const uint8_t* raw_row = s_raw + st * kMmaRawBytes + r * kQ8RowBytesT;
-        if (T == 0)
-          q8_convert_row<0>(raw_row, slab, d, r);
-        else
-          q8_convert_row<1>(raw_row, slab, d, r);
-        fence_proxy_async_smem();
-        mbar_arrive(smem_u32(&slab_full[T]));
-        mbar_arrive(smem_u32(&raw_empty[st]));
+#pragma unroll
+        for (int h2 = 0; h2 < 2; ++h2) {
+          const int qq = T + 2 * h2, i = 4 * j + qq, di = i % kMmaDRing;
+          bool ok = h2 == 1 || mbar_wait(smem_u32(&raw_full[st]), (j / kRaw) & 1, s_abort);
+          ok = ok && mbar_wait(smem_u32(&slab_free[qq]), (j & 1) ^ 1, s_abort);
+          ok = ok && mbar_wait(smem_u32(&d_free[di]), ((i / kMmaDRing) & 1) ^ 1, s_abort);
+          if (!__all_sync(0xffffffffu, ok)) {
+            live = false;
+            break;
+          }
+          uint8_t* slab = s_slab + qq * kMmaSlabBytes;
+          float* d = s_d + di * 2 * kMmaRows;
+          if (qq == 0)
+            q8_convert_quarter<0>(raw_row, slab, d, r);
+          else if (qq == 1)
+            q8_convert_quarter<1>(raw_row, slab, d, r);
+          else if (qq == 2)
+            q8_convert_quarter<2>(raw_row, slab, d, r);
+          else
+            q8_convert_quarter<3>(raw_row, slab, d, r);
+          fence_proxy_async_smem();
+          mbar_arrive(smem_u32(&slab_full[qq]));
+          mbar_arrive(smem_u32(&d_full[di]));
+        }
+        if (live) mbar_arrive(smem_u32(&raw_empty[st]));
       }
     } else {
       // ---- epilogue: thread = tile row = TMEM lane
@@ -452,21 +475,19 @@ __global__ void __launch_bounds__(kMmaThreads, 1)
         float acc[N];
 #pragma unroll
         for (int c = 0; c < N; ++c) acc[c] = 0.f;
-        for (int sl = 0; sl < 2; ++sl) {
-          const int i = 2 * j + sl, ts = i % kSlots;
-          // (the wait on slab_full, long complete, orders the team's scale writes before the
-          // reads below)
+        for (int qq = 0; qq < 4; ++qq) {
+          const int i = 4 * j + qq, ts = i % kSlots, di = i % kMmaDRing;
           bool ok = mbar_wait(smem_u32(&acc_full[ts]), (i / kSlots) & 1, s_abort);
-          ok = ok && mbar_wait(smem_u32(&slab_full[sl]), j & 1, s_abort);
+          ok = ok && mbar_wait(smem_u32(&d_full[di]), (i / kMmaDRing) & 1, s_abort);
           if (!__all_sync(0xffffffffu, ok)) {
             live = false;
             break;
           }
           tc_fence_after();
-          const uint32_t ta = tbase + (static_cast<uint32_t>(32 * q) << 16) + ts * (8 * N);
-          const float* d = s_d + sl * 4 * kMmaRows;
+          const uint32_t ta = tbase + (static_cast<uint32_t>(32 * q) << 16) + ts * (4 * N);
+          const float* d = s_d + di * 2 * kMmaRows;
 #pragma unroll
-          for (int bl = 0; bl < 4; ++bl) {
+          for (int bl = 0; bl < 2; ++bl) {
             const float dv = d[bl * kMmaRows + r];
             // (columns in chunks of 16, or 8 at N >= 48 to stay within the registers)
             constexpr int kC = N >= 48 ? 8 : 16;
@@ -488,7 +509,7 @@ __global__ void __launch_bounds__(kMmaThreads, 1)
           }
           tc_fence_before();
           mbar_arrive(smem_u32(&acc_empty[ts]));
-          mbar_arrive(smem_u32(&slab_free[sl]));
+          mbar_arrive(smem_u32(&d_free[di]));
         }
         if (!live) break;
         const long long t = blockIdx.x + static_cast<long long>(j) * gridDim.x;
