@@ -243,7 +243,11 @@ dspark_status_t dspark_early_exit_accept(const void* p1, int64_t ld_p1, const vo
  *  R      the Markov rank: 256 (other ranks: DSPARK_ERR_UNSUPPORTED).
  *  h      device [B, R] float32 states, 16-byte aligned.
  *  y      device [B, V] float32 results (row b at y + b * V).
- *  F16: float32 sums in a fixed order on the CUDA cores, the table read once per 4 states.
+ *  F16, B == 1: float32 sums in a fixed order on the CUDA cores.
+ *  F16, B > 1: on the tensor cores (tcgen05), the table read once per 64 states (loaded by
+ *    TMA tensor copies): each state scaled by a power of two and split into float16 hi + lo
+ *    (within 2^-23 of its largest |h|); the products with the exact table halves are summed
+ *    in float32 by the tensor cores, one sum per part over all R values.
  *  Q8_0, B <= 4: on the CUDA cores, one read of the table: exact integer dot products of each
  *    block's bytes with three signed-byte digit planes of the state (within 2^-22 of the
  *    block's largest |h|), combined and scaled by d in float32.

@@ -532,6 +532,70 @@ dspark_status_t markov_mma_launch(const void* table, int V, const float* h, int 
   return e == cudaSuccess ? DSPARK_OK : DSPARK_ERR_CUDA;
 }
 
+// cuTensorMapEncodeTiled from the driver, looked up once through the runtime (the library
+// links no driver library of its own).
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn tensor_map_encoder() {
+  static EncodeTiledFn fn = nullptr;
+  static bool looked = false;
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (!looked) {
+    looked = true;
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+// Batches of up to this many states take the CUDA-core F16 kernel; larger ones the
+// tensor-core kernel, 64 states per launch.
+constexpr int kMarkovF16CudaCoreStates = 1;
+
+// The F16 mat-vec on the tensor cores for nb <= N states: a tensor map over the V x 256 table
+// (boxes of 128 rows x 64 halves, 128-byte swizzle, rows past V read as zeros).
+template <int N>
+dspark_status_t markov_f16_mma_launch(const void* table, int V, const float* h, int nb, float* y,
+                                      int ldy, cudaStream_t stream) {
+  const EncodeTiledFn enc = tensor_map_encoder();
+  if (!enc) return DSPARK_ERR_UNSUPPORTED;
+  alignas(64) CUtensorMap map;
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(kMarkovRank), static_cast<cuuint64_t>(V)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(kMarkovRank) * 2};
+  const cuuint32_t box[2] = {64, kMmaRows};
+  const cuuint32_t es[2] = {1, 1};
+  if (enc(&map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void*>(table), dims, strides, box,
+          es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return DSPARK_ERR_UNSUPPORTED;
+  const void* fn = reinterpret_cast<const void*>(&markov_f16_mma_kernel<N>);
+  const size_t smem = static_cast<size_t>(f16_mma_smem(N));
+  cudaError_t e = cudaSuccess;
+  const int ctas = resident_ctas(fn, kF16MmaThreads, smem, &e);
+  if (e != cudaSuccess) return DSPARK_ERR_CUDA;
+  if (ctas < 1) return DSPARK_ERR_UNSUPPORTED;
+  const int n_tiles = (V + kMmaRows - 1) / kMmaRows;
+  const int grid = n_tiles < ctas ? n_tiles : ctas;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(grid), 1, 1);
+  cfg.blockDim = dim3(kF16MmaThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, markov_f16_mma_kernel<N>, map, V, h, nb, y, ldy);
+  return e == cudaSuccess ? DSPARK_OK : DSPARK_ERR_CUDA;
+}
+
 }  // namespace
 }  // namespace dspark
 
@@ -769,6 +833,24 @@ dspark_status_t dspark_markov_matvec(const void* table, dspark_table_t type, int
         st = markov_mma_launch<48>(table, V, hb, nb, yb, V, s);
       else
         st = markov_mma_launch<64>(table, V, hb, nb, yb, V, s);
+      if (st != DSPARK_OK) return st;
+    }
+    return DSPARK_OK;
+  }
+  if (type == DSPARK_TABLE_F16 && B > kMarkovF16CudaCoreStates) {
+    for (int b0 = 0; b0 < B; b0 += kMmaMaxStates) {
+      const int nb = B - b0 < kMmaMaxStates ? B - b0 : kMmaMaxStates;
+      const float* hb = h + static_cast<size_t>(b0) * R;
+      float* yb = y + static_cast<size_t>(b0) * V;
+      dspark_status_t st;
+      if (nb <= 16)
+        st = markov_f16_mma_launch<16>(table, V, hb, nb, yb, V, s);
+      else if (nb <= 32)
+        st = markov_f16_mma_launch<32>(table, V, hb, nb, yb, V, s);
+      else if (nb <= 48)
+        st = markov_f16_mma_launch<48>(table, V, hb, nb, yb, V, s);
+      else
+        st = markov_f16_mma_launch<64>(table, V, hb, nb, yb, V, s);
       if (st != DSPARK_OK) return st;
     }
     return DSPARK_OK;

@@ -36,6 +36,7 @@
 // bounded) and frees the tensor memory before the CTA exits.
 #pragma once
 
+#include <cuda.h>  // CUtensorMap (the type only; no driver calls here)
 #include <cuda_fp16.h>
 
 #include "common.cuh"
@@ -255,13 +256,66 @@ __device__ __forceinline__ int ilog2f(float m) {
   return be != 0 ? be - 127 : -149 + (31 - __clz(static_cast<int>(u & 0x7fffffu)));
 }
 
+// The B operand of the Markov MMAs, built by warps w0 .. w0 + NW - 1 of the CTA: state b
+// (rows nb..N-1 zero) scaled by 2^e_b (m_b 2^e_b in [2^14, 2^15)) and split into float16 hi
+// (B row b) and lo (B row N + b), 128-byte-swizzled K-major: atom k / 64, row n, 16-byte chunk
+// (k % 64) / 8 stored at chunk ((k % 64) / 8) ^ (n % 8), element k % 8. s_scale[b] and
+// s_scale[64 + b] receive 2^-e_b as two exact factors. Ends with the proxy fence that makes the
+// writes visible to the tensor cores (the caller synchronises the builders afterwards).
+template <int N, int NW>
+__device__ __forceinline__ void build_b_operand(const float* h, int nb, uint8_t* s_b,
+                                                float* s_scale, int w, int lane) {
+  constexpr int kPer = (N + NW - 1) / NW;
+  float hv[kPer][8];
+#pragma unroll
+  for (int u = 0; u < kPer; ++u) {
+    const int b = w + NW * u;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) hv[u][j] = b < nb ? __ldg(h + b * kMarkovRank + lane + 32 * j) : 0.f;
+  }
+#pragma unroll
+  for (int u = 0; u < kPer; ++u) {
+    const int b = w + NW * u;
+    if (b >= N) break;
+    float m = 0.f;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) m = max_nan(m, fabsf(hv[u][j]));  // NaN anywhere: m NaN
+    m = warp_max_nan(m);
+    int e = 0;
+    if (m > 0.f && m <= 3.402823466e38f) e = 14 - ilog2f(m);  // m 2^e in [2^14, 2^15)
+    // 2^e in two exact factors (e in [-114, 163]); 2^-e likewise
+    const int e1 = e > 127 ? 127 : e, e2 = e - e1;
+    const float f1 = pow2f(e1), f2 = pow2f(e2);
+    if (lane == 0) {
+      const int g1 = -e < -126 ? -126 : -e;
+      s_scale[b] = pow2f(g1);
+      s_scale[64 + b] = pow2f(-e - g1);
+    }
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int k = lane + 32 * j;
+      const float x = __fmul_rn(__fmul_rn(hv[u][j], f1), f2);
+      const __half hi = __float2half_rn(x);
+      // (a non-finite x keeps lo = 0: its products are those of x itself)
+      const __half lo =
+          is_finite(x) ? __float2half_rn(__fsub_rn(x, __half2float(hi))) : __float2half_rn(0.f);
+      const int off_hi = (k >> 6) * (2 * N * 128) + b * 128 +
+                         ((((k & 63) >> 3) ^ (b & 7)) << 4) + (k & 7) * 2;
+      const int off_lo = (k >> 6) * (2 * N * 128) + (N + b) * 128 +
+                         ((((k & 63) >> 3) ^ ((N + b) & 7)) << 4) + (k & 7) * 2;
+      *reinterpret_cast<__half*>(s_b + off_hi) = hi;
+      *reinterpret_cast<__half*>(s_b + off_lo) = lo;
+    }
+  }
+  fence_proxy_async_smem();
+}
+
 template <int N>
 __global__ void __launch_bounds__(kMmaThreads, 1)
     markov_q8_0_mma_kernel(const uint8_t* __restrict__ W, int V, const float* h, int nb,
                            float* y, int ldy) {
   constexpr int kRaw = mma_raw_stages(N);
   constexpr int kSlots = mma_tmem_slots(N);
-  constexpr int kStatesPerWarp = (N + 12) / 13;  // the split is done by warps 1-13
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                            ~static_cast<uintptr_t>(1023));
@@ -345,53 +399,8 @@ __global__ void __launch_bounds__(kMmaThreads, 1)
       }
     }
   } else {
-    // ---- warps 1-13: the B operand. State b (rows nb..N-1 zero) scaled by 2^e_b and split
-    // into float16 hi (B row b) and lo (B row N + b), 128-byte-swizzled K-major: atom k / 64,
-    // row n, 16-byte chunk (k % 64) / 8 stored at chunk ((k % 64) / 8) ^ (n % 8), element k % 8.
-    const int w1 = wi - 1;
-    float hv[kStatesPerWarp][8];
-#pragma unroll
-    for (int u = 0; u < kStatesPerWarp; ++u) {
-      const int b = w1 + 13 * u;
-#pragma unroll
-      for (int j = 0; j < 8; ++j)
-        hv[u][j] = b < nb ? __ldg(h + b * kMarkovRank + lane + 32 * j) : 0.f;
-    }
-#pragma unroll
-    for (int u = 0; u < kStatesPerWarp; ++u) {
-      const int b = w1 + 13 * u;
-      if (b >= N) break;
-      float m = 0.f;
-#pragma unroll
-      for (int j = 0; j < 8; ++j) m = max_nan(m, fabsf(hv[u][j]));  // NaN anywhere: m NaN
-      m = warp_max_nan(m);
-      int e = 0;
-      if (m > 0.f && m <= 3.402823466e38f) e = 14 - ilog2f(m);  // m 2^e in [2^14, 2^15)
-      // 2^e in two exact factors (e in [-114, 163]); 2^-e likewise
-      const int e1 = e > 127 ? 127 : e, e2 = e - e1;
-      const float f1 = pow2f(e1), f2 = pow2f(e2);
-      if (lane == 0) {
-        const int g1 = -e < -126 ? -126 : -e;
-        s_scale[b] = pow2f(g1);
-        s_scale[64 + b] = pow2f(-e - g1);
-      }
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const int k = lane + 32 * j;
-        const float x = __fmul_rn(__fmul_rn(hv[u][j], f1), f2);
-        const __half hi = __float2half_rn(x);
-        // (a non-finite x keeps lo = 0: its products are those of x itself)
-        const __half lo =
-            is_finite(x) ? __float2half_rn(__fsub_rn(x, __half2float(hi))) : __float2half_rn(0.f);
-        const int off_hi = (k >> 6) * (2 * N * 128) + b * 128 +
-                           ((((k & 63) >> 3) ^ (b & 7)) << 4) + (k & 7) * 2;
-        const int off_lo = (k >> 6) * (2 * N * 128) + (N + b) * 128 +
-                           ((((k & 63) >> 3) ^ ((N + b) & 7)) << 4) + (k & 7) * 2;
-        *reinterpret_cast<__half*>(s_b + off_hi) = hi;
-        *reinterpret_cast<__half*>(s_b + off_lo) = lo;
-      }
-    }
-    fence_proxy_async_smem();
+    // ---- warps 1-13: the B operand
+    build_b_operand<N, 13>(h, nb, s_b, s_scale, wi - 1, lane);
     asm volatile("bar.sync 1, %0;" ::"n"(kMmaThreads - 32) : "memory");  // warps 1-13
     const uint32_t tbase = *s_tmem;
     tc_fence_after();
@@ -521,6 +530,189 @@ __global__ void __launch_bounds__(kMmaThreads, 1)
               y[static_cast<long long>(c) * ldy + row] =
                   __fmul_rn(__fmul_rn(acc[c], s_scale[c]), s_scale[64 + c]);
         }
+      }
+    }
+  }
+
+  __syncthreads();
+  if (wi == 0) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(*s_tmem),
+                 "r"(kMmaTmemCols)
+                 : "memory");
+  }
+}
+
+// ---------------------------------------------------------------- the F16 table
+
+// The same mat-vec over an F16 table (V x 256 halves, row-major): one float32 accumulator per
+// (row, hi/lo part, state) over all 256 k, so no per-block scale and no conversion. The tensor
+// memory accelerator (TMA) loads each quarter tile (128 rows x 64 halves) straight into a
+// 128-byte-swizzled A stage, 8 stages (128 KB) in flight. One CTA per SM, 6 warps: warp 0 one
+// lane issues the TMA loads, warp 1 one lane the MMAs (4 K-steps per quarter, 16 per tile,
+// N = 2 x 16..64, into the tile's accumulator slot; a commit frees each stage, another marks
+// the tile's accumulators ready), warps 2-5 read the accumulators (thread = row = TMEM lane)
+// and write y = (D_hi + D_lo) 2^-e_b; warps 1-5 build the B operand first.
+//   y[b, r] = 2^-e_b (sum_k W[r, k] hi[b, k] + sum_k W[r, k] lo[b, k])
+// Every product is exact in float32; the tensor cores sum them in float32.
+constexpr int kF16MmaThreads = 192;
+constexpr int kF16Stages = 8;                    // A stages of 16 KB
+constexpr int kF16StageBytes = kMmaRows * 128;   // 128 rows x 64 halves
+
+__host__ __device__ constexpr int f16_tmem_slots(int n) { return 512 / (2 * n) < 4 ? 512 / (2 * n) : 4; }
+__host__ __device__ constexpr int f16_mma_smem(int n) {
+  return 4 * 2 * n * 128 + kF16Stages * kF16StageBytes + 1024 + 1024;
+}
+
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int x, int y,
+                                            uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes "
+      "[%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
+      : "memory");
+}
+
+template <int N>
+__global__ void __launch_bounds__(kF16MmaThreads, 1)
+    markov_f16_mma_kernel(const __grid_constant__ CUtensorMap tmap, int V, const float* h, int nb,
+                          float* y, int ldy) {
+  constexpr int kSlots = f16_tmem_slots(N);
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                           ~static_cast<uintptr_t>(1023));
+  uint8_t* s_b = sm;                                  // 4 atoms x 2N rows x 128 B
+  uint8_t* s_a = sm + 4 * 2 * N * 128;                // kF16Stages x 16 KB
+  uint64_t* bars = reinterpret_cast<uint64_t*>(s_a + kF16Stages * kF16StageBytes);
+  uint64_t* a_full = bars;                            // [8] TMA (expect_tx) + bytes
+  uint64_t* a_free = bars + 8;                        // [8] MMA commit
+  uint64_t* acc_full = bars + 16;                     // [4] MMA commit
+  uint64_t* acc_empty = bars + 20;                    // [4] the epilogue (128)
+  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(bars + 24);
+  volatile int* s_abort = reinterpret_cast<volatile int*>(bars + 25);
+  float* s_scale = reinterpret_cast<float*>(bars + 26);  // [2][64]
+
+  const int tid = threadIdx.x, wi = tid >> 5, lane = tid & 31;
+  const int n_tiles = (V + kMmaRows - 1) / kMmaRows;
+  const int my_tiles = blockIdx.x < n_tiles ? (n_tiles - 1 - blockIdx.x) / gridDim.x + 1 : 0;
+
+  if (tid == 0) {
+    for (int i = 0; i < kF16Stages; ++i) {
+      mbar_init(smem_u32(&a_full[i]), 1);
+      mbar_init(smem_u32(&a_free[i]), 1);
+    }
+    for (int i = 0; i < 4; ++i) {
+      mbar_init(smem_u32(&acc_full[i]), 1);
+      mbar_init(smem_u32(&acc_empty[i]), kMmaTeam);
+    }
+    *s_abort = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap)) : "memory");
+  }
+  if (wi == 0) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(s_tmem)),
+                 "r"(kMmaTmemCols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    tc_fence_before();
+  }
+  __syncthreads();
+
+  grid_dependency_wait();  // h comes from the kernel before (programmatic launch)
+  grid_dependents_launch();
+
+  if (wi == 0) {
+    // ---- producer: one TMA load per quarter tile
+    if (lane == 0) {
+      const int n_items = 4 * my_tiles;
+      int armed = 0;
+      for (int i = 0; i < n_items; ++i) {
+        const int st = i % kF16Stages;
+        if (!mbar_wait(smem_u32(&a_free[st]), ((i / kF16Stages) & 1) ^ 1, s_abort)) break;
+        const int t = blockIdx.x + (i >> 2) * gridDim.x;
+        mbar_arrive_tx(smem_u32(&a_full[st]), kF16StageBytes);
+        tma_load_2d(smem_u32(s_a + st * kF16StageBytes), &tmap, 64 * (i & 3), t * kMmaRows,
+                    smem_u32(&a_full[st]));
+        armed = i + 1;
+      }
+      if (*s_abort) {
+        for (int i = armed - kF16Stages < 0 ? 0 : armed - kF16Stages; i < armed; ++i) {
+          const uint32_t bar = smem_u32(&a_full[i % kF16Stages]);
+          const long long t0 = clock64();
+          while (!mbar_try(bar, (i / kF16Stages) & 1) && clock64() - t0 < (1ll << 31)) {
+          }
+        }
+      }
+    }
+  } else {
+    build_b_operand<N, 5>(h, nb, s_b, s_scale, wi - 1, lane);
+    asm volatile("bar.sync 1, %0;" ::"n"(kF16MmaThreads - 32) : "memory");  // warps 1-5
+    const uint32_t tbase = *s_tmem;
+    tc_fence_after();
+    if (wi == 1) {
+      // ---- MMA issuer
+      if (lane == 0) {
+        constexpr uint32_t idesc = mma_idesc_f16(2 * N);
+        const uint32_t b0 = smem_u32(s_b);
+        int last = -1;
+        bool live = true;
+        for (int j = 0; j < my_tiles && live; ++j) {
+          const int ts = j % kSlots;
+          if (!mbar_wait(smem_u32(&acc_empty[ts]), ((j / kSlots) & 1) ^ 1, s_abort)) break;
+          for (int qq = 0; qq < 4; ++qq) {
+            const int i = 4 * j + qq, st = i % kF16Stages;
+            if (!mbar_wait(smem_u32(&a_full[st]), (i / kF16Stages) & 1, s_abort)) {
+              live = false;
+              break;
+            }
+            tc_fence_after();
+            const uint32_t a0 = smem_u32(s_a + st * kF16StageBytes);
+#pragma unroll
+            for (int w = 0; w < 4; ++w)
+              mma_f16(tbase + ts * (2 * N), sw128_desc(a0 + 32 * w),
+                      sw128_desc(b0 + qq * (2 * N * 128) + 32 * w), idesc, (qq | w) != 0);
+            mma_commit(smem_u32(&a_free[st]));
+          }
+          if (!live) break;
+          mma_commit(smem_u32(&acc_full[ts]));
+          last = j;
+        }
+        if (*s_abort && last >= 0) {
+          const uint32_t bar = smem_u32(&acc_full[last % kSlots]);
+          const long long t0 = clock64();
+          while (!mbar_try(bar, (last / kSlots) & 1) && clock64() - t0 < (1ll << 31)) {
+          }
+        }
+      }
+    } else {
+      // ---- epilogue: thread = tile row = TMEM lane
+      const int q = wi & 3;
+      const int r = 32 * q + lane;
+      for (int j = 0; j < my_tiles; ++j) {
+        const int ts = j % kSlots;
+        if (!__all_sync(0xffffffffu,
+                        mbar_wait(smem_u32(&acc_full[ts]), (j / kSlots) & 1, s_abort)))
+          break;
+        tc_fence_after();
+        const uint32_t ta = tbase + (static_cast<uint32_t>(32 * q) << 16) + ts * (2 * N);
+        const long long row = static_cast<long long>(blockIdx.x + j * gridDim.x) * kMmaRows + r;
+#pragma unroll
+        for (int c = 0; c < N; c += 16) {
+          float vh[16], vl[16];
+          tmem_ld16(ta + c, vh);
+          tmem_ld16(ta + N + c, vl);
+          tmem_ld_wait();
+          if (row < V) {
+#pragma unroll
+            for (int k = 0; k < 16; ++k)
+              if (c + k < nb)
+                y[static_cast<long long>(c + k) * ldy + row] = __fmul_rn(
+                    __fmul_rn(__fadd_rn(vh[k], vl[k]), s_scale[c + k]), s_scale[64 + c + k]);
+          }
+        }
+        tc_fence_before();
+        mbar_arrive(smem_u32(&acc_empty[ts]));
       }
     }
   }

@@ -7,7 +7,9 @@ by a power of two, is split into float16 hi + lo within 2^-23 of its largest |h|
 64 products q * part are exact and summed in float32 (at most a few roundings of 2^-24 per
 MMA step of 16 products), then scaled by d and the 8 blocks added by float32 FMAs. The same
 2 R 2^-24 sum |W h| covers the sums; the tests add 2^-22 max_k |h[b, k]| sum_k |W[v, k]| for
-the split. One to four Q8_0 states take the CUDA-core kernel: exact integer dot products with
+the split. F16 with two or more states runs on the tensor cores the same way (products of the
+exact table halves with the two parts, one float32 accumulator per part over all 256 k) and
+gets the same added term. One to four Q8_0 states take the CUDA-core kernel: exact integer dot products with
 three signed-byte digit planes of the state, which represent it within 2^-22 of each block's
 largest |h| (so within the same added term), then a few float32 roundings per block.
 """
@@ -35,10 +37,9 @@ def _check(V, B, fmt, seed=4):
     W = mk.f16_table(raw) if fmt == "f16" else mk.q8_0_table(raw, R)
     ref = mk.markov_matvec(W, H)
     bound = 2 * R * 2.0 ** -24 * mk.abs_products(W, H) + 1e-30
-    if fmt == "q8_0":
-        hmax = np.abs(H.astype(np.float64)).max(axis=1)                  # [B]
-        wsum = np.abs(W).sum(axis=1)                                      # [V]
-        bound = bound + 2.0 ** -22 * hmax[:, None] * wsum[None, :]
+    hmax = np.abs(H.astype(np.float64)).max(axis=1)                      # [B]
+    wsum = np.abs(W).sum(axis=1)                                          # [V]
+    bound = bound + 2.0 ** -22 * hmax[:, None] * wsum[None, :]
     err = np.abs(y.cpu().numpy().astype(np.float64) - ref)
     assert np.all(err <= bound), (fmt, V, B, float((err / bound).max()))
     assert bd.pipeline_timeouts() == 0
@@ -50,10 +51,11 @@ def test_serving_vocab(fmt, B):
     _check(129280, B, fmt)
 
 
+@pytest.mark.parametrize("fmt", ["f16", "q8_0"])
 @pytest.mark.parametrize("B", [5, 16, 17, 48, 64, 65, 130])
-def test_q8_0_many_states(B):
+def test_many_states(fmt, B):
     """One read of the table per 64 states on the tensor cores (N = 16, 32, 48, 64 and splits)."""
-    _check(129280, B, "q8_0", seed=7)
+    _check(129280, B, fmt, seed=7)
 
 
 @pytest.mark.parametrize("fmt", ["f16", "q8_0"])
@@ -62,10 +64,11 @@ def test_ragged_vocab(fmt, V):
     _check(V, 2, fmt, seed=5)
 
 
+@pytest.mark.parametrize("fmt", ["f16", "q8_0"])
 @pytest.mark.parametrize("V", [1, 127, 128, 129, 1000, 18943, 262144])
-def test_ragged_vocab_tensor_cores(V):
+def test_ragged_vocab_tensor_cores(fmt, V):
     """Partial last tiles and grids smaller than the SM count on the tensor-core path."""
-    _check(V, 6, "q8_0", seed=9)
+    _check(V, 6, fmt, seed=9)
 
 
 def test_one_hot_state_reads_a_column():
@@ -80,11 +83,12 @@ def test_one_hot_state_reads_a_column():
 
 
 
-def test_q8_0_state_scales():
+@pytest.mark.parametrize("fmt", ["f16", "q8_0"])
+def test_state_scales(fmt):
     """States of very different magnitudes (each is scaled by its own power of two), a zero
     state and one with a single nonzero entry, in one launch."""
     V = 5000
-    raw = wl.markov_table(V, R, "q8_0", seed=8)
+    raw = wl.markov_table(V, R, fmt, seed=8)
     H = wl.markov_states(6, R, seed=8).astype(np.float64)
     H[0] *= 1e-30
     H[1] *= 1e20
@@ -93,9 +97,10 @@ def test_q8_0_state_scales():
     H[3, 200] = -3.0
     H[4] *= 2.0 ** -140  # subnormal float32 states
     H = H.astype(np.float32)
-    y = bd.markov_matvec(torch.from_numpy(raw).to(DEV), "q8_0", torch.from_numpy(H).to(DEV))
+    t = torch.from_numpy(raw.view(np.int16) if fmt == "f16" else raw).to(DEV)
+    y = bd.markov_matvec(t, fmt, torch.from_numpy(H).to(DEV))
     torch.cuda.synchronize()
-    W = mk.q8_0_table(raw, R)
+    W = mk.f16_table(raw) if fmt == "f16" else mk.q8_0_table(raw, R)
     ref = mk.markov_matvec(W, H)
     bound = 2 * R * 2.0 ** -24 * mk.abs_products(W, H) + \
         2.0 ** -22 * np.abs(H.astype(np.float64)).max(axis=1)[:, None] * np.abs(W).sum(axis=1)[None, :]
