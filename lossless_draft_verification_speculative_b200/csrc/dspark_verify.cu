@@ -500,9 +500,11 @@ dspark_status_t markov_launch(const void* table, dspark_table_t type, int V, con
   return e == cudaSuccess ? DSPARK_OK : DSPARK_ERR_CUDA;
 }
 
-// Batches of up to this many states take the CUDA-core Q8_0 kernel (one launch; faster there);
-// larger ones the tensor-core kernel, 64 states per launch.
-constexpr int kMarkovCudaCoreStates = 4;
+// Q8_0 routing by the number of states (measured on a 129280-row table): one state on the
+// CUDA-core kernel (8.0 us; the integer tensor-core kernel takes 10.8), 2 to kI8MaxStates on the
+// integer tensor cores (four states: 11.3 us against 15.3 on the CUDA cores), more on the
+// float16 tensor-core kernel, 64 states per launch.
+constexpr int kMarkovCudaCoreStates = 1;
 
 // The Q8_0 mat-vec on the tensor cores for nb <= N states (N = 16, 32, 48 or 64): one CTA per
 // SM over the 128-row tiles.
@@ -593,6 +595,45 @@ dspark_status_t markov_f16_mma_launch(const void* table, int V, const float* h, 
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   e = cudaLaunchKernelEx(&cfg, markov_f16_mma_kernel<N>, map, V, h, nb, y, ldy);
+  return e == cudaSuccess ? DSPARK_OK : DSPARK_ERR_CUDA;
+}
+
+// The Q8_0 mat-vec on the integer tensor cores for NB <= 5 states: a tensor map over the
+// V x 272-byte table (boxes of 128 rows x 128 bytes, 128-byte swizzle, bytes past the row and
+// rows past V read as zeros).
+template <int NB>
+dspark_status_t markov_i8_launch(const void* table, int V, const float* h, float* y, int ldy,
+                                 cudaStream_t stream) {
+  const EncodeTiledFn enc = tensor_map_encoder();
+  if (!enc) return DSPARK_ERR_UNSUPPORTED;
+  alignas(64) CUtensorMap map;
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(kQ8RowBytes), static_cast<cuuint64_t>(V)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(kQ8RowBytes)};
+  const cuuint32_t box[2] = {128, kMmaRows};
+  const cuuint32_t es[2] = {1, 1};
+  if (enc(&map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(table), dims, strides, box,
+          es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return DSPARK_ERR_UNSUPPORTED;
+  const void* fn = reinterpret_cast<const void*>(&markov_q8_0_i8_kernel<NB>);
+  const size_t smem = static_cast<size_t>(i8_mma_smem());
+  cudaError_t e = cudaSuccess;
+  const int ctas = resident_ctas(fn, kI8Threads, smem, &e);
+  if (e != cudaSuccess) return DSPARK_ERR_CUDA;
+  if (ctas < 1) return DSPARK_ERR_UNSUPPORTED;
+  const int n_tiles = (V + kMmaRows - 1) / kMmaRows;
+  const int grid = n_tiles < ctas ? n_tiles : ctas;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(grid), 1, 1);
+  cfg.blockDim = dim3(kI8Threads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, markov_q8_0_i8_kernel<NB>, map, V, h, y, ldy);
   return e == cudaSuccess ? DSPARK_OK : DSPARK_ERR_CUDA;
 }
 
@@ -819,6 +860,15 @@ dspark_status_t dspark_markov_matvec(const void* table, dspark_table_t type, int
   if (R != kMarkovRank) return DSPARK_ERR_UNSUPPORTED;
   if (!aligned(table, 16) || !aligned(h, 16) || !aligned(y, 4)) return DSPARK_ERR_UNSUPPORTED;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (type == DSPARK_TABLE_Q8_0 && B > kMarkovCudaCoreStates && B <= kI8MaxStates) {
+    switch (B) {
+      case 1: return markov_i8_launch<1>(table, V, h, y, V, s);
+      case 2: return markov_i8_launch<2>(table, V, h, y, V, s);
+      case 3: return markov_i8_launch<3>(table, V, h, y, V, s);
+      case 4: return markov_i8_launch<4>(table, V, h, y, V, s);
+      default: return markov_i8_launch<5>(table, V, h, y, V, s);
+    }
+  }
   if (type == DSPARK_TABLE_Q8_0 && B > kMarkovCudaCoreStates) {
     for (int b0 = 0; b0 < B; b0 += kMmaMaxStates) {
       const int nb = B - b0 < kMmaMaxStates ? B - b0 : kMmaMaxStates;

@@ -12,7 +12,7 @@
 //    butterfly (each round halves the values a lane carries): 2 states x 4 rows cost 9
 //    shuffles instead of 40. With 3 or 4 states the products run as packed f32x2 FMAs (even
 //    and odd elements in the two halves of the accumulator).
-//  - Q8_0 (1 to 4 states; more take the tensor-core kernel): a row is 8 blocks of 34 bytes
+//  - Q8_0 (one state; more take the tensor-core kernels): a row is 8 blocks of 34 bytes
 //    (272 bytes, so rows start 16-byte aligned). A group of 8 consecutive rows (2176 bytes) is
 //    copied by 16-byte asynchronous copies into one of the warp's two shared buffers, so the
 //    next group is in flight while the warp decodes this one; lane l decodes blocks (row l/8,
@@ -263,11 +263,14 @@ __global__ void __launch_bounds__(kMarkovThreads, NB <= 2 ? 4 : 3) markov_q8_0_k
   grid_dependents_launch();
   long long v0 = static_cast<long long>(gw) * kQ8Rows;
   if (v0 < V) fetch(v0, 0);
-  // the states' digits: warp w takes (state, block) pairs w, w + 8, ...
-  for (int t = wi; t < NB * kQ8Blocks; t += kMarkovThreads / 32) {
-    const int b = t / kQ8Blocks, j = t % kQ8Blocks;
-    q8_state_digits(h[b * kMarkovRank + j * 32 + lane], j, lane, s_dig[b], s_ex[b]);
-  }
+  static_assert(kMarkovThreads / 32 == kQ8Blocks, "one warp per table block");
+  // the states' digits: warp w takes (state, block) pairs w, w + 8, ..., all of its state
+  // values loaded before any is used
+  float hvs[NB];
+#pragma unroll
+  for (int u = 0; u < NB; ++u) hvs[u] = __ldg(h + u * kMarkovRank + wi * 32 + lane);
+#pragma unroll
+  for (int u = 0; u < NB; ++u) q8_state_digits(hvs[u], wi, lane, s_dig[u], s_ex[u]);
   __syncthreads();
   int xb[NB];  // this lane's block exponent per state
 #pragma unroll

@@ -726,4 +726,320 @@ __global__ void __launch_bounds__(kF16MmaThreads, 1)
   }
 }
 
+// ---------------------------------------------------------------- Q8_0, few states, int8
+
+// The Q8_0 mat-vec for 1 to 5 states on the integer tensor cores (kind::i8), with no
+// conversion: the table bytes are the A operand as stored. TMA copies each tile's 272-byte rows
+// in 3 windows of 128 bytes (128 rows x 128 bytes, 128-byte swizzle; the bytes past 272 read as
+// zeros) into one shared stage. Block j of a row (scale bytes 34 j, 34 j + 1, then 32 signed
+// bytes) lies in the 32-byte K steps k0 = floor(34 j / 32) and k0 + 1; its MMA pair multiplies
+// both steps by B operands that hold the state's digits at the block's 32 byte positions and
+// zeros elsewhere (so the scale bytes and the neighbouring blocks drop out), into the block's
+// own 16 int32 columns: column 3 s + p is plane p of state s (three signed-byte digit planes
+// per state and block, as in the CUDA-core kernel). The sums are exact. The epilogue (thread =
+// row = TMEM lane) reads the block's scale d from the staged bytes and adds
+//   d 2^(x_sj - X_s) (A + (B + C / 254) / 254)
+// over the 8 blocks (x_sj the block's digit exponent, X_s the state's largest), then writes
+// 2^X_s times the sum. One CTA per SM, 6 warps: warp 0 one lane issues the TMA copies (4 tile
+// stages, 192 KB), warp 1 one lane the 16 MMAs per tile and their commit, warps 2-5 the
+// epilogue, which also releases the stage (its scale bytes are read there); warps 1-5 build the
+// digits first.
+constexpr int kI8Threads = 192;
+constexpr int kI8MaxStates = 5;                    // 3 planes x 5 states <= N = 16
+constexpr int kI8N = 16;
+constexpr int kI8Windows = 3;                      // 128-byte windows per 272-byte row
+constexpr int kI8WinBytes = kMmaRows * 128;        // 16384
+constexpr int kI8TileBytes = kI8Windows * kI8WinBytes;  // 49152
+constexpr int kI8Stages = 4;
+constexpr int kI8BBytes = 8 * 2 * kI8N * 32;       // (block, K step) B operands: 8 KB
+constexpr int kI8Slots = 4;                        // accumulator slots of 8 x 16 columns
+
+__host__ __device__ constexpr int i8_mma_smem() {
+  return kI8Stages * kI8TileBytes + kI8BBytes + 1024 + 1024;
+}
+
+// Shared-memory descriptor of a K-major operand in the 32-byte swizzle layout: rows of 32
+// bytes, 8-row groups 256 bytes apart, the 16-byte chunk c of row r stored at c ^ ((r / 4) % 2).
+__device__ __forceinline__ uint64_t sw32_desc(uint32_t saddr) {
+  return static_cast<uint64_t>((saddr >> 4) & 0x3FFFu) | (1ull << 16) |  // leading offset (unused)
+         (16ull << 32) |                                                // group stride 256 B
+         (1ull << 46) |                                                 // descriptor version
+         (6ull << 61);                                                  // 32-byte swizzle
+}
+
+// Instruction descriptor: kind::i8, A and B signed 8-bit, K-major, D signed 32-bit, M = 128, N.
+__host__ __device__ constexpr uint32_t mma_idesc_s8(int n) {
+  return (2u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(n >> 3) << 17) |
+         (static_cast<uint32_t>(128 >> 4) << 24);
+}
+
+__device__ __forceinline__ void mma_s8(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                       uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// 4 consecutive 32-bit TMEM columns of this warp's 32 lanes.
+__device__ __forceinline__ void tmem_ld4(uint32_t taddr, float* v) {
+  uint32_t r[4];
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x4.b32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(taddr)
+               : "memory");
+#pragma unroll
+  for (int i = 0; i < 4; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// Byte offset of (row n, byte k) in a 32-byte-swizzled K-major operand.
+__device__ __forceinline__ int sw32_off(int n, int k) {
+  return n * 32 + ((((k >> 4) ^ (n >> 2)) & 1) << 4) + (k & 15);
+}
+// Byte offset of (row n, byte k < 128) in a 128-byte-swizzled atom.
+__device__ __forceinline__ int sw128_off(int n, int k) {
+  return n * 128 + ((((k >> 4) ^ n) & 7) << 4) + (k & 15);
+}
+
+template <int NB>
+__global__ void __launch_bounds__(kI8Threads, 1)
+    markov_q8_0_i8_kernel(const __grid_constant__ CUtensorMap tmap, int V, const float* h,
+                          float* y, int ldy) {
+  // TMEM columns read per block (3 NB used) and blocks per load batch (64 registers)
+  constexpr int kLd = NB == 1 ? 4 : (NB == 2 ? 8 : 16);
+  constexpr int kBatch = 64 / kLd < 8 ? 64 / kLd : 8;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                           ~static_cast<uintptr_t>(1023));
+  uint8_t* s_a = sm;                                   // kI8Stages x 3 windows x 16 KB
+  uint8_t* s_b = sm + kI8Stages * kI8TileBytes;        // [block][K step 0/1][16 x 32 B]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(s_b + kI8BBytes);
+  uint64_t* t_full = bars;          // [4] TMA (expect_tx) + bytes
+  uint64_t* t_free = bars + 4;      // [4] the epilogue (128)
+  uint64_t* acc_full = bars + 8;    // [4] MMA commit
+  uint64_t* acc_empty = bars + 12;  // [4] the epilogue (128)
+  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(bars + 16);
+  volatile int* s_abort = reinterpret_cast<volatile int*>(bars + 17);
+  int* s_x = reinterpret_cast<int*>(bars + 18);        // [5][8] block exponents
+
+  const int tid = threadIdx.x, wi = tid >> 5, lane = tid & 31;
+  const int n_tiles = (V + kMmaRows - 1) / kMmaRows;
+  const int my_tiles = blockIdx.x < n_tiles ? (n_tiles - 1 - blockIdx.x) / gridDim.x + 1 : 0;
+
+  if (tid == 0) {
+    for (int i = 0; i < 4; ++i) {
+      mbar_init(smem_u32(&t_full[i]), 1);
+      mbar_init(smem_u32(&t_free[i]), kMmaTeam);
+      mbar_init(smem_u32(&acc_full[i]), 1);
+      mbar_init(smem_u32(&acc_empty[i]), kMmaTeam);
+    }
+    *s_abort = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap)) : "memory");
+  }
+  if (wi == 0) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(s_tmem)),
+                 "r"(kMmaTmemCols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    tc_fence_before();
+  }
+  // the B operands start as zeros (warps 1-5)
+  for (int i = tid - 32; i >= 0 && i < kI8BBytes / 16; i += kI8Threads - 32)
+    reinterpret_cast<uint4*>(s_b)[i] = make_uint4(0, 0, 0, 0);
+  __syncthreads();
+
+  grid_dependency_wait();  // h comes from the kernel before (programmatic launch)
+  grid_dependents_launch();
+
+  if (wi == 0) {
+    // ---- producer: 3 TMA copies per tile into one stage
+    if (lane == 0) {
+      int armed = 0;
+      for (int j = 0; j < my_tiles; ++j) {
+        const int st = j % kI8Stages;
+        if (!mbar_wait(smem_u32(&t_free[st]), ((j / kI8Stages) & 1) ^ 1, s_abort)) break;
+        const int t = blockIdx.x + j * gridDim.x;
+        mbar_arrive_tx(smem_u32(&t_full[st]), kI8TileBytes);
+#pragma unroll
+        for (int w = 0; w < kI8Windows; ++w)
+          tma_load_2d(smem_u32(s_a + st * kI8TileBytes + w * kI8WinBytes), &tmap, 128 * w,
+                      t * kMmaRows, smem_u32(&t_full[st]));
+        armed = j + 1;
+      }
+      if (*s_abort) {
+        for (int j = armed - kI8Stages < 0 ? 0 : armed - kI8Stages; j < armed; ++j) {
+          const uint32_t bar = smem_u32(&t_full[j % kI8Stages]);
+          const long long t0 = clock64();
+          while (!mbar_try(bar, (j / kI8Stages) & 1) && clock64() - t0 < (1ll << 31)) {
+          }
+        }
+      }
+    }
+  } else {
+    // ---- warps 1-5: digits of (state s, block j) pairs t = s * 8 + j, warp w taking pairs
+    // w - 1, w + 4, ...; all of a warp's state values are loaded before any is used
+    constexpr int kPairs = (NB * kQ8Blocks + 4) / 5;
+    float hvs[kPairs];
+#pragma unroll
+    for (int u = 0; u < kPairs; ++u) {
+      const int t = wi - 1 + 5 * u;
+      hvs[u] = t < NB * kQ8Blocks ? __ldg(h + (t / kQ8Blocks) * kMarkovRank + (t % kQ8Blocks) * 32 + lane) : 0.f;
+    }
+#pragma unroll
+    for (int u = 0; u < kPairs; ++u) {
+      const int t = wi - 1 + 5 * u;
+      if (t >= NB * kQ8Blocks) break;
+      const int st = t / kQ8Blocks, j = t % kQ8Blocks;
+      const float hv = hvs[u];
+      const float ah = fabsf(hv);
+      const uint32_t mb = __reduce_max_sync(0xffffffffu, __float_as_uint(ah));
+      const float m = __uint_as_float(mb);
+      int x = 0;
+      if (m > 0.f && m <= 3.402823466e38f) {
+        const int be = static_cast<int>(mb >> 23);
+        const int lg = be != 0 ? be - 127 : -149 + (31 - __clz(static_cast<int>(mb & 0x7fffffu)));
+        x = lg - 6;
+        if (mul_pow2(m, -x) > 127.f) x += 1;
+      }
+      const float v = mul_pow2(hv, -x);
+      const float a = rintf(v);
+      const float r1 = __fmul_rn(__fsub_rn(v, a), 254.f);
+      const float bb = rintf(r1);
+      const float c = rintf(__fmul_rn(__fsub_rn(r1, bb), 254.f));
+      // element lane of block j is table byte g = 34 j + 2 + lane: K step g / 32, byte g % 32
+      const int g = 34 * j + 2 + lane, w = (g >> 5) - (34 * j >> 5);
+      uint8_t* bm = s_b + (j * 2 + w) * (kI8N * 32);
+      bm[sw32_off(3 * st + 0, g & 31)] = static_cast<uint8_t>(static_cast<int8_t>(a));
+      bm[sw32_off(3 * st + 1, g & 31)] = static_cast<uint8_t>(static_cast<int8_t>(bb));
+      bm[sw32_off(3 * st + 2, g & 31)] = static_cast<uint8_t>(static_cast<int8_t>(c));
+      if (lane == 0) s_x[st * 8 + j] = m <= 3.402823466e38f ? x : 1024;  // 1024: non-finite
+    }
+    fence_proxy_async_smem();
+    asm volatile("bar.sync 1, %0;" ::"n"(kI8Threads - 32) : "memory");  // warps 1-5
+    const uint32_t tbase = *s_tmem;
+    tc_fence_after();
+    if (wi == 1) {
+      // ---- MMA issuer: per tile, per block, its two 32-byte K steps into the block's columns
+      if (lane == 0) {
+        constexpr uint32_t idesc = mma_idesc_s8(kI8N);
+        const uint32_t b0 = smem_u32(s_b);
+        int last = -1;
+        for (int j = 0; j < my_tiles; ++j) {
+          const int st = j % kI8Stages, ts = j % kI8Slots;
+          if (!mbar_wait(smem_u32(&t_full[st]), (j / kI8Stages) & 1, s_abort)) break;
+          if (!mbar_wait(smem_u32(&acc_empty[ts]), ((j / kI8Slots) & 1) ^ 1, s_abort)) break;
+          tc_fence_after();
+          const uint32_t a0 = smem_u32(s_a + st * kI8TileBytes);
+#pragma unroll
+          for (int blk = 0; blk < kQ8Blocks; ++blk) {
+            const int k0 = 34 * blk >> 5;
+#pragma unroll
+            for (int w = 0; w < 2; ++w) {
+              const int k = k0 + w;  // 32-byte K step: window k / 4, 32 (k % 4) bytes in
+              mma_s8(tbase + ts * (kQ8Blocks * kI8N) + blk * kI8N,
+                     sw128_desc(a0 + (k >> 2) * kI8WinBytes + 32 * (k & 3)),
+                     sw32_desc(b0 + (blk * 2 + w) * (kI8N * 32)), idesc, w);
+            }
+          }
+          mma_commit(smem_u32(&acc_full[ts]));
+          last = j;
+        }
+        if (*s_abort && last >= 0) {
+          const uint32_t bar = smem_u32(&acc_full[last % kI8Slots]);
+          const long long t0 = clock64();
+          while (!mbar_try(bar, (last / kI8Slots) & 1) && clock64() - t0 < (1ll << 31)) {
+          }
+        }
+      }
+    } else {
+      // ---- epilogue: thread = tile row = TMEM lane
+      const int q = wi & 3;
+      const int r = 32 * q + lane;
+      // per state: X_s and the block factors 2^(x_sj - X_s) (0 below 2^-126)
+      int X[NB];
+      float gf[NB][kQ8Blocks];
+#pragma unroll
+      for (int s2 = 0; s2 < NB; ++s2) {
+        int mx = s_x[s2 * 8];
+#pragma unroll
+        for (int j = 1; j < kQ8Blocks; ++j) mx = max(mx, s_x[s2 * 8 + j]);
+        X[s2] = mx;
+#pragma unroll
+        for (int j = 0; j < kQ8Blocks; ++j) {
+          const int dx = s_x[s2 * 8 + j] - mx;
+          gf[s2][j] = dx >= -126 ? pow2f(dx) : 0.f;
+        }
+      }
+      for (int j = 0; j < my_tiles; ++j) {
+        const int st = j % kI8Stages, ts = j % kI8Slots;
+        if (!__all_sync(0xffffffffu,
+                        mbar_wait(smem_u32(&acc_full[ts]), (j / kI8Slots) & 1, s_abort)))
+          break;
+        tc_fence_after();
+        const uint32_t ta =
+            tbase + (static_cast<uint32_t>(32 * q) << 16) + ts * (kQ8Blocks * kI8N);
+        const uint8_t* tile = s_a + st * kI8TileBytes;
+        float acc[NB];
+#pragma unroll
+        for (int s2 = 0; s2 < NB; ++s2) acc[s2] = 0.f;
+#pragma unroll
+        for (int b0 = 0; b0 < kQ8Blocks; b0 += kBatch) {
+          float v[kBatch][kLd];
+          float dd[kBatch];
+#pragma unroll
+          for (int u = 0; u < kBatch; ++u) {
+            if constexpr (kLd == 4)
+              tmem_ld4(ta + (b0 + u) * kI8N, v[u]);
+            else if constexpr (kLd == 8)
+              tmem_ld8(ta + (b0 + u) * kI8N, v[u]);
+            else
+              tmem_ld16(ta + (b0 + u) * kI8N, v[u]);
+          }
+#pragma unroll
+          for (int u = 0; u < kBatch; ++u) {
+            // the block's scale: bytes 34 blk .. 34 blk + 1 (even; one 16-byte chunk)
+            const int o = 34 * (b0 + u);
+            dd[u] = __half2float(*reinterpret_cast<const __half*>(
+                tile + (o >> 7) * kI8WinBytes + sw128_off(r, o & 127)));
+          }
+          tmem_ld_wait();
+#pragma unroll
+          for (int u = 0; u < kBatch; ++u) {
+#pragma unroll
+            for (int s2 = 0; s2 < NB; ++s2) {
+              const int A = __float_as_int(v[u][3 * s2]), Bv = __float_as_int(v[u][3 * s2 + 1]),
+                        C = __float_as_int(v[u][3 * s2 + 2]);
+              float f = __fmaf_rn(small_int_to_float(C), 1.f / 254.f, small_int_to_float(Bv));
+              f = __fmaf_rn(f, 1.f / 254.f, small_int_to_float(A));
+              acc[s2] = __fmaf_rn(__fmul_rn(dd[u], gf[s2][b0 + u]), f, acc[s2]);
+            }
+          }
+        }
+        tc_fence_before();
+        mbar_arrive(smem_u32(&acc_empty[ts]));
+        mbar_arrive(smem_u32(&t_free[st]));
+        const long long row = static_cast<long long>(blockIdx.x + j * gridDim.x) * kMmaRows + r;
+        if (row < V) {
+#pragma unroll
+          for (int s2 = 0; s2 < NB; ++s2)
+            y[static_cast<long long>(s2) * ldy + row] =
+                X[s2] >= 1024 ? __int_as_float(0x7fc00000) : mul_pow2(acc[s2], X[s2]);
+        }
+      }
+    }
+  }
+
+  __syncthreads();
+  if (wi == 0) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(*s_tmem),
+                 "r"(kMmaTmemCols)
+                 : "memory");
+  }
+}
+
 }  // namespace dspark

@@ -1,17 +1,17 @@
 """The Markov-head table mat-vec on the GPU against the float64 oracle.
 
-Tolerance, from the arithmetic. F16: each output is a float32 sum of R = 256 products (8 per
-lane, then a butterfly), so its error is below (R + 8) * 2^-24 * sum_k |W[v, k] h[b, k]|; the
-tests allow twice R * 2^-24 times that sum, plus 1e-30. Q8_0 (tensor cores): the state, scaled
-by a power of two, is split into float16 hi + lo within 2^-23 of its largest |h|; each block's
-64 products q * part are exact and summed in float32 (at most a few roundings of 2^-24 per
-MMA step of 16 products), then scaled by d and the 8 blocks added by float32 FMAs. The same
-2 R 2^-24 sum |W h| covers the sums; the tests add 2^-22 max_k |h[b, k]| sum_k |W[v, k]| for
-the split. F16 with two or more states runs on the tensor cores the same way (products of the
-exact table halves with the two parts, one float32 accumulator per part over all 256 k) and
-gets the same added term. One to four Q8_0 states take the CUDA-core kernel: exact integer dot products with
-three signed-byte digit planes of the state, which represent it within 2^-22 of each block's
-largest |h| (so within the same added term), then a few float32 roundings per block.
+Tolerance, from the arithmetic. F16, one state: each output is a float32 sum of R = 256
+products (8 per lane, then a butterfly), so its error is below (R + 8) 2^-24 sum_k |W[v, k]
+h[b, k]|; the tests allow twice R 2^-24 times that sum, plus 1e-30. F16 with two or more states
+and Q8_0 with more than five (tensor cores): the state, scaled by a power of two, is split into
+float16 hi + lo within 2^-23 of its largest |h|; the products of the exact table values with
+the parts are exact and summed in float32 (F16: one sum per part over all 256 k; Q8_0: per
+block of 32, then scaled by d and the 8 blocks added by float32 FMAs). The same 2 R 2^-24
+sum |W h| covers the sums; the tests add 2^-22 max_k |h[b, k]| sum_k |W[v, k]| for the split.
+One to five Q8_0 states take exact integer dot products with three signed-byte digit planes of
+the state (on the CUDA cores for one state, the integer tensor cores for two to five), which
+represent it within 2^-22 of each block's largest |h| (so within the same added term), then a
+few float32 roundings per block.
 """
 
 import numpy as np
@@ -59,9 +59,10 @@ def test_many_states(fmt, B):
 
 
 @pytest.mark.parametrize("fmt", ["f16", "q8_0"])
+@pytest.mark.parametrize("B", [1, 2])
 @pytest.mark.parametrize("V", [1, 7, 8, 9, 63, 65, 127, 128, 129, 1000, 262144])
-def test_ragged_vocab(fmt, V):
-    _check(V, 2, fmt, seed=5)
+def test_ragged_vocab(fmt, B, V):
+    _check(V, B, fmt, seed=5)
 
 
 @pytest.mark.parametrize("fmt", ["f16", "q8_0"])
@@ -83,19 +84,20 @@ def test_one_hot_state_reads_a_column():
 
 
 
-@pytest.mark.parametrize("fmt", ["f16", "q8_0"])
-def test_state_scales(fmt):
+@pytest.mark.parametrize("fmt,nst", [("f16", 6), ("q8_0", 5), ("q8_0", 6)])
+def test_state_scales(fmt, nst):
     """States of very different magnitudes (each is scaled by its own power of two), a zero
-    state and one with a single nonzero entry, in one launch."""
+    state and one with a single nonzero entry, in one launch (five Q8_0 states take the
+    integer tensor-core kernel, six the float16 one)."""
     V = 5000
     raw = wl.markov_table(V, R, fmt, seed=8)
-    H = wl.markov_states(6, R, seed=8).astype(np.float64)
+    H = wl.markov_states(nst, R, seed=8).astype(np.float64)
     H[0] *= 1e-30
     H[1] *= 1e20
     H[2] = 0.0
     H[3] = 0.0
     H[3, 200] = -3.0
-    H[4] *= 2.0 ** -140  # subnormal float32 states
+    H[4, :128] *= 2.0 ** -140  # subnormal float32 values in half the blocks
     H = H.astype(np.float32)
     t = torch.from_numpy(raw.view(np.int16) if fmt == "f16" else raw).to(DEV)
     y = bd.markov_matvec(t, fmt, torch.from_numpy(H).to(DEV))
