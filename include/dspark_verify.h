@@ -267,6 +267,16 @@ dspark_status_t dspark_markov_matvec(const void* table, dspark_table_t type, int
  * Synchronous (waits for the device). DSPARK_ERR_INVALID_ARG for a NULL count. */
 dspark_status_t dspark_pipeline_timeouts(unsigned long long* count);
 
+/* For tests of the timeout path only: dspark_markov_matvec with each CTA's first table copy
+ * withheld in its pipelined tensor-core kernels, so that the waits for it run out (about a
+ * second) and the kernels give up as described above: the call returns DSPARK_OK, y is left
+ * incomplete and dspark_pipeline_timeouts grows. DSPARK_ERR_UNSUPPORTED where the call would
+ * take a CUDA-core kernel (one state), which has no waits. Same arguments as
+ * dspark_markov_matvec. */
+dspark_status_t dspark_markov_matvec_withheld(const void* table, dspark_table_t type, int V,
+                                              int R, const float* h, int B, float* y,
+                                              void* stream);
+
 /* speculative_sample_accept without a workspace argument. The pages have no counterpart of
  * this entry point: it exists for callers that cannot allocate device memory where they
  * verify (a serving loop whose KV-cache pool took all free HBM at start-up and left no

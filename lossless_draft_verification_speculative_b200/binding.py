@@ -136,6 +136,8 @@ def load_library(build_if_missing: bool = True) -> ctypes.CDLL:
                                              ctypes.c_float, vp, AcceptOut, vp, sz, vp]
     lib.dspark_markov_matvec.restype = i32
     lib.dspark_markov_matvec.argtypes = [vp, i32, i32, i32, vp, i32, vp, vp]
+    lib.dspark_markov_matvec_withheld.restype = i32
+    lib.dspark_markov_matvec_withheld.argtypes = [vp, i32, i32, i32, vp, i32, vp, vp]
     lib.dspark_pipeline_timeouts.restype = i32
     lib.dspark_pipeline_timeouts.argtypes = [ctypes.POINTER(ctypes.c_ulonglong)]
     lib.dspark_quench_reset.restype = i32
@@ -404,7 +406,7 @@ MARKOV_TABLE_CODES = {"f16": 0, "q8_0": 1}
 
 
 def markov_matvec(table: torch.Tensor, fmt: str, h: torch.Tensor, *,
-                  out: Optional[torch.Tensor] = None) -> torch.Tensor:
+                  out: Optional[torch.Tensor] = None, _withhold: bool = False) -> torch.Tensor:
     """The drafter's Markov-head table mat-vec on the GPU: y[b, v] = sum_k W[v, k] h[b, k].
 
     ``table`` holds markov_w2 as the drafter files store it: fmt "f16", a [V, R] float16 (or
@@ -427,11 +429,20 @@ def markov_matvec(table: torch.Tensor, fmt: str, h: torch.Tensor, *,
     y = out if out is not None else torch.empty(B, V, dtype=torch.float32, device=h.device)
     if y.shape != (B, V) or y.dtype != torch.float32 or not y.is_contiguous():
         raise ValueError("out must be a contiguous float32 [B, V] tensor")
-    rc = lib.dspark_markov_matvec(_ptr(table), MARKOV_TABLE_CODES[fmt], V, R, _ptr(h), B,
-                                  _ptr(y), _stream_handle(h.device))
+    fn = lib.dspark_markov_matvec_withheld if _withhold else lib.dspark_markov_matvec
+    rc = fn(_ptr(table), MARKOV_TABLE_CODES[fmt], V, R, _ptr(h), B, _ptr(y),
+            _stream_handle(h.device))
     if rc != DSPARK_OK:
         raise DsparkError(rc, "dspark_markov_matvec")
     return y
+
+
+def markov_matvec_withheld(table: torch.Tensor, fmt: str, h: torch.Tensor, *,
+                           out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """markov_matvec with the first table copy of every CTA withheld, for tests of the timeout
+    path only: the pipelined kernels' waits run out (about a second), they give up, and
+    ``pipeline_timeouts()`` grows; the result is incomplete."""
+    return markov_matvec(table, fmt, h, out=out, _withhold=True)
 
 
 def pipeline_timeouts(device=None) -> int:

@@ -510,7 +510,7 @@ constexpr int kMarkovCudaCoreStates = 1;
 // SM over the 128-row tiles.
 template <int N>
 dspark_status_t markov_mma_launch(const void* table, int V, const float* h, int nb, float* y,
-                                  int ldy, cudaStream_t stream) {
+                                  int ldy, cudaStream_t stream, int withhold) {
   const void* fn = reinterpret_cast<const void*>(&markov_q8_0_mma_kernel<N>);
   const size_t smem = static_cast<size_t>(mma_q8_smem(N).total);
   cudaError_t e = cudaSuccess;
@@ -530,7 +530,7 @@ dspark_status_t markov_mma_launch(const void* table, int V, const float* h, int 
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   e = cudaLaunchKernelEx(&cfg, markov_q8_0_mma_kernel<N>, static_cast<const uint8_t*>(table), V,
-                         h, nb, y, ldy);
+                         h, nb, y, ldy, withhold);
   return e == cudaSuccess ? DSPARK_OK : DSPARK_ERR_CUDA;
 }
 
@@ -564,7 +564,7 @@ constexpr int kMarkovF16CudaCoreStates = 1;
 // (boxes of 128 rows x 64 halves, 128-byte swizzle, rows past V read as zeros).
 template <int N>
 dspark_status_t markov_f16_mma_launch(const void* table, int V, const float* h, int nb, float* y,
-                                      int ldy, cudaStream_t stream) {
+                                      int ldy, cudaStream_t stream, int withhold) {
   const EncodeTiledFn enc = tensor_map_encoder();
   if (!enc) return DSPARK_ERR_UNSUPPORTED;
   alignas(64) CUtensorMap map;
@@ -594,7 +594,7 @@ dspark_status_t markov_f16_mma_launch(const void* table, int V, const float* h, 
   cfg.stream = stream;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  e = cudaLaunchKernelEx(&cfg, markov_f16_mma_kernel<N>, map, V, h, nb, y, ldy);
+  e = cudaLaunchKernelEx(&cfg, markov_f16_mma_kernel<N>, map, V, h, nb, y, ldy, withhold);
   return e == cudaSuccess ? DSPARK_OK : DSPARK_ERR_CUDA;
 }
 
@@ -603,7 +603,7 @@ dspark_status_t markov_f16_mma_launch(const void* table, int V, const float* h, 
 // rows past V read as zeros).
 template <int NB>
 dspark_status_t markov_i8_launch(const void* table, int V, const float* h, float* y, int ldy,
-                                 cudaStream_t stream) {
+                                 cudaStream_t stream, int withhold) {
   const EncodeTiledFn enc = tensor_map_encoder();
   if (!enc) return DSPARK_ERR_UNSUPPORTED;
   alignas(64) CUtensorMap map;
@@ -633,7 +633,7 @@ dspark_status_t markov_i8_launch(const void* table, int V, const float* h, float
   cfg.stream = stream;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  e = cudaLaunchKernelEx(&cfg, markov_q8_0_i8_kernel<NB>, map, V, h, y, ldy);
+  e = cudaLaunchKernelEx(&cfg, markov_q8_0_i8_kernel<NB>, map, V, h, y, ldy, withhold);
   return e == cudaSuccess ? DSPARK_OK : DSPARK_ERR_CUDA;
 }
 
@@ -641,6 +641,85 @@ dspark_status_t markov_i8_launch(const void* table, int V, const float* h, float
 }  // namespace dspark
 
 using namespace dspark;
+
+namespace dspark {
+namespace {
+// The Markov mat-vec dispatch; withhold != 0 (tests of the timeout path) is only accepted
+// where the call takes a pipelined tensor-core kernel.
+dspark_status_t markov_matvec_impl(const void* table, dspark_table_t type, int V, int R,
+                                   const float* h, int B, float* y, void* stream, int withhold) {
+  if (type != DSPARK_TABLE_F16 && type != DSPARK_TABLE_Q8_0) return DSPARK_ERR_INVALID_ARG;
+  if (V < 0 || R < 1 || B < 0) return DSPARK_ERR_INVALID_ARG;
+  if (V == 0 || B == 0) return DSPARK_OK;
+  if (!table || !h || !y) return DSPARK_ERR_INVALID_ARG;
+  if (R != kMarkovRank) return DSPARK_ERR_UNSUPPORTED;
+  if (!aligned(table, 16) || !aligned(h, 16) || !aligned(y, 4)) return DSPARK_ERR_UNSUPPORTED;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (withhold && ((type == DSPARK_TABLE_Q8_0 && B <= kMarkovCudaCoreStates) ||
+                   (type == DSPARK_TABLE_F16 && B <= kMarkovF16CudaCoreStates)))
+    return DSPARK_ERR_UNSUPPORTED;
+  if (type == DSPARK_TABLE_Q8_0 && B > kMarkovCudaCoreStates && B <= kI8MaxStates) {
+    switch (B) {
+      case 1: return markov_i8_launch<1>(table, V, h, y, V, s, withhold);
+      case 2: return markov_i8_launch<2>(table, V, h, y, V, s, withhold);
+      case 3: return markov_i8_launch<3>(table, V, h, y, V, s, withhold);
+      case 4: return markov_i8_launch<4>(table, V, h, y, V, s, withhold);
+      default: return markov_i8_launch<5>(table, V, h, y, V, s, withhold);
+    }
+  }
+  if (type == DSPARK_TABLE_Q8_0 && B > kMarkovCudaCoreStates) {
+    for (int b0 = 0; b0 < B; b0 += kMmaMaxStates) {
+      const int nb = B - b0 < kMmaMaxStates ? B - b0 : kMmaMaxStates;
+      const float* hb = h + static_cast<size_t>(b0) * R;
+      float* yb = y + static_cast<size_t>(b0) * V;
+      dspark_status_t st;
+      if (nb <= 16)
+        st = markov_mma_launch<16>(table, V, hb, nb, yb, V, s, withhold);
+      else if (nb <= 32)
+        st = markov_mma_launch<32>(table, V, hb, nb, yb, V, s, withhold);
+      else if (nb <= 48)
+        st = markov_mma_launch<48>(table, V, hb, nb, yb, V, s, withhold);
+      else
+        st = markov_mma_launch<64>(table, V, hb, nb, yb, V, s, withhold);
+      if (st != DSPARK_OK) return st;
+    }
+    return DSPARK_OK;
+  }
+  if (type == DSPARK_TABLE_F16 && B > kMarkovF16CudaCoreStates) {
+    for (int b0 = 0; b0 < B; b0 += kMmaMaxStates) {
+      const int nb = B - b0 < kMmaMaxStates ? B - b0 : kMmaMaxStates;
+      const float* hb = h + static_cast<size_t>(b0) * R;
+      float* yb = y + static_cast<size_t>(b0) * V;
+      dspark_status_t st;
+      if (nb <= 16)
+        st = markov_f16_mma_launch<16>(table, V, hb, nb, yb, V, s, withhold);
+      else if (nb <= 32)
+        st = markov_f16_mma_launch<32>(table, V, hb, nb, yb, V, s, withhold);
+      else if (nb <= 48)
+        st = markov_f16_mma_launch<48>(table, V, hb, nb, yb, V, s, withhold);
+      else
+        st = markov_f16_mma_launch<64>(table, V, hb, nb, yb, V, s, withhold);
+      if (st != DSPARK_OK) return st;
+    }
+    return DSPARK_OK;
+  }
+  for (int b0 = 0; b0 < B; b0 += kMarkovMaxStates) {
+    const int nb = B - b0 < kMarkovMaxStates ? B - b0 : kMarkovMaxStates;
+    const float* hb = h + static_cast<size_t>(b0) * R;
+    float* yb = y + static_cast<size_t>(b0) * V;
+    dspark_status_t st;
+    switch (nb) {
+      case 1: st = markov_launch<1>(table, type, V, hb, yb, V, s); break;
+      case 2: st = markov_launch<2>(table, type, V, hb, yb, V, s); break;
+      case 3: st = markov_launch<3>(table, type, V, hb, yb, V, s); break;
+      default: st = markov_launch<4>(table, type, V, hb, yb, V, s); break;
+    }
+    if (st != DSPARK_OK) return st;
+  }
+  return DSPARK_OK;
+}
+}  // namespace
+}  // namespace dspark
 
 extern "C" {
 
@@ -853,72 +932,13 @@ dspark_status_t dspark_early_exit_accept(const void* p1, int64_t ld_p1, const vo
 
 dspark_status_t dspark_markov_matvec(const void* table, dspark_table_t type, int V, int R,
                                      const float* h, int B, float* y, void* stream) {
-  if (type != DSPARK_TABLE_F16 && type != DSPARK_TABLE_Q8_0) return DSPARK_ERR_INVALID_ARG;
-  if (V < 0 || R < 1 || B < 0) return DSPARK_ERR_INVALID_ARG;
-  if (V == 0 || B == 0) return DSPARK_OK;
-  if (!table || !h || !y) return DSPARK_ERR_INVALID_ARG;
-  if (R != kMarkovRank) return DSPARK_ERR_UNSUPPORTED;
-  if (!aligned(table, 16) || !aligned(h, 16) || !aligned(y, 4)) return DSPARK_ERR_UNSUPPORTED;
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (type == DSPARK_TABLE_Q8_0 && B > kMarkovCudaCoreStates && B <= kI8MaxStates) {
-    switch (B) {
-      case 1: return markov_i8_launch<1>(table, V, h, y, V, s);
-      case 2: return markov_i8_launch<2>(table, V, h, y, V, s);
-      case 3: return markov_i8_launch<3>(table, V, h, y, V, s);
-      case 4: return markov_i8_launch<4>(table, V, h, y, V, s);
-      default: return markov_i8_launch<5>(table, V, h, y, V, s);
-    }
-  }
-  if (type == DSPARK_TABLE_Q8_0 && B > kMarkovCudaCoreStates) {
-    for (int b0 = 0; b0 < B; b0 += kMmaMaxStates) {
-      const int nb = B - b0 < kMmaMaxStates ? B - b0 : kMmaMaxStates;
-      const float* hb = h + static_cast<size_t>(b0) * R;
-      float* yb = y + static_cast<size_t>(b0) * V;
-      dspark_status_t st;
-      if (nb <= 16)
-        st = markov_mma_launch<16>(table, V, hb, nb, yb, V, s);
-      else if (nb <= 32)
-        st = markov_mma_launch<32>(table, V, hb, nb, yb, V, s);
-      else if (nb <= 48)
-        st = markov_mma_launch<48>(table, V, hb, nb, yb, V, s);
-      else
-        st = markov_mma_launch<64>(table, V, hb, nb, yb, V, s);
-      if (st != DSPARK_OK) return st;
-    }
-    return DSPARK_OK;
-  }
-  if (type == DSPARK_TABLE_F16 && B > kMarkovF16CudaCoreStates) {
-    for (int b0 = 0; b0 < B; b0 += kMmaMaxStates) {
-      const int nb = B - b0 < kMmaMaxStates ? B - b0 : kMmaMaxStates;
-      const float* hb = h + static_cast<size_t>(b0) * R;
-      float* yb = y + static_cast<size_t>(b0) * V;
-      dspark_status_t st;
-      if (nb <= 16)
-        st = markov_f16_mma_launch<16>(table, V, hb, nb, yb, V, s);
-      else if (nb <= 32)
-        st = markov_f16_mma_launch<32>(table, V, hb, nb, yb, V, s);
-      else if (nb <= 48)
-        st = markov_f16_mma_launch<48>(table, V, hb, nb, yb, V, s);
-      else
-        st = markov_f16_mma_launch<64>(table, V, hb, nb, yb, V, s);
-      if (st != DSPARK_OK) return st;
-    }
-    return DSPARK_OK;
-  }
-  for (int b0 = 0; b0 < B; b0 += kMarkovMaxStates) {
-    const int nb = B - b0 < kMarkovMaxStates ? B - b0 : kMarkovMaxStates;
-    const float* hb = h + static_cast<size_t>(b0) * R;
-    float* yb = y + static_cast<size_t>(b0) * V;
-    dspark_status_t st;
-    switch (nb) {
-      case 1: st = markov_launch<1>(table, type, V, hb, yb, V, s); break;
-      case 2: st = markov_launch<2>(table, type, V, hb, yb, V, s); break;
-      case 3: st = markov_launch<3>(table, type, V, hb, yb, V, s); break;
-      default: st = markov_launch<4>(table, type, V, hb, yb, V, s); break;
-    }
-    if (st != DSPARK_OK) return st;
-  }
-  return DSPARK_OK;
+  return markov_matvec_impl(table, type, V, R, h, B, y, stream, 0);
+}
+
+dspark_status_t dspark_markov_matvec_withheld(const void* table, dspark_table_t type, int V,
+                                              int R, const float* h, int B, float* y,
+                                              void* stream) {
+  return markov_matvec_impl(table, type, V, R, h, B, y, stream, 1);
 }
 
 dspark_status_t dspark_pipeline_timeouts(unsigned long long* count) {

@@ -33,7 +33,8 @@
 // slots in tensor memory (4 N columns each). Every mbarrier wait is bounded (about a second);
 // a wait that runs out sets an abort flag that ends every role's loop, counts the event in a
 // device counter (dspark_pipeline_timeouts), lets the copies and MMAs in flight finish (again
-// bounded) and frees the tensor memory before the CTA exits.
+// bounded) and frees the tensor memory before the CTA exits. `withhold` (tests of that path
+// only) makes each CTA's producer skip its first copy, so the waits for it run out.
 #pragma once
 
 #include <cuda.h>  // CUtensorMap (the type only; no driver calls here)
@@ -313,7 +314,7 @@ __device__ __forceinline__ void build_b_operand(const float* h, int nb, uint8_t*
 template <int N>
 __global__ void __launch_bounds__(kMmaThreads, 1)
     markov_q8_0_mma_kernel(const uint8_t* __restrict__ W, int V, const float* h, int nb,
-                           float* y, int ldy) {
+                           float* y, int ldy, int withhold) {
   constexpr int kRaw = mma_raw_stages(N);
   constexpr int kSlots = mma_tmem_slots(N);
   extern __shared__ uint8_t smem_raw[];
@@ -383,6 +384,7 @@ __global__ void __launch_bounds__(kMmaThreads, 1)
         const long long t = blockIdx.x + static_cast<long long>(j) * gridDim.x;
         const int rows = V - t * kMmaRows < kMmaRows ? static_cast<int>(V - t * kMmaRows) : kMmaRows;
         const uint32_t bytes = static_cast<uint32_t>(rows * kQ8RowBytesT);
+        if (withhold && j == 0) continue;  // (timeout test: this tile never arrives)
         mbar_arrive_tx(smem_u32(&raw_full[st]), bytes);
         bulk_copy_g2s(smem_u32(s_raw + st * kMmaRawBytes), W + t * kMmaRows * kQ8RowBytesT,
                       bytes, smem_u32(&raw_full[st]));
@@ -391,6 +393,7 @@ __global__ void __launch_bounds__(kMmaThreads, 1)
       if (*s_abort) {
         // let the copies in flight land before the CTA's shared memory goes away
         for (int j = armed - kRaw < 0 ? 0 : armed - kRaw; j < armed; ++j) {
+          if (withhold && j == 0) continue;
           const uint32_t bar = smem_u32(&raw_full[j % kRaw]);
           const long long t0 = clock64();
           while (!mbar_try(bar, (j / kRaw) & 1) && clock64() - t0 < (1ll << 31)) {
@@ -576,7 +579,7 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map
 template <int N>
 __global__ void __launch_bounds__(kF16MmaThreads, 1)
     markov_f16_mma_kernel(const __grid_constant__ CUtensorMap tmap, int V, const float* h, int nb,
-                          float* y, int ldy) {
+                          float* y, int ldy, int withhold) {
   constexpr int kSlots = f16_tmem_slots(N);
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -631,6 +634,7 @@ __global__ void __launch_bounds__(kF16MmaThreads, 1)
         const int st = i % kF16Stages;
         if (!mbar_wait(smem_u32(&a_free[st]), ((i / kF16Stages) & 1) ^ 1, s_abort)) break;
         const int t = blockIdx.x + (i >> 2) * gridDim.x;
+        if (withhold && i == 0) continue;  // (timeout test: this stage never arrives)
         mbar_arrive_tx(smem_u32(&a_full[st]), kF16StageBytes);
         tma_load_2d(smem_u32(s_a + st * kF16StageBytes), &tmap, 64 * (i & 3), t * kMmaRows,
                     smem_u32(&a_full[st]));
@@ -638,6 +642,7 @@ __global__ void __launch_bounds__(kF16MmaThreads, 1)
       }
       if (*s_abort) {
         for (int i = armed - kF16Stages < 0 ? 0 : armed - kF16Stages; i < armed; ++i) {
+          if (withhold && i == 0) continue;
           const uint32_t bar = smem_u32(&a_full[i % kF16Stages]);
           const long long t0 = clock64();
           while (!mbar_try(bar, (i / kF16Stages) & 1) && clock64() - t0 < (1ll << 31)) {
@@ -806,7 +811,7 @@ __device__ __forceinline__ int sw128_off(int n, int k) {
 template <int NB>
 __global__ void __launch_bounds__(kI8Threads, 1)
     markov_q8_0_i8_kernel(const __grid_constant__ CUtensorMap tmap, int V, const float* h,
-                          float* y, int ldy) {
+                          float* y, int ldy, int withhold) {
   // TMEM columns read per block (3 NB used) and blocks per load batch (64 registers)
   constexpr int kLd = NB == 1 ? 4 : (NB == 2 ? 8 : 16);
   constexpr int kBatch = 64 / kLd < 8 ? 64 / kLd : 8;
@@ -863,6 +868,7 @@ __global__ void __launch_bounds__(kI8Threads, 1)
         const int st = j % kI8Stages;
         if (!mbar_wait(smem_u32(&t_free[st]), ((j / kI8Stages) & 1) ^ 1, s_abort)) break;
         const int t = blockIdx.x + j * gridDim.x;
+        if (withhold && j == 0) continue;  // (timeout test: this tile never arrives)
         mbar_arrive_tx(smem_u32(&t_full[st]), kI8TileBytes);
 #pragma unroll
         for (int w = 0; w < kI8Windows; ++w)
@@ -872,6 +878,7 @@ __global__ void __launch_bounds__(kI8Threads, 1)
       }
       if (*s_abort) {
         for (int j = armed - kI8Stages < 0 ? 0 : armed - kI8Stages; j < armed; ++j) {
+          if (withhold && j == 0) continue;
           const uint32_t bar = smem_u32(&t_full[j % kI8Stages]);
           const long long t0 = clock64();
           while (!mbar_try(bar, (j / kI8Stages) & 1) && clock64() - t0 < (1ll << 31)) {

@@ -29,6 +29,7 @@ R = 256
 
 
 def _check(V, B, fmt, seed=4):
+    timeouts = bd.pipeline_timeouts()
     raw = wl.markov_table(V, R, fmt, seed=seed)
     H = wl.markov_states(B, R, seed=seed)
     t = torch.from_numpy(raw.view(np.int16) if fmt == "f16" else raw).to(DEV)
@@ -42,7 +43,7 @@ def _check(V, B, fmt, seed=4):
     bound = bound + 2.0 ** -22 * hmax[:, None] * wsum[None, :]
     err = np.abs(y.cpu().numpy().astype(np.float64) - ref)
     assert np.all(err <= bound), (fmt, V, B, float((err / bound).max()))
-    assert bd.pipeline_timeouts() == 0
+    assert bd.pipeline_timeouts() == timeouts
 
 
 @pytest.mark.parametrize("fmt", ["f16", "q8_0"])
@@ -84,6 +85,24 @@ def test_one_hot_state_reads_a_column():
 
 
 
+@pytest.mark.parametrize("fmt,B", [("f16", 4), ("q8_0", 3), ("q8_0", 8)])
+def test_timeout_path(fmt, B):
+    """Each tensor-core kernel (F16; Q8_0 integer; Q8_0 float16) with its first copies withheld:
+    the waits for them run out, the kernels give up and free what they hold, the counter grows,
+    and the device stays usable: the next normal call is correct."""
+    V = 20000
+    raw = wl.markov_table(V, R, fmt, seed=10)
+    t = torch.from_numpy(raw.view(np.int16) if fmt == "f16" else raw).to(DEV)
+    h = torch.from_numpy(wl.markov_states(B, R, seed=10)).to(DEV)
+    before = bd.pipeline_timeouts()
+    bd.markov_matvec_withheld(t, fmt, h)
+    torch.cuda.synchronize()
+    assert bd.pipeline_timeouts() > before
+    _check(V, B, fmt, seed=10)
+    with pytest.raises(bd.DsparkError):  # one state: the CUDA-core kernels have no waits
+        bd.markov_matvec_withheld(t, fmt, h[:1].contiguous())
+
+
 @pytest.mark.parametrize("fmt,nst", [("f16", 6), ("q8_0", 5), ("q8_0", 6)])
 def test_state_scales(fmt, nst):
     """States of very different magnitudes (each is scaled by its own power of two), a zero
@@ -112,4 +131,3 @@ def test_state_scales(fmt, nst):
     assert np.all(err <= bound + 2.0 ** -149)
     assert np.all(y.cpu().numpy()[2] == 0.0)
     assert np.array_equal(y.cpu().numpy()[3].astype(np.float64), W[:, 200] * -3.0)
-    assert bd.pipeline_timeouts() == 0
