@@ -501,8 +501,8 @@ dspark_status_t markov_launch(const void* table, dspark_table_t type, int V, con
 }
 
 // Q8_0 routing by the number of states (measured on a 129280-row table): one state on the
-// CUDA-core kernel (8.0 us; the integer tensor-core kernel takes 10.8), 2 to kI8MaxStates on the
-// integer tensor cores (four states: 11.3 us against 15.3 on the CUDA cores), more on the
+// CUDA-core kernel (8.0 us; the integer tensor-core kernel takes 10.0), 2 to kI8MaxStates on the
+// integer tensor cores (four states: 10.5 us against 15.3 on the CUDA cores), more on the
 // float16 tensor-core kernel, 64 states per launch.
 constexpr int kMarkovCudaCoreStates = 1;
 
@@ -616,7 +616,7 @@ dspark_status_t markov_i8_launch(const void* table, int V, const float* h, float
           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
     return DSPARK_ERR_UNSUPPORTED;
   const void* fn = reinterpret_cast<const void*>(&markov_q8_0_i8_kernel<NB>);
-  const size_t smem = static_cast<size_t>(i8_mma_smem());
+  const size_t smem = static_cast<size_t>(i8_mma_smem(NB));
   cudaError_t e = cudaSuccess;
   const int ctas = resident_ctas(fn, kI8Threads, smem, &e);
   if (e != cudaSuccess) return DSPARK_ERR_CUDA;

@@ -120,6 +120,31 @@ __device__ __forceinline__ void tc_fence_after() {
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
 }
 
+// The CTA's tensor memory: all 512 columns (one CTA per SM), allocated by one warp, which
+// writes the base address to *slot; freed by one warp once every MMA and load is done.
+__device__ __forceinline__ void tmem_alloc_all(uint32_t* slot) {
+  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                   smem_u32(slot)),
+               "r"(kMmaTmemCols)
+               : "memory");
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  tc_fence_before();
+}
+__device__ __forceinline__ void tmem_free_all(uint32_t base) {
+  tc_fence_after();
+  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(base),
+               "r"(kMmaTmemCols)
+               : "memory");
+}
+
+// After an abort: wait (about a second at most) for the phase of the given parity of `bar` to
+// complete, i.e. for the asynchronous copy or the MMAs it tracks to land.
+__device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity) {
+  const long long t0 = clock64();
+  while (!mbar_try(bar, parity) && clock64() - t0 < (1ll << 31)) {
+  }
+}
+
 // Shared-memory matrix descriptor of a K-major operand in the 128-byte swizzle layout: rows of
 // 128 bytes, 8-row groups 1024 bytes apart (the group stride), the 16-byte chunk c of row r
 // stored at chunk c ^ (r % 8); the group base is 1024-byte aligned. A K step of 16 halves
@@ -361,14 +386,7 @@ __global__ void __launch_bounds__(kMmaThreads, 1)
     *s_abort = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
-  if (wi == 0) {
-    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
-                     smem_u32(s_tmem)),
-                 "r"(kMmaTmemCols)
-                 : "memory");
-    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
-    tc_fence_before();
-  }
+  if (wi == 0) tmem_alloc_all(s_tmem);
   __syncthreads();  // barriers initialised, tensor memory allocated
 
   grid_dependency_wait();  // h comes from the kernel before (programmatic launch)
@@ -394,10 +412,7 @@ __global__ void __launch_bounds__(kMmaThreads, 1)
         // let the copies in flight land before the CTA's shared memory goes away
         for (int j = armed - kRaw < 0 ? 0 : armed - kRaw; j < armed; ++j) {
           if (withhold && j == 0) continue;
-          const uint32_t bar = smem_u32(&raw_full[j % kRaw]);
-          const long long t0 = clock64();
-          while (!mbar_try(bar, (j / kRaw) & 1) && clock64() - t0 < (1ll << 31)) {
-          }
+          drain_wait(smem_u32(&raw_full[j % kRaw]), (j / kRaw) & 1);
         }
       }
     }
@@ -438,10 +453,7 @@ __global__ void __launch_bounds__(kMmaThreads, 1)
         if (*s_abort && issued > 0) {
           // the last commit completes once every MMA issued before it has
           const int i = issued - 1;
-          const uint32_t bar = smem_u32(&acc_full[i % kSlots]);
-          const long long t0 = clock64();
-          while (!mbar_try(bar, (i / kSlots) & 1) && clock64() - t0 < (1ll << 31)) {
-          }
+          drain_wait(smem_u32(&acc_full[i % kSlots]), (i / kSlots) & 1);
         }
       }
     } else if (wi < 10) {
@@ -538,12 +550,7 @@ __global__ void __launch_bounds__(kMmaThreads, 1)
   }
 
   __syncthreads();
-  if (wi == 0) {
-    tc_fence_after();
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(*s_tmem),
-                 "r"(kMmaTmemCols)
-                 : "memory");
-  }
+  if (wi == 0) tmem_free_all(*s_tmem);
 }
 
 // ---------------------------------------------------------------- the F16 table
@@ -612,14 +619,7 @@ __global__ void __launch_bounds__(kF16MmaThreads, 1)
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap)) : "memory");
   }
-  if (wi == 0) {
-    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
-                     smem_u32(s_tmem)),
-                 "r"(kMmaTmemCols)
-                 : "memory");
-    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
-    tc_fence_before();
-  }
+  if (wi == 0) tmem_alloc_all(s_tmem);
   __syncthreads();
 
   grid_dependency_wait();  // h comes from the kernel before (programmatic launch)
@@ -643,10 +643,7 @@ __global__ void __launch_bounds__(kF16MmaThreads, 1)
       if (*s_abort) {
         for (int i = armed - kF16Stages < 0 ? 0 : armed - kF16Stages; i < armed; ++i) {
           if (withhold && i == 0) continue;
-          const uint32_t bar = smem_u32(&a_full[i % kF16Stages]);
-          const long long t0 = clock64();
-          while (!mbar_try(bar, (i / kF16Stages) & 1) && clock64() - t0 < (1ll << 31)) {
-          }
+          drain_wait(smem_u32(&a_full[i % kF16Stages]), (i / kF16Stages) & 1);
         }
       }
     }
@@ -684,10 +681,7 @@ __global__ void __launch_bounds__(kF16MmaThreads, 1)
           last = j;
         }
         if (*s_abort && last >= 0) {
-          const uint32_t bar = smem_u32(&acc_full[last % kSlots]);
-          const long long t0 = clock64();
-          while (!mbar_try(bar, (last / kSlots) & 1) && clock64() - t0 < (1ll << 31)) {
-          }
+          drain_wait(smem_u32(&acc_full[last % kSlots]), (last / kSlots) & 1);
         }
       }
     } else {
@@ -723,12 +717,7 @@ __global__ void __launch_bounds__(kF16MmaThreads, 1)
   }
 
   __syncthreads();
-  if (wi == 0) {
-    tc_fence_after();
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(*s_tmem),
-                 "r"(kMmaTmemCols)
-                 : "memory");
-  }
+  if (wi == 0) tmem_free_all(*s_tmem);
 }
 
 // ---------------------------------------------------------------- Q8_0, few states, int8
@@ -736,31 +725,34 @@ __global__ void __launch_bounds__(kF16MmaThreads, 1)
 // The Q8_0 mat-vec for 1 to 5 states on the integer tensor cores (kind::i8), with no
 // conversion: the table bytes are the A operand as stored. TMA copies each tile's 272-byte rows
 // in 3 windows of 128 bytes (128 rows x 128 bytes, 128-byte swizzle; the bytes past 272 read as
-// zeros) into one shared stage. Block j of a row (scale bytes 34 j, 34 j + 1, then 32 signed
-// bytes) lies in the 32-byte K steps k0 = floor(34 j / 32) and k0 + 1; its MMA pair multiplies
-// both steps by B operands that hold the state's digits at the block's 32 byte positions and
-// zeros elsewhere (so the scale bytes and the neighbouring blocks drop out), into the block's
-// own 16 int32 columns: column 3 s + p is plane p of state s (three signed-byte digit planes
-// per state and block, as in the CUDA-core kernel). The sums are exact. The epilogue (thread =
-// row = TMEM lane) reads the block's scale d from the staged bytes and adds
+// zeros) into one shared stage, and 9 MMAs (one per 32-byte K step) accumulate the whole row
+// into one set of int32 columns: column j 3 NB + p NB + s belongs to block j, digit plane p,
+// state s (three signed-byte digit planes per state and block, as in the CUDA-core kernel).
+// B column (j, p, s) holds those digits at block j's 32 byte positions (34 j + 2 ..) and zeros
+// everywhere else, so each column sums block j's products alone: the scale bytes and the other
+// blocks drop out, and the sums are exact. The epilogue (thread = row = TMEM lane) reads each
+// block's scale d from the staged bytes and adds
 //   d 2^(x_sj - X_s) (A + (B + C / 254) / 254)
 // over the 8 blocks (x_sj the block's digit exponent, X_s the state's largest), then writes
-// 2^X_s times the sum. One CTA per SM, 6 warps: warp 0 one lane issues the TMA copies (4 tile
-// stages, 192 KB), warp 1 one lane the 16 MMAs per tile and their commit, warps 2-5 the
-// epilogue, which also releases the stage (its scale bytes are read there); warps 1-5 build the
-// digits first.
+// 2^X_s times the sum. One CTA per SM, 6 warps: warp 0 one lane issues the TMA copies (3-4
+// tile stages), warp 1 one lane the 9 MMAs per tile and their commit, warps 2-5 the epilogue,
+// which also releases the stage (its scale bytes are read there); warps 1-5 build the digits
+// first.
 constexpr int kI8Threads = 192;
-constexpr int kI8MaxStates = 5;                    // 3 planes x 5 states <= N = 16
-constexpr int kI8N = 16;
+constexpr int kI8MaxStates = 5;
 constexpr int kI8Windows = 3;                      // 128-byte windows per 272-byte row
 constexpr int kI8WinBytes = kMmaRows * 128;        // 16384
 constexpr int kI8TileBytes = kI8Windows * kI8WinBytes;  // 49152
-constexpr int kI8Stages = 4;
-constexpr int kI8BBytes = 8 * 2 * kI8N * 32;       // (block, K step) B operands: 8 KB
-constexpr int kI8Slots = 4;                        // accumulator slots of 8 x 16 columns
+constexpr int kI8KSteps = 9;                       // 32-byte K steps covering 272 bytes
 
-__host__ __device__ constexpr int i8_mma_smem() {
-  return kI8Stages * kI8TileBytes + kI8BBytes + 1024 + 1024;
+// MMA N for NB states (8 blocks x 3 planes x NB, rounded up to 16), its tile stages and
+// accumulator slots in the 512 TMEM columns
+__host__ __device__ constexpr int i8_n(int nb) { return (24 * nb + 15) / 16 * 16; }
+__host__ __device__ constexpr int i8_stages(int nb) { return nb <= 4 ? 4 : 3; }
+__host__ __device__ constexpr int i8_slots(int nb) { return 512 / i8_n(nb) < 4 ? 512 / i8_n(nb) : 4; }
+__host__ __device__ constexpr int i8_b_bytes(int nb) { return kI8KSteps * i8_n(nb) * 32; }
+__host__ __device__ constexpr int i8_mma_smem(int nb) {
+  return i8_stages(nb) * kI8TileBytes + i8_b_bytes(nb) + 1024 + 1024;
 }
 
 // Shared-memory descriptor of a K-major operand in the 32-byte swizzle layout: rows of 32
@@ -812,15 +804,16 @@ template <int NB>
 __global__ void __launch_bounds__(kI8Threads, 1)
     markov_q8_0_i8_kernel(const __grid_constant__ CUtensorMap tmap, int V, const float* h,
                           float* y, int ldy, int withhold) {
-  // TMEM columns read per block (3 NB used) and blocks per load batch (64 registers)
-  constexpr int kLd = NB == 1 ? 4 : (NB == 2 ? 8 : 16);
-  constexpr int kBatch = 64 / kLd < 8 ? 64 / kLd : 8;
+  constexpr int kN = i8_n(NB);
+  constexpr int kStages = i8_stages(NB);
+  constexpr int kSlots = i8_slots(NB);
+  constexpr int kBBytes = i8_b_bytes(NB);
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                            ~static_cast<uintptr_t>(1023));
-  uint8_t* s_a = sm;                                   // kI8Stages x 3 windows x 16 KB
-  uint8_t* s_b = sm + kI8Stages * kI8TileBytes;        // [block][K step 0/1][16 x 32 B]
-  uint64_t* bars = reinterpret_cast<uint64_t*>(s_b + kI8BBytes);
+  uint8_t* s_a = sm;                                   // kStages x 3 windows x 16 KB
+  uint8_t* s_b = sm + kStages * kI8TileBytes;          // [K step][kN x 32 B]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(s_b + kBBytes);
   uint64_t* t_full = bars;          // [4] TMA (expect_tx) + bytes
   uint64_t* t_free = bars + 4;      // [4] the epilogue (128)
   uint64_t* acc_full = bars + 8;    // [4] MMA commit
@@ -844,16 +837,9 @@ __global__ void __launch_bounds__(kI8Threads, 1)
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap)) : "memory");
   }
-  if (wi == 0) {
-    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
-                     smem_u32(s_tmem)),
-                 "r"(kMmaTmemCols)
-                 : "memory");
-    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
-    tc_fence_before();
-  }
+  if (wi == 0) tmem_alloc_all(s_tmem);
   // the B operands start as zeros (warps 1-5)
-  for (int i = tid - 32; i >= 0 && i < kI8BBytes / 16; i += kI8Threads - 32)
+  for (int i = tid - 32; i >= 0 && i < kBBytes / 16; i += kI8Threads - 32)
     reinterpret_cast<uint4*>(s_b)[i] = make_uint4(0, 0, 0, 0);
   __syncthreads();
 
@@ -865,8 +851,8 @@ __global__ void __launch_bounds__(kI8Threads, 1)
     if (lane == 0) {
       int armed = 0;
       for (int j = 0; j < my_tiles; ++j) {
-        const int st = j % kI8Stages;
-        if (!mbar_wait(smem_u32(&t_free[st]), ((j / kI8Stages) & 1) ^ 1, s_abort)) break;
+        const int st = j % kStages;
+        if (!mbar_wait(smem_u32(&t_free[st]), ((j / kStages) & 1) ^ 1, s_abort)) break;
         const int t = blockIdx.x + j * gridDim.x;
         if (withhold && j == 0) continue;  // (timeout test: this tile never arrives)
         mbar_arrive_tx(smem_u32(&t_full[st]), kI8TileBytes);
@@ -877,12 +863,9 @@ __global__ void __launch_bounds__(kI8Threads, 1)
         armed = j + 1;
       }
       if (*s_abort) {
-        for (int j = armed - kI8Stages < 0 ? 0 : armed - kI8Stages; j < armed; ++j) {
+        for (int j = armed - kStages < 0 ? 0 : armed - kStages; j < armed; ++j) {
           if (withhold && j == 0) continue;
-          const uint32_t bar = smem_u32(&t_full[j % kI8Stages]);
-          const long long t0 = clock64();
-          while (!mbar_try(bar, (j / kI8Stages) & 1) && clock64() - t0 < (1ll << 31)) {
-          }
+          drain_wait(smem_u32(&t_full[j % kStages]), (j / kStages) & 1);
         }
       }
     }
@@ -917,12 +900,14 @@ __global__ void __launch_bounds__(kI8Threads, 1)
       const float r1 = __fmul_rn(__fsub_rn(v, a), 254.f);
       const float bb = rintf(r1);
       const float c = rintf(__fmul_rn(__fsub_rn(r1, bb), 254.f));
-      // element lane of block j is table byte g = 34 j + 2 + lane: K step g / 32, byte g % 32
-      const int g = 34 * j + 2 + lane, w = (g >> 5) - (34 * j >> 5);
-      uint8_t* bm = s_b + (j * 2 + w) * (kI8N * 32);
-      bm[sw32_off(3 * st + 0, g & 31)] = static_cast<uint8_t>(static_cast<int8_t>(a));
-      bm[sw32_off(3 * st + 1, g & 31)] = static_cast<uint8_t>(static_cast<int8_t>(bb));
-      bm[sw32_off(3 * st + 2, g & 31)] = static_cast<uint8_t>(static_cast<int8_t>(c));
+      // element lane of block j is table byte g = 34 j + 2 + lane: K step g / 32, byte g % 32;
+      // B columns j 3 NB + p NB + st
+      const int g = 34 * j + 2 + lane;
+      uint8_t* bm = s_b + (g >> 5) * (kN * 32);
+      const int n0 = j * 3 * NB + st;
+      bm[sw32_off(n0, g & 31)] = static_cast<uint8_t>(static_cast<int8_t>(a));
+      bm[sw32_off(n0 + NB, g & 31)] = static_cast<uint8_t>(static_cast<int8_t>(bb));
+      bm[sw32_off(n0 + 2 * NB, g & 31)] = static_cast<uint8_t>(static_cast<int8_t>(c));
       if (lane == 0) s_x[st * 8 + j] = m <= 3.402823466e38f ? x : 1024;  // 1024: non-finite
     }
     fence_proxy_async_smem();
@@ -932,34 +917,24 @@ __global__ void __launch_bounds__(kI8Threads, 1)
     if (wi == 1) {
       // ---- MMA issuer: per tile, per block, its two 32-byte K steps into the block's columns
       if (lane == 0) {
-        constexpr uint32_t idesc = mma_idesc_s8(kI8N);
+        constexpr uint32_t idesc = mma_idesc_s8(kN);
         const uint32_t b0 = smem_u32(s_b);
         int last = -1;
         for (int j = 0; j < my_tiles; ++j) {
-          const int st = j % kI8Stages, ts = j % kI8Slots;
-          if (!mbar_wait(smem_u32(&t_full[st]), (j / kI8Stages) & 1, s_abort)) break;
-          if (!mbar_wait(smem_u32(&acc_empty[ts]), ((j / kI8Slots) & 1) ^ 1, s_abort)) break;
+          const int st = j % kStages, ts = j % kSlots;
+          if (!mbar_wait(smem_u32(&t_full[st]), (j / kStages) & 1, s_abort)) break;
+          if (!mbar_wait(smem_u32(&acc_empty[ts]), ((j / kSlots) & 1) ^ 1, s_abort)) break;
           tc_fence_after();
           const uint32_t a0 = smem_u32(s_a + st * kI8TileBytes);
 #pragma unroll
-          for (int blk = 0; blk < kQ8Blocks; ++blk) {
-            const int k0 = 34 * blk >> 5;
-#pragma unroll
-            for (int w = 0; w < 2; ++w) {
-              const int k = k0 + w;  // 32-byte K step: window k / 4, 32 (k % 4) bytes in
-              mma_s8(tbase + ts * (kQ8Blocks * kI8N) + blk * kI8N,
-                     sw128_desc(a0 + (k >> 2) * kI8WinBytes + 32 * (k & 3)),
-                     sw32_desc(b0 + (blk * 2 + w) * (kI8N * 32)), idesc, w);
-            }
-          }
+          for (int k = 0; k < kI8KSteps; ++k)  // K step k: window k / 4, 32 (k % 4) bytes in
+            mma_s8(tbase + ts * kN, sw128_desc(a0 + (k >> 2) * kI8WinBytes + 32 * (k & 3)),
+                   sw32_desc(b0 + k * (kN * 32)), idesc, k != 0);
           mma_commit(smem_u32(&acc_full[ts]));
           last = j;
         }
         if (*s_abort && last >= 0) {
-          const uint32_t bar = smem_u32(&acc_full[last % kI8Slots]);
-          const long long t0 = clock64();
-          while (!mbar_try(bar, (last / kI8Slots) & 1) && clock64() - t0 < (1ll << 31)) {
-          }
+          drain_wait(smem_u32(&acc_full[last % kSlots]), (last / kSlots) & 1);
         }
       }
     } else {
@@ -982,48 +957,38 @@ __global__ void __launch_bounds__(kI8Threads, 1)
         }
       }
       for (int j = 0; j < my_tiles; ++j) {
-        const int st = j % kI8Stages, ts = j % kI8Slots;
+        const int st = j % kStages, ts = j % kSlots;
         if (!__all_sync(0xffffffffu,
-                        mbar_wait(smem_u32(&acc_full[ts]), (j / kI8Slots) & 1, s_abort)))
+                        mbar_wait(smem_u32(&acc_full[ts]), (j / kSlots) & 1, s_abort)))
           break;
         tc_fence_after();
-        const uint32_t ta =
-            tbase + (static_cast<uint32_t>(32 * q) << 16) + ts * (kQ8Blocks * kI8N);
+        const uint32_t ta = tbase + (static_cast<uint32_t>(32 * q) << 16) + ts * kN;
         const uint8_t* tile = s_a + st * kI8TileBytes;
+        float v[kN];
+#pragma unroll
+        for (int c = 0; c < kN; c += 16) tmem_ld16(ta + c, v + c);
+        float dd[kQ8Blocks];
+#pragma unroll
+        for (int blk = 0; blk < kQ8Blocks; ++blk) {
+          // the block's scale: bytes 34 blk .. 34 blk + 1 (even; one 16-byte chunk)
+          const int o = 34 * blk;
+          dd[blk] = __half2float(*reinterpret_cast<const __half*>(
+              tile + (o >> 7) * kI8WinBytes + sw128_off(r, o & 127)));
+        }
+        tmem_ld_wait();
         float acc[NB];
 #pragma unroll
         for (int s2 = 0; s2 < NB; ++s2) acc[s2] = 0.f;
 #pragma unroll
-        for (int b0 = 0; b0 < kQ8Blocks; b0 += kBatch) {
-          float v[kBatch][kLd];
-          float dd[kBatch];
+        for (int blk = 0; blk < kQ8Blocks; ++blk) {
 #pragma unroll
-          for (int u = 0; u < kBatch; ++u) {
-            if constexpr (kLd == 4)
-              tmem_ld4(ta + (b0 + u) * kI8N, v[u]);
-            else if constexpr (kLd == 8)
-              tmem_ld8(ta + (b0 + u) * kI8N, v[u]);
-            else
-              tmem_ld16(ta + (b0 + u) * kI8N, v[u]);
-          }
-#pragma unroll
-          for (int u = 0; u < kBatch; ++u) {
-            // the block's scale: bytes 34 blk .. 34 blk + 1 (even; one 16-byte chunk)
-            const int o = 34 * (b0 + u);
-            dd[u] = __half2float(*reinterpret_cast<const __half*>(
-                tile + (o >> 7) * kI8WinBytes + sw128_off(r, o & 127)));
-          }
-          tmem_ld_wait();
-#pragma unroll
-          for (int u = 0; u < kBatch; ++u) {
-#pragma unroll
-            for (int s2 = 0; s2 < NB; ++s2) {
-              const int A = __float_as_int(v[u][3 * s2]), Bv = __float_as_int(v[u][3 * s2 + 1]),
-                        C = __float_as_int(v[u][3 * s2 + 2]);
-              float f = __fmaf_rn(small_int_to_float(C), 1.f / 254.f, small_int_to_float(Bv));
-              f = __fmaf_rn(f, 1.f / 254.f, small_int_to_float(A));
-              acc[s2] = __fmaf_rn(__fmul_rn(dd[u], gf[s2][b0 + u]), f, acc[s2]);
-            }
+          for (int s2 = 0; s2 < NB; ++s2) {
+            const int c0 = blk * 3 * NB + s2;
+            const int A = __float_as_int(v[c0]), Bv = __float_as_int(v[c0 + NB]),
+                      C = __float_as_int(v[c0 + 2 * NB]);
+            float f = __fmaf_rn(small_int_to_float(C), 1.f / 254.f, small_int_to_float(Bv));
+            f = __fmaf_rn(f, 1.f / 254.f, small_int_to_float(A));
+            acc[s2] = __fmaf_rn(__fmul_rn(dd[blk], gf[s2][blk]), f, acc[s2]);
           }
         }
         tc_fence_before();
@@ -1041,12 +1006,7 @@ __global__ void __launch_bounds__(kI8Threads, 1)
   }
 
   __syncthreads();
-  if (wi == 0) {
-    tc_fence_after();
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(*s_tmem),
-                 "r"(kMmaTmemCols)
-                 : "memory");
-  }
+  if (wi == 0) tmem_free_all(*s_tmem);
 }
 
 }  // namespace dspark
