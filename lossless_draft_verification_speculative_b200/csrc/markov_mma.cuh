@@ -1,9 +1,13 @@
-// The Markov-head mat-vec y[b, v] = sum_k W[v, k] h[b, k] over a GGUF Q8_0 table, on the
-// fifth-generation tensor cores (tcgen05), for 1 to 64 states per launch with one read of the
-// table (the DeepSeek-V4-Flash DSpark drafter card, "Files": markov_w2 in Q8_0, 8 blocks of
-// 34 bytes per row of R = 256; the engine reads it four times per draft block).
+// The Markov-head mat-vec y[b, v] = sum_k W[v, k] h[b, k] on the fifth-generation tensor cores
+// (tcgen05), with one read of the table per launch (the DeepSeek-V4-Flash DSpark drafter card,
+// "Files": markov_w2 in F16 or Q8_0, 8 blocks of 34 bytes per row of R = 256 in Q8_0; the engine
+// reads it four times per draft block). Three kernels:
+//  - markov_q8_0_mma_kernel (below): Q8_0, up to 64 states, the bytes converted to float16;
+//  - markov_f16_mma_kernel: F16, up to 64 states, the table loaded by TMA as stored;
+//  - markov_q8_0_i8_kernel: Q8_0, up to 5 states, integer MMAs on the bytes as stored.
+// The host (dspark_markov_matvec) picks one by format and number of states.
 //
-// Exact operands. A Q8_0 value is d q with q a signed byte, exact in float16; the block scale
+// markov_q8_0_mma_kernel. Exact operands. A Q8_0 value is d q with q a signed byte, exact in float16; the block scale
 // d is per (row, block of 32), so each block gets its own float32 accumulators and d is
 // applied afterwards. Each state h_b is scaled by a power of two 2^e_b (m_b 2^e_b in
 // [2^14, 2^15), m_b = max_k |h[b, k]|) and split into float16 parts hi + lo, which represent it
