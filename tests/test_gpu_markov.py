@@ -131,3 +131,26 @@ def test_state_scales(fmt, nst):
     assert np.all(err <= bound + 2.0 ** -149)
     assert np.all(y.cpu().numpy()[2] == 0.0)
     assert np.array_equal(y.cpu().numpy()[3].astype(np.float64), W[:, 200] * -3.0)
+
+
+@pytest.mark.parametrize("fmt,B", [("f16", 1), ("f16", 4), ("q8_0", 1), ("q8_0", 3), ("q8_0", 7)])
+def test_nonfinite_states(fmt, B):
+    """A state holding a NaN or an infinity gives non-finite results (on every kernel path:
+    CUDA cores at one state, the tensor-core kernels above); the other states are unaffected."""
+    V = 3000
+    raw = wl.markov_table(V, R, fmt, seed=11)
+    W = mk.f16_table(raw) if fmt == "f16" else mk.q8_0_table(raw, R)
+    H = wl.markov_states(B, R, seed=11)
+    bad = 0
+    H[bad, 5] = np.nan if B % 2 else np.inf
+    t = torch.from_numpy(raw.view(np.int16) if fmt == "f16" else raw).to(DEV)
+    y = bd.markov_matvec(t, fmt, torch.from_numpy(H).to(DEV))
+    torch.cuda.synchronize()
+    y = y.cpu().numpy().astype(np.float64)
+    assert not np.isfinite(y[bad]).any()
+    if B > 1:
+        good = H[1:]
+        ref = mk.markov_matvec(W, good)
+        bound = 2 * R * 2.0 ** -24 * mk.abs_products(W, good) + 1e-30 + \
+            2.0 ** -22 * np.abs(good.astype(np.float64)).max(axis=1)[:, None] * np.abs(W).sum(axis=1)[None, :]
+        assert np.all(np.abs(y[1:] - ref) <= bound)
