@@ -96,3 +96,15 @@ def test_optional_result_fields_may_be_absent():
 def test_greedy_at_zero_temperature_needs_no_uniforms():
     with pytest.raises(RuntimeError, match="CUDA tensors only"):
         _static(T=0.0, uniforms=None, Q=None)
+
+
+def test_markov_wrappers_check_before_launch():
+    """markov_matvec and its test-only withheld variant reject an unknown table format and a
+    table that is not on the GPU before anything reaches the library."""
+    table = torch.zeros(16, 272, dtype=torch.uint8)
+    h = torch.zeros(1, 256, dtype=torch.float32)
+    for fn in (bd.markov_matvec, bd.markov_matvec_withheld):
+        with pytest.raises(ValueError, match="fmt"):
+            fn(table, "q4_0", h)
+        with pytest.raises(ValueError, match="CUDA"):
+            fn(table, "q8_0", h)
