@@ -695,7 +695,7 @@ def time_markov_matvec(dev, n=50, replays=5):
         nbytes = t0.numel() * t0.element_size()
         copies = -(-200_000_000 // nbytes)
         tabs = [t0] + [t0.clone() for _ in range(copies - 1)]
-        for B in (1, 4, 64):
+        for B in (1, 4, 8, 64):
             h = torch.from_numpy(wl.markov_states(B, MARKOV_R)).to(dev)
             y = torch.empty(B, MARKOV_V, device=dev)
             with torch.cuda.stream(stream):

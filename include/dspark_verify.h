@@ -248,11 +248,11 @@ dspark_status_t dspark_early_exit_accept(const void* p1, int64_t ld_p1, const vo
  *    TMA tensor copies): each state scaled by a power of two and split into float16 hi + lo
  *    (within 2^-23 of its largest |h|); the products with the exact table halves are summed
  *    in float32 by the tensor cores, one sum per part over all R values.
- *  Q8_0, B <= 5: one read of the table; exact integer dot products of each block's bytes with
+ *  Q8_0, B <= 10: one read of the table; exact integer dot products of each block's bytes with
  *    three signed-byte digit planes of the state (within 2^-22 of the block's largest |h|),
  *    combined and scaled by d in float32: on the CUDA cores for B == 1, on the integer tensor
- *    cores (tcgen05 kind::i8, the table loaded as stored by TMA) for B = 2..5.
- *  Q8_0, B > 5: on the tensor cores (tcgen05), the table read once per 64 states. Each state is
+ *    cores (tcgen05 kind::i8, the table loaded as stored by TMA) for B = 2..10.
+ *  Q8_0, B > 10: on the tensor cores (tcgen05), the table read once per 64 states. Each state is
  *    scaled by a power of two and split into float16 parts hi + lo (within 2^-23 of its
  *    largest |h|); each block's 32 products q * part are exact and summed in float32 by the
  *    tensor cores, then scaled by d and the 8 blocks added by float32 FMAs in a fixed order.

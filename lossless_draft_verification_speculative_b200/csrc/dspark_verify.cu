@@ -501,9 +501,9 @@ dspark_status_t markov_launch(const void* table, dspark_table_t type, int V, con
 }
 
 // Q8_0 routing by the number of states (measured on a 129280-row table): one state on the
-// CUDA-core kernel (8.0 us; the integer tensor-core kernel takes 10.0), 2 to kI8MaxStates on the
-// integer tensor cores (four states: 10.5 us against 15.3 on the CUDA cores), more on the
-// float16 tensor-core kernel, 64 states per launch.
+// CUDA-core kernel (8.0 us; the integer tensor-core kernel takes 10.0), 2 to kI8MaxStates (10)
+// on the integer tensor cores (four states: 10.5 us against 15.3 on the CUDA cores), more on
+// the float16 tensor-core kernel, 64 states per launch.
 constexpr int kMarkovCudaCoreStates = 1;
 
 // The Q8_0 mat-vec on the tensor cores for nb <= N states (N = 16, 32, 48 or 64): one CTA per
@@ -664,7 +664,12 @@ dspark_status_t markov_matvec_impl(const void* table, dspark_table_t type, int V
       case 2: return markov_i8_launch<2>(table, V, h, y, V, s, withhold);
       case 3: return markov_i8_launch<3>(table, V, h, y, V, s, withhold);
       case 4: return markov_i8_launch<4>(table, V, h, y, V, s, withhold);
-      default: return markov_i8_launch<5>(table, V, h, y, V, s, withhold);
+      case 5: return markov_i8_launch<5>(table, V, h, y, V, s, withhold);
+      case 6: return markov_i8_launch<6>(table, V, h, y, V, s, withhold);
+      case 7: return markov_i8_launch<7>(table, V, h, y, V, s, withhold);
+      case 8: return markov_i8_launch<8>(table, V, h, y, V, s, withhold);
+      case 9: return markov_i8_launch<9>(table, V, h, y, V, s, withhold);
+      default: return markov_i8_launch<10>(table, V, h, y, V, s, withhold);
     }
   }
   if (type == DSPARK_TABLE_Q8_0 && B > kMarkovCudaCoreStates) {

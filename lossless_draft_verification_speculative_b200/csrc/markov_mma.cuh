@@ -4,7 +4,7 @@
 // reads it four times per draft block). Three kernels:
 //  - markov_q8_0_mma_kernel (below): Q8_0, up to 64 states, the bytes converted to float16;
 //  - markov_f16_mma_kernel: F16, up to 64 states, the table loaded by TMA as stored;
-//  - markov_q8_0_i8_kernel: Q8_0, up to 5 states, integer MMAs on the bytes as stored.
+//  - markov_q8_0_i8_kernel: Q8_0, up to 10 states, integer MMAs on the bytes as stored.
 // The host (dspark_markov_matvec) picks one by format and number of states.
 //
 // markov_q8_0_mma_kernel. Exact operands. A Q8_0 value is d q with q a signed byte, exact in float16; the block scale
@@ -726,12 +726,13 @@ __global__ void __launch_bounds__(kF16MmaThreads, 1)
 
 // ---------------------------------------------------------------- Q8_0, few states, int8
 
-// The Q8_0 mat-vec for 1 to 5 states on the integer tensor cores (kind::i8), with no
+// The Q8_0 mat-vec for 1 to 10 states on the integer tensor cores (kind::i8), with no
 // conversion: the table bytes are the A operand as stored. TMA copies each tile's 272-byte rows
 // in 3 windows of 128 bytes (128 rows x 128 bytes, 128-byte swizzle; the bytes past 272 read as
 // zeros) into one shared stage, and 9 MMAs (one per 32-byte K step) accumulate the whole row
-// into one set of int32 columns: column j 3 NB + p NB + s belongs to block j, digit plane p,
-// state s (three signed-byte digit planes per state and block, as in the CUDA-core kernel).
+// into one set of int32 columns: column j G + p NB + s belongs to block j, digit plane p,
+// state s (three signed-byte digit planes per state and block, as in the CUDA-core kernel;
+// G = 3 NB, or 3 NB rounded up to 8 beyond 5 states).
 // B column (j, p, s) holds those digits at block j's 32 byte positions (34 j + 2 ..) and zeros
 // everywhere else, so each column sums block j's products alone: the scale bytes and the other
 // blocks drop out, and the sums are exact. The epilogue (thread = row = TMEM lane) reads each
@@ -743,15 +744,19 @@ __global__ void __launch_bounds__(kF16MmaThreads, 1)
 // which also releases the stage (its scale bytes are read there); warps 1-5 build the digits
 // first.
 constexpr int kI8Threads = 192;
-constexpr int kI8MaxStates = 5;
+constexpr int kI8MaxStates = 10;
 constexpr int kI8Windows = 3;                      // 128-byte windows per 272-byte row
 constexpr int kI8WinBytes = kMmaRows * 128;        // 16384
 constexpr int kI8TileBytes = kI8Windows * kI8WinBytes;  // 49152
 constexpr int kI8KSteps = 9;                       // 32-byte K steps covering 272 bytes
 
-// MMA N for NB states (8 blocks x 3 planes x NB, rounded up to 16), its tile stages and
-// accumulator slots in the 512 TMEM columns
-__host__ __device__ constexpr int i8_n(int nb) { return (24 * nb + 15) / 16 * 16; }
+// Columns per block: 3 NB (up to 5 states, blocks packed), else 3 NB rounded up to 8 (so each
+// block's columns load as whole 8-column groups); MMA N for NB states (8 blocks, rounded up to
+// 16), its tile stages and accumulator slots in the 512 TMEM columns
+__host__ __device__ constexpr int i8_g(int nb) { return nb <= 5 ? 3 * nb : (3 * nb + 7) / 8 * 8; }
+__host__ __device__ constexpr int i8_n(int nb) {
+  return nb <= 5 ? (24 * nb + 15) / 16 * 16 : 8 * i8_g(nb);
+}
 __host__ __device__ constexpr int i8_stages(int nb) { return nb <= 4 ? 4 : 3; }
 __host__ __device__ constexpr int i8_slots(int nb) { return 512 / i8_n(nb) < 4 ? 512 / i8_n(nb) : 4; }
 __host__ __device__ constexpr int i8_b_bytes(int nb) { return kI8KSteps * i8_n(nb) * 32; }
@@ -809,6 +814,7 @@ __global__ void __launch_bounds__(kI8Threads, 1)
     markov_q8_0_i8_kernel(const __grid_constant__ CUtensorMap tmap, int V, const float* h,
                           float* y, int ldy, int withhold) {
   constexpr int kN = i8_n(NB);
+  constexpr int kG = i8_g(NB);
   constexpr int kStages = i8_stages(NB);
   constexpr int kSlots = i8_slots(NB);
   constexpr int kBBytes = i8_b_bytes(NB);
@@ -824,7 +830,7 @@ __global__ void __launch_bounds__(kI8Threads, 1)
   uint64_t* acc_empty = bars + 12;  // [4] the epilogue (128)
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(bars + 16);
   volatile int* s_abort = reinterpret_cast<volatile int*>(bars + 17);
-  int* s_x = reinterpret_cast<int*>(bars + 18);        // [5][8] block exponents
+  int* s_x = reinterpret_cast<int*>(bars + 18);        // [NB][8] block exponents
 
   const int tid = threadIdx.x, wi = tid >> 5, lane = tid & 31;
   const int n_tiles = (V + kMmaRows - 1) / kMmaRows;
@@ -905,10 +911,10 @@ __global__ void __launch_bounds__(kI8Threads, 1)
       const float bb = rintf(r1);
       const float c = rintf(__fmul_rn(__fsub_rn(r1, bb), 254.f));
       // element lane of block j is table byte g = 34 j + 2 + lane: K step g / 32, byte g % 32;
-      // B columns j 3 NB + p NB + st
+      // B columns j kG + p NB + st
       const int g = 34 * j + 2 + lane;
       uint8_t* bm = s_b + (g >> 5) * (kN * 32);
-      const int n0 = j * 3 * NB + st;
+      const int n0 = j * kG + st;
       bm[sw32_off(n0, g & 31)] = static_cast<uint8_t>(static_cast<int8_t>(a));
       bm[sw32_off(n0 + NB, g & 31)] = static_cast<uint8_t>(static_cast<int8_t>(bb));
       bm[sw32_off(n0 + 2 * NB, g & 31)] = static_cast<uint8_t>(static_cast<int8_t>(c));
@@ -945,19 +951,23 @@ __global__ void __launch_bounds__(kI8Threads, 1)
       // ---- epilogue: thread = tile row = TMEM lane
       const int q = wi & 3;
       const int r = 32 * q + lane;
-      // per state: X_s and the block factors 2^(x_sj - X_s) (0 below 2^-126)
+      // per state: X_s and (up to 5 states, in registers) the block factors 2^(x_sj - X_s)
+      // (0 below 2^-126)
       int X[NB];
-      float gf[NB][kQ8Blocks];
+      constexpr int kGf = NB <= 5 ? NB : 1;
+      float gf[kGf][kQ8Blocks];
 #pragma unroll
       for (int s2 = 0; s2 < NB; ++s2) {
         int mx = s_x[s2 * 8];
 #pragma unroll
         for (int j = 1; j < kQ8Blocks; ++j) mx = max(mx, s_x[s2 * 8 + j]);
         X[s2] = mx;
+        if constexpr (NB <= 5) {
 #pragma unroll
-        for (int j = 0; j < kQ8Blocks; ++j) {
-          const int dx = s_x[s2 * 8 + j] - mx;
-          gf[s2][j] = dx >= -126 ? pow2f(dx) : 0.f;
+          for (int j = 0; j < kQ8Blocks; ++j) {
+            const int dx = s_x[s2 * 8 + j] - mx;
+            gf[s2][j] = dx >= -126 ? pow2f(dx) : 0.f;
+          }
         }
       }
       for (int j = 0; j < my_tiles; ++j) {
@@ -968,9 +978,6 @@ __global__ void __launch_bounds__(kI8Threads, 1)
         tc_fence_after();
         const uint32_t ta = tbase + (static_cast<uint32_t>(32 * q) << 16) + ts * kN;
         const uint8_t* tile = s_a + st * kI8TileBytes;
-        float v[kN];
-#pragma unroll
-        for (int c = 0; c < kN; c += 16) tmem_ld16(ta + c, v + c);
         float dd[kQ8Blocks];
 #pragma unroll
         for (int blk = 0; blk < kQ8Blocks; ++blk) {
@@ -979,20 +986,40 @@ __global__ void __launch_bounds__(kI8Threads, 1)
           dd[blk] = __half2float(*reinterpret_cast<const __half*>(
               tile + (o >> 7) * kI8WinBytes + sw128_off(r, o & 127)));
         }
-        tmem_ld_wait();
         float acc[NB];
 #pragma unroll
         for (int s2 = 0; s2 < NB; ++s2) acc[s2] = 0.f;
+        // block blk's plane digits of state s2, as integers, into acc
+        auto add_block = [&](const float* vb, int blk, float gfac, int s2) {
+          const int A = __float_as_int(vb[s2]), Bv = __float_as_int(vb[s2 + NB]),
+                    C = __float_as_int(vb[s2 + 2 * NB]);
+          float f = __fmaf_rn(small_int_to_float(C), 1.f / 254.f, small_int_to_float(Bv));
+          f = __fmaf_rn(f, 1.f / 254.f, small_int_to_float(A));
+          acc[s2] = __fmaf_rn(__fmul_rn(dd[blk], gfac), f, acc[s2]);
+        };
+        if constexpr (NB <= 5) {
+          // every column at once, one wait
+          float v[kN];
 #pragma unroll
-        for (int blk = 0; blk < kQ8Blocks; ++blk) {
+          for (int c = 0; c < kN; c += 16) tmem_ld16(ta + c, v + c);
+          tmem_ld_wait();
 #pragma unroll
-          for (int s2 = 0; s2 < NB; ++s2) {
-            const int c0 = blk * 3 * NB + s2;
-            const int A = __float_as_int(v[c0]), Bv = __float_as_int(v[c0 + NB]),
-                      C = __float_as_int(v[c0 + 2 * NB]);
-            float f = __fmaf_rn(small_int_to_float(C), 1.f / 254.f, small_int_to_float(Bv));
-            f = __fmaf_rn(f, 1.f / 254.f, small_int_to_float(A));
-            acc[s2] = __fmaf_rn(__fmul_rn(dd[blk], gf[s2][blk]), f, acc[s2]);
+          for (int blk = 0; blk < kQ8Blocks; ++blk)
+#pragma unroll
+            for (int s2 = 0; s2 < NB; ++s2) add_block(v + blk * kG, blk, gf[s2][blk], s2);
+        } else {
+          // block by block: its kG columns as 8-column loads, one wait each
+#pragma unroll
+          for (int blk = 0; blk < kQ8Blocks; ++blk) {
+            float v[kG];
+#pragma unroll
+            for (int c = 0; c < kG; c += 8) tmem_ld8(ta + blk * kG + c, v + c);
+            tmem_ld_wait();
+#pragma unroll
+            for (int s2 = 0; s2 < NB; ++s2) {
+              const int dx = s_x[s2 * 8 + blk] - X[s2];
+              add_block(v, blk, dx >= -126 ? pow2f(dx) : 0.f, s2);
+            }
           }
         }
         tc_fence_before();
