@@ -466,18 +466,17 @@ dspark_status_t static_scratch_address(void** addr) {
   return DSPARK_OK;
 }
 
-// The Markov-head mat-vec for up to kMarkovMaxStates states per launch.
-template <int NB>
+// The Markov-head mat-vec for one state on the CUDA cores.
 dspark_status_t markov_launch(const void* table, dspark_table_t type, int V, const float* h,
-                              float* y, int ldy, cudaStream_t stream) {
+                              float* y, cudaStream_t stream) {
   const bool q8 = type == DSPARK_TABLE_Q8_0;
-  const void* fn = q8 ? reinterpret_cast<const void*>(&markov_q8_0_kernel<NB>)
-                      : reinterpret_cast<const void*>(&markov_f16_kernel<NB>);
+  const void* fn = q8 ? reinterpret_cast<const void*>(&markov_q8_0_kernel)
+                      : reinterpret_cast<const void*>(&markov_f16_kernel);
   cudaError_t e = cudaSuccess;
   const int ctas = resident_ctas(fn, kMarkovThreads, 0, &e);
   if (e != cudaSuccess) return DSPARK_ERR_CUDA;
   if (ctas < 1) return DSPARK_ERR_UNSUPPORTED;
-  const long long rows_per_cta = (kMarkovThreads / 32) * (q8 ? kQ8Rows : (NB == 1 ? 8 : 4));
+  const long long rows_per_cta = (kMarkovThreads / 32) * (q8 ? kQ8Rows : 8);
   const long long want = (V + rows_per_cta - 1) / rows_per_cta;
   const int grid = static_cast<int>(want < ctas ? want : ctas);
   cudaLaunchAttribute attr[1];
@@ -491,11 +490,11 @@ dspark_status_t markov_launch(const void* table, dspark_table_t type, int V, con
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   if (q8) {
-    e = cudaLaunchKernelEx(&cfg, markov_q8_0_kernel<NB>, static_cast<const uint8_t*>(table), V,
-                           h, y, ldy);
+    e = cudaLaunchKernelEx(&cfg, markov_q8_0_kernel, static_cast<const uint8_t*>(table), V, h,
+                           y);
   } else {
-    e = cudaLaunchKernelEx(&cfg, markov_f16_kernel<NB>, static_cast<const uint16_t*>(table), V,
-                           h, y, ldy);
+    e = cudaLaunchKernelEx(&cfg, markov_f16_kernel, static_cast<const uint16_t*>(table), V, h,
+                           y);
   }
   return e == cudaSuccess ? DSPARK_OK : DSPARK_ERR_CUDA;
 }
@@ -598,9 +597,9 @@ dspark_status_t markov_f16_mma_launch(const void* table, int V, const float* h, 
   return e == cudaSuccess ? DSPARK_OK : DSPARK_ERR_CUDA;
 }
 
-// The Q8_0 mat-vec on the integer tensor cores for NB <= 5 states: a tensor map over the
-// V x 272-byte table (boxes of 128 rows x 128 bytes, 128-byte swizzle, bytes past the row and
-// rows past V read as zeros).
+// The Q8_0 mat-vec on the integer tensor cores for NB <= kI8MaxStates states: a tensor map
+// over the V x 272-byte table (boxes of 128 rows x 128 bytes, 128-byte swizzle, bytes past the
+// row and rows past V read as zeros).
 template <int NB>
 dspark_status_t markov_i8_launch(const void* table, int V, const float* h, float* y, int ldy,
                                  cudaStream_t stream, int withhold) {
@@ -660,7 +659,6 @@ dspark_status_t markov_matvec_impl(const void* table, dspark_table_t type, int V
     return DSPARK_ERR_UNSUPPORTED;
   if (type == DSPARK_TABLE_Q8_0 && B > kMarkovCudaCoreStates && B <= kI8MaxStates) {
     switch (B) {
-      case 1: return markov_i8_launch<1>(table, V, h, y, V, s, withhold);
       case 2: return markov_i8_launch<2>(table, V, h, y, V, s, withhold);
       case 3: return markov_i8_launch<3>(table, V, h, y, V, s, withhold);
       case 4: return markov_i8_launch<4>(table, V, h, y, V, s, withhold);
@@ -708,20 +706,8 @@ dspark_status_t markov_matvec_impl(const void* table, dspark_table_t type, int V
     }
     return DSPARK_OK;
   }
-  for (int b0 = 0; b0 < B; b0 += kMarkovMaxStates) {
-    const int nb = B - b0 < kMarkovMaxStates ? B - b0 : kMarkovMaxStates;
-    const float* hb = h + static_cast<size_t>(b0) * R;
-    float* yb = y + static_cast<size_t>(b0) * V;
-    dspark_status_t st;
-    switch (nb) {
-      case 1: st = markov_launch<1>(table, type, V, hb, yb, V, s); break;
-      case 2: st = markov_launch<2>(table, type, V, hb, yb, V, s); break;
-      case 3: st = markov_launch<3>(table, type, V, hb, yb, V, s); break;
-      default: st = markov_launch<4>(table, type, V, hb, yb, V, s); break;
-    }
-    if (st != DSPARK_OK) return st;
-  }
-  return DSPARK_OK;
+  // one state (B == 1 here)
+  return markov_launch(table, type, V, h, y, s);
 }
 }  // namespace
 }  // namespace dspark

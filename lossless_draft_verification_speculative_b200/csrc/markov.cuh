@@ -2,17 +2,14 @@
 // markov_w2 (V rows of R = 256 values; the DeepSeek-V4-Flash DSpark drafter card ships it in
 // F16 or in GGUF Q8_0 and says the ds4 engine reads it in full four times per draft block).
 //
-// The table is read once per call; the work per byte is a few multiply-adds, so the kernel is
-// an HBM stream. One CTA of 8 warps per resident slot walks groups of rows grid-stride; a warp
-// keeps a group's loads in flight together:
-//  - F16: a row is 512 bytes, one 16-byte piece (8 halves) per lane; 8 rows per group (4 with
-//    several states: with 2 states, 8 rows took 15.1 us per 129280-row call and 4 rows 12.7). Lane l holds h[b, 8l .. 8l+7] in registers and multiplies its pieces.
-//    With one state each row's 32 partial sums are added by its own butterfly (8 independent
-//    chains); with more, the group's (row, state) partial sums are added by one transposed
-//    butterfly (each round halves the values a lane carries): 2 states x 4 rows cost 9
-//    shuffles instead of 40. With 3 or 4 states the products run as packed f32x2 FMAs (even
-//    and odd elements in the two halves of the accumulator).
-//  - Q8_0 (one state; more take the tensor-core kernels): a row is 8 blocks of 34 bytes
+// These are the one-state kernels (several states take the tensor-core kernels). The table is
+// read once per call; the work per byte is a few multiply-adds, so the kernel is an HBM
+// stream. One CTA of 8 warps per resident slot walks groups of rows grid-stride; a warp keeps
+// a group's loads in flight together:
+//  - F16: a row is 512 bytes, one 16-byte piece (8 halves) per lane; 8 rows per group. Lane l
+//    holds h[8l .. 8l+7] in registers and multiplies its pieces; each row's 32 partial sums are
+//    added by its own butterfly (8 independent chains).
+//  - Q8_0: a row is 8 blocks of 34 bytes
 //    (272 bytes, so rows start 16-byte aligned). A group of 8 consecutive rows (2176 bytes) is
 //    copied by 16-byte asynchronous copies into one of the warp's two shared buffers, so the
 //    next group is in flight while the warp decodes this one; lane l decodes blocks (row l/8,
@@ -34,7 +31,6 @@ namespace dspark {
 
 constexpr int kMarkovRank = 256;     // R: the only rank the drafters ship
 constexpr int kMarkovThreads = 256;  // 8 warps per CTA
-constexpr int kMarkovMaxStates = 4;  // states per launch (the host splits larger batches)
 constexpr int kQ8RowBytes = kMarkovRank / 32 * 34;  // 272
 constexpr int kQ8Rows = 8;                          // rows per warp group (Q8_0)
 
@@ -49,57 +45,21 @@ __device__ __forceinline__ void unpack_f16x8(const uint4& w, float* f) {
   }
 }
 
-__host__ __device__ constexpr int pow2_ceil(int x) { return x <= 1 ? 1 : 2 * pow2_ceil((x + 1) / 2); }
-
-// Warp sum of M values per lane (M a power of two <= 32), transposed: in round t (t < log2 M)
-// lanes exchange half of their values with the lane 16 >> t away and keep the sums of the
-// other half, then the last rounds add a single value. Lane l ends with the total over the
-// warp of value index sum_t (bit (4 - t) of l) * (M >> (t + 1)); every lane that shares those
-// bits holds the same total.
-template <int M>
-__device__ __forceinline__ float warp_transpose_sum(float (&v)[M], int lane) {
-  int off = 16;
-#pragma unroll
-  for (int half = M / 2; half >= 1; half /= 2, off >>= 1) {
-    const bool upper = (lane & off) != 0;
-#pragma unroll
-    for (int j = 0; j < half; ++j) {
-      const float keep = upper ? v[j + half] : v[j];
-      const float give = upper ? v[j] : v[j + half];
-      v[j] = __fadd_rn(keep, __shfl_xor_sync(0xffffffffu, give, off));
-    }
-  }
-  float s = v[0];
-#pragma unroll
-  for (; off >= 1; off >>= 1) s = __fadd_rn(s, __shfl_xor_sync(0xffffffffu, s, off));
-  return s;
-}
-template <int M>
-__device__ __forceinline__ int transpose_sum_index(int lane) {
-  int idx = 0, off = 16;
-#pragma unroll
-  for (int half = M / 2; half >= 1; half /= 2, off >>= 1)
-    if (lane & off) idx += half;
-  return idx;
-}
-
-template <int NB>
 __global__ void __launch_bounds__(kMarkovThreads) markov_f16_kernel(const uint16_t* __restrict__ W,
                                                                     int V, const float* h,
-                                                                    float* y, int ldy) {
-  constexpr int ROWS = NB == 1 ? 8 : 4;
+                                                                    float* y) {
+  constexpr int ROWS = 8;
   grid_dependency_wait();  // h comes from the kernel before (programmatic launch)
   grid_dependents_launch();
   const int lane = threadIdx.x & 31;
   const int gw = blockIdx.x * (kMarkovThreads / 32) + (threadIdx.x >> 5);
   const int nw = gridDim.x * (kMarkovThreads / 32);
-  float hr[NB][8];
-#pragma unroll
-  for (int b = 0; b < NB; ++b) {
-    const float4 a = __ldg(reinterpret_cast<const float4*>(h + b * kMarkovRank + 8 * lane));
-    const float4 c = __ldg(reinterpret_cast<const float4*>(h + b * kMarkovRank + 8 * lane + 4));
-    hr[b][0] = a.x; hr[b][1] = a.y; hr[b][2] = a.z; hr[b][3] = a.w;
-    hr[b][4] = c.x; hr[b][5] = c.y; hr[b][6] = c.z; hr[b][7] = c.w;
+  float hr[8];
+  {
+    const float4 a = __ldg(reinterpret_cast<const float4*>(h + 8 * lane));
+    const float4 c = __ldg(reinterpret_cast<const float4*>(h + 8 * lane + 4));
+    hr[0] = a.x; hr[1] = a.y; hr[2] = a.z; hr[3] = a.w;
+    hr[4] = c.x; hr[5] = c.y; hr[6] = c.z; hr[7] = c.w;
   }
   for (long long v0 = static_cast<long long>(gw) * ROWS; v0 < V;
        v0 += static_cast<long long>(nw) * ROWS) {
@@ -108,52 +68,16 @@ __global__ void __launch_bounds__(kMarkovThreads) markov_f16_kernel(const uint16
     for (int r = 0; r < ROWS; ++r)
       w[r] = v0 + r < V ? ld_stream16(W + (v0 + r) * kMarkovRank + 8 * lane)
                         : make_uint4(0, 0, 0, 0);
-    if constexpr (NB == 1) {
-      // one state: a butterfly per row, the rows' chains independent of one another
+    // a butterfly per row, the rows' chains independent of one another
 #pragma unroll
-      for (int r = 0; r < ROWS; ++r) {
-        float f[8];
-        unpack_f16x8(w[r], f);
-        float acc = __fmul_rn(f[0], hr[0][0]);
+    for (int r = 0; r < ROWS; ++r) {
+      float f[8];
+      unpack_f16x8(w[r], f);
+      float acc = __fmul_rn(f[0], hr[0]);
 #pragma unroll
-        for (int e = 1; e < 8; ++e) acc = __fmaf_rn(f[e], hr[0][e], acc);
-        acc = warp_sum(acc);
-        if (lane == 0 && v0 + r < V) y[v0 + r] = acc;
-      }
-    } else {
-      constexpr int M = pow2_ceil(ROWS * NB);
-      float part[M];
-#pragma unroll
-      for (int m = ROWS * NB; m < M; ++m) part[m] = 0.f;
-#pragma unroll
-      for (int r = 0; r < ROWS; ++r) {
-        float f[8];
-        unpack_f16x8(w[r], f);
-#pragma unroll
-        for (int b = 0; b < NB; ++b) {
-          if constexpr (NB == 2) {  // (3 or 4 states: packed pairs, fewer instructions)
-            float acc = __fmul_rn(f[0], hr[b][0]);
-#pragma unroll
-            for (int e = 1; e < 8; ++e) acc = __fmaf_rn(f[e], hr[b][e], acc);
-            part[r * NB + b] = acc;
-            continue;
-          }
-          // even and odd elements in the two halves of a packed accumulator
-          uint64_t acc = fma2(pk2(f[0], f[1]), pk2(hr[b][0], hr[b][1]), 0ull);
-#pragma unroll
-          for (int e = 2; e < 8; e += 2)
-            acc = fma2(pk2(f[e], f[e + 1]), pk2(hr[b][e], hr[b][e + 1]), acc);
-          float lo, hi;
-          upk2(acc, lo, hi);
-          part[r * NB + b] = __fadd_rn(lo, hi);
-        }
-      }
-      const float tot = warp_transpose_sum<M>(part, lane);
-      const int idx = transpose_sum_index<M>(lane);
-      if ((lane & (32 / M - 1)) == 0 && idx < ROWS * NB) {
-        const int r = idx / NB, b = idx % NB;
-        if (v0 + r < V) y[static_cast<long long>(b) * ldy + v0 + r] = tot;
-      }
+      for (int e = 1; e < 8; ++e) acc = __fmaf_rn(f[e], hr[e], acc);
+      acc = warp_sum(acc);
+      if (lane == 0 && v0 + r < V) y[v0 + r] = acc;
     }
   }
 }
@@ -170,8 +94,8 @@ __device__ __forceinline__ void cp_async_wait() {
   asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
-// The states as signed-byte digits, for the Q8_0 products on the integer dot-product unit
-// (__dp4a): per state b and table block j (32 values), a power-of-two scale s = 2^x (the
+// The state as signed-byte digits, for the Q8_0 products on the integer dot-product unit
+// (__dp4a): per table block j (32 values), a power-of-two scale s = 2^x (the
 // smallest with max_i |h_i| / s <= 127 over the block; 2^0 for an all-zero block) and three
 // digit planes with
 //   h_i = s (a_i + (b_i + (c_i + e_i) / 254) / 254),   |a_i|, |b_i|, |c_i| <= 127, |e_i| <= 1/2,
@@ -179,7 +103,7 @@ __device__ __forceinline__ void cp_async_wait() {
 // s (A + (B + C / 254) / 254) + err with A = sum_i q_i a_i etc. exact 32-bit dot products of
 // signed bytes (|A| <= 32 * 128 * 127 < 2^22) and |err| <= s / (2 * 254^2) sum_i |q_i|
 // < 2^-22 max_i |h_i| sum_i |q_i| (s < 2 max_i |h_i| / 127); the rest is float32 rounding of
-// the combination. Layout per state: [plane][block][12 words], 8 words of digits and 4 of
+// the combination. Layout: [plane][block][12 words], 8 words of digits and 4 of
 // padding, so that the 8 lanes of a row, one per block, read their 16-byte words from 8
 // disjoint groups of 4 banks.
 constexpr int kQ8Planes = 3;
@@ -194,7 +118,7 @@ __device__ __forceinline__ float mul_pow2(float x, int k) {
                    __int_as_float((k - k1 + 127) << 23));
 }
 
-// One warp: the digits of state b's block j (lane i holds element i) into dig (the state's
+// One warp: the digits of the state's block j (lane i holds element i) into dig (the state's
 // words) and the block's exponent x into ex[j].
 __device__ __forceinline__ void q8_state_digits(float hv, int j, int lane, int8_t* dig, int* ex) {
   const float ah = fabsf(hv);
@@ -228,18 +152,17 @@ __device__ __forceinline__ float small_int_to_float(int x) {
 
 // A warp's groups are double-buffered: the copy of its next group is in flight while it
 // decodes the current one. Lane l takes blocks (row l/8, block l%8) and (row 4 + l/8, block
-// l%8): for each state, three integer dot-product chains over the block's 32 signed bytes
+// l%8): three integer dot-product chains over the block's 32 signed bytes
 // (read as aligned 32-bit words, funnel-shifted when the block starts 2 bytes into a word)
 // against the state's digit planes, then s (A + (B + C / 254) / 254) times the block scale d;
 // the 8 blocks of a row are added by a butterfly over the lanes of the row.
-template <int NB>
-__global__ void __launch_bounds__(kMarkovThreads, NB <= 2 ? 4 : 3) markov_q8_0_kernel(
-    const uint8_t* __restrict__ W, int V, const float* h, float* y, int ldy) {
+__global__ void __launch_bounds__(kMarkovThreads, 4) markov_q8_0_kernel(
+    const uint8_t* __restrict__ W, int V, const float* h, float* y) {
   constexpr int kGroupBytes = kQ8Rows * kQ8RowBytes;  // 2176
   constexpr int kPieces = kGroupBytes / 16;           // 136 16-byte pieces per group
   __shared__ __align__(16) uint8_t s_rows[kMarkovThreads / 32][2][kGroupBytes];
-  __shared__ __align__(16) int8_t s_dig[NB][kQ8StateWords * 4];
-  __shared__ int s_ex[NB][kQ8Blocks];
+  __shared__ __align__(16) int8_t s_dig[kQ8StateWords * 4];
+  __shared__ int s_ex[kQ8Blocks];
   const int lane = threadIdx.x & 31, wi = threadIdx.x >> 5;
   const int blk = lane & 7;
   const int gw = blockIdx.x * (kMarkovThreads / 32) + wi;
@@ -264,17 +187,10 @@ __global__ void __launch_bounds__(kMarkovThreads, NB <= 2 ? 4 : 3) markov_q8_0_k
   long long v0 = static_cast<long long>(gw) * kQ8Rows;
   if (v0 < V) fetch(v0, 0);
   static_assert(kMarkovThreads / 32 == kQ8Blocks, "one warp per table block");
-  // the states' digits: warp w takes (state, block) pairs w, w + 8, ..., all of its state
-  // values loaded before any is used
-  float hvs[NB];
-#pragma unroll
-  for (int u = 0; u < NB; ++u) hvs[u] = __ldg(h + u * kMarkovRank + wi * 32 + lane);
-#pragma unroll
-  for (int u = 0; u < NB; ++u) q8_state_digits(hvs[u], wi, lane, s_dig[u], s_ex[u]);
+  // the state's digits: warp w takes block w
+  q8_state_digits(__ldg(h + wi * 32 + lane), wi, lane, s_dig, s_ex);
   __syncthreads();
-  int xb[NB];  // this lane's block exponent per state
-#pragma unroll
-  for (int b = 0; b < NB; ++b) xb[b] = s_ex[b][blk];
+  const int xb = s_ex[blk];  // this lane's block exponent
   for (int st = 0; v0 < V; v0 += stride, st ^= 1) {
     if (v0 + stride < V) {
       fetch(v0 + stride, st ^ 1);
@@ -300,31 +216,28 @@ __global__ void __launch_bounds__(kMarkovThreads, NB <= 2 ? 4 : 3) markov_q8_0_k
         q[k] = static_cast<int>(__funnelshift_r(lo, hi, sh));
         lo = hi;
       }
+      int acc[kQ8Planes];
 #pragma unroll
-      for (int b = 0; b < NB; ++b) {
-        int acc[kQ8Planes];
-#pragma unroll
-        for (int pl = 0; pl < kQ8Planes; ++pl) {
-          const int4* dg = reinterpret_cast<const int4*>(s_dig[b]) +
-                           (pl * kQ8Blocks + blk) * (kQ8DigWords / 4);
-          const int4 g0 = dg[0], g1 = dg[1];
-          int a = __dp4a(q[0], g0.x, 0);
-          a = __dp4a(q[1], g0.y, a);
-          a = __dp4a(q[2], g0.z, a);
-          a = __dp4a(q[3], g0.w, a);
-          a = __dp4a(q[4], g1.x, a);
-          a = __dp4a(q[5], g1.y, a);
-          a = __dp4a(q[6], g1.z, a);
-          acc[pl] = __dp4a(q[7], g1.w, a);
-        }
-        float f = __fmaf_rn(small_int_to_float(acc[2]), 1.f / 254.f, small_int_to_float(acc[1]));
-        f = __fmaf_rn(f, 1.f / 254.f, small_int_to_float(acc[0]));
-        // d s f; a non-finite state block gives NaN
-        float s = xb[b] == 1024 ? __int_as_float(0x7fc00000) : mul_pow2(__fmul_rn(d, f), xb[b]);
-#pragma unroll
-        for (int o = 1; o < 8; o <<= 1) s = __fadd_rn(s, __shfl_xor_sync(0xffffffffu, s, o));
-        if (blk == 0 && v0 + row < V) y[static_cast<long long>(b) * ldy + v0 + row] = s;
+      for (int pl = 0; pl < kQ8Planes; ++pl) {
+        const int4* dg = reinterpret_cast<const int4*>(s_dig) +
+                         (pl * kQ8Blocks + blk) * (kQ8DigWords / 4);
+        const int4 g0 = dg[0], g1 = dg[1];
+        int a = __dp4a(q[0], g0.x, 0);
+        a = __dp4a(q[1], g0.y, a);
+        a = __dp4a(q[2], g0.z, a);
+        a = __dp4a(q[3], g0.w, a);
+        a = __dp4a(q[4], g1.x, a);
+        a = __dp4a(q[5], g1.y, a);
+        a = __dp4a(q[6], g1.z, a);
+        acc[pl] = __dp4a(q[7], g1.w, a);
       }
+      float f = __fmaf_rn(small_int_to_float(acc[2]), 1.f / 254.f, small_int_to_float(acc[1]));
+      f = __fmaf_rn(f, 1.f / 254.f, small_int_to_float(acc[0]));
+      // d s f; a non-finite state block gives NaN
+      float s = xb == 1024 ? __int_as_float(0x7fc00000) : mul_pow2(__fmul_rn(d, f), xb);
+#pragma unroll
+      for (int o = 1; o < 8; o <<= 1) s = __fadd_rn(s, __shfl_xor_sync(0xffffffffu, s, o));
+      if (blk == 0 && v0 + row < V) y[v0 + row] = s;
     }
     __syncwarp();  // the buffer is refilled two groups on
   }
