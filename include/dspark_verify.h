@@ -261,10 +261,10 @@ typedef enum { DSPARK_TABLE_F16 = 0, DSPARK_TABLE_Q8_0 = 1 } dspark_table_t;
 dspark_status_t dspark_markov_matvec(const void* table, dspark_table_t type, int V, int R,
                                      const float* h, int B, float* y, void* stream);
 
-/* The number of waits inside the library's pipelined kernels (the Q8_0 mat-vec) that ran out
- * (about a second each) on the current device since the library was loaded: 0 unless a kernel
- * gave up; a kernel that gives up frees its resources and leaves its outputs incomplete.
- * Synchronous (waits for the device). DSPARK_ERR_INVALID_ARG for a NULL count. */
+/* The number of waits inside the library's pipelined kernels (the tensor-core mat-vecs) that
+ * ran out (about a second each) on the current device since the library was loaded: 0 unless
+ * a kernel gave up; a kernel that gives up frees its resources and leaves its outputs
+ * incomplete. Synchronous (waits for the device). DSPARK_ERR_INVALID_ARG for a NULL count. */
 dspark_status_t dspark_pipeline_timeouts(unsigned long long* count);
 
 /* For tests of the timeout path only: dspark_markov_matvec with each CTA's first table copy
